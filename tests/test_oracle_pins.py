@@ -1,0 +1,387 @@
+"""Pins for the CPU oracle: it is checked here against things other than itself.
+
+Each test compares the oracle with one of: a value the pages print, a
+hand-derived worked example of the stated definition (tests/golden/), a closed
+form, a library routine that computes the same mathematics a different way, or
+brute force on tiny inputs.  All run on the CPU.
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+from mixed_precision_moe_router_b200 import inputs
+from tests import golden
+
+
+# ----------------------------------------------------------------------------
+# byte accounting and block quantisation
+# ----------------------------------------------------------------------------
+
+def test_byte_accounting_matches_pages():
+    hdr, _ = golden.load("byte_accounting.txt")
+    bpw = oracle.bits_per_weight(hdr["bits"])
+    assert bpw == hdr["bits_per_weight"]
+    gb = hdr["params"] * bpw / 8 / 1e9
+    assert abs(gb - hdr["gigabytes"]) < 0.005
+    # the packed row size plus its scales gives the same cost per weight
+    K = 2048
+    per_row = oracle.packed_row_bytes(K, 4) + 2 * K // 32
+    assert per_row * 8 / K == hdr["bits_per_weight"]
+    assert oracle.packed_row_bytes(K, 3) * 8 / K == 3
+    assert oracle.packed_row_bytes(K, 8) == K
+
+
+def _block(ws):
+    w = np.zeros((1, 32), np.float32)
+    ws = ws if isinstance(ws, list) else [ws]
+    w[0, : len(ws)] = np.asarray(ws, np.float32)
+    return w
+
+
+@pytest.mark.parametrize("case", golden.load("quant_examples.txt")[1], ids=lambda c: c["name"])
+def test_quantize_hand_examples(case):
+    w = _block(case["w"])
+    q, d = oracle.quantize_rows(w, case["bits"])
+    assert float(d[0, 0]) == case["d"]
+    exp = case["q"] if isinstance(case["q"], list) else [case["q"]]
+    assert q[0, : len(exp)].tolist() == exp
+    assert not q[0, len(exp):].any()
+
+
+@pytest.mark.parametrize("bits", [8, 4, 3])
+def test_quantize_roundtrip_bound(bits):
+    rng = np.random.default_rng(bits)
+    w = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    w[3, :32] *= 1e-4  # a block with a tiny scale
+    w[5, 32:64] = 0.0  # an all-zero block
+    packed, d = oracle.quantize_pack(w, bits)
+    back = oracle.dequantize_f32(packed, d, bits, 256)
+    blocks = w.reshape(64, 8, 32)
+    amax = np.abs(blocks).max(axis=2, keepdims=True).astype(np.float64)
+    dd = d.astype(np.float64)[..., None]
+    err = np.abs(back.reshape(64, 8, 32) - blocks.astype(np.float64))
+    assert np.all(err <= dd / 2 + amax * 2.0 ** -11 + 1e-30)
+    assert np.all(back.reshape(64, 8, 32)[5, 1] == 0)
+    # every code stays within +-qmax and the block maximum reaches +-qmax
+    q, _ = oracle.quantize_rows(w, bits)
+    qmax = oracle.QMAX[bits]
+    assert np.abs(q).max() <= qmax
+    top = np.abs(q.reshape(64, 8, 32)).max(axis=2)
+    # (only for normal fp16 scales: a subnormal scale is rounded coarsely)
+    normal = d.astype(np.float64) >= 2.0 ** -14
+    assert np.all(top[normal] == qmax)
+
+
+def test_quantize_uses_division_not_reciprocal():
+    """Find weights where w/d and w*(1/d) round to different codes; the definition
+    (fp32 division, half away from zero) decides, and the oracle must follow it."""
+    d = np.float32(np.float16(0.0999755859375))
+    found = 0
+    for n in range(1, 127):
+        target = np.float32((n + 0.5) * float(d))
+        for cand in (np.nextafter(target, np.float32(0)), target, np.nextafter(target, np.float32(1e9))):
+            cand = np.float32(cand)
+            by_div = np.float32(cand / d)
+            by_rcp = np.float32(cand * np.float32(np.float32(1) / d))
+            if by_div == by_rcp:
+                continue
+            # block: the maximum pins d to exactly fp16(0.1) * 127 / 127
+            w = np.zeros((1, 32), np.float32)
+            w[0, 0] = np.float32(127) * d
+            w[0, 1] = cand
+            q, dq = oracle.quantize_rows(w, 8)
+            assert np.float32(dq[0, 0]) == d
+            r = Fraction(float(by_div))
+            expect = int(math.floor(r + Fraction(1, 2)))  # r > 0: half away from zero
+            assert q[0, 1] == min(expect, 127)
+            found += 1
+    assert found > 0
+
+
+# ----------------------------------------------------------------------------
+# packing
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", golden.load("pack_examples.txt")[1], ids=lambda c: c["name"])
+def test_pack_hand_examples(case):
+    q = np.zeros((1, 32), np.int64)
+    qs = case["q"] if isinstance(case["q"], list) else [case["q"]]
+    q[0, : len(qs)] = qs
+    packed = oracle.pack_rows(q, case["bits"])
+    expect = [int(str(b), 16) for b in case["bytes"]]
+    assert packed[0].tolist() == expect
+    assert oracle.unpack_rows(packed, case["bits"], 32).tolist() == q.tolist()
+
+
+@pytest.mark.parametrize("bits", [8, 4, 3])
+def test_pack_roundtrip_all_codes(bits):
+    qmax = oracle.QMAX[bits]
+    rng = np.random.default_rng(10 + bits)
+    q = rng.integers(-qmax, qmax + 1, size=(7, 256))
+    q[0, : 2 * qmax + 1] = np.arange(-qmax, qmax + 1)
+    packed = oracle.pack_rows(q, bits)
+    assert packed.shape == (7, oracle.packed_row_bytes(256, bits))
+    assert np.array_equal(oracle.unpack_rows(packed, bits, 256), q)
+
+
+def test_dequant_is_exact_product():
+    rng = np.random.default_rng(3)
+    for bits in (8, 4, 3):
+        w = (rng.standard_normal((4, 64)) * 0.02).astype(np.float32)
+        q, d = oracle.quantize_rows(w, bits)
+        packed = oracle.pack_rows(q, bits)
+        f32 = oracle.dequantize_f32(packed, d, bits, 64)
+        for r in range(4):
+            for i in range(64):
+                exact = Fraction(float(d[r, i // 32])) * int(q[r, i])
+                assert Fraction(float(f32[r, i])) == exact
+        f16 = oracle.dequantize_f16(packed, d, bits, 64)
+        ref = torch.from_numpy(f32).to(torch.float16).numpy()  # library RNE fp32 -> fp16
+        assert np.array_equal(f16.view(np.uint16), ref.view(np.uint16))
+
+
+# ----------------------------------------------------------------------------
+# router / top-k / weights
+# ----------------------------------------------------------------------------
+
+def _bf16_values(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16).float().numpy()
+
+
+def test_router_logits_exact_on_bf16_inputs():
+    x = _bf16_values((3, 64), 1)
+    w = _bf16_values((5, 64), 2, 0.02)
+    b = np.array([0.5, -0.25, 0.0, 1.0, -2.0], np.float32)
+    L = oracle.router_logits(x, w, b)
+    for t in range(3):
+        for e in range(5):
+            exact = sum(Fraction(float(x[t, h])) * Fraction(float(w[e, h])) for h in range(64))
+            exact += Fraction(float(b[e]))
+            assert abs(Fraction(L[t, e]) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
+
+
+def test_topk_brute_force():
+    rng = np.random.default_rng(5)
+    for trial in range(20):
+        E = int(rng.integers(2, 40))
+        k = int(rng.integers(1, E + 1))
+        L = np.round(rng.standard_normal((4, E)), 1)  # coarse values -> many ties
+        idx, w = oracle.select_topk(L, k)
+        for t in range(4):
+            ranked = sorted(range(E), key=lambda e: (-L[t, e], e))[:k]
+            assert idx[t].tolist() == ranked
+            z = [math.exp(L[t, e]) for e in ranked]
+            assert np.allclose(w[t], [v / math.fsum(z) for v in z], rtol=1e-13, atol=0)
+
+
+def test_topk_ties_go_to_lower_id():
+    L = np.array([[1.0, 3.0, 3.0, 2.0, 3.0, 0.0]])
+    idx, w = oracle.select_topk(L, 4)
+    assert idx[0].tolist() == [1, 2, 4, 3]
+    assert np.allclose(w[0, :3], w[0, 0])
+
+
+def test_topk_full_k_is_softmax():
+    rng = np.random.default_rng(6)
+    L = rng.standard_normal((3, 16)) * 3
+    idx, w = oracle.select_topk(L, 16)
+    p = scipy.special.softmax(L, axis=1)
+    for t in range(3):
+        assert np.allclose(w[t], p[t, idx[t]], rtol=1e-12, atol=0)
+
+
+def test_topk_weights_renormalised_softmax():
+    rng = np.random.default_rng(7)
+    L = rng.standard_normal((5, 32))
+    idx, w = oracle.select_topk(L, 6)
+    p = scipy.special.softmax(L, axis=1)
+    for t in range(5):
+        sel = p[t, idx[t]]
+        assert np.allclose(w[t], sel / sel.sum(), rtol=1e-12)
+        assert abs(w[t].sum() - 1) < 1e-12
+        assert np.all(np.diff(w[t]) <= 0)
+    # a constant shift of all logits changes nothing
+    idx2, w2 = oracle.select_topk(L + 123.0, 6)
+    assert np.array_equal(idx, idx2) and np.allclose(w, w2, rtol=1e-12)
+
+
+def test_topk_margin():
+    L = np.array([[5.0, 4.0, 3.5, 3.4, 0.0]])
+    assert oracle.topk_margin(L, 2)[0] == pytest.approx(0.5)
+    assert oracle.topk_margin(L, 3)[0] == pytest.approx(0.1)
+
+
+# ----------------------------------------------------------------------------
+# bucketize
+# ----------------------------------------------------------------------------
+
+def test_bucketize_brute_force():
+    rng = np.random.default_rng(8)
+    for trial in range(30):
+        E = int(rng.integers(1, 20))
+        k = int(rng.integers(1, E + 1))
+        T = int(rng.integers(0, 12))
+        idx = np.array([rng.permutation(E)[:k] for _ in range(T)], np.int32).reshape(T, k)
+        off, srt, pos = oracle.bucketize(idx, E)
+        pairs = sorted((int(e), s) for s, e in enumerate(idx.reshape(-1)))
+        assert srt.tolist() == [s for _, s in pairs]
+        for e in range(E):
+            assert off[e + 1] - off[e] == sum(1 for p in pairs if p[0] == e)
+        assert off[0] == 0 and off[E] == T * k
+        assert np.array_equal(srt[pos], np.arange(T * k))
+
+
+# ----------------------------------------------------------------------------
+# FFN, combine, rounding
+# ----------------------------------------------------------------------------
+
+def test_silu_closed_form():
+    g = np.array([-30.0, -1.0, 0.0, 1.0, 2.5, 30.0])
+    assert np.allclose(oracle.silu(g), g * scipy.special.expit(g), rtol=1e-15, atol=1e-300)
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    assert oracle.silu(np.array([1.0]))[0] == pytest.approx(0.7310585786300049, rel=1e-15)
+
+
+def test_ffn_identity_weights_closed_form():
+    """With W_gate = c*I, W_up = I, W_down = I the layer is y = silu(c x) * x
+    elementwise: a swapped gate/up, a transposed operand or a missing factor fails."""
+    n = 8
+    c = 1.7
+    wgu = np.concatenate([c * np.eye(n), np.eye(n)])
+    x = np.linspace(-3, 3, 2 * n).reshape(2, n)
+    y = oracle.expert_ffn(x, wgu, np.eye(n))
+    assert np.allclose(y, c * x * scipy.special.expit(c * x) * x, rtol=1e-14, atol=1e-15)
+    # a permutation as W_down permutes the output
+    P = np.eye(n)[::-1]
+    assert np.allclose(oracle.expert_ffn(x, wgu, P), y[:, ::-1], rtol=1e-14)
+
+
+def test_round_bf16_matches_library_on_fp32_values():
+    rng = np.random.default_rng(9)
+    v = np.concatenate([rng.standard_normal(5000) * 10.0 ** rng.integers(-30, 30, 5000),
+                        [0.0, -0.0, 1e-40, -3e-39, 3.0e38]]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).float().numpy().astype(np.float64)
+    assert np.array_equal(oracle.round_bf16(v.astype(np.float64)), ref)
+
+
+def test_round_bf16_ties_and_single_rounding():
+    one = 1.0
+    assert oracle.round_bf16(np.array([one + 2 ** -8]))[0] == 1.0  # tie -> even
+    assert oracle.round_bf16(np.array([one + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
+    # just above the tie: a double rounding through fp32 would land on the tie and go
+    # to even (1.0); the correct single rounding goes up
+    v = one + 2 ** -8 + 2 ** -40
+    assert oracle.round_bf16(np.array([v]))[0] == 1 + 2 ** -7
+
+
+def test_combine_single_slot_is_rounding():
+    rng = np.random.default_rng(10)
+    y = rng.standard_normal((3, 16))
+    out = oracle.combine(y, None, np.ones((3, 1)))
+    assert np.array_equal(out, oracle.round_bf16(y))
+    out2, nxt = oracle.combine(y, np.zeros((3, 16)), np.ones((3, 1)), residual=np.ones((3, 16)))
+    assert np.array_equal(out2, out)
+    assert np.array_equal(nxt, oracle.round_bf16(1.0 + out))
+
+
+# ----------------------------------------------------------------------------
+# the whole layer: brute-force dense evaluation and tier-split invariance
+# ----------------------------------------------------------------------------
+
+def _tiny_layer(shelf_split=None):
+    cfg = inputs.TINY
+    seed = inputs.layer_seed(cfg)
+    x = inputs.activations(8, cfg.H, seed=seed).float().numpy()
+    wr, bias = inputs.router(cfg, seed)
+    wr = wr.float().numpy()
+    src = [tuple(t.numpy() for t in inputs.expert_source(cfg, seed, e)) for e in range(cfg.E + 1)]
+    ranges = shelf_split or cfg.tier_ranges()
+    shelves = [oracle.build_shelf(bits, first, src[first:first + n]) for bits, first, n in ranges]
+    shared = oracle.build_shelf(8, cfg.E, [src[cfg.E]])
+    return cfg, x, wr, bias, shelves, shared
+
+
+def test_layer_brute_force_dense():
+    """Every expert evaluated for every token, masked by the top-k and weighted,
+    must equal the sparse routed evaluation."""
+    cfg, x, wr, bias, shelves, shared = _tiny_layer()
+    res = oracle.moe_layer(x, wr, bias, cfg.k, shelves, shared, cfg.H, cfg.I)
+    T = x.shape[0]
+    # brute force: independent loops over (token, expert)
+    logits = np.zeros((T, cfg.E))
+    for t in range(T):
+        for e in range(cfg.E):
+            logits[t, e] = math.fsum(float(a) * float(b) for a, b in zip(x[t], wr[e]))
+    dense = np.zeros((T, cfg.E, cfg.H))
+    for e in range(cfg.E):
+        wgu, wdn = oracle.shelf_of(shelves, e).weights(e, cfg.H, cfg.I)
+        for t in range(T):
+            g = wgu[: cfg.I].astype(np.float64) @ x[t]
+            u = wgu[cfg.I:].astype(np.float64) @ x[t]
+            h = g * scipy.special.expit(g) * u
+            dense[t, e] = wdn.astype(np.float64) @ h
+    wgu, wdn = shared.weights(cfg.E, cfg.H, cfg.I)
+    total = np.zeros((T, cfg.H))
+    for t in range(T):
+        order = sorted(range(cfg.E), key=lambda e: (-logits[t, e], e))[: cfg.k]
+        p = scipy.special.softmax(logits[t])
+        mask = np.zeros(cfg.E)
+        mask[order] = p[order] / p[order].sum()
+        g = wgu[: cfg.I].astype(np.float64) @ x[t]
+        u = wgu[cfg.I:].astype(np.float64) @ x[t]
+        total[t] = mask @ dense[t] + wdn.astype(np.float64) @ (g * scipy.special.expit(g) * u)
+        assert res["topk_idx"][t].tolist() == order
+    pre = np.einsum("tj,tjh->th", res["topk_w"], res["y_slots"].reshape(T, cfg.k, -1)) + res["y_shared"]
+    assert np.allclose(pre, total, rtol=1e-12, atol=1e-14)
+    assert np.array_equal(res["out"], oracle.round_bf16(total)) or \
+        np.max(np.abs(res["out"] - oracle.round_bf16(total))) <= 2 ** -8 * np.abs(total).max()
+    assert np.allclose(res["topk_w"].sum(axis=1), 1.0, atol=1e-12)
+
+
+def test_layer_tier_split_invariance():
+    """The same 8-bit weights in one table or split over three tables give the same
+    output: each shelf computes only its ids and the results add up."""
+    cfg = inputs.TINY
+    one = _tiny_layer(shelf_split=[(8, 0, 16)])
+    three = _tiny_layer(shelf_split=[(8, 0, 5), (8, 5, 2), (8, 7, 9)])
+    r1 = oracle.moe_layer(*one[1:4], cfg.k, one[4], one[5], cfg.H, cfg.I)
+    r3 = oracle.moe_layer(*three[1:4], cfg.k, three[4], three[5], cfg.H, cfg.I)
+    assert np.array_equal(r1["out"], r3["out"])
+
+
+# ----------------------------------------------------------------------------
+# the synthetic workload reproduces the pages' routing skew
+# ----------------------------------------------------------------------------
+
+def test_zipf_routing_share():
+    hdr, _ = golden.load("routing_skew.txt")
+    cfg = inputs.DECODE
+    x = inputs.activations(4096, cfg.H, seed=inputs.X_SEED).float().numpy()
+    wr, bias = inputs.router(cfg, inputs.layer_seed(cfg, 0))
+    L = oracle.router_logits(x, wr.float().numpy(), bias.numpy())
+    idx, _ = oracle.select_topk(L, cfg.k)
+    counts = np.bincount(idx.reshape(-1), minlength=cfg.E)
+    top = int(cfg.E * hdr["top_fraction"])
+    share = np.sort(counts)[::-1][:top].sum() / counts.sum()
+    assert abs(share - hdr["token_share"]) < hdr["tolerance"]
+    # ids are popularity ranks: the 8-bit tier (ids < 128) carries that share
+    assert abs(counts[:128].sum() / counts.sum() - hdr["token_share"]) < hdr["tolerance"] + 0.01
+
+
+def test_draft_batch_overlap():
+    """Correlated drafts share about 60% of the base token's top-10 experts."""
+    cfg = inputs.DECODE
+    wr, bias = inputs.router(cfg, inputs.layer_seed(cfg, 0))
+    overlaps = []
+    for s in range(8):
+        x = inputs.correlated_activations(5, cfg.H, seed=100 + s).float().numpy()
+        idx, _ = oracle.select_topk(oracle.router_logits(x, wr.float().numpy(), bias.numpy()), cfg.k)
+        base = set(idx[0].tolist())
+        overlaps += [len(base & set(idx[t].tolist())) / cfg.k for t in range(1, 5)]
+    assert 0.45 < float(np.mean(overlaps)) < 0.75
