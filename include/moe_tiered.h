@@ -1,0 +1,251 @@
+/*
+ * moe_tiered.h -- C ABI of the tiered mixed-precision MoE layer (B200, sm_100a).
+ *
+ * One routed mixture-of-experts FFN layer in which a single routing decision
+ * drives several expert tables ("shelves") stored at different precisions:
+ * popular experts in 8-bit blocks, rarer ones in 4-bit and 3-bit blocks.
+ *
+ * Sources, cited by page title and section:
+ *   [P1] "I ran a 125B model on three RTX 3090s at 80 tokens/s by teaching
+ *        llama.cpp which experts matter" (dev.to)
+ *   [P2] "Running Qwen3.8-Flash-Next 125B on Three RTX 3090s at 80 Tokens per
+ *        Second" (n1n.ai)
+ *   [P3] "flashnext-2x3090" README (gitlite mirror)
+ *   [P5] "Qwen3.8-Flash-Next hits 39 tok/s on a 24GB GPU, provided you bring
+ *        96GB of system RAM" (deniz.in)
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise; the
+ *     caller allocates and owns all of them.  The library never allocates,
+ *     frees or synchronises: each call only enqueues kernels on `stream`
+ *     (a cudaStream_t; NULL is the legacy default stream).
+ *   - Tensors are dense, row-major, with the last index contiguous.  bf16 and
+ *     fp16 values are passed as their uint16_t bit patterns.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Expert ids are signed int32.  No call ever writes a "skip" sentinel as an
+ *     expert id, and no id reaches an address computation before it has been
+ *     range-checked ([P1] "the four bugs, briefly": a -1 "skip" promoted to
+ *     unsigned read four billion rows past a buffer).
+ *   - Return value: MOE_OK, or an error code after which nothing was enqueued;
+ *     moe_last_error() then describes it (per host thread).  Errors found by a
+ *     kernel (data-dependent) are OR-ed into an optional device status word as
+ *     MOE_STATUS_* bits; the caller clears it and reads it when it wants.
+ *   - Calls are asynchronous and contain no host synchronisation, so a
+ *     sequence of them can be captured into a CUDA graph.
+ */
+#ifndef MOE_TIERED_H
+#define MOE_TIERED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+/* return codes */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG 1 /* a size, pointer, alignment or layout is invalid */
+#define MOE_ERR_UNSUPPORTED 2 /* valid, but outside what the kernels implement */
+#define MOE_ERR_WORKSPACE 3   /* workspace missing or smaller than required */
+#define MOE_ERR_CUDA 4        /* a CUDA launch failed */
+
+/* device status bits (OR-ed into the optional int32 status word) */
+#define MOE_STATUS_BAD_EXPERT_ID 0x1 /* an id outside [0,E) was seen and skipped;
+                                        outputs of that token are undefined */
+#define MOE_STATUS_FP16_RANGE 0x2    /* the tensor-core path met an activation
+                                        beyond the fp16 range (|v| > 65504) */
+#define MOE_STATUS_TIMEOUT 0x4       /* a bounded device-side wait gave up */
+
+#define MOE_BLOCK 32     /* weights per quantisation block (one fp16 scale) */
+#define MOE_MAX_TIERS 4  /* shelves per layer */
+#define MOE_MAX_TOPK 32
+#define MOE_MAX_EXPERTS 1024
+
+/*
+ * Packed shelf format ([P1] "step 4: three shelves, all on the GPU": each
+ * shelf is one expert table at one precision; [P3] "Why the model fits at
+ * all": a 4-bit code plus a 16-bit scale per 32 weights is 4.5 bits/weight).
+ *
+ * A weight matrix [rows][K] (K % 64 == 0) is stored as two arrays:
+ *   qs    uint8  [rows][K*bits/8]   codes, row by row
+ *   scale uint16 [rows][K/32]       fp16 scale d of each block of 32 weights
+ * and dequantises to w = d * q (exact in fp32).  Per block of 32:
+ *   d = fp16_rne(fp32(amax) / fp32(qmax)), qmax = 2^(bits-1) - 1,
+ *   q = clamp(round_half_away(fp32(w) / fp32(d)), -qmax, qmax); d == 0 -> q = 0.
+ * Codes within a row:
+ *   bits 8: the int8 value q.
+ *   bits 4: c = q + 8; weight 2m in the low nibble of byte m, 2m+1 in the high.
+ *   bits 3: c = q + 4; a low plane of K/4 bytes (bits 0-1 of weight i at bit
+ *           2*(i%4) of byte i/4) followed by a high plane of K/8 bytes (bit 2
+ *           of weight i at bit i%8 of byte K/4 + i/8).
+ */
+size_t moe_packed_row_bytes(int32_t K, int32_t bits);
+
+/*
+ * One shelf: experts [first_expert, first_expert + n_experts) at `bits`.
+ * Per expert (expert j of the shelf at index j), hidden H, intermediate I:
+ *   gu_qs    [n_experts][2*I][H*bits/8]   gate rows 0..I-1, up rows I..2I-1
+ *   gu_scale [n_experts][2*I][H/32]
+ *   dn_qs    [n_experts][H][I*bits/8]
+ *   dn_scale [n_experts][H][I/32]
+ */
+typedef struct moe_tier {
+    int32_t bits;          /* 8, 4 or 3 */
+    int32_t first_expert;  /* first id of this shelf's contiguous id range */
+    int32_t n_experts;     /* experts on the shelf (0 for an unused shared slot) */
+    int32_t reserved;      /* must be 0 */
+    const uint8_t *gu_qs;
+    const uint16_t *gu_scale;
+    const uint8_t *dn_qs;
+    const uint16_t *dn_scale;
+} moe_tier;
+
+/*
+ * A layer's expert weights ([P1] "step 4": experts are reordered hottest-first
+ * into one table per precision).  The shelves must cover the ids [0, E)
+ * exactly, without overlap.  `shared` is the always-on shared expert
+ * ([P5] "What the model actually is": 10 routed plus 1 shared expert);
+ * shared.n_experts is 1, or 0 for a layer without one; shared.first_expert
+ * is ignored.  The descriptor itself is a HOST struct, read during the call.
+ */
+typedef struct moe_layer_weights {
+    int32_t H;        /* hidden size, % 64 == 0 */
+    int32_t I;        /* expert intermediate size, % 64 == 0 */
+    int32_t E;        /* routed experts, 1..MOE_MAX_EXPERTS */
+    int32_t n_tiers;  /* 1..MOE_MAX_TIERS */
+    moe_tier tiers[MOE_MAX_TIERS];
+    moe_tier shared;
+} moe_layer_weights;
+
+/* FFN execution path */
+#define MOE_FFN_AUTO 0 /* per expert: GEMV below the token threshold, GEMM above */
+#define MOE_FFN_GEMV 1 /* every expert through the CUDA-core GEMV */
+#define MOE_FFN_GEMM 2 /* every expert through the tcgen05 GEMM */
+
+/* Description of the most recent error on the calling host thread. */
+const char *moe_last_error(void);
+const char *moe_version(void);
+
+/*
+ * moe_quantize: source fp32 rows -> packed shelf rows (format above).
+ *   src   float  [rows][K]  (device)
+ *   qs    uint8  [rows][K*bits/8], scale uint16 [rows][K/32]  (device, written)
+ * The codes and scales are bit-identical to the definition above.
+ */
+int moe_quantize(const float *src, int64_t rows, int32_t K, int32_t bits,
+                 uint8_t *qs, uint16_t *scale, moe_stream_t stream);
+
+/*
+ * moe_dequantize: packed rows -> w = d*q as fp32 (exact) and/or as the fp16
+ * value fp16_rne(d*q) that the tensor-core path stages.  Either output may be
+ * NULL, not both.  Sizes [rows][K].
+ */
+int moe_dequantize(const uint8_t *qs, const uint16_t *scale, int64_t rows,
+                   int32_t K, int32_t bits, float *out_f32, uint16_t *out_f16,
+                   moe_stream_t stream);
+
+/*
+ * moe_router_topk: the router ([P1] "a small dictionary": a router picks the
+ * best 10 of 512 experts for each word).
+ *   logit[t,e] = sum_h x[t,h] * w_router[e,h] + bias[e]    (fp32 accumulate)
+ *   topk_idx[t,j] = the k largest logits, ordered by (logit desc, id asc)
+ *   topk_w[t,j]   = exp(l_j - l_0) / sum_{i<k} exp(l_i - l_0)
+ *                   (the softmax over all E restricted to the k, renormalised)
+ *   x        bf16 [T][H];  w_router bf16 [E][H];  bias fp32 [E] or NULL
+ *   logits   fp32 [T][E] or NULL (written when given)
+ *   topk_idx int32 [T][k];  topk_w fp32 [T][k]
+ *   workspace: moe_router_workspace_size() bytes (may be 0 -> NULL allowed)
+ * Limits: 1 <= k <= min(E, MOE_MAX_TOPK), E <= MOE_MAX_EXPERTS, H % 64 == 0.
+ * T == 0 enqueues nothing.
+ */
+size_t moe_router_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
+int moe_router_topk(const uint16_t *x, const uint16_t *w_router, const float *bias,
+                    int32_t T, int32_t H, int32_t E, int32_t k, float *logits,
+                    int32_t *topk_idx, float *topk_w, void *workspace,
+                    size_t workspace_bytes, moe_stream_t stream);
+
+/* moe_topk_softmax: the selection and weights of moe_router_topk, applied to
+ * given fp32 logits [T][E].  Same outputs, same limits. */
+int moe_topk_softmax(const float *logits, int32_t T, int32_t E, int32_t k,
+                     int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
+/*
+ * moe_bucketize: token -> expert grouping ([P1] "the four bugs, briefly": the
+ * grouping helper must see each expert at most once per token and must never
+ * drop a slot).  Slot s = t*k + j.
+ *   expert_offsets int32 [E+1]: exclusive prefix sum of per-expert counts
+ *   sorted_slot    int32 [T*k]: the slots of expert e, ascending, at
+ *                               [expert_offsets[e], expert_offsets[e+1])
+ *   slot_pos       int32 [T*k]: inverse map, sorted_slot[slot_pos[s]] == s
+ *   active         int32 [E+1]: active[0] = number of experts with at least
+ *                               one slot, then their ids ascending
+ *   status         int32 [1] or NULL: MOE_STATUS_BAD_EXPERT_ID if an id is
+ *                               outside [0,E); that slot is left out
+ *                               (slot_pos[s] = -1).
+ * Limits: T*k <= 2^24.
+ */
+int moe_bucketize(const int32_t *topk_idx, int32_t T, int32_t k, int32_t E,
+                  int32_t *expert_offsets, int32_t *sorted_slot, int32_t *slot_pos,
+                  int32_t *active, int32_t *status, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn_tiered: the tiered SwiGLU expert FFN ([P1] "step 4":
+ * mul_mat_id takes an id range, each shelf computes only the ids on it, and
+ * the shelf results add up; the decode path fuses gate, up and activation).
+ * Every (expert e, slot s) pair with expert_offsets/sorted_slot/active from
+ * moe_bucketize, plus the shared expert for every token:
+ *   g = W_gate[e] x[t], u = W_up[e] x[t], h = silu(g) * u, y = W_down[e] h
+ *   y_slots  fp32 [T*k][H]  (row s = t*k+j)
+ *   y_shared fp32 [T][H]    (NULL iff the layer has no shared expert)
+ * `mode` is MOE_FFN_AUTO / _GEMV / _GEMM.  The GEMV path dequantises to fp32
+ * (exact) and accumulates in fp32; the GEMM path stages w, x and h in fp16 and
+ * accumulates in fp32 (tcgen05), reporting MOE_STATUS_FP16_RANGE if x or h
+ * leaves the fp16 range.
+ * workspace: moe_ffn_workspace_size() bytes.
+ */
+size_t moe_ffn_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k,
+                              int32_t mode);
+int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t T,
+                          int32_t k, const int32_t *expert_offsets,
+                          const int32_t *sorted_slot, const int32_t *active,
+                          float *y_slots, float *y_shared, void *workspace,
+                          size_t workspace_bytes, int32_t mode, int32_t *status,
+                          moe_stream_t stream);
+
+/*
+ * moe_combine: out[t] = bf16_rne( sum_{j<k} topk_w[t,j] * y_slots[t*k+j]
+ *                                 + y_shared[t] )
+ * summed in that fixed order ([P1] "step 4": the results simply add up).
+ * With residual != NULL also x_next[t] = bf16_rne(residual[t] + out[t]).
+ *   y_slots fp32 [T*k][H]; y_shared fp32 [T][H] or NULL; topk_w fp32 [T][k]
+ *   residual bf16 [T][H] or NULL; out bf16 [T][H]; x_next bf16 [T][H] (needed
+ *   iff residual is given).
+ */
+int moe_combine(const float *y_slots, const float *y_shared, const float *topk_w,
+                int32_t T, int32_t k, int32_t H, const uint16_t *residual,
+                uint16_t *out, uint16_t *x_next, moe_stream_t stream);
+
+/*
+ * moe_layer_forward: router -> bucketize -> tiered FFN -> combine, with every
+ * intermediate in `workspace` (moe_layer_workspace_size() bytes).
+ *   x bf16 [T][H]; w_router bf16 [E][H]; bias fp32 [E] or NULL
+ *   out bf16 [T][H]; with residual != NULL (normally residual == x) also
+ *   x_next = bf16(residual + out).
+ * Same limits as the calls it chains.  Capturable into a CUDA graph.
+ */
+size_t moe_layer_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k,
+                                int32_t mode);
+int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router,
+                      const float *bias, const uint16_t *x, int32_t T, int32_t k,
+                      const uint16_t *residual, uint16_t *out, uint16_t *x_next,
+                      void *workspace, size_t workspace_bytes, int32_t mode,
+                      int32_t *status, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_TIERED_H */

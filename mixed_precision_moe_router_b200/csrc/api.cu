@@ -1,0 +1,376 @@
+// C ABI entry points: argument validation, workspace carving and launches.
+// Every check here runs on the host before anything is enqueued; nothing here
+// allocates, frees or synchronises.
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "ffn.cuh"
+
+// launchers defined next to their kernels
+cudaError_t moe_launch_quantize(const float *, int64_t, int, int, uint8_t *, uint16_t *, cudaStream_t);
+cudaError_t moe_launch_dequantize(const uint8_t *, const uint16_t *, int64_t, int, int, float *, uint16_t *,
+                                  cudaStream_t);
+cudaError_t moe_configure_router();
+cudaError_t moe_launch_router_logits(const uint16_t *, const uint16_t *, const float *, int, int, int, float *,
+                                     cudaStream_t);
+cudaError_t moe_launch_topk(const float *, int, int, int, int32_t *, float *, cudaStream_t);
+cudaError_t moe_configure_bucketize();
+cudaError_t moe_launch_bucketize(const int32_t *, int, int, int32_t *, int32_t *, int32_t *, int32_t *, int32_t *,
+                                 cudaStream_t);
+cudaError_t moe_configure_ffn_gemv();
+cudaError_t moe_launch_ffn_gemv(const moe::FfnParams &, cudaStream_t);
+cudaError_t moe_configure_ffn_gemm();
+cudaError_t moe_launch_ffn_gemm(const moe::FfnParams &, void *ws, size_t ws_bytes, cudaStream_t);
+size_t moe_ffn_gemm_workspace(const moe_layer_weights *, int T, int k);
+cudaError_t moe_launch_combine(const float *, const float *, const float *, int, int, int, const uint16_t *,
+                               uint16_t *, uint16_t *, cudaStream_t);
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int ok() {
+    g_err.clear();
+    return MOE_OK;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Kernel attributes (dynamic shared memory limits) are set once per device.
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+cudaError_t g_dev_err[kMaxDevices];
+
+int ensure_configured() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::call_once(g_dev_once[dev], [dev]() {
+        cudaError_t r = moe_configure_router();
+        if (r == cudaSuccess) r = moe_configure_bucketize();
+        if (r == cudaSuccess) r = moe_configure_ffn_gemv();
+        if (r == cudaSuccess) r = moe_configure_ffn_gemm();
+        g_dev_err[dev] = r;
+    });
+    if (g_dev_err[dev] != cudaSuccess) return cuda_fail(g_dev_err[dev], "kernel configuration");
+    return MOE_OK;
+}
+
+bool valid_bits(int b) { return b == 8 || b == 4 || b == 3; }
+
+size_t align_up(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+int check_tier(const moe_tier &t, const char *name, int idx) {
+    if (!valid_bits(t.bits)) return fail(MOE_ERR_INVALID_ARG, "%s[%d].bits = %d (want 8, 4 or 3)", name, idx, t.bits);
+    if (t.reserved != 0) return fail(MOE_ERR_INVALID_ARG, "%s[%d].reserved must be 0", name, idx);
+    if (!t.gu_qs || !t.gu_scale || !t.dn_qs || !t.dn_scale)
+        return fail(MOE_ERR_INVALID_ARG, "%s[%d] has a NULL table pointer", name, idx);
+    if (!aligned16(t.gu_qs) || !aligned16(t.gu_scale) || !aligned16(t.dn_qs) || !aligned16(t.dn_scale))
+        return fail(MOE_ERR_INVALID_ARG, "%s[%d] table pointer not 16-byte aligned", name, idx);
+    return MOE_OK;
+}
+
+int check_weights(const moe_layer_weights *w) {
+    if (!w) return fail(MOE_ERR_INVALID_ARG, "weights descriptor is NULL");
+    if (w->H <= 0 || w->H % 128 != 0) return fail(MOE_ERR_INVALID_ARG, "H = %d must be a positive multiple of 128", w->H);
+    if (w->I <= 0 || w->I % 128 != 0) return fail(MOE_ERR_INVALID_ARG, "I = %d must be a positive multiple of 128", w->I);
+    if (w->H > 16384 || w->I > 16384) return fail(MOE_ERR_UNSUPPORTED, "H and I are limited to 16384");
+    if (w->E < 1 || w->E > MOE_MAX_EXPERTS) return fail(MOE_ERR_INVALID_ARG, "E = %d outside [1, %d]", w->E, MOE_MAX_EXPERTS);
+    if (w->n_tiers < 1 || w->n_tiers > MOE_MAX_TIERS)
+        return fail(MOE_ERR_INVALID_ARG, "n_tiers = %d outside [1, %d]", w->n_tiers, MOE_MAX_TIERS);
+    long covered = 0;
+    for (int i = 0; i < w->n_tiers; ++i) {
+        const moe_tier &t = w->tiers[i];
+        if (t.n_experts < 1) return fail(MOE_ERR_INVALID_ARG, "tiers[%d].n_experts = %d", i, t.n_experts);
+        if (t.first_expert < 0 || t.first_expert + t.n_experts > w->E)
+            return fail(MOE_ERR_INVALID_ARG, "tiers[%d] id range [%d, %d) outside [0, %d)", i, t.first_expert,
+                        t.first_expert + t.n_experts, w->E);
+        for (int j = 0; j < i; ++j) {
+            const moe_tier &o = w->tiers[j];
+            if (t.first_expert < o.first_expert + o.n_experts && o.first_expert < t.first_expert + t.n_experts)
+                return fail(MOE_ERR_INVALID_ARG, "tiers[%d] and tiers[%d] overlap", j, i);
+        }
+        covered += t.n_experts;
+        int r = check_tier(t, "tiers", i);
+        if (r) return r;
+    }
+    if (covered != w->E) return fail(MOE_ERR_INVALID_ARG, "tiers cover %ld of %d expert ids", covered, w->E);
+    if (w->shared.n_experts != 0 && w->shared.n_experts != 1)
+        return fail(MOE_ERR_INVALID_ARG, "shared.n_experts = %d (want 0 or 1)", w->shared.n_experts);
+    if (w->shared.n_experts == 1) {
+        int r = check_tier(w->shared, "shared", 0);
+        if (r) return r;
+    }
+    return MOE_OK;
+}
+
+int check_k(int T, int E, int k) {
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %d", T);
+    if (E < 1 || E > MOE_MAX_EXPERTS) return fail(MOE_ERR_INVALID_ARG, "E = %d outside [1, %d]", E, MOE_MAX_EXPERTS);
+    if (k < 1 || k > E || k > MOE_MAX_TOPK) return fail(MOE_ERR_INVALID_ARG, "k = %d outside [1, min(E, %d)]", k, MOE_MAX_TOPK);
+    if (static_cast<int64_t>(T) * k > (1 << 24)) return fail(MOE_ERR_UNSUPPORTED, "T*k = %lld exceeds 2^24", (long long)T * k);
+    return MOE_OK;
+}
+
+moe::FfnParams make_params(const moe_layer_weights *w, const uint16_t *x, int T, int k, const int32_t *offsets,
+                           const int32_t *sorted, const int32_t *active, float *y_slots, float *y_shared,
+                           float *h, int32_t *status) {
+    moe::FfnParams p;
+    p.w = *w;
+    p.E = w->E;
+    p.T = T;
+    p.k = k;
+    p.has_shared = w->shared.n_experts == 1;
+    const long ma = static_cast<long>(T) * k;
+    p.max_active = static_cast<int>(ma < w->E ? ma : w->E);
+    p.x = x;
+    p.offsets = offsets;
+    p.sorted = sorted;
+    p.active = active;
+    p.h = h;
+    p.y_slots = y_slots;
+    p.y_shared = y_shared;
+    p.status = status;
+    return p;
+}
+
+size_t ffn_ws_bytes(const moe_layer_weights *w, int T, int k, int mode) {
+    const size_t rows = static_cast<size_t>(T) * k + static_cast<size_t>(T);
+    size_t gemv = align_up(rows * w->I * sizeof(float));
+    size_t gemm = mode == MOE_FFN_GEMV ? 0 : moe_ffn_gemm_workspace(w, T, k);
+    return (gemv > gemm ? gemv : gemm) + 256;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_err.c_str(); }
+
+const char *moe_version(void) { return "moe_tiered 0.1 (sm_100a)"; }
+
+size_t moe_packed_row_bytes(int32_t K, int32_t bits) {
+    if (K <= 0 || K % 64 != 0 || !valid_bits(bits)) return 0;
+    return static_cast<size_t>(K) * bits / 8;
+}
+
+int moe_quantize(const float *src, int64_t rows, int32_t K, int32_t bits, uint8_t *qs, uint16_t *scale,
+                 moe_stream_t stream) {
+    if (!valid_bits(bits)) return fail(MOE_ERR_INVALID_ARG, "bits = %d (want 8, 4 or 3)", bits);
+    if (K <= 0 || K % 64 != 0) return fail(MOE_ERR_INVALID_ARG, "K = %d must be a positive multiple of 64", K);
+    if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "rows = %lld", (long long)rows);
+    if (rows == 0) return ok();
+    if (!src || !qs || !scale) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(src) || !aligned16(qs) || !aligned16(scale)) return fail(MOE_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+    int r = ensure_configured();
+    if (r) return r;
+    cudaError_t e = moe_launch_quantize(src, rows, K, bits, qs, scale, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "quantize launch");
+}
+
+int moe_dequantize(const uint8_t *qs, const uint16_t *scale, int64_t rows, int32_t K, int32_t bits, float *out_f32,
+                   uint16_t *out_f16, moe_stream_t stream) {
+    if (!valid_bits(bits)) return fail(MOE_ERR_INVALID_ARG, "bits = %d (want 8, 4 or 3)", bits);
+    if (K <= 0 || K % 64 != 0) return fail(MOE_ERR_INVALID_ARG, "K = %d must be a positive multiple of 64", K);
+    if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "rows = %lld", (long long)rows);
+    if (!out_f32 && !out_f16) return fail(MOE_ERR_INVALID_ARG, "both outputs are NULL");
+    if (rows == 0) return ok();
+    if (!qs || !scale) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    int r = ensure_configured();
+    if (r) return r;
+    cudaError_t e = moe_launch_dequantize(qs, scale, rows, K, bits, out_f32, out_f16,
+                                          reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "dequantize launch");
+}
+
+size_t moe_router_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k) {
+    (void)H;
+    (void)k;
+    if (T <= 0 || E <= 0) return 0;
+    return align_up(static_cast<size_t>(T) * E * sizeof(float));
+}
+
+int moe_router_topk(const uint16_t *x, const uint16_t *w_router, const float *bias, int32_t T, int32_t H, int32_t E,
+                    int32_t k, float *logits, int32_t *topk_idx, float *topk_w, void *workspace,
+                    size_t workspace_bytes, moe_stream_t stream) {
+    int r = check_k(T, E, k);
+    if (r) return r;
+    if (H <= 0 || H % 64 != 0 || H > 16384) return fail(MOE_ERR_INVALID_ARG, "H = %d must be a multiple of 64 in (0, 16384]", H);
+    if (T == 0) return ok();
+    if (!x || !w_router || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(x) || !aligned16(w_router)) return fail(MOE_ERR_INVALID_ARG, "x / w_router not 16-byte aligned");
+    float *lg = logits;
+    if (!lg) {
+        if (!workspace || workspace_bytes < moe_router_workspace_size(T, H, E, k))
+            return fail(MOE_ERR_WORKSPACE, "router workspace needs %zu bytes", moe_router_workspace_size(T, H, E, k));
+        lg = static_cast<float *>(workspace);
+    }
+    r = ensure_configured();
+    if (r) return r;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = moe_launch_router_logits(x, w_router, bias, T, H, E, lg, s);
+    if (e == cudaSuccess) e = moe_launch_topk(lg, T, E, k, topk_idx, topk_w, s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "router launch");
+}
+
+int moe_topk_softmax(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *topk_idx, float *topk_w,
+                     moe_stream_t stream) {
+    int r = check_k(T, E, k);
+    if (r) return r;
+    if (T == 0) return ok();
+    if (!logits || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    r = ensure_configured();
+    if (r) return r;
+    cudaError_t e = moe_launch_topk(logits, T, E, k, topk_idx, topk_w, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "top-k launch");
+}
+
+int moe_bucketize(const int32_t *topk_idx, int32_t T, int32_t k, int32_t E, int32_t *expert_offsets,
+                  int32_t *sorted_slot, int32_t *slot_pos, int32_t *active, int32_t *status, moe_stream_t stream) {
+    int r = check_k(T, E, k);
+    if (r) return r;
+    if (!expert_offsets || !active) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (T > 0 && (!topk_idx || !sorted_slot || !slot_pos)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    r = ensure_configured();
+    if (r) return r;
+    cudaError_t e = moe_launch_bucketize(topk_idx, T * k, E, expert_offsets, sorted_slot, slot_pos, active, status,
+                                         reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "bucketize launch");
+}
+
+size_t moe_ffn_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k, int32_t mode) {
+    if (!w || T < 0 || k < 1) return 0;
+    return ffn_ws_bytes(w, T, k, mode);
+}
+
+int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t k,
+                          const int32_t *expert_offsets, const int32_t *sorted_slot, const int32_t *active,
+                          float *y_slots, float *y_shared, void *workspace, size_t workspace_bytes, int32_t mode,
+                          int32_t *status, moe_stream_t stream) {
+    int r = check_weights(w);
+    if (r) return r;
+    r = check_k(T, w->E, k);
+    if (r) return r;
+    if (mode != MOE_FFN_AUTO && mode != MOE_FFN_GEMV && mode != MOE_FFN_GEMM)
+        return fail(MOE_ERR_INVALID_ARG, "mode = %d", mode);
+    if (T == 0) return ok();
+    if (!x || !expert_offsets || !sorted_slot || !active || !y_slots)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    const bool has_shared = w->shared.n_experts == 1;
+    if (has_shared != (y_shared != nullptr))
+        return fail(MOE_ERR_INVALID_ARG, "y_shared must be given iff the layer has a shared expert");
+    if (!aligned16(x) || !aligned16(y_slots) || (y_shared && !aligned16(y_shared)))
+        return fail(MOE_ERR_INVALID_ARG, "x / y pointers not 16-byte aligned");
+    const size_t need = ffn_ws_bytes(w, T, k, mode);
+    if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "ffn workspace needs %zu bytes", need);
+    r = ensure_configured();
+    if (r) return r;
+    float *h = static_cast<float *>(workspace);
+    moe::FfnParams p = make_params(w, x, T, k, expert_offsets, sorted_slot, active, y_slots, y_shared, h, status);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (mode == MOE_FFN_GEMM) e = moe_launch_ffn_gemm(p, workspace, workspace_bytes, s);
+    else e = moe_launch_ffn_gemv(p, s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ffn launch");
+}
+
+int moe_combine(const float *y_slots, const float *y_shared, const float *topk_w, int32_t T, int32_t k, int32_t H,
+                const uint16_t *residual, uint16_t *out, uint16_t *x_next, moe_stream_t stream) {
+    if (T < 0 || k < 1 || k > MOE_MAX_TOPK) return fail(MOE_ERR_INVALID_ARG, "T = %d, k = %d", T, k);
+    if (H <= 0 || H % 4 != 0) return fail(MOE_ERR_INVALID_ARG, "H = %d must be a positive multiple of 4", H);
+    if (T == 0) return ok();
+    if (!y_slots || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (!out && !residual) return fail(MOE_ERR_INVALID_ARG, "out is NULL and there is no residual");
+    if (residual && !x_next) return fail(MOE_ERR_INVALID_ARG, "x_next is required with a residual");
+    if (!aligned16(y_slots) || (y_shared && !aligned16(y_shared)))
+        return fail(MOE_ERR_INVALID_ARG, "y pointers not 16-byte aligned");
+    cudaError_t e = moe_launch_combine(y_slots, y_shared, topk_w, T, k, H, residual, out, x_next,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "combine launch");
+}
+
+namespace {
+struct LayerWs {
+    float *logits;
+    int32_t *idx;
+    float *tw;
+    int32_t *offsets, *sorted, *pos, *active;
+    float *y_slots, *y_shared;
+    void *ffn_ws;
+    size_t ffn_bytes;
+    size_t total;
+};
+
+LayerWs carve(const moe_layer_weights *w, int T, int k, int mode, char *base) {
+    LayerWs L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *p = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return p;
+    };
+    const size_t S = static_cast<size_t>(T) * k;
+    L.logits = reinterpret_cast<float *>(take(static_cast<size_t>(T) * w->E * sizeof(float)));
+    L.idx = reinterpret_cast<int32_t *>(take(S * sizeof(int32_t)));
+    L.tw = reinterpret_cast<float *>(take(S * sizeof(float)));
+    L.offsets = reinterpret_cast<int32_t *>(take((w->E + 1) * sizeof(int32_t)));
+    L.sorted = reinterpret_cast<int32_t *>(take(S * sizeof(int32_t)));
+    L.pos = reinterpret_cast<int32_t *>(take(S * sizeof(int32_t)));
+    L.active = reinterpret_cast<int32_t *>(take((w->E + 1) * sizeof(int32_t)));
+    L.y_slots = reinterpret_cast<float *>(take(S * w->H * sizeof(float)));
+    L.y_shared = reinterpret_cast<float *>(take(static_cast<size_t>(T) * w->H * sizeof(float)));
+    L.ffn_bytes = ffn_ws_bytes(w, T, k, mode);
+    L.ffn_ws = take(L.ffn_bytes);
+    L.total = off;
+    return L;
+}
+}  // namespace
+
+size_t moe_layer_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k, int32_t mode) {
+    if (!w || T < 0 || k < 1 || w->E < 1) return 0;
+    return carve(w, T, k, mode, nullptr).total;
+}
+
+int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router, const float *bias, const uint16_t *x,
+                      int32_t T, int32_t k, const uint16_t *residual, uint16_t *out, uint16_t *x_next,
+                      void *workspace, size_t workspace_bytes, int32_t mode, int32_t *status, moe_stream_t stream) {
+    int r = check_weights(w);
+    if (r) return r;
+    r = check_k(T, w->E, k);
+    if (r) return r;
+    if (T == 0) return ok();
+    const size_t need = moe_layer_workspace_size(w, T, k, mode);
+    if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "layer workspace needs %zu bytes", need);
+    if (!aligned16(workspace)) return fail(MOE_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    LayerWs L = carve(w, T, k, mode, static_cast<char *>(workspace));
+    r = moe_router_topk(x, w_router, bias, T, w->H, w->E, k, L.logits, L.idx, L.tw, nullptr, 0, stream);
+    if (r) return r;
+    r = moe_bucketize(L.idx, T, k, w->E, L.offsets, L.sorted, L.pos, L.active, status, stream);
+    if (r) return r;
+    r = moe_expert_ffn_tiered(w, x, T, k, L.offsets, L.sorted, L.active, L.y_slots,
+                              w->shared.n_experts == 1 ? L.y_shared : nullptr, L.ffn_ws, L.ffn_bytes, mode, status,
+                              stream);
+    if (r) return r;
+    return moe_combine(L.y_slots, w->shared.n_experts == 1 ? L.y_shared : nullptr, L.tw, T, k, w->H, residual, out,
+                       x_next, stream);
+}
+
+}  // extern "C"

@@ -8,4 +8,4 @@ from .moe_oracle import (BLOCK, QMAX, Shelf, bits_per_weight, bucketize,  # noqa
                          build_shelf, combine, dequantize_f16, dequantize_f32,
                          expert_ffn, moe_layer, pack_rows, packed_row_bytes,
                          quantize_pack, quantize_rows, round_bf16, router_logits,
-                         select_topk, shelf_of, silu, topk_margin, unpack_rows)
+                         select_topk, shelf_of, shelves_lookup, silu, topk_margin, unpack_rows)

@@ -336,14 +336,19 @@ def shelf_of(shelves, e):
     return hits[0]
 
 
-def moe_layer(x, w_router, bias, k, shelves, shared, H, I, residual=None,
-              experts=None):
+def shelves_lookup(shelves, H, I):
+    """Expert id -> dequantised fp32 (gate_up, down) from a list of shelves."""
+    def get(e):
+        return shelf_of(shelves, e).weights(e, H, I)
+    return get
+
+
+def moe_layer(x, w_router, bias, k, expert_weights, shared_weights, H, I, residual=None):
     """One routed MoE layer: router -> top-k -> bucketize -> tiered FFN -> combine.
 
-    ``shelves`` is a list of :class:`Shelf` covering [0, E) exactly; ``shared``
-    is a Shelf holding the one shared expert (or None).  ``experts`` optionally
-    maps an expert id to already-dequantised (gate_up, down) fp32 arrays, to
-    avoid dequantising one expert twice across calls.
+    ``expert_weights(e)`` returns expert e's dequantised fp32 (gate_up [2I,H],
+    down [H,I]) from whichever shelf owns it (see :func:`shelves_lookup`);
+    ``shared_weights`` is the shared expert's pair, or None.
 
     Returns a dict with every intermediate the library exposes.
     """
@@ -359,15 +364,11 @@ def moe_layer(x, w_router, bias, k, shelves, shared, H, I, residual=None,
         if lo == hi:
             continue  # an expert nobody chose costs nothing
         slots = sorted_slot[lo:hi]
-        if experts is not None and e in experts:
-            wgu, wdn = experts[e]
-        else:
-            wgu, wdn = shelf_of(shelves, e).weights(e, H, I)
+        wgu, wdn = expert_weights(e)
         y_slots[slots] = expert_ffn(x[slots // k], wgu, wdn)
     y_shared = None
-    if shared is not None:
-        wgu, wdn = shared.weights(shared.first, H, I)
-        y_shared = expert_ffn(x, wgu, wdn)
+    if shared_weights is not None:
+        y_shared = expert_ffn(x, *shared_weights)
     res = combine(y_slots, y_shared, w, residual)
     out, x_next = (res if residual is not None else (res, None))
     return dict(logits=logits, topk_idx=idx, topk_w=w, expert_offsets=offsets,

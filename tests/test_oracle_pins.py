@@ -311,7 +311,8 @@ def test_layer_brute_force_dense():
     """Every expert evaluated for every token, masked by the top-k and weighted,
     must equal the sparse routed evaluation."""
     cfg, x, wr, bias, shelves, shared = _tiny_layer()
-    res = oracle.moe_layer(x, wr, bias, cfg.k, shelves, shared, cfg.H, cfg.I)
+    res = oracle.moe_layer(x, wr, bias, cfg.k, oracle.shelves_lookup(shelves, cfg.H, cfg.I),
+                           shared.weights(cfg.E, cfg.H, cfg.I), cfg.H, cfg.I)
     T = x.shape[0]
     # brute force: independent loops over (token, expert)
     logits = np.zeros((T, cfg.E))
@@ -350,8 +351,10 @@ def test_layer_tier_split_invariance():
     cfg = inputs.TINY
     one = _tiny_layer(shelf_split=[(8, 0, 16)])
     three = _tiny_layer(shelf_split=[(8, 0, 5), (8, 5, 2), (8, 7, 9)])
-    r1 = oracle.moe_layer(*one[1:4], cfg.k, one[4], one[5], cfg.H, cfg.I)
-    r3 = oracle.moe_layer(*three[1:4], cfg.k, three[4], three[5], cfg.H, cfg.I)
+    r1 = oracle.moe_layer(*one[1:4], cfg.k, oracle.shelves_lookup(one[4], cfg.H, cfg.I),
+                          one[5].weights(cfg.E, cfg.H, cfg.I), cfg.H, cfg.I)
+    r3 = oracle.moe_layer(*three[1:4], cfg.k, oracle.shelves_lookup(three[4], cfg.H, cfg.I),
+                          three[5].weights(cfg.E, cfg.H, cfg.I), cfg.H, cfg.I)
     assert np.array_equal(r1["out"], r3["out"])
 
 
