@@ -1,0 +1,335 @@
+"""Benchmark of the tiered MoE layer on B200.
+
+Default workload (one GPU): decode, one token at a time through 48 stacked MoE
+layers of the decode configuration (hidden 2048, 512 experts of intermediate
+512 on three shelves -- ids 0-127 at 8 bits, 128-319 at 4 bits, 320-511 at
+3 bits, blocks of 32 with fp16 scales -- plus one 8-bit shared expert, top-10
+Zipf-skewed routing, bf16 residual stream).  The 48 layers have independent
+seeded weights (~49.5 GB resident), so no layer's weights are in L2 when it
+runs.  One step = one token through all 48 layers; the metric counts
+layer-tokens (tokens x layers) per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun), every rank runs its own replica on its own tokens: the
+layer has no exchange step, so scaling is weak and there is no collective on
+the data path (only the timing max-reduce).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixed_precision_moe_router_b200 import inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; decode expert-weight GB/s vs HBM peak; prefill TFLOP/s"
+UNIT = "layer-tokens/s"
+N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
+KERNELS_PER_LAYER = 6  # router logits, top-k, bucketize, gate_up, down, combine (+1 rmsnorm per step)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait()
+            self.th.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 4 + i and r[4 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def build_stack(cfg, n_layers, device):
+    from mixed_precision_moe_router_b200 import binding as B
+    layers, routers = [], []
+    for l in range(n_layers):
+        seed = inputs.layer_seed(cfg, l)
+        layers.append(B.build_layer(cfg, seed, device))
+        routers.append(inputs.router(cfg, seed, device))
+    torch.cuda.synchronize()
+    return layers, routers
+
+
+def expert_bytes(cfg, layer, e):
+    return layer.nbytes_expert(e)
+
+
+def run_native(args, rank, world):
+    from mixed_precision_moe_router_b200 import binding as B
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    cfg = inputs.DECODE
+    T = 1
+    layers, routers = build_stack(cfg, N_LAYERS, device)
+    k = cfg.k
+    x0 = inputs.activations(T, cfg.H, seed=inputs.X_SEED + 1000 * rank, device=device)
+    nws = B.layer_workspace_size(layers[0], T, k, B.FFN_AUTO)
+    ws = torch.empty(nws, dtype=torch.uint8, device=device)
+    # residual stream xs[l] (bf16) and the normalised input ns[l] each layer reads
+    xs = [x0.clone()] + [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device) for _ in range(N_LAYERS)]
+    ns = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device) for _ in range(N_LAYERS + 1)]
+    outs = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device) for _ in range(N_LAYERS)]
+
+    def step():
+        B.rmsnorm(xs[0], out=ns[0])
+        for l in range(N_LAYERS):
+            wr, bias = routers[l]
+            B.layer_forward(layers[l], wr, bias, ns[l], k, residual=xs[l], workspace=ws, out=outs[l],
+                            x_next=xs[l + 1], x_next_norm=ns[l + 1])
+
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        step()  # first run outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        time.sleep(0.3)
+        cur = torch.cuda.current_stream(device)
+        ev0.record(cur)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(cur)
+        torch.cuda.synchronize()
+        time.sleep(0.2)
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * T * N_LAYERS * args.steps / (ms / 1e3)
+
+    # per-call timing of the FFN (the dominant kernels) and algorithmic bytes
+    hbm, tf, peak_kind = peaks()
+    ffn_ms, ffn_bytes = [], []
+    with torch.cuda.stream(stream):
+        for l in range(N_LAYERS):
+            wr, bias = routers[l]
+            idx, w, _ = B.router_topk(ns[l], wr, bias, k)
+            off, srt, pos, act = B.bucketize(idx, cfg.E)
+            torch.cuda.synchronize()
+            touched = sorted(set(idx.cpu().numpy().reshape(-1).tolist()))
+            ffn_bytes.append(sum(layers[l].nbytes_expert(e) for e in touched) + layers[l].nbytes_expert(cfg.E))
+            # one call per layer: the previous layer's FFN (other weights) ran in between,
+            # so this layer's experts are not L2-resident
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            B.expert_ffn(layers[l], ns[l], k, off, srt, act, mode=B.FFN_AUTO)
+            b.record(stream)
+            b.synchronize()
+            ffn_ms.append(a.elapsed_time(b))
+    avg_ms = float(np.mean(ffn_ms))
+    avg_bytes = float(np.mean(ffn_bytes))
+    achieved = avg_bytes / (avg_ms / 1e3) / 1e9
+
+    # end to end through the public API: pinned host input, eager calls, host output
+    h_in = x0.cpu().pin_memory()
+    h_out = torch.empty(T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    with torch.cuda.stream(stream):
+        for i in range(e2e_steps + 2):
+            if i == 2:
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            xs[0].copy_(h_in, non_blocking=True)
+            step()
+            h_out.copy_(xs[N_LAYERS], non_blocking=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = world * T * N_LAYERS / (e2e_ms / 1e3)
+    del graph
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "decode: 48 stacked MoE layers (H=2048, I=512, E=512, top-10 + 1 shared, "
+                               "shelves 128x8-bit/192x4-bit/192x3-bit, Zipf routing), 1 token per step per GPU",
+                   "global_batch": world * T, "layers": N_LAYERS, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: ~1.37 GB of distinct expert weights touched per step",
+                   "graph": "one CUDA graph per step (48 x layer_forward)"},
+        "roofline": {"bound": "hbm", "kernel": "expert FFN (gate_up + down GEMV launches of one layer)",
+                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": None, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": round(avg_bytes), "avg_launch_us": round(avg_ms * 1e3, 2)},
+        "e2e": {"value": round(e2e_val, 1), "unit": UNIT,
+                "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2},
+        "gpu_launches": args.steps * (N_LAYERS * KERNELS_PER_LAYER + 1),
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+class OracleStack:
+    """The oracle on the same stack: packs (by the oracle's own quantiser) the
+    experts each layer touches for one token, outside any timed region."""
+
+    def __init__(self, n_layers):
+        import oracle
+        self.oracle = oracle
+        cfg = self.cfg = inputs.DECODE
+        x = inputs.activations(1, cfg.H, seed=inputs.X_SEED).float().numpy()
+        n = oracle.rms_norm(x).astype(np.float32)
+        self.layers = []
+        for l in range(n_layers):
+            seed = inputs.layer_seed(cfg, l)
+            wr, bias = inputs.router(cfg, seed)
+            wrn, bn = wr.float().numpy(), bias.numpy()
+            idx, _ = oracle.select_topk(oracle.router_logits(n, wrn, bn), cfg.k)
+            packed = {}
+            for e in [int(v) for v in idx.reshape(-1)] + [cfg.E]:
+                wgu, wdn = inputs.expert_source(cfg, seed, e)
+                bits = cfg.shared_bits if e == cfg.E else [b for b, f, n in cfg.tier_ranges() if f <= e < f + n][0]
+                packed[e] = (bits, oracle.quantize_pack(wgu.numpy(), bits), oracle.quantize_pack(wdn.numpy(), bits))
+            self.layers.append((x, n, wrn, bn, packed))
+            r = self.run(l)
+            x, n = r["x_next"].astype(np.float32), r["n_next"].astype(np.float32)
+
+    def run(self, l):
+        o, cfg = self.oracle, self.cfg
+        x, n, wrn, bn, packed = self.layers[l]
+
+        def weights(e):
+            bits, (gq, gs), (dq, ds) = packed[e]
+            return o.dequantize_f32(gq, gs, bits, cfg.H), o.dequantize_f32(dq, ds, bits, cfg.I)
+        return o.moe_layer(n, wrn, bn, cfg.k, weights, weights(cfg.E), cfg.H, cfg.I, residual=x)
+
+
+def cpu_baseline(budget_s=15.0, n_layers=4):
+    """The oracle as it stands, timed on the host (one thread) on a bounded
+    sample of the same workload: one token through the first ``n_layers``
+    layers of the stack, repeated until about ``budget_s`` seconds of work."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        st = OracleStack(n_layers)
+        done, total = 0, 0.0
+        while total < budget_s:
+            t0 = time.perf_counter()
+            st.run(done % n_layers)
+            total += time.perf_counter() - t0
+            done += 1
+    return {"value": round(done / total, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} layer-tokens: 1 token through the first {n_layers} layers of the stack, "
+                      "repeated (fp64 numpy oracle incl. dequantisation, 1 thread; packing not timed)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=inputs.N_STACK,
+                    help="stack depth; the benchmark is defined at 48, fewer only for profiler captures")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+    global N_LAYERS
+    N_LAYERS = args.layers
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        from threadpoolctl import threadpool_limits
+        t0 = time.perf_counter()
+        with threadpool_limits(limits=1):
+            st = OracleStack(4)
+            times = []
+            for i in range(args.warmup + args.steps):
+                a = time.perf_counter()
+                st.run(i % 4)
+                times.append(time.perf_counter() - a)
+        v = float(args.steps / sum(times[args.warmup:]))
+        sample = f"each step: 1 token through one of the first 4 layers of the stack (fp64 numpy oracle, 1 thread)"
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / v, 3) if v else None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "decode: 48 stacked MoE layers, 1 token (oracle sample)"},
+            "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": round(time.perf_counter() - t0, 1)}))
+        return
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    line = run_native(args, rank, world)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

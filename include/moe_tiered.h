@@ -63,6 +63,7 @@ typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
 #define MOE_MAX_TIERS 4  /* shelves per layer */
 #define MOE_MAX_TOPK 32
 #define MOE_MAX_EXPERTS 1024
+#define MOE_NORM_EPS 1e-6f /* epsilon of the residual-stream RMS norm */
 
 /*
  * Packed shelf format ([P1] "step 4: three shelves, all on the GPU": each
@@ -219,21 +220,30 @@ int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t
  * moe_combine: out[t] = bf16_rne( sum_{j<k} topk_w[t,j] * y_slots[t*k+j]
  *                                 + y_shared[t] )
  * summed in that fixed order ([P1] "step 4": the results simply add up).
- * With residual != NULL also x_next[t] = bf16_rne(residual[t] + out[t]).
+ * With residual != NULL it also advances the bf16 residual stream of a stack
+ * of layers ([P5] "What the model actually is": 48 layers, residual design):
+ *   x_next[t] = bf16_rne(residual[t] + out[t])
+ *   x_next_norm[t] = bf16_rne(x_next[t] / sqrt(mean_h(x_next[t]^2) + MOE_NORM_EPS))
+ * (the RMS-normalised stream that the next layer reads; NULL to skip).
  *   y_slots fp32 [T*k][H]; y_shared fp32 [T][H] or NULL; topk_w fp32 [T][k]
- *   residual bf16 [T][H] or NULL; out bf16 [T][H]; x_next bf16 [T][H] (needed
- *   iff residual is given).
+ *   residual bf16 [T][H] or NULL; out bf16 [T][H] (may be NULL when a residual
+ *   is given); x_next, x_next_norm bf16 [T][H] (x_next needed iff residual).
  */
 int moe_combine(const float *y_slots, const float *y_shared, const float *topk_w,
                 int32_t T, int32_t k, int32_t H, const uint16_t *residual,
-                uint16_t *out, uint16_t *x_next, moe_stream_t stream);
+                uint16_t *out, uint16_t *x_next, uint16_t *x_next_norm,
+                moe_stream_t stream);
+
+/* moe_rmsnorm: n[t] = bf16_rne(x[t] / sqrt(mean_h(x[t]^2) + MOE_NORM_EPS)),
+ * the input of the first layer of a stack.  x, n bf16 [T][H], H % 4 == 0. */
+int moe_rmsnorm(const uint16_t *x, int32_t T, int32_t H, uint16_t *n, moe_stream_t stream);
 
 /*
  * moe_layer_forward: router -> bucketize -> tiered FFN -> combine, with every
  * intermediate in `workspace` (moe_layer_workspace_size() bytes).
- *   x bf16 [T][H]; w_router bf16 [E][H]; bias fp32 [E] or NULL
- *   out bf16 [T][H]; with residual != NULL (normally residual == x) also
- *   x_next = bf16(residual + out).
+ *   x bf16 [T][H] (the layer input); w_router bf16 [E][H]; bias fp32 [E] or NULL
+ *   out bf16 [T][H]; with residual != NULL also x_next and x_next_norm as in
+ *   moe_combine (in a stack: x = the normalised stream, residual = the stream).
  * Same limits as the calls it chains.  Capturable into a CUDA graph.
  */
 size_t moe_layer_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k,
@@ -241,7 +251,7 @@ size_t moe_layer_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k
 int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router,
                       const float *bias, const uint16_t *x, int32_t T, int32_t k,
                       const uint16_t *residual, uint16_t *out, uint16_t *x_next,
-                      void *workspace, size_t workspace_bytes, int32_t mode,
+                      uint16_t *x_next_norm, void *workspace, size_t workspace_bytes, int32_t mode,
                       int32_t *status, moe_stream_t stream);
 
 #ifdef __cplusplus

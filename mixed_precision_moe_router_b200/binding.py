@@ -54,10 +54,11 @@ SIGNATURES = [
     ("moe_ffn_workspace_size", c_size, [ctypes.POINTER(LayerWeights), c_i32, c_i32, c_i32]),
     ("moe_expert_ffn_tiered", c_i32, [ctypes.POINTER(LayerWeights), c_vp, c_i32, c_i32, c_vp, c_vp, c_vp,
                                       c_vp, c_vp, c_vp, c_size, c_i32, c_vp, c_vp]),
-    ("moe_combine", c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    ("moe_combine", c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    ("moe_rmsnorm", c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp]),
     ("moe_layer_workspace_size", c_size, [ctypes.POINTER(LayerWeights), c_i32, c_i32, c_i32]),
     ("moe_layer_forward", c_i32, [ctypes.POINTER(LayerWeights), c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp,
-                                  c_vp, c_vp, c_size, c_i32, c_vp, c_vp]),
+                                  c_vp, c_vp, c_vp, c_size, c_i32, c_vp, c_vp]),
 ]
 
 _lib = None
@@ -280,15 +281,25 @@ def expert_ffn(layer, x, k, offsets, sorted_slot, active, mode=FFN_AUTO, status=
     return y_slots, y_shared
 
 
-def combine(y_slots, y_shared, topk_w, residual=None, want_out=True):
+def combine(y_slots, y_shared, topk_w, residual=None, want_out=True, want_norm=True):
+    """Returns out, or (out, x_next, x_next_norm) when a residual is given."""
     T, k = topk_w.shape
     H = y_slots.shape[1]
     dev = y_slots.device
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev) if want_out else None
     x_next = torch.empty(T, H, dtype=torch.bfloat16, device=dev) if residual is not None else None
+    n_next = torch.empty(T, H, dtype=torch.bfloat16, device=dev) if residual is not None and want_norm else None
     _check(lib().moe_combine(_ptr(y_slots), _ptr(y_shared), _ptr(topk_w), T, k, H, _ptr(residual), _ptr(out),
-                             _ptr(x_next), _stream()))
-    return out if residual is None else (out, x_next)
+                             _ptr(x_next), _ptr(n_next), _stream()))
+    return out if residual is None else (out, x_next, n_next)
+
+
+def rmsnorm(x, out=None):
+    _need(x, torch.bfloat16, name="x")
+    T, H = x.shape
+    n = out if out is not None else torch.empty_like(x)
+    _check(lib().moe_rmsnorm(_ptr(x), T, H, _ptr(n), _stream()))
+    return n
 
 
 def layer_workspace_size(layer, T, k, mode=FFN_AUTO):
@@ -296,9 +307,9 @@ def layer_workspace_size(layer, T, k, mode=FFN_AUTO):
 
 
 def layer_forward(layer, w_router, bias, x, k, residual=None, mode=FFN_AUTO, workspace=None, out=None,
-                  x_next=None, status=None):
+                  x_next=None, x_next_norm=None, status=None):
     """One MoE layer through the library's fused entry point.  Returns out, or
-    (out, x_next) when a residual is given."""
+    (out, x_next, x_next_norm) when a residual is given."""
     _need(x, torch.bfloat16, name="x")
     T = x.shape[0]
     dev = x.device
@@ -308,9 +319,12 @@ def layer_forward(layer, w_router, bias, x, k, residual=None, mode=FFN_AUTO, wor
         workspace = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
     if out is None:
         out = torch.empty(T, layer.H, dtype=torch.bfloat16, device=dev)
-    if residual is not None and x_next is None:
-        x_next = torch.empty(T, layer.H, dtype=torch.bfloat16, device=dev)
+    if residual is not None:
+        if x_next is None:
+            x_next = torch.empty(T, layer.H, dtype=torch.bfloat16, device=dev)
+        if x_next_norm is None:
+            x_next_norm = torch.empty(T, layer.H, dtype=torch.bfloat16, device=dev)
     _check(lib().moe_layer_forward(ctypes.byref(d), _ptr(w_router), _ptr(bias), _ptr(x), T, k, _ptr(residual),
-                                   _ptr(out), _ptr(x_next), _ptr(workspace), workspace.numel(), mode,
-                                   _ptr(status), _stream()))
-    return out if residual is None else (out, x_next)
+                                   _ptr(out), _ptr(x_next), _ptr(x_next_norm), _ptr(workspace), workspace.numel(),
+                                   mode, _ptr(status), _stream()))
+    return out if residual is None else (out, x_next, x_next_norm)

@@ -20,13 +20,15 @@ cudaError_t moe_launch_topk(const float *, int, int, int, int32_t *, float *, cu
 cudaError_t moe_configure_bucketize();
 cudaError_t moe_launch_bucketize(const int32_t *, int, int, int32_t *, int32_t *, int32_t *, int32_t *, int32_t *,
                                  cudaStream_t);
-cudaError_t moe_configure_ffn_gemv();
-cudaError_t moe_launch_ffn_gemv(const moe::FfnParams &, cudaStream_t);
+cudaError_t moe_configure_ffn_stream();
+cudaError_t moe_launch_ffn_stream(const moe::FfnParams &, cudaStream_t);
+bool moe_ffn_stream_supported(int H, int I);
 cudaError_t moe_configure_ffn_gemm();
 cudaError_t moe_launch_ffn_gemm(const moe::FfnParams &, void *ws, size_t ws_bytes, cudaStream_t);
 size_t moe_ffn_gemm_workspace(const moe_layer_weights *, int T, int k);
 cudaError_t moe_launch_combine(const float *, const float *, const float *, int, int, int, const uint16_t *,
-                               uint16_t *, uint16_t *, cudaStream_t);
+                               uint16_t *, uint16_t *, uint16_t *, cudaStream_t);
+cudaError_t moe_launch_rmsnorm(const uint16_t *, int, int, uint16_t *, cudaStream_t);
 
 namespace {
 
@@ -66,7 +68,7 @@ int ensure_configured() {
     std::call_once(g_dev_once[dev], [dev]() {
         cudaError_t r = moe_configure_router();
         if (r == cudaSuccess) r = moe_configure_bucketize();
-        if (r == cudaSuccess) r = moe_configure_ffn_gemv();
+        if (r == cudaSuccess) r = moe_configure_ffn_stream();
         if (r == cudaSuccess) r = moe_configure_ffn_gemm();
         g_dev_err[dev] = r;
     });
@@ -146,15 +148,21 @@ moe::FfnParams make_params(const moe_layer_weights *w, const uint16_t *x, int T,
     p.sorted = sorted;
     p.active = active;
     p.h = h;
+    p.ctr = nullptr;
     p.y_slots = y_slots;
     p.y_shared = y_shared;
     p.status = status;
     return p;
 }
 
+size_t ffn_ctr_bytes(const moe_layer_weights *w, int T, int k) {
+    const long ma = static_cast<long>(T) * k;
+    return align_up((static_cast<size_t>(ma < w->E ? ma : w->E) + 1) * sizeof(int));
+}
+
 size_t ffn_ws_bytes(const moe_layer_weights *w, int T, int k, int mode) {
     const size_t rows = static_cast<size_t>(T) * k + static_cast<size_t>(T);
-    size_t gemv = align_up(rows * w->I * sizeof(float));
+    size_t gemv = align_up(rows * w->I * sizeof(float)) + ffn_ctr_bytes(w, T, k);
     size_t gemm = mode == MOE_FFN_GEMV ? 0 : moe_ffn_gemm_workspace(w, T, k);
     return (gemv > gemm ? gemv : gemm) + 256;
 }
@@ -283,17 +291,26 @@ int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t
     if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "ffn workspace needs %zu bytes", need);
     r = ensure_configured();
     if (r) return r;
+    if (mode != MOE_FFN_GEMM && !moe_ffn_stream_supported(w->H, w->I))
+        return fail(MOE_ERR_UNSUPPORTED, "GEMV path supports H, I <= 2048");
     float *h = static_cast<float *>(workspace);
     moe::FfnParams p = make_params(w, x, T, k, expert_offsets, sorted_slot, active, y_slots, y_shared, h, status);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (mode == MOE_FFN_GEMM) e = moe_launch_ffn_gemm(p, workspace, workspace_bytes, s);
-    else e = moe_launch_ffn_gemv(p, s);
+    if (mode == MOE_FFN_GEMM) {
+        e = moe_launch_ffn_gemm(p, workspace, workspace_bytes, s);
+    } else {
+        const size_t hb = align_up((static_cast<size_t>(T) * k + T) * w->I * sizeof(float));
+        p.ctr = reinterpret_cast<int *>(static_cast<char *>(workspace) + hb);
+        e = cudaMemsetAsync(p.ctr, 0, ffn_ctr_bytes(w, T, k), s);
+        if (e == cudaSuccess) e = moe_launch_ffn_stream(p, s);
+    }
     return e == cudaSuccess ? ok() : cuda_fail(e, "ffn launch");
 }
 
 int moe_combine(const float *y_slots, const float *y_shared, const float *topk_w, int32_t T, int32_t k, int32_t H,
-                const uint16_t *residual, uint16_t *out, uint16_t *x_next, moe_stream_t stream) {
+                const uint16_t *residual, uint16_t *out, uint16_t *x_next, uint16_t *x_next_norm,
+                moe_stream_t stream) {
     if (T < 0 || k < 1 || k > MOE_MAX_TOPK) return fail(MOE_ERR_INVALID_ARG, "T = %d, k = %d", T, k);
     if (H <= 0 || H % 4 != 0) return fail(MOE_ERR_INVALID_ARG, "H = %d must be a positive multiple of 4", H);
     if (T == 0) return ok();
@@ -302,9 +319,21 @@ int moe_combine(const float *y_slots, const float *y_shared, const float *topk_w
     if (residual && !x_next) return fail(MOE_ERR_INVALID_ARG, "x_next is required with a residual");
     if (!aligned16(y_slots) || (y_shared && !aligned16(y_shared)))
         return fail(MOE_ERR_INVALID_ARG, "y pointers not 16-byte aligned");
-    cudaError_t e = moe_launch_combine(y_slots, y_shared, topk_w, T, k, H, residual, out, x_next,
+    if (x_next_norm && !residual) return fail(MOE_ERR_INVALID_ARG, "x_next_norm needs a residual");
+    cudaError_t e = moe_launch_combine(y_slots, y_shared, topk_w, T, k, H, residual, out, x_next, x_next_norm,
                                        reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "combine launch");
+}
+
+int moe_rmsnorm(const uint16_t *x, int32_t T, int32_t H, uint16_t *n, moe_stream_t stream) {
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %d", T);
+    if (H <= 0 || H % 4 != 0) return fail(MOE_ERR_INVALID_ARG, "H = %d must be a positive multiple of 4", H);
+    if (T == 0) return ok();
+    if (!x || !n) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(x) & 7u) || (reinterpret_cast<uintptr_t>(n) & 7u))
+        return fail(MOE_ERR_INVALID_ARG, "x / n not 8-byte aligned");
+    cudaError_t e = moe_launch_rmsnorm(x, T, H, n, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "rmsnorm launch");
 }
 
 namespace {
@@ -351,7 +380,8 @@ size_t moe_layer_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k
 
 int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router, const float *bias, const uint16_t *x,
                       int32_t T, int32_t k, const uint16_t *residual, uint16_t *out, uint16_t *x_next,
-                      void *workspace, size_t workspace_bytes, int32_t mode, int32_t *status, moe_stream_t stream) {
+                      uint16_t *x_next_norm, void *workspace, size_t workspace_bytes, int32_t mode, int32_t *status,
+                      moe_stream_t stream) {
     int r = check_weights(w);
     if (r) return r;
     r = check_k(T, w->E, k);
@@ -370,7 +400,7 @@ int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router, cons
                               stream);
     if (r) return r;
     return moe_combine(L.y_slots, w->shared.n_experts == 1 ? L.y_shared : nullptr, L.tw, T, k, w->H, residual, out,
-                       x_next, stream);
+                       x_next, x_next_norm, stream);
 }
 
 }  // extern "C"

@@ -1,5 +1,6 @@
 // Combine: out[t] = bf16(sum_j w[t,j] * y[t*k+j] + y_shared[t]), fixed order;
-// optional residual stream x_next = bf16(residual + out).
+// optional residual stream x_next = bf16(residual + out) and its RMS-normalised
+// copy n_next = bf16(x_next / sqrt(mean(x_next^2) + eps)), the next layer's input.
 //
 // [P1] "step 4: three shelves, all on the GPU": the per-shelf results simply
 // add up; with one shared expert always on ([P5] "What the model actually is").
@@ -7,58 +8,111 @@
 
 namespace moe {
 
-// One thread per 4 consecutive hidden elements of one token.
-__global__ void __launch_bounds__(256)
+constexpr int kCombineThreads = 256;
+
+__device__ __forceinline__ float block_sum(float v, float *red) {
+    v = warp_sum(v);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float s = 0.f;
+    if (threadIdx.x < 32) {
+        s = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+        s = warp_sum(s);
+        if (threadIdx.x == 0) red[0] = s;
+    }
+    __syncthreads();
+    return red[0];
+}
+
+__device__ __forceinline__ uint2 pack4(uint16_t a, uint16_t b, uint16_t c, uint16_t d) {
+    return make_uint2(static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16),
+                      static_cast<uint32_t>(c) | (static_cast<uint32_t>(d) << 16));
+}
+
+// One CTA per token; each thread owns 4-element chunks c = threadIdx.x + i*blockDim.
+__global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const float *__restrict__ y, const float *__restrict__ ysh, const float *__restrict__ w,
                int T, int k, int H, const uint16_t *__restrict__ res, uint16_t *__restrict__ out,
-               uint16_t *__restrict__ xnext) {
-    const int per_tok = H / 4;
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= static_cast<int64_t>(T) * per_tok) return;
-    const int t = static_cast<int>(idx / per_tok);
-    const int c = static_cast<int>(idx - static_cast<int64_t>(t) * per_tok);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-        const float wj = w[static_cast<size_t>(t) * k + j];
-        const float4 v = reinterpret_cast<const float4 *>(y + (static_cast<size_t>(t) * k + j) * H)[c];
-        a.x = fmaf(wj, v.x, a.x);
-        a.y = fmaf(wj, v.y, a.y);
-        a.z = fmaf(wj, v.z, a.z);
-        a.w = fmaf(wj, v.w, a.w);
+               uint16_t *__restrict__ xnext, uint16_t *__restrict__ nnext, float eps) {
+    __shared__ float red[32];
+    const int t = blockIdx.x;
+    const int chunks = H / 4;
+    const size_t row = static_cast<size_t>(t) * H;
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const float wj = w[static_cast<size_t>(t) * k + j];
+            const float4 v = reinterpret_cast<const float4 *>(y + (static_cast<size_t>(t) * k + j) * H)[c];
+            a.x = fmaf(wj, v.x, a.x);
+            a.y = fmaf(wj, v.y, a.y);
+            a.z = fmaf(wj, v.z, a.z);
+            a.w = fmaf(wj, v.w, a.w);
+        }
+        if (ysh) {
+            const float4 v = reinterpret_cast<const float4 *>(ysh + row)[c];
+            a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+        }
+        const uint16_t o0 = f32_to_bf16_rne(a.x), o1 = f32_to_bf16_rne(a.y);
+        const uint16_t o2 = f32_to_bf16_rne(a.z), o3 = f32_to_bf16_rne(a.w);
+        if (out) *reinterpret_cast<uint2 *>(out + row + 4 * c) = pack4(o0, o1, o2, o3);
+        if (res) {
+            const uint2 r = *reinterpret_cast<const uint2 *>(res + row + 4 * c);
+            const uint16_t n0 = f32_to_bf16_rne(bf16lo(r.x) + bf16_to_f32(o0));
+            const uint16_t n1 = f32_to_bf16_rne(bf16hi(r.x) + bf16_to_f32(o1));
+            const uint16_t n2 = f32_to_bf16_rne(bf16lo(r.y) + bf16_to_f32(o2));
+            const uint16_t n3 = f32_to_bf16_rne(bf16hi(r.y) + bf16_to_f32(o3));
+            *reinterpret_cast<uint2 *>(xnext + row + 4 * c) = pack4(n0, n1, n2, n3);
+            const float f0 = bf16_to_f32(n0), f1 = bf16_to_f32(n1), f2 = bf16_to_f32(n2), f3 = bf16_to_f32(n3);
+            ss = fmaf(f0, f0, fmaf(f1, f1, fmaf(f2, f2, fmaf(f3, f3, ss))));
+        }
     }
-    if (ysh) {
-        const float4 v = reinterpret_cast<const float4 *>(ysh + static_cast<size_t>(t) * H)[c];
-        a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+    if (!res || !nnext) return;  // uniform across the CTA
+    const float tot = block_sum(ss, red);
+    const float rinv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(xnext + row + 4 * c);
+        *reinterpret_cast<uint2 *>(nnext + row + 4 * c) =
+            pack4(f32_to_bf16_rne(bf16lo(v.x) * rinv), f32_to_bf16_rne(bf16hi(v.x) * rinv),
+                  f32_to_bf16_rne(bf16lo(v.y) * rinv), f32_to_bf16_rne(bf16hi(v.y) * rinv));
     }
-    const uint16_t o0 = f32_to_bf16_rne(a.x), o1 = f32_to_bf16_rne(a.y);
-    const uint16_t o2 = f32_to_bf16_rne(a.z), o3 = f32_to_bf16_rne(a.w);
-    const size_t base = static_cast<size_t>(t) * H + 4 * c;
-    if (out) {
-        uint2 pk;
-        pk.x = static_cast<uint32_t>(o0) | (static_cast<uint32_t>(o1) << 16);
-        pk.y = static_cast<uint32_t>(o2) | (static_cast<uint32_t>(o3) << 16);
-        *reinterpret_cast<uint2 *>(out + base) = pk;
+}
+
+// n = bf16(x / sqrt(mean(x^2) + eps)), one CTA per token.
+__global__ void __launch_bounds__(kCombineThreads)
+rmsnorm_kernel(const uint16_t *__restrict__ x, int H, float eps, uint16_t *__restrict__ n) {
+    __shared__ float red[32];
+    const size_t row = static_cast<size_t>(blockIdx.x) * H;
+    const int chunks = H / 4;
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(x + row + 4 * c);
+        const float f0 = bf16lo(v.x), f1 = bf16hi(v.x), f2 = bf16lo(v.y), f3 = bf16hi(v.y);
+        ss = fmaf(f0, f0, fmaf(f1, f1, fmaf(f2, f2, fmaf(f3, f3, ss))));
     }
-    if (res) {
-        const uint2 r = *reinterpret_cast<const uint2 *>(res + base);
-        const uint16_t n0 = f32_to_bf16_rne(bf16lo(r.x) + bf16_to_f32(o0));
-        const uint16_t n1 = f32_to_bf16_rne(bf16hi(r.x) + bf16_to_f32(o1));
-        const uint16_t n2 = f32_to_bf16_rne(bf16lo(r.y) + bf16_to_f32(o2));
-        const uint16_t n3 = f32_to_bf16_rne(bf16hi(r.y) + bf16_to_f32(o3));
-        uint2 pk;
-        pk.x = static_cast<uint32_t>(n0) | (static_cast<uint32_t>(n1) << 16);
-        pk.y = static_cast<uint32_t>(n2) | (static_cast<uint32_t>(n3) << 16);
-        *reinterpret_cast<uint2 *>(xnext + base) = pk;
+    const float tot = block_sum(ss, red);
+    const float rinv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(x + row + 4 * c);
+        *reinterpret_cast<uint2 *>(n + row + 4 * c) =
+            pack4(f32_to_bf16_rne(bf16lo(v.x) * rinv), f32_to_bf16_rne(bf16hi(v.x) * rinv),
+                  f32_to_bf16_rne(bf16lo(v.y) * rinv), f32_to_bf16_rne(bf16hi(v.y) * rinv));
     }
 }
 
 }  // namespace moe
 
 cudaError_t moe_launch_combine(const float *y, const float *ysh, const float *w, int T, int k, int H,
-                               const uint16_t *res, uint16_t *out, uint16_t *xnext, cudaStream_t s) {
-    const int64_t n = static_cast<int64_t>(T) * (H / 4);
-    const int threads = 256;
-    const int64_t grid = (n + threads - 1) / threads;
-    moe::combine_kernel<<<static_cast<unsigned>(grid), threads, 0, s>>>(y, ysh, w, T, k, H, res, out, xnext);
+                               const uint16_t *res, uint16_t *out, uint16_t *xnext, uint16_t *nnext,
+                               cudaStream_t s) {
+    moe::combine_kernel<<<T, moe::kCombineThreads, 0, s>>>(y, ysh, w, T, k, H, res, out, xnext, nnext,
+                                                           MOE_NORM_EPS);
+    return cudaGetLastError();
+}
+
+cudaError_t moe_launch_rmsnorm(const uint16_t *x, int T, int H, uint16_t *n, cudaStream_t s) {
+    moe::rmsnorm_kernel<<<T, moe::kCombineThreads, 0, s>>>(x, H, MOE_NORM_EPS, n);
     return cudaGetLastError();
 }

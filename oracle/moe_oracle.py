@@ -278,12 +278,27 @@ def round_bf16(v):
 # ---------------------------------------------------------------------------
 # Combine and the residual stream
 # [P1] "step 4": the three shelf results simply add up.
+# [P5] "What the model actually is": 48 layers, a residual design.
 # READING: out[t] = bf16( sum_j w[t,j] * y[t*k+j] + y_shared[t] ) summed in the
-# fixed order j = 0..k-1, then the shared expert; with a residual input the
-# layer also returns x_next = bf16( x + out ) (no normalisation).
+# fixed order j = 0..k-1, then the shared expert.  In a stack the residual
+# stream is bf16, x_next = bf16( x + out ), and each MoE layer reads the RMS-
+# normalised stream n = bf16( x / sqrt(mean(x^2) + eps) ) (pre-norm, no learned
+# gain, eps = 1e-6): without a norm the SwiGLU blocks, which grow like |x|^2,
+# drive the stack to overflow within about 14 layers.
 # ---------------------------------------------------------------------------
 
+NORM_EPS = 1e-6
+
+
+def rms_norm(x, eps=NORM_EPS):
+    """bf16( x / sqrt(mean(x^2) + eps) ) per row, in fp64."""
+    x = np.asarray(x, np.float64)
+    r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return round_bf16(x / r)
+
+
 def combine(y_slots, y_shared, topk_w, residual=None):
+    """Returns out, or (out, x_next, n_next) when a residual is given."""
     y = np.asarray(y_slots, np.float64)
     w = np.asarray(topk_w, np.float64)
     T, k = w.shape
@@ -293,7 +308,8 @@ def combine(y_slots, y_shared, topk_w, residual=None):
     out = round_bf16(s)
     if residual is None:
         return out
-    return out, round_bf16(np.asarray(residual, np.float64) + out)
+    x_next = round_bf16(np.asarray(residual, np.float64) + out)
+    return out, x_next, rms_norm(x_next)
 
 
 # ---------------------------------------------------------------------------
@@ -370,7 +386,24 @@ def moe_layer(x, w_router, bias, k, expert_weights, shared_weights, H, I, residu
     if shared_weights is not None:
         y_shared = expert_ffn(x, *shared_weights)
     res = combine(y_slots, y_shared, w, residual)
-    out, x_next = (res if residual is not None else (res, None))
+    out, x_next, n_next = (res if residual is not None else (res, None, None))
     return dict(logits=logits, topk_idx=idx, topk_w=w, expert_offsets=offsets,
                 sorted_slot=sorted_slot, slot_pos=slot_pos, y_slots=y_slots,
-                y_shared=y_shared, out=out, x_next=x_next)
+                y_shared=y_shared, out=out, x_next=x_next, n_next=n_next)
+
+
+def moe_stack(x0, layers, k, H, I):
+    """Free-running stack: n_0 = rms_norm(x_0); per layer out = MoE(n_l),
+    x_{l+1} = bf16(x_l + out), n_{l+1} = rms_norm(x_{l+1}).
+
+    ``layers`` is a list of (w_router, bias, expert_weights, shared_weights).
+    Returns the per-layer results (each holding its input n under key "n")."""
+    x = np.asarray(x0, np.float64)
+    n = rms_norm(x)
+    results = []
+    for (wr, bias, ew, sw) in layers:
+        r = moe_layer(n.astype(np.float32), wr, bias, k, ew, sw, H, I, residual=x)
+        r["n"], r["x"] = n, x
+        results.append(r)
+        x, n = r["x_next"], r["n_next"]
+    return results

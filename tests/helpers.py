@@ -34,6 +34,30 @@ def to_np(t):
     return t.detach().cpu().numpy()
 
 
+def _prepare_expert(args):
+    """Worker: oracle quantisation + dequantisation of one expert (runs in a
+    spawned process; pure numpy, no GPU)."""
+    wgu, wdn, bits, H, I = args
+    gq, gs = oracle.quantize_pack(wgu, bits)
+    dq, ds = oracle.quantize_pack(wdn, bits)
+    return oracle.dequantize_f32(gq, gs, bits, H), oracle.dequantize_f32(dq, ds, bits, I)
+
+
+_POOL = None
+
+
+def pool():
+    """A process pool started with 'spawn' (safe after CUDA is initialised)."""
+    global _POOL
+    if _POOL is None:
+        import concurrent.futures
+        import multiprocessing
+        import os
+        n = max(1, min(32, (os.cpu_count() or 2) - 1))
+        _POOL = concurrent.futures.ProcessPoolExecutor(n, mp_context=multiprocessing.get_context("spawn"))
+    return _POOL
+
+
 class OracleExperts:
     """Expert id -> dequantised fp32 weights, quantised by the oracle from the
     generator's source weights (drawn on ``device`` like the GPU layer's)."""
@@ -42,6 +66,18 @@ class OracleExperts:
         self.cfg, self.seed, self.device = cfg, seed, device
         self._cache = {}
         self._packed = {}
+
+    def prefetch(self, experts):
+        """Prepare several experts in parallel (worker processes)."""
+        todo = [int(e) for e in sorted(set(int(v) for v in experts)) if int(e) not in self._cache]
+        if not todo:
+            return
+        jobs = []
+        for e in todo:
+            wgu, wdn = inputs.expert_source(self.cfg, self.seed, e, self.device)
+            jobs.append((wgu.cpu().numpy(), wdn.cpu().numpy(), self.bits(e), self.cfg.H, self.cfg.I))
+        for e, res in zip(todo, pool().map(_prepare_expert, jobs)):
+            self._cache[e] = res
 
     def bits(self, e):
         if e == self.cfg.E:

@@ -25,7 +25,7 @@ def header_functions():
 def test_library_exports_every_declared_symbol():
     L = B.lib()
     declared = header_functions()
-    assert len(declared) >= 14
+    assert len(declared) >= 15
     for name in declared:
         assert hasattr(L, name), name
     assert declared == {n for n, _, _ in B.SIGNATURES}
@@ -102,8 +102,10 @@ def test_router_and_quantize_reject_bad_args():
     assert L.moe_router_topk(p, p, None, 4, 256, 16, 2, None, p, p, None, 0, None) == B.MOE_ERR_WORKSPACE
     assert L.moe_topk_softmax(p, 4, 16, 0, p, p, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_bucketize(p, 4, 2, 16, None, p, p, p, None, None) == B.MOE_ERR_INVALID_ARG
-    assert L.moe_combine(p, None, p, 4, 2, 6, None, p, None, None) == B.MOE_ERR_INVALID_ARG
-    assert L.moe_combine(p, None, p, 4, 2, 256, p, p, None, None) == B.MOE_ERR_INVALID_ARG  # residual w/o x_next
+    assert L.moe_combine(p, None, p, 4, 2, 6, None, p, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(p, None, p, 4, 2, 256, p, p, None, None, None) == B.MOE_ERR_INVALID_ARG  # no x_next
+    assert L.moe_combine(p, None, p, 4, 2, 256, None, p, None, p, None) == B.MOE_ERR_INVALID_ARG  # norm w/o res
+    assert L.moe_rmsnorm(p, 4, 6, p, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_dequantize(p, p, 4, 128, 8, None, None, None) == B.MOE_ERR_INVALID_ARG
 
 

@@ -285,9 +285,24 @@ def test_combine_single_slot_is_rounding():
     y = rng.standard_normal((3, 16))
     out = oracle.combine(y, None, np.ones((3, 1)))
     assert np.array_equal(out, oracle.round_bf16(y))
-    out2, nxt = oracle.combine(y, np.zeros((3, 16)), np.ones((3, 1)), residual=np.ones((3, 16)))
+    out2, nxt, nrm = oracle.combine(y, np.zeros((3, 16)), np.ones((3, 1)), residual=np.ones((3, 16)))
     assert np.array_equal(out2, out)
     assert np.array_equal(nxt, oracle.round_bf16(1.0 + out))
+    assert np.array_equal(nrm, oracle.rms_norm(nxt))
+
+
+def test_rms_norm_closed_forms_and_library():
+    # a constant row normalises to ones (up to eps); sign and scale are preserved
+    c = np.full((2, 64), 3.0)
+    assert np.allclose(oracle.rms_norm(c), 1.0, atol=2 ** -8)
+    v = np.array([[3.0, -4.0] * 8])          # rms = sqrt(12.5)
+    assert np.allclose(oracle.rms_norm(v), oracle.round_bf16(v / np.sqrt(12.5 + oracle.NORM_EPS)), rtol=0)
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((5, 256)) * 7
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (256,), eps=oracle.NORM_EPS).numpy()
+    assert np.allclose(oracle.rms_norm(x), oracle.round_bf16(ref), rtol=0, atol=0) or \
+        np.max(np.abs(oracle.rms_norm(x) - ref)) <= 2 ** -8 * np.max(np.abs(ref))
+    assert np.array_equal(oracle.rms_norm(x * 2 ** 5), oracle.rms_norm(x))  # exact scale invariance
 
 
 # ----------------------------------------------------------------------------
