@@ -24,7 +24,8 @@ cudaError_t moe_configure_ffn_stream();
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &, cudaStream_t);
 bool moe_ffn_stream_supported(int H, int I);
 cudaError_t moe_configure_ffn_gemm();
-cudaError_t moe_launch_ffn_gemm(const moe::FfnParams &, void *ws, size_t ws_bytes, cudaStream_t);
+cudaError_t moe_launch_ffn_gemm(const moe::FfnParams &, void *ws, size_t ws_bytes, cudaStream_t, int min_count);
+bool moe_ffn_gemm_supported(int H, int I);
 size_t moe_ffn_gemm_workspace(const moe_layer_weights *, int T, int k);
 cudaError_t moe_launch_combine(const float *, const float *, const float *, int, int, int, const uint16_t *,
                                uint16_t *, uint16_t *, uint16_t *, cudaStream_t);
@@ -149,6 +150,7 @@ moe::FfnParams make_params(const moe_layer_weights *w, const uint16_t *x, int T,
     p.active = active;
     p.h = h;
     p.ctr = nullptr;
+    p.max_count = 0x7fffffff;
     p.y_slots = y_slots;
     p.y_shared = y_shared;
     p.status = status;
@@ -160,11 +162,23 @@ size_t ffn_ctr_bytes(const moe_layer_weights *w, int T, int k) {
     return align_up((static_cast<size_t>(ma < w->E ? ma : w->E) + 1) * sizeof(int));
 }
 
-size_t ffn_ws_bytes(const moe_layer_weights *w, int T, int k, int mode) {
+// Token count from which an expert goes through the tensor-core GEMM in
+// MOE_FFN_AUTO mode (below it the streaming GEMV reads the weights once anyway
+// and wastes no tensor-core columns).
+constexpr int kGemmMinTokens = 24;
+
+bool uses_gemv(int mode) { return mode != MOE_FFN_GEMM; }
+bool uses_gemm(int mode, int T) { return mode == MOE_FFN_GEMM || (mode == MOE_FFN_AUTO && T >= kGemmMinTokens); }
+
+size_t gemv_ws_bytes(const moe_layer_weights *w, int T, int k) {
     const size_t rows = static_cast<size_t>(T) * k + static_cast<size_t>(T);
-    size_t gemv = align_up(rows * w->I * sizeof(float)) + ffn_ctr_bytes(w, T, k);
-    size_t gemm = mode == MOE_FFN_GEMV ? 0 : moe_ffn_gemm_workspace(w, T, k);
-    return (gemv > gemm ? gemv : gemm) + 256;
+    return align_up(rows * w->I * sizeof(float)) + ffn_ctr_bytes(w, T, k);
+}
+
+size_t ffn_ws_bytes(const moe_layer_weights *w, int T, int k, int mode) {
+    const size_t gemv = uses_gemv(mode) ? gemv_ws_bytes(w, T, k) : 0;
+    const size_t gemm = uses_gemm(mode, T) ? align_up(moe_ffn_gemm_workspace(w, T, k)) : 0;
+    return gemv + gemm + 256;
 }
 
 }  // namespace
@@ -291,19 +305,27 @@ int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t
     if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "ffn workspace needs %zu bytes", need);
     r = ensure_configured();
     if (r) return r;
-    if (mode != MOE_FFN_GEMM && !moe_ffn_stream_supported(w->H, w->I))
+    if (uses_gemv(mode) && !moe_ffn_stream_supported(w->H, w->I))
         return fail(MOE_ERR_UNSUPPORTED, "GEMV path supports H, I <= 2048");
-    float *h = static_cast<float *>(workspace);
+    if (uses_gemm(mode, T) && !moe_ffn_gemm_supported(w->H, w->I))
+        return fail(MOE_ERR_UNSUPPORTED, "GEMM path needs H %% 128 == 0 and I %% 64 == 0");
+    char *ws = static_cast<char *>(workspace);
+    float *h = reinterpret_cast<float *>(ws);
     moe::FfnParams p = make_params(w, x, T, k, expert_offsets, sorted_slot, active, y_slots, y_shared, h, status);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    if (mode == MOE_FFN_GEMM) {
-        e = moe_launch_ffn_gemm(p, workspace, workspace_bytes, s);
-    } else {
+    cudaError_t e = cudaSuccess;
+    const bool gemm = uses_gemm(mode, T);
+    const int split = mode == MOE_FFN_GEMM ? 1 : kGemmMinTokens;  // GEMM takes experts with >= split tokens
+    if (uses_gemv(mode)) {
         const size_t hb = align_up((static_cast<size_t>(T) * k + T) * w->I * sizeof(float));
-        p.ctr = reinterpret_cast<int *>(static_cast<char *>(workspace) + hb);
+        p.ctr = reinterpret_cast<int *>(ws + hb);
+        p.max_count = gemm ? split - 1 : 0x7fffffff;
         e = cudaMemsetAsync(p.ctr, 0, ffn_ctr_bytes(w, T, k), s);
         if (e == cudaSuccess) e = moe_launch_ffn_stream(p, s);
+    }
+    if (e == cudaSuccess && gemm) {
+        char *gws = ws + (uses_gemv(mode) ? gemv_ws_bytes(w, T, k) : 0);
+        e = moe_launch_ffn_gemm(p, gws, 0, s, split);
     }
     return e == cudaSuccess ? ok() : cuda_fail(e, "ffn launch");
 }

@@ -13,6 +13,7 @@ struct FfnParams {
     const int32_t *offsets, *sorted, *active;
     float *h;             // fp32 [T*k + T][I] (GEMV path)
     int *ctr;             // [max_active + 1] gate_up tiles done per slot (zeroed per call)
+    int max_count;        // GEMV path: experts with more tokens are left to the GEMM path
     float *y_slots;       // fp32 [T*k][H]
     float *y_shared;      // fp32 [T][H]
     int32_t *status;

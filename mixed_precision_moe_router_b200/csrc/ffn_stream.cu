@@ -28,10 +28,11 @@ namespace moe {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kStreamThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kGuPairs = 8;                                  // gate/up row pairs per tile
+constexpr int kGuPairs = 16;                                 // gate/up row pairs per tile (2 per warp)
 constexpr int kDnRows = 64;                                  // down rows per tile
 constexpr int kMaxStages = 6;
 constexpr int kMaxRegK = 2048;  // activations held in registers: K <= 2048
+constexpr int kMaxSmemEntries = 2048;  // token-entry tables kept in shared memory up to this size
 
 __host__ __device__ __forceinline__ int row_bytes(int K, int bits) { return K * bits / 8; }
 __host__ __device__ __forceinline__ int gu_tile_bytes(int H, int bits) {
@@ -40,9 +41,18 @@ __host__ __device__ __forceinline__ int gu_tile_bytes(int H, int bits) {
 __host__ __device__ __forceinline__ int dn_tile_bytes(int I, int bits) {
     return kDnRows * (row_bytes(I, bits) + I / 16);
 }
+// Work estimate used to balance tiles over CTAs: bytes moved plus a share for
+// the per-weight dequant/FMA work, which is the same for every precision.
+__host__ __device__ __forceinline__ long long gu_tile_cost(int H, int bits) {
+    return gu_tile_bytes(H, bits) + static_cast<long long>(2 * kGuPairs) * H / 2;
+}
+__host__ __device__ __forceinline__ long long dn_tile_cost(int I, int bits) {
+    return dn_tile_bytes(I, bits) + static_cast<long long>(kDnRows) * I / 2;
+}
 
 struct SlotTabs {  // per expert slot, in shared memory
     int *expert, *bits, *count, *first;
+    int *tok, *row;  // entries [first, first + count) of every slot: token and h/y row
 };
 
 // Shelf pointers of expert e, read from the kernel parameters with constant
@@ -100,11 +110,11 @@ __device__ __forceinline__ void for_each_tile(const FfnParams &p, const SlotTabs
         long long total = 0;
         for (int a = 0; a < n_slots; ++a)
             total += static_cast<long long>(nt) *
-                     (phase == 0 ? gu_tile_bytes(p.w.H, st.bits[a]) : dn_tile_bytes(p.w.I, st.bits[a]));
+                     (phase == 0 ? gu_tile_cost(p.w.H, st.bits[a]) : dn_tile_cost(p.w.I, st.bits[a]));
         const long long lo = total * c / G, hi = total * (c + 1) / G;
         long long off = 0;
         for (int a = 0; a < n_slots && off < hi; ++a) {
-            const long long tb = phase == 0 ? gu_tile_bytes(p.w.H, st.bits[a]) : dn_tile_bytes(p.w.I, st.bits[a]);
+            const long long tb = phase == 0 ? gu_tile_cost(p.w.H, st.bits[a]) : dn_tile_cost(p.w.I, st.bits[a]);
             const long long end = off + nt * tb;
             if (end > lo) {
                 const long long b0 = lo > off ? (lo - off + tb - 1) / tb : 0;
@@ -219,20 +229,47 @@ __device__ __forceinline__ void load_act_f32(const float *row, int K, int lane, 
     }
 }
 
-// token and output row of the n-th entry of slot a
+// token and output row of the n-th entry of slot a (tables built in the prologue)
 __device__ __forceinline__ void slot_entry(const FfnParams &p, const SlotTabs &st, int a, int n, int &tok,
                                            int &row) {
-    if (st.expert[a] == p.E) {
-        tok = n;
-        row = p.T * p.k + n;
+    const int j = st.first[a] + n;
+    if (st.tok) {
+        tok = st.tok[j];
+        row = st.row[j];
+    } else if (j >= p.T * p.k) {  // shared expert
+        tok = j - p.T * p.k;
+        row = j;
     } else {
-        const int s = p.sorted[st.first[a] + n];
-        tok = s / p.k;
-        row = s;
+        row = p.sorted[j];
+        tok = row / p.k;
     }
 }
 
-// gate_up tile: warp w computes pair i = 8*tile + w for every token of the slot.
+// Sum each of N values over the 32 lanes with N-1 + log2(32/N) shuffles instead
+// of 5N: at every step each lane keeps half of its values and swaps the other
+// half.  On return lane l holds the full sum of value (l / (32 / N)) % N.
+template <int N>
+__device__ __forceinline__ float transpose_reduce(float (&v)[N]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int n = N, o = 16; n > 1; n >>= 1, o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? v[i] : v[i + n / 2];
+            const float keep = upper ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    float r = v[0];
+    constexpr int rest = 32 / N;  // lanes still holding partial sums of the same value
+#pragma unroll
+    for (int o = rest / 2; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+    return r;
+}
+
+// gate_up tile: warp w computes pairs i = 16*tile + 2*w + {0, 1} for every
+// token of the slot.  h is written with plain stores; the caller publishes it.
 template <int BITS, int UPL>
 __device__ __forceinline__ void consume_gu(const FfnParams &p, const SlotTabs &st, int a, int tile,
                                            const uint8_t *stage, float *act, int &act_key) {
@@ -241,11 +278,12 @@ __device__ __forceinline__ void consume_gu(const FfnParams &p, const SlotTabs &s
     constexpr int W = UnitW<BITS>::W;
     const int U = H / W;
     const int rb = row_bytes(H, BITS);
-    const uint8_t *gq = stage + warp * rb;
-    const uint8_t *uq = stage + kGuPairs * rb + warp * rb;
-    const uint16_t *gs = reinterpret_cast<const uint16_t *>(stage + 2 * kGuPairs * rb) + warp * (H / 32);
-    const uint16_t *us = gs + kGuPairs * (H / 32);
-    const int i = tile * kGuPairs + warp;
+    const int nsc = H / 32;
+    const uint8_t *q0 = stage + (2 * warp) * rb;                 // gate rows 2w, 2w+1
+    const uint8_t *q1 = stage + (kGuPairs + 2 * warp) * rb;      // up rows
+    const uint16_t *s0 = reinterpret_cast<const uint16_t *>(stage + 2 * kGuPairs * rb) + (2 * warp) * nsc;
+    const uint16_t *s1 = s0 + kGuPairs * nsc;
+    const int i0 = tile * kGuPairs + 2 * warp;
     for (int n = 0; n < st.count[a]; ++n) {
         int tok, row;
         slot_entry(p, st, a, n, tok, row);
@@ -254,20 +292,24 @@ __device__ __forceinline__ void consume_gu(const FfnParams &p, const SlotTabs &s
             load_act_bf16<BITS, UPL>(p.x + static_cast<size_t>(tok) * H, H, lane, act);
             act_key = key;
         }
-        float g = 0.f, u = 0.f;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};  // g(i0), g(i0+1), u(i0), u(i0+1)
 #pragma unroll
         for (int j = 0; j < UPL; ++j) {
             const int un = lane + 32 * j;
             if (un < U) {
-                g += unit_dot<BITS>(gq, gs, H, un, act + W * j);
-                u += unit_dot<BITS>(uq, us, H, un, act + W * j);
+                v[0] += unit_dot<BITS>(q0, s0, H, un, act + W * j);
+                v[1] += unit_dot<BITS>(q0 + rb, s0 + nsc, H, un, act + W * j);
+                v[2] += unit_dot<BITS>(q1, s1, H, un, act + W * j);
+                v[3] += unit_dot<BITS>(q1 + rb, s1 + nsc, H, un, act + W * j);
             }
         }
-        g = warp_sum(g);
-        u = warp_sum(u);
-        if (lane == 0) {
-            p.h[static_cast<size_t>(row) * I + i] = g / (1.0f + expf(-g)) * u;
-            __threadfence();  // published before this warp counts the tile done
+        // lane l ends with value (l / 8) % 4: lanes 0 and 8 hold the two gates,
+        // 16 and 24 the two ups
+        const float r = transpose_reduce<4>(v);
+        const float up = __shfl_down_sync(0xffffffffu, r, 16);
+        if (lane == 0 || lane == 8) {
+            const int i = i0 + (lane >> 3);
+            p.h[static_cast<size_t>(row) * I + i] = r / (1.0f + expf(-r)) * up;
         }
     }
 }
@@ -275,7 +317,7 @@ __device__ __forceinline__ void consume_gu(const FfnParams &p, const SlotTabs &s
 // down tile: warp w computes rows 64*tile + 8*w + r (r < 8) for every token.
 template <int BITS, int UPL>
 __device__ __forceinline__ void consume_dn(const FfnParams &p, const SlotTabs &st, int a, int tile,
-                                           const uint8_t *stage, float *act) {
+                                           const uint8_t *stage, float *act, int &act_key) {
     const int H = p.w.H, I = p.w.I;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int W = UnitW<BITS>::W;
@@ -286,7 +328,11 @@ __device__ __forceinline__ void consume_dn(const FfnParams &p, const SlotTabs &s
     for (int n = 0; n < st.count[a]; ++n) {
         int tok, row;
         slot_entry(p, st, a, n, tok, row);
-        load_act_f32<BITS, UPL>(p.h + static_cast<size_t>(row) * I, I, lane, act);
+        const int key = -(row * 16 + BITS) - 2;
+        if (key != act_key) {
+            load_act_f32<BITS, UPL>(p.h + static_cast<size_t>(row) * I, I, lane, act);
+            act_key = key;
+        }
         float acc[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
@@ -299,18 +345,11 @@ __device__ __forceinline__ void consume_dn(const FfnParams &p, const SlotTabs &s
             }
             acc[r] = v;
         }
-        // reduce the R row sums across the warp: after the butterfly lane r holds row r
-#pragma unroll
-        for (int r = 0; r < R; ++r) acc[r] = warp_sum(acc[r]);
+        // lane l ends with the full sum of row (l / 4) % 8
+        const float res = transpose_reduce<R>(acc);
         float *dst = row >= p.T * p.k ? p.y_shared + static_cast<size_t>(row - p.T * p.k) * H
                                       : p.y_slots + static_cast<size_t>(row) * H;
-        if (lane < R) {
-            float v = acc[0];
-#pragma unroll
-            for (int r = 1; r < R; ++r)
-                if (lane == r) v = acc[r];
-            dst[tile * kDnRows + warp * R + lane] = v;
-        }
+        if ((lane & 3) == 0) dst[tile * kDnRows + warp * R + (lane >> 2)] = res;
     }
 }
 
@@ -336,17 +375,16 @@ __device__ __forceinline__ void consume_tile(const FfnParams &p, const SlotTabs 
             consume_gu<3, 1>(p, st, a, tile, stage, act, act_key);
         }
     } else {
-        act_key = -1;
         const int upl = upl_of(p.w.I, bits);
         if (bits == 8) {
-            if (upl <= 1) consume_dn<8, 1>(p, st, a, tile, stage, act);
-            else if (upl <= 2) consume_dn<8, 2>(p, st, a, tile, stage, act);
-            else consume_dn<8, 4>(p, st, a, tile, stage, act);
+            if (upl <= 1) consume_dn<8, 1>(p, st, a, tile, stage, act, act_key);
+            else if (upl <= 2) consume_dn<8, 2>(p, st, a, tile, stage, act, act_key);
+            else consume_dn<8, 4>(p, st, a, tile, stage, act, act_key);
         } else if (bits == 4) {
-            if (upl <= 1) consume_dn<4, 1>(p, st, a, tile, stage, act);
-            else consume_dn<4, 2>(p, st, a, tile, stage, act);
+            if (upl <= 1) consume_dn<4, 1>(p, st, a, tile, stage, act, act_key);
+            else consume_dn<4, 2>(p, st, a, tile, stage, act, act_key);
         } else {
-            consume_dn<3, 1>(p, st, a, tile, stage, act);
+            consume_dn<3, 1>(p, st, a, tile, stage, act, act_key);
         }
     }
 }
@@ -407,9 +445,25 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, StreamSmem &
     float act[64];
     int act_key = -1;
     int i = 0;
-    const int gu_done = (I / kGuPairs) * kConsumerWarps;  // one count per consumer warp per tile
+    // h of a slot is published (fence + count) once per warp when the warp
+    // leaves that slot: the count target is (gate_up tiles) x (consumer warps)
+    // contributions, each contribution counting its tiles.
+    int pend_slot = -1, pend_tiles = 0;
+    const int gu_done = (I / kGuPairs) * kConsumerWarps;
+    auto publish = [&]() {
+        if (pend_slot >= 0) {
+            __syncwarp();
+            if (lane == 0 || lane == 8) __threadfence();  // the two lanes that wrote h
+            __syncwarp();
+            if (lane == 0) atomicAdd(p.ctr + pend_slot, pend_tiles);
+        }
+        pend_slot = -1;
+        pend_tiles = 0;
+    };
     for_each_tile(p, S.st, n_slots, [&](int phase, int a, int tile) {
         if (*static_cast<volatile int *>(S.abort)) return;
+        if (phase == 0 && a != pend_slot) publish();
+        if (phase == 1 && pend_slot >= 0) publish();
         const int s = i % nstages;
         const uint32_t par = (i / nstages) & 1;
         bool ok = mbar_wait(&S.full[s], par);
@@ -426,12 +480,14 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, StreamSmem &
         }
         consume_tile(p, S.st, phase, a, tile, S.stages + static_cast<size_t>(s) * stage_bytes, act, act_key);
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&S.empty[s]);
-            if (phase == 0) atomicAdd(p.ctr + a, 1);
+        if (lane == 0) mbar_arrive(&S.empty[s]);
+        if (phase == 0) {
+            pend_slot = a;
+            ++pend_tiles;
         }
         ++i;
     });
+    publish();
 }
 
 __global__ void __launch_bounds__(kStreamThreads, 1)
@@ -449,6 +505,11 @@ ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
     S.st.bits = tabs + max_slots;
     S.st.count = tabs + 2 * max_slots;
     S.st.first = tabs + 3 * max_slots;
+    // entry tables in shared memory when they fit, else read from global
+    const int n_ent = p.T * p.k + p.T;
+    const bool ent_smem = n_ent <= kMaxSmemEntries;
+    S.st.tok = ent_smem ? tabs + 4 * max_slots : nullptr;
+    S.st.row = ent_smem ? S.st.tok + n_ent : nullptr;
     // slot table: active routed experts, then the shared expert
     const int n_active = min(p.active[0], p.max_active);
     for (int a = threadIdx.x; a < n_active; a += blockDim.x) {
@@ -456,17 +517,34 @@ ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
         const bool bad = e < 0 || e >= p.E;
         if (bad) e = 0;
         const int f = p.offsets[e];
+        const int cnt = bad ? 0 : p.offsets[e + 1] - f;
         S.st.expert[a] = e;
         S.st.bits[a] = expert_bits(p, e);
         S.st.first[a] = f;
-        S.st.count[a] = bad ? 0 : p.offsets[e + 1] - f;
+        S.st.count[a] = cnt > p.max_count ? 0 : cnt;  // larger groups go to the tensor-core path
+    }
+    // entries: routed slots in sorted order (first = expert offset), then the
+    // shared expert's T tokens at [T*k, T*k + T)
+    const int S_ = p.T * p.k;
+    const int n_routed = min(p.offsets[p.E], S_);
+    if (ent_smem) {
+        for (int j = threadIdx.x; j < n_routed; j += blockDim.x) {
+            const int sl = p.sorted[j];
+            const bool okj = sl >= 0 && sl < S_;
+            S.st.tok[j] = okj ? sl / p.k : 0;
+            S.st.row[j] = okj ? sl : 0;
+        }
+        for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
+            S.st.tok[S_ + t] = t;
+            S.st.row[S_ + t] = S_ + t;
+        }
     }
     if (threadIdx.x == 0) {
         if (p.has_shared) {
             S.st.expert[n_active] = p.E;
             S.st.bits[n_active] = p.w.shared.bits;
-            S.st.first[n_active] = 0;
-            S.st.count[n_active] = p.T;
+            S.st.first[n_active] = S_;
+            S.st.count[n_active] = p.T > p.max_count ? 0 : p.T;
         }
         for (int s = 0; s < nstages; ++s) {
             mbar_init(&S.full[s], 1);
@@ -482,12 +560,14 @@ ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
 
 }  // namespace moe
 
-size_t moe_ffn_stream_smem(int H, int I, int max_slots, int *nstages, int *stage_bytes) {
+size_t moe_ffn_stream_smem(int H, int I, int max_slots, int n_ent, int *nstages, int *stage_bytes) {
     int sb = moe::gu_tile_bytes(H, 8);
     const int d = moe::dn_tile_bytes(I, 8);
     if (d > sb) sb = d;
     sb = (sb + 1023) & ~1023;
-    const size_t tail = 2 * moe::kMaxStages * sizeof(uint64_t) + 16 + 4 * sizeof(int) * static_cast<size_t>(max_slots);
+    const size_t ent = n_ent <= moe::kMaxSmemEntries ? 2 * sizeof(int) * static_cast<size_t>(n_ent) : 0;
+    const size_t tail =
+        2 * moe::kMaxStages * sizeof(uint64_t) + 16 + 4 * sizeof(int) * static_cast<size_t>(max_slots) + ent;
     const size_t budget = 220 * 1024;
     int ns = static_cast<int>((budget - tail) / sb);
     if (ns > moe::kMaxStages) ns = moe::kMaxStages;
@@ -507,7 +587,8 @@ bool moe_ffn_stream_supported(int H, int I) {
 // counters (int[max_active + 1]) must be zero on entry; the caller clears them.
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     int nstages = 0, stage_bytes = 0;
-    const size_t smem = moe_ffn_stream_smem(p.w.H, p.w.I, p.max_active + 1, &nstages, &stage_bytes);
+    const size_t smem =
+        moe_ffn_stream_smem(p.w.H, p.w.I, p.max_active + 1, p.T * p.k + p.T, &nstages, &stage_bytes);
     if (nstages < 2) return cudaErrorInvalidConfiguration;
     int dev = 0;
     cudaGetDevice(&dev);

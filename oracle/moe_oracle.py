@@ -255,6 +255,33 @@ def expert_ffn(x, w_gate_up, w_down):
     return h @ np.asarray(w_down, np.float64).T
 
 
+def round_f16(v):
+    """Round to the nearest fp16 value, ties to even (one rounding from fp64)."""
+    v = np.asarray(v, np.float64)
+    out = np.zeros_like(v)
+    nz = (v != 0) & np.isfinite(v)
+    m, e = np.frexp(v[nz])
+    step_exp = np.maximum(e - 11, -24)  # 11 significant bits; subnormal grid 2**-24
+    r = np.ldexp(np.rint(np.ldexp(v[nz], -step_exp)), step_exp)
+    r = np.where(np.abs(r) > 65504.0, np.copysign(np.inf, r), r)
+    out[nz] = r
+    out[~np.isfinite(v)] = v[~np.isfinite(v)]
+    return out
+
+
+def expert_ffn_f16_staged(x, w_gate_up_f16, w_down_f16):
+    """The tensor-core path's arithmetic: x, the dequantised weights and h are
+    each rounded to fp16; products and sums are exact (fp64 here, fp32 on the
+    tensor cores).  ``w_*_f16`` are the fp16 staging values fp16(d*q)."""
+    x16 = round_f16(x)
+    wgu = np.asarray(w_gate_up_f16, np.float64)
+    I = wgu.shape[0] // 2
+    g = x16 @ wgu[:I].T
+    u = x16 @ wgu[I:].T
+    h16 = round_f16(silu(g) * u)
+    return h16 @ np.asarray(w_down_f16, np.float64).T
+
+
 # ---------------------------------------------------------------------------
 # Rounding to bf16 (outputs and the residual stream are bf16)
 # ---------------------------------------------------------------------------

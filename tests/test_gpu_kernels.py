@@ -191,7 +191,7 @@ def _tiny():
     return cfg, seed, layer
 
 
-@pytest.mark.parametrize("mode", [B.FFN_GEMV])
+@pytest.mark.parametrize("mode", [B.FFN_GEMV, B.FFN_GEMM])
 def test_ffn_tiny_matches_oracle(mode):
     cfg, seed, layer = _tiny()
     T = 8
@@ -231,7 +231,7 @@ def _layer_check(cfg, seed, layer, x, mode, ox=None):
     return out, xn_gpu, res
 
 
-@pytest.mark.parametrize("mode", [B.FFN_GEMV, B.FFN_AUTO])
+@pytest.mark.parametrize("mode", [B.FFN_GEMV, B.FFN_AUTO, B.FFN_GEMM])
 def test_layer_tiny_matches_oracle(mode):
     cfg, seed, layer = _tiny()
     x = inputs.activations(8, cfg.H, seed=seed, device=DEV)
@@ -273,3 +273,34 @@ def test_gemv_batch_invariance():
     for t in (0, 4, 8):
         one = B.layer_forward(layer, wr, bias, x[t:t + 1].contiguous(), cfg.k, mode=B.FFN_GEMV)
         assert torch.equal(one[0], full[t])
+
+
+@pytest.mark.parametrize("T", [1, 13, 40, 300])
+def test_gemm_path_matches_f16_staged_oracle(T):
+    """The tensor-core path against the oracle's fp16-staged arithmetic: the same
+    staged operands with exact accumulation, so only fp32 accumulation order
+    separates them (tight bound), for token counts from 1 to several M tiles."""
+    cfg, seed, layer = _tiny()
+    x = inputs.activations(T, cfg.H, seed=seed + 100 + T, device=DEV)
+    g = torch.Generator().manual_seed(T)
+    ids = torch.stack([torch.randperm(cfg.E, generator=g)[: cfg.k] for _ in range(T)]).to(torch.int32).to(DEV)
+    off, srt, pos, act = B.bucketize(ids, cfg.E)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y, ysh = B.expert_ffn(layer, x, cfg.k, off, srt, act, mode=B.FFN_GEMM, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ox = Hh.OracleExperts(cfg, seed, DEV)
+    xn = x.float().cpu().numpy()
+    idn = ids.cpu().numpy().reshape(-1)
+
+    def staged(e, rows):
+        (gq, gs), (dq, ds) = ox.packed(e)
+        b = ox.bits(e)
+        return oracle.expert_ffn_f16_staged(rows, oracle.dequantize_f16(gq, gs, b, cfg.H),
+                                            oracle.dequantize_f16(dq, ds, b, cfg.I))
+    exp = np.stack([staged(int(idn[s]), xn[s // cfg.k: s // cfg.k + 1])[0] for s in range(T * cfg.k)])
+    got = y.cpu().numpy()
+    scale = np.abs(exp).max()
+    assert np.max(np.abs(got - exp)) < 5e-4 * scale, np.max(np.abs(got - exp)) / scale
+    esh = staged(cfg.E, xn)
+    assert np.max(np.abs(ysh.cpu().numpy() - esh)) < 5e-4 * np.abs(esh).max()

@@ -403,3 +403,27 @@ def test_draft_batch_overlap():
         base = set(idx[0].tolist())
         overlaps += [len(base & set(idx[t].tolist())) / cfg.k for t in range(1, 5)]
     assert 0.45 < float(np.mean(overlaps)) < 0.75
+
+
+def test_round_f16_matches_library():
+    rng = np.random.default_rng(12)
+    v = np.concatenate([rng.standard_normal(4000) * 10.0 ** rng.integers(-9, 5, 4000),
+                        [0.0, 65504.0, 65520.0, 2.0 ** -24, 3 * 2.0 ** -26]]).astype(np.float32)
+    ref = v.astype(np.float16).astype(np.float64)  # numpy: RNE fp32 -> fp16
+    assert np.array_equal(oracle.round_f16(v.astype(np.float64)), ref)
+
+
+def test_f16_staged_ffn_equals_exact_when_staging_is_lossless():
+    """With integer weights (d = 1) and small integer activations every staged
+    value is exactly representable, so the staged FFN equals the fp64 one up to
+    the rounding of h, which is exact too when silu(g)*u is representable."""
+    rng = np.random.default_rng(13)
+    n, I = 64, 32
+    wgu = rng.integers(-3, 4, size=(2 * I, n)).astype(np.float64)
+    wdn = rng.integers(-3, 4, size=(n, I)).astype(np.float64)
+    x = rng.integers(-2, 3, size=(5, n)).astype(np.float64)
+    y_exact = oracle.expert_ffn(x, wgu, wdn)
+    y_staged = oracle.expert_ffn_f16_staged(x, wgu, wdn)
+    h = oracle.silu(x @ wgu[:I].T) * (x @ wgu[I:].T)
+    assert np.allclose(y_staged, oracle.round_f16(h) @ wdn.T, rtol=0, atol=0)
+    assert np.max(np.abs(y_staged - y_exact)) <= np.abs(h).max() * 2.0 ** -11 * np.abs(wdn).sum(axis=1).max()
