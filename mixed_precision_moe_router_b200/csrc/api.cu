@@ -165,7 +165,7 @@ size_t ffn_ctr_bytes(const moe_layer_weights *w, int T, int k) {
 // Token count from which an expert goes through the tensor-core GEMM in
 // MOE_FFN_AUTO mode (below it the streaming GEMV reads the weights once anyway
 // and wastes no tensor-core columns).
-constexpr int kGemmMinTokens = 24;
+constexpr int kGemmMinTokens = 8;
 
 bool uses_gemv(int mode) { return mode != MOE_FFN_GEMM; }
 bool uses_gemm(int mode, int T) { return mode == MOE_FFN_GEMM || (mode == MOE_FFN_AUTO && T >= kGemmMinTokens); }

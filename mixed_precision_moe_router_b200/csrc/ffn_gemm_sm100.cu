@@ -15,17 +15,18 @@
 // Operands are staged in fp16 (w = fp16_rne(d*q); x and h in fp16, whose range
 // is checked), accumulation is fp32 in tensor memory.
 //
-// Warp roles (352 threads, one CTA per SM, persistent over tiles):
-//   warps 0-3  dequant: each thread owns one tile row; its packed codes and
-//              scales stream through a 4-deep cp.async ring in shared memory,
-//              then are converted with packed half2 arithmetic and stored in
-//              the 128B-swizzled K-major layout the MMA reads.
-//   warps 4-7  epilogue: tcgen05.ld of their 32 accumulator lanes.
-//   warps 8-9  token rows: cp.async gather of fp16 rows (zero-filled past the
-//              expert's last token).
-//   warp  10   allocates 512 TMEM columns; lane 0 issues tcgen05.mma and
-//              tcgen05.commit.  Two accumulators let the epilogue of one tile
-//              overlap the MMAs of the next.
+// Warp roles (480 threads, one CTA per SM, persistent over tiles):
+//   warps 0-7  dequant: thread (warp w, lane l) owns tile row 32*(w%4)+l, which
+//              is the tensor-memory lane its warp may access, and half of each
+//              64-wide K chunk; its packed codes and scales stream through a
+//              4-deep cp.async ring in shared memory, are converted with packed
+//              half2 arithmetic and stored straight into tensor memory
+//              (tcgen05.st), where the MMA reads its A operand.
+//   warps 8-11 epilogue: tcgen05.ld of their 32 accumulator lanes.
+//   warps 12-13 token rows: cp.async gather of fp16 rows into 128B-swizzled
+//              K-major shared memory (zero-filled past the expert's last token).
+//   warp  14   allocates 512 TMEM columns (two 128-column accumulators, then the
+//              A stages); lane 0 issues tcgen05.mma and tcgen05.commit.
 #include "common.cuh"
 #include "ffn.cuh"
 #include "sync.cuh"
@@ -35,17 +36,19 @@ namespace gemm {
 
 constexpr int BM = 128;        // weight rows per tile (MMA M)
 constexpr int BK = 64;         // K elements per stage (128 bytes of fp16: one swizzle row)
-constexpr int MAXN = 256;      // tokens per accumulator (MMA N)
-constexpr int STAGES = 3;
+constexpr int MAXN = 128;      // tokens per accumulator (MMA N)
+constexpr int STAGES = 6;
 constexpr int RAW = 4;         // cp.async depth of the dequant producers
-constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = MAXN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int RAW_ROW = 80;    // per producer thread and raw stage: 64 code bytes + 4 scale bytes (+pad)
-constexpr int RAW_BYTES = BM * RAW_ROW;
-constexpr int WARPS = 11;
+constexpr int STAGE_BYTES = B_BYTES;           // shared memory holds the token tile only
+constexpr int ACC_COLS = 2 * MAXN;             // two fp32 accumulators
+constexpr int A_COLS = BK / 2;                 // one fp16 A stage in TMEM: 2 values per column
+constexpr int DQ_THREADS = 2 * BM;  // two dequant warps per TMEM lane quarter, 32 weights per thread
+constexpr int RAW_ROW = 48;         // per dequant thread and raw stage: 32 code bytes + 4 scale bytes (+pad)
+constexpr int RAW_BYTES = DQ_THREADS * RAW_ROW;
+constexpr int WARPS = 15;
 constexpr int THREADS = WARPS * 32;
-constexpr int EPI_WARP0 = 4, BPROD_WARP0 = 8, MMA_WARP = 10;
+constexpr int EPI_WARP0 = 8, BPROD_WARP0 = 12, MMA_WARP = 14;
 constexpr int BPROD_THREADS = 64;
 constexpr int TMEM_COLS = 512;
 
@@ -97,6 +100,29 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+
+// A from tensor memory (row m in lane m, two fp16 per column), B from shared memory
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Issue a 16-column store into tensor memory; completion is awaited later with
+// tmem_st_wait() so that it overlaps the next chunk's conversion.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -219,6 +245,60 @@ __device__ __forceinline__ void dequant3(const uint8_t *raw, uint32_t d2a, uint3
     }
 }
 
+// 32-weight variants (one quantisation block, one scale pair d2)
+__device__ __forceinline__ void dequant8_32(const uint8_t *raw, uint32_t d2, uint32_t (&o)[16]) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(raw);
+    const uint32_t bias = 0x64806480u;
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+        const uint4 w = q[v];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t u = ws[m] ^ 0x80808080u;
+            o[v * 8 + 2 * m] = hmul2_u(hsub2_u(__byte_perm(u, 0x64646464u, 0x4140), bias), d2);
+            o[v * 8 + 2 * m + 1] = hmul2_u(hsub2_u(__byte_perm(u, 0x64646464u, 0x4342), bias), d2);
+        }
+    }
+}
+
+__device__ __forceinline__ void dequant4_32(const uint8_t *raw, uint32_t d2, uint32_t (&o)[16]) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(raw);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t bias = 0x64086408u;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        uint32_t P[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) P[j] = hsub2_u(((ws[m] >> (4 * j)) & 0x000f000fu) | 0x64006400u, bias);
+        o[4 * m] = hmul2_u(__byte_perm(P[0], P[1], 0x5410), d2);
+        o[4 * m + 1] = hmul2_u(__byte_perm(P[2], P[3], 0x5410), d2);
+        o[4 * m + 2] = hmul2_u(__byte_perm(P[0], P[1], 0x7632), d2);
+        o[4 * m + 3] = hmul2_u(__byte_perm(P[2], P[3], 0x7632), d2);
+    }
+}
+
+__device__ __forceinline__ void dequant3_32(const uint8_t *raw, uint32_t d2, uint32_t (&o)[16]) {
+    const uint2 lo = *reinterpret_cast<const uint2 *>(raw);
+    const uint32_t hi = *reinterpret_cast<const uint32_t *>(raw + 8);
+    const uint32_t lw[2] = {lo.x, lo.y};
+    const uint32_t bias = 0x64046404u;
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        const uint32_t hw = hi >> (16 * p);
+        const uint32_t Y = ((hw & 0xffu) | ((hw & 0xff00u) << 8)) << 2;
+        uint32_t P[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            P[j] = hsub2_u(((lw[p] >> (2 * j)) & 0x00030003u) | ((Y >> j) & 0x00040004u) | 0x64006400u, bias);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            o[p * 8 + j] = hmul2_u(__byte_perm(P[2 * j], P[2 * j + 1], 0x5410), d2);
+            o[p * 8 + 4 + j] = hmul2_u(__byte_perm(P[2 * j], P[2 * j + 1], 0x7632), d2);
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // slots and tiles
 // ---------------------------------------------------------------------------
@@ -295,83 +375,104 @@ __device__ __forceinline__ void fail(const Params &P, const Shared &S) {
 // ---------------------------------------------------------------------------
 // roles
 // ---------------------------------------------------------------------------
-// Dequant producer: thread r streams row r of every tile's weight block.
-__device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, int total_tiles) {
-    const int r = threadIdx.x;  // 0..127
+// Dequant producer: threads 2r and 2r+1 stream the two 32-weight halves of
+// row r of every tile's 64-wide K chunk.
+__device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, int total_tiles, uint32_t tmem) {
+    const int tid = threadIdx.x;  // 0..255
+    const int warp = tid >> 5, lane = tid & 31;
+    const int r = 32 * (warp & 3) + lane;  // tile row = TMEM lane this warp may access
+    const int half = warp >> 2;            // which 32 of the chunk's 64 weights
     const int nmt = n_mtiles(P), NK = n_kchunks(P);
     const int K = P.phase == 0 ? P.f.w.H : P.f.w.I;
     const int G = gridDim.x;
     const int my_tiles = total_tiles > static_cast<int>(blockIdx.x)
                              ? (total_tiles - static_cast<int>(blockIdx.x) + G - 1) / G : 0;
     const int nchunks = my_tiles * NK;
-    uint8_t *raw_me = S.raw + r * RAW_ROW;
+    uint8_t *raw_me = S.raw + tid * RAW_ROW;
     const uint32_t raw_me_s = smem_u32(raw_me);
 
-    // source of linear chunk L of this thread: (row pointer, scale pointer, kc, bits)
-    auto chunk_src = [&](int L, int &bits, const uint8_t *&qrow, const uint16_t *&srow, int &kc) {
-        const int t = blockIdx.x + (L / NK) * G;
-        kc = L % NK;
-        const Tile tl = tile_of(S.slots, nmt, t);
-        const int e = S.slots.expert[tl.slot];
+    // Row source of this thread for the tile holding linear chunk L; recomputed
+    // only when a cursor crosses into the next tile.
+    struct RowCtx {
+        int tile_local = -1, bits = 8;
+        const uint8_t *qrow = nullptr;
+        const uint16_t *srow = nullptr;
+    };
+    auto locate = [&](RowCtx &c, int L) {
+        const int tl_local = L / NK;
+        if (tl_local == c.tile_local) return;
+        c.tile_local = tl_local;
+        const Tile tl = tile_of(S.slots, nmt, blockIdx.x + tl_local * G);
         const uint8_t *qs;
         const uint16_t *sc;
-        expert_rows(P, e, bits, qs, sc);
-        int row;
-        if (P.phase == 0) row = ((r & 1) ? P.f.w.I : 0) + tl.mt * (BM / 2) + (r >> 1);
-        else row = tl.mt * BM + r;
-        qrow = qs + static_cast<size_t>(row) * (K * bits / 8);
-        srow = sc + static_cast<size_t>(row) * (K / 32);
+        expert_rows(P, S.slots.expert[tl.slot], c.bits, qs, sc);
+        const int row = P.phase == 0 ? ((r & 1) ? P.f.w.I : 0) + tl.mt * (BM / 2) + (r >> 1) : tl.mt * BM + r;
+        c.qrow = qs + static_cast<size_t>(row) * (K * c.bits / 8);
+        c.srow = sc + static_cast<size_t>(row) * (K / 32);
     };
+    RowCtx ci, cp;  // issue-ahead and processing cursors
     auto issue = [&](int L) {
         if (L < nchunks) {
-            int bits, kc;
-            const uint8_t *qrow;
-            const uint16_t *srow;
-            chunk_src(L, bits, qrow, srow, kc);
+            locate(ci, L);
+            const int kc = L % NK;
+            const uint8_t *qrow = ci.qrow;
             const uint32_t dst = raw_me_s + (L % RAW) * RAW_BYTES;
-            if (bits == 8) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) cp_async16(dst + 16 * c, qrow + kc * 64 + 16 * c, 16);
-            } else if (bits == 4) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c) cp_async16(dst + 16 * c, qrow + kc * 32 + 16 * c, 16);
+            const int blk = 2 * kc + half;  // 32-weight block index within the row
+            if (ci.bits == 8) {
+                cp_async16(dst, qrow + 32 * blk, 16);
+                cp_async16(dst + 16, qrow + 32 * blk + 16, 16);
+            } else if (ci.bits == 4) {
+                cp_async16(dst, qrow + 16 * blk, 16);
             } else {
-                cp_async16(dst, qrow + kc * 16, 16);
-                cp_async8(dst + 16, qrow + K / 4 + kc * 8);
+                cp_async8(dst, qrow + 8 * blk);
+                cp_async4(dst + 8, qrow + K / 4 + 4 * blk);
             }
-            cp_async4(dst + 64, srow + 2 * kc);
+            cp_async4(dst + 32, ci.srow + 2 * kc);  // both scales of the 64-wide chunk
         }
         cp_async_commit();
     };
 #pragma unroll 1
     for (int L = 0; L < RAW - 1; ++L) issue(L);
+    int pend = -1;  // stage whose TMEM store is in flight and not yet signalled
 #pragma unroll 1
     for (int L = 0; L < nchunks; ++L) {
         issue(L + RAW - 1);
         cp_async_wait<RAW - 1>();
-        if (aborted(S)) break;
-        int bits, kc;
-        const uint8_t *qrow;
-        const uint16_t *srow;
-        chunk_src(L, bits, qrow, srow, kc);
+        if (__any_sync(0xffffffffu, aborted(S))) break;  // warp-uniform exit (tcgen05.st is warp-wide)
+        locate(cp, L);
+        const int bits = cp.bits;
         const uint8_t *raw = raw_me + (L % RAW) * RAW_BYTES;
-        const uint32_t sc2 = *reinterpret_cast<const uint32_t *>(raw + 64);
-        const uint32_t d2a = (sc2 & 0xffffu) | (sc2 << 16);   // (d0, d0)
-        const uint32_t d2b = (sc2 >> 16) | (sc2 & 0xffff0000u);  // (d1, d1)
-        uint32_t o[32];
-        if (bits == 8) dequant8(raw, d2a, d2b, o);
-        else if (bits == 4) dequant4(raw, d2a, d2b, o);
-        else dequant3(raw, d2a, d2b, o);
+        const uint32_t sc2 = *reinterpret_cast<const uint32_t *>(raw + 32);
+        const uint32_t d = half ? (sc2 >> 16) : (sc2 & 0xffffu);
+        const uint32_t d2 = d | (d << 16);
+        uint32_t o[16];
+        if (bits == 8) dequant8_32(raw, d2, o);
+        else if (bits == 4) dequant4_32(raw, d2, o);
+        else dequant3_32(raw, d2, o);
+        if (pend >= 0) {  // the previous chunk's store has had a whole conversion to land
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&S.full_a[pend]);
+            pend = -1;
+        }
         const int s = L % STAGES;
-        if (!mbar_wait(&S.empty[s], ((L / STAGES) & 1) ^ 1)) { fail(P, S); break; }
-        uint8_t *A = S.stages + s * STAGE_BYTES;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4 *>(A + sw128(r, c)) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        fence_proxy_async();
-        mbar_arrive(&S.full_a[s]);
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&S.empty[s], ((L / STAGES) & 1) ^ 1));
+        if (!ok) { fail(P, S); break; }
+        tc_fence_after();
+        // lanes 32*(warp%4).. of the stage's A columns; this thread's row and half
+        tmem_st16(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + ACC_COLS + s * A_COLS + 16 * half, o);
+        pend = s;
+    }
+    if (pend >= 0) {
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&S.full_a[pend]);
     }
     cp_async_wait<0>();
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Token-row producer: 64 threads gather the fp16 rows of the tile's tokens.
@@ -382,7 +483,6 @@ __device__ __forceinline__ void role_tokens(const Params &P, const Shared &S, in
     const int G = gridDim.x;
     const int S_ = P.f.T * P.f.k;
     int q = 0;  // linear chunk counter
-    int pending = -1;
 #pragma unroll 1
     for (int t = blockIdx.x; t < total_tiles; t += G) {
         const Tile tl = tile_of(S.slots, nmt, t);
@@ -410,7 +510,7 @@ __device__ __forceinline__ void role_tokens(const Params &P, const Shared &S, in
         for (int kc = 0; kc < NK; ++kc, ++q) {
             const int s = q % STAGES;
             if (!mbar_wait(&S.empty[s], ((q / STAGES) & 1) ^ 1)) { fail(P, S); break; }
-            const uint32_t B = smem_u32(S.stages + s * STAGE_BYTES + A_BYTES);
+            const uint32_t B = smem_u32(S.stages + s * STAGE_BYTES);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int j = b + 64 * m;
@@ -421,21 +521,12 @@ __device__ __forceinline__ void role_tokens(const Params &P, const Shared &S, in
                     for (int c = 0; c < 8; ++c) cp_async16(B + sw128(j, c), row + 8 * c, n);
                 }
             }
-            cp_async_commit();
-            if (pending >= 0) {
-                cp_async_wait<1>();
-                fence_proxy_async();
-                mbar_arrive(&S.full_b[pending]);
-            }
-            pending = s;
+            // the stage's arrival fires when this thread's copies have landed
+            cp_async_arrive_noinc(&S.full_b[s]);
         }
         if (aborted(S)) break;
     }
     cp_async_wait<0>();
-    if (pending >= 0) {
-        fence_proxy_async();
-        mbar_arrive(&S.full_b[pending]);
-    }
 }
 
 // MMA issuer (one thread).
@@ -460,11 +551,11 @@ __device__ __forceinline__ void role_mma(const Params &P, const Shared &S, int t
             const uint32_t par = (q / STAGES) & 1;
             if (!mbar_wait(&S.full_a[s], par) || !mbar_wait(&S.full_b[s], par)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t A = smem_u32(S.stages + s * STAGE_BYTES);
-            const uint64_t ad = smem_desc_sw128(A), bd = smem_desc_sw128(A + A_BYTES);
+            const uint64_t bd = smem_desc_sw128(smem_u32(S.stages + s * STAGE_BYTES));
+            const uint32_t a = tmem + ACC_COLS + s * A_COLS;
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k)  // 16 fp16 = 32 bytes per MMA step along K
-                mma_f16(d, ad + 2 * k, bd + 2 * k, idesc, (kc | k) != 0);
+            for (int k = 0; k < BK / 16; ++k)  // K step of 16: 8 TMEM columns of A, 32 bytes of B
+                mma_f16_ts(d, a + 8 * k, bd + 2 * k, idesc, (kc | k) != 0);
             mma_commit(&S.empty[s]);
         }
         if (!ok) { fail(P, S); break; }
@@ -504,7 +595,7 @@ __device__ __forceinline__ void role_epilogue(const Params &P, const Shared &S, 
                     const float g = __uint_as_float(v[j]);
                     const float u = __shfl_down_sync(0xffffffffu, g, 1);
                     if (!(lane & 1) && c0 + j < nvalid) {
-                        const float hv = g / (1.0f + expf(-g)) * u;
+                        const float hv = __fdividef(g, 1.0f + __expf(-g)) * u;
                         range_bad |= !(fabsf(hv) <= 65504.0f);
                         const int ent = first + tl.nc * MAXN + c0 + j;
                         P.h16[static_cast<size_t>(ent) * I + i] = __half_as_ushort(__float2half_rn(hv));
@@ -599,7 +690,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_gemm_kernel(const Params P) {
             }
             S.slots.tile0[n] = acc;
             for (int s = 0; s < STAGES; ++s) {
-                mbar_init(&S.full_a[s], BM);
+                mbar_init(&S.full_a[s], DQ_THREADS);
                 mbar_init(&S.full_b[s], BPROD_THREADS);
                 mbar_init(&S.empty[s], 1);
             }
@@ -627,7 +718,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_gemm_kernel(const Params P) {
     const uint32_t tmem = *S.tmem_slot;
     const int total_tiles = S.slots.tile0[S.slots.n];
 
-    if (warp < 4) role_dequant(P, S, total_tiles);
+    if (warp < EPI_WARP0) role_dequant(P, S, total_tiles, tmem);
     else if (warp < BPROD_WARP0) role_epilogue(P, S, total_tiles, tmem);
     else if (warp < MMA_WARP) role_tokens(P, S, total_tiles);
     else if (threadIdx.x == MMA_WARP * 32) role_mma(P, S, total_tiles, tmem);
@@ -678,9 +769,11 @@ size_t moe_ffn_gemm_workspace(const moe_layer_weights *w, int T, int k) {
     return x16 + h16;
 }
 
+constexpr size_t kMaxDynSmem = 232448 - 1024;  // 227 KB opt-in limit per CTA on sm_100, less static smem
+
 cudaError_t moe_configure_ffn_gemm() {
     return cudaFuncSetAttribute(moe::gemm::ffn_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(gemm_smem_bytes(MOE_MAX_EXPERTS + 1)));
+                                static_cast<int>(kMaxDynSmem));
 }
 
 bool moe_ffn_gemm_supported(int H, int I) {
@@ -705,6 +798,7 @@ cudaError_t moe_launch_ffn_gemm(const moe::FfnParams &f, void *ws, size_t, cudaS
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = gemm_smem_bytes(f.max_active + 1);
+    if (smem > kMaxDynSmem) return cudaErrorInvalidConfiguration;  // too many experts for the slot tables
     for (int phase = 0; phase < 2; ++phase) {
         P.phase = phase;
         moe::gemm::ffn_gemm_kernel<<<sms, moe::gemm::THREADS, smem, s>>>(P);
