@@ -17,6 +17,9 @@ cudaError_t moe_configure_router();
 cudaError_t moe_launch_router_logits(const uint16_t *, const uint16_t *, const float *, int, int, int, float *,
                                      cudaStream_t);
 cudaError_t moe_launch_topk(const float *, int, int, int, int32_t *, float *, cudaStream_t);
+bool moe_router_gemm_supported(int T, int H, int E);
+cudaError_t moe_launch_router_gemm(const uint16_t *, const uint16_t *, const float *, int, int, int, float *,
+                                   cudaStream_t);
 cudaError_t moe_configure_bucketize();
 cudaError_t moe_launch_bucketize(const int32_t *, int, int, int32_t *, int32_t *, int32_t *, int32_t *, int32_t *,
                                  cudaStream_t);
@@ -248,7 +251,9 @@ int moe_router_topk(const uint16_t *x, const uint16_t *w_router, const float *bi
     r = ensure_configured();
     if (r) return r;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = moe_launch_router_logits(x, w_router, bias, T, H, E, lg, s);
+    // prefill-sized batches: the logits are a dense bf16 GEMM on the tensor cores
+    cudaError_t e = moe_router_gemm_supported(T, H, E) ? moe_launch_router_gemm(x, w_router, bias, T, H, E, lg, s)
+                                                       : moe_launch_router_logits(x, w_router, bias, T, H, E, lg, s);
     if (e == cudaSuccess) e = moe_launch_topk(lg, T, E, k, topk_idx, topk_w, s);
     return e == cudaSuccess ? ok() : cuda_fail(e, "router launch");
 }

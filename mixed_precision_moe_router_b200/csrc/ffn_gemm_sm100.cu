@@ -35,16 +35,17 @@ namespace moe {
 namespace gemm {
 
 constexpr int BM = 128;        // weight rows per tile (MMA M)
-constexpr int BK = 64;         // K elements per stage (128 bytes of fp16: one swizzle row)
+constexpr int BK = 128;        // K elements per stage (two 128-byte swizzle atoms of fp16 per token row)
 constexpr int MAXN = 128;      // tokens per accumulator (MMA N)
-constexpr int STAGES = 6;
+constexpr int STAGES = 4;
 constexpr int RAW = 4;         // cp.async depth of the dequant producers
-constexpr int B_BYTES = MAXN * BK * 2;
+constexpr int B_HALF = MAXN * 128;             // one 64-wide K half of the token tile (128 B rows)
+constexpr int B_BYTES = 2 * B_HALF;
 constexpr int STAGE_BYTES = B_BYTES;           // shared memory holds the token tile only
 constexpr int ACC_COLS = 2 * MAXN;             // two fp32 accumulators
 constexpr int A_COLS = BK / 2;                 // one fp16 A stage in TMEM: 2 values per column
-constexpr int DQ_THREADS = 2 * BM;  // two dequant warps per TMEM lane quarter, 32 weights per thread
-constexpr int RAW_ROW = 48;         // per dequant thread and raw stage: 32 code bytes + 4 scale bytes (+pad)
+constexpr int DQ_THREADS = 2 * BM;  // two dequant warps per TMEM lane quarter, 64 weights per thread
+constexpr int RAW_ROW = 80;         // per dequant thread and raw stage: 64 code bytes + 4 scale bytes (+pad)
 constexpr int RAW_BYTES = DQ_THREADS * RAW_ROW;
 constexpr int WARPS = 15;
 constexpr int THREADS = WARPS * 32;
@@ -54,7 +55,11 @@ constexpr int TMEM_COLS = 512;
 
 struct Params {
     FfnParams f;
-    int phase;              // 0: gate_up, 1: down
+    int phase;              // 0: gate_up, 1: down, 2: router logits
+    // router mode: logits[t][e] = x[t] . w_router[e] + bias[e], bf16 operands
+    const uint16_t *wr;     // bf16 [E][H]
+    const float *bias;      // [E] or null
+    float *logits;          // fp32 [T][E]
     const uint16_t *x16;    // fp16 [T][H]
     uint16_t *h16;          // fp16 [T*k + T][I], expert-grouped rows
     int min_count;          // experts with fewer tokens are left to the GEMV path
@@ -122,6 +127,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
         "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -154,8 +170,9 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 
 // Instruction descriptor: kind::f16, A = B = fp16, D = fp32, both K-major,
 // M = 128, N = n.
-__device__ __forceinline__ uint32_t idesc_f16(int n) {
-    return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+__device__ __forceinline__ uint32_t idesc_f16(int n, bool bf16 = false) {
+    const uint32_t ab = bf16 ? ((1u << 7) | (1u << 10)) : 0u;  // A and B format: 0 = fp16, 1 = bf16
+    return (1u << 4) | ab | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
 }
 
 // byte offset of 16-byte chunk c of row r in a 128B-swizzled K-major tile
@@ -308,10 +325,10 @@ struct Slots {
 };
 
 __device__ __forceinline__ int n_mtiles(const Params &P) {
-    return P.phase == 0 ? (2 * P.f.w.I) / BM : P.f.w.H / BM;
+    return P.phase == 0 ? (2 * P.f.w.I) / BM : (P.phase == 1 ? P.f.w.H / BM : P.f.E / BM);
 }
 __device__ __forceinline__ int n_kchunks(const Params &P) {
-    return (P.phase == 0 ? P.f.w.H : P.f.w.I) / BK;
+    return (P.phase == 1 ? P.f.w.I : P.f.w.H) / BK;
 }
 
 struct Tile {
@@ -410,6 +427,40 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
         c.qrow = qs + static_cast<size_t>(row) * (K * c.bits / 8);
         c.srow = sc + static_cast<size_t>(row) * (K / 32);
     };
+    if (P.phase == 2) {  // router: bf16 weight rows go to tensor memory unchanged
+        int pend = -1;
+#pragma unroll 1
+        for (int L = 0; L < nchunks; ++L) {
+            const Tile tl = tile_of(S.slots, nmt, blockIdx.x + (L / NK) * G);
+            const int kc = L % NK;
+            const uint16_t *src = P.wr + static_cast<size_t>(tl.mt * BM + r) * P.f.w.H + kc * BK + 64 * half;
+            uint32_t o[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(src + 8 * c);
+                o[4 * c] = q.x; o[4 * c + 1] = q.y; o[4 * c + 2] = q.z; o[4 * c + 3] = q.w;
+            }
+            if (pend >= 0) {
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.full_a[pend]);
+                pend = -1;
+            }
+            const int s = L % STAGES;
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.empty[s], ((L / STAGES) & 1) ^ 1))) { fail(P, S); break; }
+            tc_fence_after();
+            tmem_st32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + ACC_COLS + s * A_COLS + 32 * half, o);
+            pend = s;
+        }
+        if (pend >= 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.full_a[pend]);
+        }
+        return;
+    }
     RowCtx ci, cp;  // issue-ahead and processing cursors
     auto issue = [&](int L) {
         if (L < nchunks) {
@@ -417,17 +468,18 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
             const int kc = L % NK;
             const uint8_t *qrow = ci.qrow;
             const uint32_t dst = raw_me_s + (L % RAW) * RAW_BYTES;
-            const int blk = 2 * kc + half;  // 32-weight block index within the row
+            const int blk = 4 * kc + 2 * half;  // first of this thread's two 32-weight blocks
             if (ci.bits == 8) {
-                cp_async16(dst, qrow + 32 * blk, 16);
-                cp_async16(dst + 16, qrow + 32 * blk + 16, 16);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) cp_async16(dst + 16 * c, qrow + 32 * blk + 16 * c, 16);
             } else if (ci.bits == 4) {
                 cp_async16(dst, qrow + 16 * blk, 16);
+                cp_async16(dst + 16, qrow + 16 * blk + 16, 16);
             } else {
-                cp_async8(dst, qrow + 8 * blk);
-                cp_async4(dst + 8, qrow + K / 4 + 4 * blk);
+                cp_async16(dst, qrow + 8 * blk, 16);
+                cp_async8(dst + 16, qrow + K / 4 + 4 * blk);
             }
-            cp_async4(dst + 32, ci.srow + 2 * kc);  // both scales of the 64-wide chunk
+            cp_async4(dst + 64, ci.srow + blk);  // the scales of its two blocks
         }
         cp_async_commit();
     };
@@ -442,17 +494,33 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
         locate(cp, L);
         const int bits = cp.bits;
         const uint8_t *raw = raw_me + (L % RAW) * RAW_BYTES;
-        const uint32_t sc2 = *reinterpret_cast<const uint32_t *>(raw + 32);
-        const uint32_t d = half ? (sc2 >> 16) : (sc2 & 0xffffu);
-        const uint32_t d2 = d | (d << 16);
-        uint32_t o[16];
-        if (bits == 8) dequant8_32(raw, d2, o);
-        else if (bits == 4) dequant4_32(raw, d2, o);
-        else dequant3_32(raw, d2, o);
+        const uint32_t sc2 = *reinterpret_cast<const uint32_t *>(raw + 64);
+        const uint32_t d2a = (sc2 & 0xffffu) | (sc2 << 16);       // (d0, d0)
+        const uint32_t d2b = (sc2 >> 16) | (sc2 & 0xffff0000u);   // (d1, d1)
+        uint32_t o[32];
+        uint32_t(&o0)[16] = *reinterpret_cast<uint32_t(*)[16]>(o);
+        uint32_t(&o1)[16] = *reinterpret_cast<uint32_t(*)[16]>(o + 16);
+        if (bits == 8) {
+            dequant8_32(raw, d2a, o0);
+            dequant8_32(raw + 32, d2b, o1);
+        } else if (bits == 4) {
+            dequant4_32(raw, d2a, o0);
+            dequant4_32(raw + 16, d2b, o1);
+        } else {
+            // lo plane: 8 bytes per block; hi plane: 4 bytes per block
+            uint8_t tmp[16];
+            *reinterpret_cast<uint2 *>(tmp) = *reinterpret_cast<const uint2 *>(raw);
+            *reinterpret_cast<uint32_t *>(tmp + 8) = *reinterpret_cast<const uint32_t *>(raw + 16);
+            dequant3_32(tmp, d2a, o0);
+            *reinterpret_cast<uint2 *>(tmp) = *reinterpret_cast<const uint2 *>(raw + 8);
+            *reinterpret_cast<uint32_t *>(tmp + 8) = *reinterpret_cast<const uint32_t *>(raw + 20);
+            dequant3_32(tmp, d2b, o1);
+        }
         if (pend >= 0) {  // the previous chunk's store has had a whole conversion to land
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&S.full_a[pend]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.full_a[pend]);  // one arrival per warp
             pend = -1;
         }
         const int s = L % STAGES;
@@ -460,13 +528,14 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
         if (!ok) { fail(P, S); break; }
         tc_fence_after();
         // lanes 32*(warp%4).. of the stage's A columns; this thread's row and half
-        tmem_st16(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + ACC_COLS + s * A_COLS + 16 * half, o);
+        tmem_st32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + ACC_COLS + s * A_COLS + 32 * half, o);
         pend = s;
     }
     if (pend >= 0) {
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&S.full_a[pend]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.full_a[pend]);
     }
     cp_async_wait<0>();
 }
@@ -479,7 +548,7 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
 __device__ __forceinline__ void role_tokens(const Params &P, const Shared &S, int total_tiles) {
     const int b = threadIdx.x - BPROD_WARP0 * 32;  // 0..63
     const int nmt = n_mtiles(P), NK = n_kchunks(P);
-    const int K = P.phase == 0 ? P.f.w.H : P.f.w.I;
+    const int K = P.phase == 1 ? P.f.w.I : P.f.w.H;
     const int G = gridDim.x;
     const int S_ = P.f.T * P.f.k;
     int q = 0;  // linear chunk counter
@@ -498,7 +567,9 @@ __device__ __forceinline__ void role_tokens(const Params &P, const Shared &S, in
             src[m] = nullptr;
             if (j < nvalid) {
                 const int ent = first + tl.nc * MAXN + j;
-                if (P.phase == 0) {
+                if (P.phase == 2) {
+                    src[m] = P.f.x + static_cast<size_t>(ent) * K;  // token rows in order, bf16
+                } else if (P.phase == 0) {
                     const int tok = ent >= S_ ? ent - S_ : P.f.sorted[ent] / P.f.k;
                     src[m] = P.x16 + static_cast<size_t>(tok) * K;
                 } else {
@@ -518,7 +589,9 @@ __device__ __forceinline__ void role_tokens(const Params &P, const Shared &S, in
                     const uint16_t *row = src[m] ? src[m] + kc * BK : P.x16;
                     const int n = src[m] ? 16 : 0;  // zero-fill rows past the last token
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) cp_async16(B + sw128(j, c), row + 8 * c, n);
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) cp_async16(B + h * B_HALF + sw128(j, c), row + 64 * h + 8 * c, n);
                 }
             }
             // the stage's arrival fires when this thread's copies have landed
@@ -539,7 +612,7 @@ __device__ __forceinline__ void role_mma(const Params &P, const Shared &S, int t
         const Tile tl = tile_of(S.slots, nmt, t);
         const int nvalid = min(MAXN, S.slots.count[tl.slot] - tl.nc * MAXN);
         const int Nt = (nvalid + 15) & ~15;
-        const uint32_t idesc = idesc_f16(Nt);
+        const uint32_t idesc = idesc_f16(Nt, P.phase == 2);
         const int buf = acc & 1;
         if (!mbar_wait(&S.acc_empty[buf], ((acc >> 1) & 1) ^ 1)) { fail(P, S); break; }
         tc_fence_after();
@@ -551,11 +624,13 @@ __device__ __forceinline__ void role_mma(const Params &P, const Shared &S, int t
             const uint32_t par = (q / STAGES) & 1;
             if (!mbar_wait(&S.full_a[s], par) || !mbar_wait(&S.full_b[s], par)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t bd = smem_desc_sw128(smem_u32(S.stages + s * STAGE_BYTES));
+            const uint32_t b0 = smem_u32(S.stages + s * STAGE_BYTES);
             const uint32_t a = tmem + ACC_COLS + s * A_COLS;
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k)  // K step of 16: 8 TMEM columns of A, 32 bytes of B
-                mma_f16_ts(d, a + 8 * k, bd + 2 * k, idesc, (kc | k) != 0);
+            for (int k = 0; k < BK / 16; ++k) {  // K step of 16: 8 TMEM columns of A, 32 bytes of a B half
+                const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * B_HALF) + 2 * (k & 3);
+                mma_f16_ts(d, a + 8 * k, bd, idesc, (kc | k) != 0);
+            }
             mma_commit(&S.empty[s]);
         }
         if (!ok) { fail(P, S); break; }
@@ -581,41 +656,59 @@ __device__ __forceinline__ void role_epilogue(const Params &P, const Shared &S, 
         const int first = S.slots.first[tl.slot];
         const int nvalid = min(MAXN, S.slots.count[tl.slot] - tl.nc * MAXN);
         const int buf = acc & 1;
-        if (!mbar_wait(&S.acc_full[buf], (acc >> 1) & 1)) { fail(P, S); break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&S.acc_full[buf], (acc >> 1) & 1))) { fail(P, S); break; }
         tc_fence_after();
         const int row = 32 * q + lane;  // accumulator lane = tile row
 #pragma unroll 1
         for (int c0 = 0; c0 < nvalid; c0 += 32) {
             uint32_t v[32];
             tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + buf * MAXN + c0, v);
-            if (P.phase == 0) {
-                const int i = tl.mt * (BM / 2) + (row >> 1);  // pair index
+            if (P.phase == 2) {
+                const int e = tl.mt * BM + row;
+                const float b = P.bias ? P.bias[e] : 0.f;
+                float *lg = P.logits + static_cast<size_t>(tl.nc * MAXN + c0) * P.f.E + e;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float g = __uint_as_float(v[j]);
-                    const float u = __shfl_down_sync(0xffffffffu, g, 1);
-                    if (!(lane & 1) && c0 + j < nvalid) {
+                for (int j = 0; j < 32; ++j)
+                    if (c0 + j < nvalid) lg[static_cast<size_t>(j) * P.f.E] = __uint_as_float(v[j]) + b;
+            } else if (P.phase == 0) {
+                // lanes 2p and 2p+1 hold gate and up of pair p; each lane finishes
+                // every other column so both lanes of a pair do the SwiGLU work
+                const int i = tl.mt * (BM / 2) + (row >> 1);  // pair index
+                const bool odd = lane & 1;
+                uint16_t *hbase = P.h16 + static_cast<size_t>(first + tl.nc * MAXN + c0) * I + i;
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const float a0 = __uint_as_float(v[j]), a1 = __uint_as_float(v[j + 1]);
+                    const float recv = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+                    const float g = odd ? recv : a0;  // even: g_j      odd: g_{j+1}
+                    const float u = odd ? a1 : recv;  // even: u_j      odd: u_{j+1}
+                    const int col = j + (odd ? 1 : 0);
+                    if (c0 + col < nvalid) {
                         const float hv = __fdividef(g, 1.0f + __expf(-g)) * u;
                         range_bad |= !(fabsf(hv) <= 65504.0f);
-                        const int ent = first + tl.nc * MAXN + c0 + j;
-                        P.h16[static_cast<size_t>(ent) * I + i] = __half_as_ushort(__float2half_rn(hv));
+                        hbase[static_cast<size_t>(col) * I] = __half_as_ushort(__float2half_rn(hv));
                     }
                 }
             } else {
                 const int n = tl.mt * BM + row;
+                // one coalesced load of the 32 destination rows, then broadcast per column
+                const int my_ent = first + tl.nc * MAXN + c0 + lane;
+                int my_row = -1;
+                if (c0 + lane < nvalid) my_row = my_ent >= S_ ? -(my_ent - S_) - 2 : P.f.sorted[my_ent];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    if (c0 + j < nvalid) {
-                        const int ent = first + tl.nc * MAXN + c0 + j;
-                        float *dst = ent >= S_ ? P.f.y_shared + static_cast<size_t>(ent - S_) * H
-                                               : P.f.y_slots + static_cast<size_t>(P.f.sorted[ent]) * H;
+                    const int dr = __shfl_sync(0xffffffffu, my_row, j);
+                    if (dr != -1) {
+                        float *dst = dr <= -2 ? P.f.y_shared + static_cast<size_t>(-dr - 2) * H
+                                              : P.f.y_slots + static_cast<size_t>(dr) * H;
                         dst[n] = __uint_as_float(v[j]);
                     }
                 }
             }
         }
         tc_fence_before();
-        mbar_arrive(&S.acc_empty[buf]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);  // one arrival per epilogue warp
     }
     if (range_bad) status_or(P.f.status, MOE_STATUS_FP16_RANGE);
 }
@@ -650,7 +743,17 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_gemm_kernel(const Params P) {
 
     const int warp = threadIdx.x >> 5;
     // slot table: routed experts with at least min_count tokens, then the shared expert
-    if (warp == 0) {
+    // (router mode: one slot holding every token)
+    if (warp == 0 && P.phase == 2) {
+        if (threadIdx.x == 0) {
+            S.slots.expert[0] = -1;
+            S.slots.count[0] = P.f.T;
+            S.slots.first[0] = 0;
+            S.slots.n = 1;
+            S.slots.tile0[0] = 0;
+            S.slots.tile0[1] = ((P.f.T + MAXN - 1) / MAXN) * n_mtiles(P);
+        }
+    } else if (warp == 0) {
         const int n_active = min(P.f.active[0], P.f.max_active);
         int n = 0;
         for (int a0 = 0; a0 < n_active; a0 += 32) {
@@ -689,19 +792,21 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_gemm_kernel(const Params P) {
                 acc += ((S.slots.count[a] + MAXN - 1) / MAXN) * nmt;
             }
             S.slots.tile0[n] = acc;
-            for (int s = 0; s < STAGES; ++s) {
-                mbar_init(&S.full_a[s], DQ_THREADS);
-                mbar_init(&S.full_b[s], BPROD_THREADS);
-                mbar_init(&S.empty[s], 1);
-            }
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(&S.acc_full[b], 1);
-                mbar_init(&S.acc_empty[b], 4 * 32);
-            }
-            mbar_init(S.fin, 1);
-            *S.abort = 0;
-            mbar_fence_init();
         }
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&S.full_a[s], DQ_THREADS / 32);  // one arrival per dequant warp
+            mbar_init(&S.full_b[s], BPROD_THREADS);
+            mbar_init(&S.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.acc_full[b], 1);
+            mbar_init(&S.acc_empty[b], 4);
+        }
+        mbar_init(S.fin, 1);
+        *S.abort = 0;
+        mbar_fence_init();
     }
     if (warp == MMA_WARP) {
         tmem_alloc(S.tmem_slot, TMEM_COLS);
@@ -779,6 +884,35 @@ cudaError_t moe_configure_ffn_gemm() {
 bool moe_ffn_gemm_supported(int H, int I) {
     return H % moe::gemm::BM == 0 && I % (moe::gemm::BM / 2) == 0 && H % moe::gemm::BK == 0 &&
            I % moe::gemm::BK == 0;
+}
+
+bool moe_router_gemm_supported(int T, int H, int E) {
+    return T >= 64 && E % moe::gemm::BM == 0 && H % moe::gemm::BK == 0;
+}
+
+// Router logits on the tensor cores: logits[t][e] = x[t] . w_router[e] + bias[e].
+cudaError_t moe_launch_router_gemm(const uint16_t *x, const uint16_t *wr, const float *bias, int T, int H, int E,
+                                   float *logits, cudaStream_t s) {
+    moe::gemm::Params P{};
+    P.f.w.H = H;
+    P.f.w.I = 128;
+    P.f.E = E;
+    P.f.T = T;
+    P.f.k = 1;
+    P.f.max_active = 1;
+    P.f.x = x;
+    P.phase = 2;
+    P.wr = wr;
+    P.bias = bias;
+    P.logits = logits;
+    P.min_count = 1;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tiles = ((T + moe::gemm::MAXN - 1) / moe::gemm::MAXN) * (E / moe::gemm::BM);
+    const int grid = tiles < sms ? tiles : sms;
+    moe::gemm::ffn_gemm_kernel<<<grid, moe::gemm::THREADS, gemm_smem_bytes(2), s>>>(P);
+    return cudaGetLastError();
 }
 
 // Runs the experts with at least `min_count` tokens (and the shared expert when

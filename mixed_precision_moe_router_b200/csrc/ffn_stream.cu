@@ -510,19 +510,48 @@ ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
     const bool ent_smem = n_ent <= kMaxSmemEntries;
     S.st.tok = ent_smem ? tabs + 4 * max_slots : nullptr;
     S.st.row = ent_smem ? S.st.tok + n_ent : nullptr;
-    // slot table: active routed experts, then the shared expert
-    const int n_active = min(p.active[0], p.max_active);
-    for (int a = threadIdx.x; a < n_active; a += blockDim.x) {
-        int e = p.active[1 + a];
-        const bool bad = e < 0 || e >= p.E;
-        if (bad) e = 0;
-        const int f = p.offsets[e];
-        const int cnt = bad ? 0 : p.offsets[e + 1] - f;
-        S.st.expert[a] = e;
-        S.st.bits[a] = expert_bits(p, e);
-        S.st.first[a] = f;
-        S.st.count[a] = cnt > p.max_count ? 0 : cnt;  // larger groups go to the tensor-core path
+    // slot table: active routed experts with work for this path (compacted),
+    // then the shared expert
+    __shared__ int n_keep;
+    if (threadIdx.x == 0) n_keep = 0;
+    __syncthreads();
+    const int n_active_all = min(p.active[0], p.max_active);
+    for (int a0 = 0; a0 < n_active_all; a0 += blockDim.x) {
+        const int a = a0 + threadIdx.x;
+        int e = -1, f = 0, cnt = 0;
+        if (a < n_active_all) {
+            e = p.active[1 + a];
+            if (e >= 0 && e < p.E) {
+                f = p.offsets[e];
+                cnt = p.offsets[e + 1] - f;
+            }
+        }
+        const bool keep = a < n_active_all && e >= 0 && e < p.E && cnt > 0 && cnt <= p.max_count;
+        // order-preserving compaction within this block-wide step
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        __shared__ int warp_base[kStreamThreads / 32];
+        if ((threadIdx.x & 31) == 0) warp_base[threadIdx.x >> 5] = __popc(m);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int run = n_keep;
+            for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+                const int c = warp_base[w];
+                warp_base[w] = run;
+                run += c;
+            }
+            n_keep = run;
+        }
+        __syncthreads();
+        if (keep) {
+            const int pos = warp_base[threadIdx.x >> 5] + __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
+            S.st.expert[pos] = e;
+            S.st.bits[pos] = expert_bits(p, e);
+            S.st.first[pos] = f;
+            S.st.count[pos] = cnt;
+        }
+        __syncthreads();
     }
+    const int n_active = n_keep;
     // entries: routed slots in sorted order (first = expert offset), then the
     // shared expert's T tokens at [T*k, T*k + T)
     const int S_ = p.T * p.k;
@@ -540,11 +569,11 @@ ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
         }
     }
     if (threadIdx.x == 0) {
-        if (p.has_shared) {
+        if (p.has_shared && p.T <= p.max_count) {
             S.st.expert[n_active] = p.E;
             S.st.bits[n_active] = p.w.shared.bits;
             S.st.first[n_active] = S_;
-            S.st.count[n_active] = p.T > p.max_count ? 0 : p.T;
+            S.st.count[n_active] = p.T;
         }
         for (int s = 0; s < nstages; ++s) {
             mbar_init(&S.full[s], 1);
@@ -554,7 +583,7 @@ ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
         mbar_fence_init();
     }
     __syncthreads();
-    const int n_slots = n_active + (p.has_shared ? 1 : 0);
+    const int n_slots = n_active + (p.has_shared && p.T <= p.max_count ? 1 : 0);
     ffn_stream_body(p, S, n_slots, nstages, stage_bytes);
 }
 
@@ -577,7 +606,9 @@ size_t moe_ffn_stream_smem(int H, int I, int max_slots, int n_ent, int *nstages,
 }
 
 cudaError_t moe_configure_ffn_stream() {
-    return cudaFuncSetAttribute(moe::ffn_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    // the opt-in limit is 227 KB per CTA including static shared memory
+    return cudaFuncSetAttribute(moe::ffn_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                227 * 1024 - 1024);
 }
 
 bool moe_ffn_stream_supported(int H, int I) {
