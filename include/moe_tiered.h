@@ -217,6 +217,41 @@ int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t
                           moe_stream_t stream);
 
 /*
+ * moe_expert_ffn_tiered_static: the streaming (MOE_FFN_GEMV) path of
+ * moe_expert_ffn_tiered with no workspace argument.  The pages have no
+ * counterpart of this call; it exists for callers that cannot hand the
+ * library a device buffer: a C or C++ host with no device allocator of its
+ * own, whose decode loop must not call cudaMalloc/cudaFree because cudaFree
+ * waits for the whole device and so stalls every other stream on it, and a
+ * serving process that reserved its HBM for weights and KV cache up front
+ * and has nothing spare to carve a workspace from.
+ *
+ * Its scratch (the SwiGLU intermediates of every slot and the completion
+ * counters) is one array of MOE_STATIC_SCRATCH_BYTES bytes compiled into the
+ * library: every GPU that loads the library holds it until the process
+ * exits.  The call needs
+ *   align256((T*k + T) * I * 4) + align256((min(T*k, E) + 1) * 4)
+ * bytes of it (at I = 512, k = 10: up to 46 tokens) and returns
+ * MOE_ERR_UNSUPPORTED, enqueueing nothing, when that exceeds the array.
+ * Arguments, outputs and results are those of moe_expert_ffn_tiered in
+ * MOE_FFN_GEMV mode.  It allocates nothing: it clears the counters with an
+ * asynchronous memset on `stream` and launches the streaming kernel.
+ *
+ * All calls on a device share the one array and each overwrites what the
+ * previous one left there, so two calls whose work overlaps on the GPU (on
+ * different streams, or from several host threads) race and give undefined
+ * results: order them on one stream or with events.  The first call on each
+ * device looks up the array's device address (with that device current),
+ * so make that first call before any stream capture on that device.
+ */
+#define MOE_STATIC_SCRATCH_BYTES (1 << 20)
+int moe_expert_ffn_tiered_static(const moe_layer_weights *w, const uint16_t *x,
+                                 int32_t T, int32_t k, const int32_t *expert_offsets,
+                                 const int32_t *sorted_slot, const int32_t *active,
+                                 float *y_slots, float *y_shared, int32_t *status,
+                                 moe_stream_t stream);
+
+/*
  * moe_combine: out[t] = bf16_rne( sum_{j<k} topk_w[t,j] * y_slots[t*k+j]
  *                                 + y_shared[t] )
  * summed in that fixed order ([P1] "step 4": the results simply add up).

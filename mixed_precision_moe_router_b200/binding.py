@@ -25,6 +25,7 @@ STATUS_FP16_RANGE = 0x2
 STATUS_TIMEOUT = 0x4
 FFN_AUTO, FFN_GEMV, FFN_GEMM = 0, 1, 2
 MAX_TIERS = 4
+STATIC_SCRATCH_BYTES = 1 << 20  # size of the scratch array behind moe_expert_ffn_tiered_static
 
 c_i32, c_i64, c_size, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 
@@ -54,6 +55,8 @@ SIGNATURES = [
     ("moe_ffn_workspace_size", c_size, [ctypes.POINTER(LayerWeights), c_i32, c_i32, c_i32]),
     ("moe_expert_ffn_tiered", c_i32, [ctypes.POINTER(LayerWeights), c_vp, c_i32, c_i32, c_vp, c_vp, c_vp,
                                       c_vp, c_vp, c_vp, c_size, c_i32, c_vp, c_vp]),
+    ("moe_expert_ffn_tiered_static", c_i32, [ctypes.POINTER(LayerWeights), c_vp, c_i32, c_i32, c_vp, c_vp,
+                                             c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("moe_combine", c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     ("moe_rmsnorm", c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp]),
     ("moe_layer_workspace_size", c_size, [ctypes.POINTER(LayerWeights), c_i32, c_i32, c_i32]),
@@ -278,6 +281,23 @@ def expert_ffn(layer, x, k, offsets, sorted_slot, active, mode=FFN_AUTO, status=
     _check(lib().moe_expert_ffn_tiered(ctypes.byref(d), _ptr(x), T, k, _ptr(offsets), _ptr(sorted_slot),
                                        _ptr(active), _ptr(y_slots), _ptr(y_shared), _ptr(ws), nws, mode,
                                        _ptr(status), _stream()))
+    return y_slots, y_shared
+
+
+def expert_ffn_static(layer, x, k, offsets, sorted_slot, active, status=None):
+    """The streaming expert FFN through the call that takes no workspace: its
+    scratch is an array inside the library, for hosts that cannot allocate
+    device memory while they decode.  Calls on one device share that array, so
+    they must not overlap on the GPU (issue them on one stream)."""
+    _need(x, torch.bfloat16, name="x")
+    T = x.shape[0]
+    dev = x.device
+    d = layer.descriptor()
+    y_slots = torch.empty(T * k, layer.H, dtype=torch.float32, device=dev)
+    y_shared = torch.empty(T, layer.H, dtype=torch.float32, device=dev) if layer.shared is not None else None
+    _check(lib().moe_expert_ffn_tiered_static(ctypes.byref(d), _ptr(x), T, k, _ptr(offsets), _ptr(sorted_slot),
+                                              _ptr(active), _ptr(y_slots), _ptr(y_shared), _ptr(status),
+                                              _stream()))
     return y_slots, y_shared
 
 

@@ -431,3 +431,83 @@ int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router, cons
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// moe_expert_ffn_tiered_static: the streaming FFN without a caller workspace,
+// for hosts that cannot allocate device memory in their decode loop (no
+// allocator of their own, or HBM fully reserved up front; cudaFree would also
+// wait for the whole device).  Its scratch is the array below, which each GPU
+// that loads the library holds until exit; all calls on a device share it.
+// ---------------------------------------------------------------------------
+
+static __device__ __align__(256) unsigned char moe_static_scratch[MOE_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::once_flag g_scratch_once[kMaxDevices];
+void *g_scratch_ptr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up on the
+// first call per device (which therefore must not run under stream capture).
+int static_scratch(char **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::call_once(g_scratch_once[dev], [dev]() {
+        void *p = nullptr;
+        cudaError_t r = cudaGetSymbolAddress(&p, moe_static_scratch);
+        if (r != cudaSuccess) {
+            cudaGetLastError();
+            p = nullptr;
+        }
+        g_scratch_err[dev] = r;
+        g_scratch_ptr[dev] = p;
+    });
+    if (g_scratch_err[dev] != cudaSuccess) return cuda_fail(g_scratch_err[dev], "cudaGetSymbolAddress(scratch)");
+    *ptr = static_cast<char *>(g_scratch_ptr[dev]);
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" int moe_expert_ffn_tiered_static(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t k,
+                                            const int32_t *expert_offsets, const int32_t *sorted_slot,
+                                            const int32_t *active, float *y_slots, float *y_shared,
+                                            int32_t *status, moe_stream_t stream) {
+    int r = check_weights(w);
+    if (r) return r;
+    r = check_k(T, w->E, k);
+    if (r) return r;
+    if (T == 0) return ok();
+    if (!x || !expert_offsets || !sorted_slot || !active || !y_slots)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    const bool has_shared = w->shared.n_experts == 1;
+    if (has_shared != (y_shared != nullptr))
+        return fail(MOE_ERR_INVALID_ARG, "y_shared must be given iff the layer has a shared expert");
+    if (!aligned16(x) || !aligned16(y_slots) || (y_shared && !aligned16(y_shared)))
+        return fail(MOE_ERR_INVALID_ARG, "x / y pointers not 16-byte aligned");
+    const size_t need = gemv_ws_bytes(w, T, k);
+    if (need > static_cast<size_t>(MOE_STATIC_SCRATCH_BYTES))
+        return fail(MOE_ERR_UNSUPPORTED,
+                    "T = %d, k = %d, I = %d needs %zu bytes of scratch; the static array holds %d "
+                    "(use moe_expert_ffn_tiered with a workspace)",
+                    T, k, w->I, need, MOE_STATIC_SCRATCH_BYTES);
+    r = ensure_configured();
+    if (r) return r;
+    if (!moe_ffn_stream_supported(w->H, w->I)) return fail(MOE_ERR_UNSUPPORTED, "GEMV path supports H, I <= 2048");
+    char *ws = nullptr;
+    r = static_scratch(&ws);
+    if (r) return r;
+    moe::FfnParams p = make_params(w, x, T, k, expert_offsets, sorted_slot, active, y_slots, y_shared,
+                                   reinterpret_cast<float *>(ws), status);
+    // counters follow the intermediates, as in the workspace layout; they must
+    // start at zero and the previous call left its final counts there
+    const size_t hb = align_up((static_cast<size_t>(T) * k + T) * w->I * sizeof(float));
+    p.ctr = reinterpret_cast<int *>(ws + hb);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(p.ctr, 0, ffn_ctr_bytes(w, T, k), s);
+    if (e == cudaSuccess) e = moe_launch_ffn_stream(p, s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ffn launch");
+}
