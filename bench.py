@@ -35,7 +35,7 @@ from mixed_precision_moe_router_b200 import inputs  # noqa: E402
 METRIC = "MoE-layer tokens/s; decode expert-weight GB/s vs HBM peak; prefill TFLOP/s"
 UNIT = "layer-tokens/s"
 N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
-KERNELS_PER_LAYER = 6  # router logits, top-k, bucketize, gate_up, down, combine (+1 rmsnorm per step)
+KERNELS_PER_LAYER = 5  # router logits, top-k, bucketize, streaming FFN, combine (+1 rmsnorm per step)
 
 
 def peaks():
@@ -103,6 +103,163 @@ def expert_bytes(cfg, layer, e):
     return layer.nbytes_expert(e)
 
 
+def queue_ahead(cycles=60_000_000):
+    """Keep the GPU busy (~30 ms) while the host enqueues the calls that follow,
+    so that events around each call measure device time, not host latency."""
+    torch.cuda._sleep(cycles)
+
+
+def time_calls(stream, calls):
+    """Device time (ms) of each call, all enqueued behind one spin kernel."""
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+    with torch.cuda.stream(stream):
+        queue_ahead()
+        for (a, b), fn in zip(evs, calls):
+            a.record(stream)
+            fn()
+            b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+class StackRunner:
+    """T tokens through the stack as one CUDA graph of rmsnorm + n x layer_forward."""
+
+    def __init__(self, layers, routers, x0, stream):
+        from mixed_precision_moe_router_b200 import binding as B
+        self.B, self.layers, self.routers, self.stream = B, layers, routers, stream
+        cfg = inputs.DECODE
+        T = self.T = x0.shape[0]
+        dev = x0.device
+        n = len(layers)
+        self.ws = torch.empty(B.layer_workspace_size(layers[0], T, cfg.k, B.FFN_AUTO), dtype=torch.uint8,
+                              device=dev)
+        self.xs = [x0.clone()] + [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev) for _ in range(n)]
+        self.ns = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev) for _ in range(n + 1)]
+        self.outs = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev) for _ in range(n)]
+        with torch.cuda.stream(stream):
+            self.step()  # first run outside capture
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=stream):
+            self.step()
+
+    def step(self):
+        B, k = self.B, inputs.DECODE.k
+        B.rmsnorm(self.xs[0], out=self.ns[0])
+        for l, layer in enumerate(self.layers):
+            wr, bias = self.routers[l]
+            B.layer_forward(layer, wr, bias, self.ns[l], k, residual=self.xs[l], workspace=self.ws,
+                            out=self.outs[l], x_next=self.xs[l + 1], x_next_norm=self.ns[l + 1])
+
+    def time(self, steps, warmup):
+        for _ in range(warmup):
+            self.graph.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cur = torch.cuda.current_stream()
+        a.record(cur)
+        for _ in range(steps):
+            self.graph.replay()
+        b.record(cur)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+
+def ffn_flops(cfg, pairs):
+    """gate_up (2I x H) and down (H x I) products of each (token, expert) pair."""
+    return 6.0 * cfg.H * cfg.I * pairs
+
+
+def ffn_calls(layers, routers, xs, mode, stream):
+    """Route xs[l] through layer l, then return one FFN call per layer plus the
+    touched expert bytes and (token, expert) pairs of each."""
+    from mixed_precision_moe_router_b200 import binding as B
+    cfg = inputs.DECODE
+    calls, nbytes, pairs = [], [], []
+    for l, layer in enumerate(layers):
+        wr, bias = routers[l]
+        x = xs[l]
+        with torch.cuda.stream(stream):
+            idx, _, _ = B.router_topk(x, wr, bias, cfg.k)
+            off, srt, pos, act = B.bucketize(idx, cfg.E)
+        torch.cuda.synchronize()
+        touched = sorted(set(idx.cpu().numpy().reshape(-1).tolist()))
+        nbytes.append(sum(layer.nbytes_expert(e) for e in touched) + layer.nbytes_expert(cfg.E))
+        pairs.append(x.shape[0] * (cfg.k + 1))
+        calls.append(lambda layer=layer, x=x, off=off, srt=srt, act=act:
+                     B.expert_ffn(layer, x, cfg.k, off, srt, act, mode=mode))
+    return calls, nbytes, pairs
+
+
+def ffn_profile(layers, routers, xs, stream, mode=None):
+    """Mean device time of the FFN call over the layers (each layer's experts
+    are cold: the calls before it touched other layers' weights)."""
+    from mixed_precision_moe_router_b200 import binding as B
+    calls, nbytes, pairs = ffn_calls(layers, routers, xs, B.FFN_AUTO if mode is None else mode, stream)
+    time_calls(stream, calls)  # warm-up (allocator, first launches)
+    ms = time_calls(stream, calls)
+    ms_avg = float(np.mean(ms))
+    return {"ms": ms_avg, "bytes": float(np.mean(nbytes)), "pairs": float(np.mean(pairs)),
+            "gbs": float(np.mean(nbytes)) / (ms_avg / 1e3) / 1e9,
+            "tflops": ffn_flops(inputs.DECODE, float(np.mean(pairs))) / (ms_avg / 1e3) / 1e12}
+
+
+def prefill_profile(layer, router, stream, T=inputs.PREFILL_T, reps=10):
+    """One layer of the decode configuration on T prompt tokens: the whole layer
+    and its FFN call (tensor-core grouped GEMM + streaming GEMV for experts
+    with few tokens), timed on the device."""
+    from mixed_precision_moe_router_b200 import binding as B
+    cfg = inputs.DECODE
+    dev = layer_device(layer)
+    x = inputs.activations(T, cfg.H, seed=inputs.X_SEED + 11, device=dev)
+    wr, bias = router
+    ws = torch.empty(B.layer_workspace_size(layer, T, cfg.k, B.FFN_AUTO), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
+    layer_call = lambda: B.layer_forward(layer, wr, bias, x, cfg.k, workspace=ws, out=out)  # noqa: E731
+    time_calls(stream, [layer_call] * 3)
+    layer_ms = float(np.median(time_calls(stream, [layer_call] * reps)))
+    calls, _, pairs = ffn_calls([layer], [router], [x], B.FFN_AUTO, stream)
+    time_calls(stream, calls * 3)
+    ffn_ms = float(np.median(time_calls(stream, calls * reps)))
+    return {"T": T, "layer_ms": layer_ms, "ffn_ms": ffn_ms, "flops": ffn_flops(cfg, pairs[0]),
+            "tflops": ffn_flops(cfg, pairs[0]) / (ffn_ms / 1e3) / 1e12}
+
+
+def layer_device(layer):
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def run_prefill(args, rank, world):
+    """--workload prefill: one layer, 4096 tokens; the line reports layer-tokens/s
+    and the tensor-core roofline of the FFN call."""
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    layers, routers = build_stack(inputs.DECODE, 1, device)
+    stream = torch.cuda.Stream(device)
+    hbm, tf, peak_kind = peaks()
+    with ClockSampler(device.index) as clk:
+        pf = prefill_profile(layers[0], routers[0], stream, reps=max(args.steps, 3))
+    T = pf["T"]
+    return {
+        "metric": METRIC, "value": round(world * T / (pf["layer_ms"] / 1e3), 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pf["layer_ms"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": f"prefill: one MoE layer (H=2048, I=512, E=512, top-10 + 1 shared, 3 shelves, "
+                               f"Zipf routing), {T} tokens per step per GPU", "global_batch": world * T,
+                   "layers": 1, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: every expert of the layer (~0.6 GB) is read each step"},
+        "roofline": {"bound": "tensor", "kernel": "expert FFN call (f16 staging + gate_up GEMM + down GEMM)",
+                     "achieved": round(pf["tflops"], 1), "peak": tf, "unit": "TFLOP/s",
+                     "frac": round(pf["tflops"] / tf, 4), "traffic": None, "peak_kind": peak_kind + " burst",
+                     "algorithmic_flops_per_launch": pf["flops"], "avg_launch_us": round(pf["ffn_ms"] * 1e3, 1)},
+        "gpu_launches": max(args.steps, 3) * 8,
+        "clocks": clk.summary(),
+    }
+
+
 def run_native(args, rank, world):
     from mixed_precision_moe_router_b200 import binding as B
     device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -111,28 +268,10 @@ def run_native(args, rank, world):
     T = 1
     layers, routers = build_stack(cfg, N_LAYERS, device)
     k = cfg.k
-    x0 = inputs.activations(T, cfg.H, seed=inputs.X_SEED + 1000 * rank, device=device)
-    nws = B.layer_workspace_size(layers[0], T, k, B.FFN_AUTO)
-    ws = torch.empty(nws, dtype=torch.uint8, device=device)
-    # residual stream xs[l] (bf16) and the normalised input ns[l] each layer reads
-    xs = [x0.clone()] + [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device) for _ in range(N_LAYERS)]
-    ns = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device) for _ in range(N_LAYERS + 1)]
-    outs = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device) for _ in range(N_LAYERS)]
-
-    def step():
-        B.rmsnorm(xs[0], out=ns[0])
-        for l in range(N_LAYERS):
-            wr, bias = routers[l]
-            B.layer_forward(layers[l], wr, bias, ns[l], k, residual=xs[l], workspace=ws, out=outs[l],
-                            x_next=xs[l + 1], x_next_norm=ns[l + 1])
-
     stream = torch.cuda.Stream(device)
-    with torch.cuda.stream(stream):
-        step()  # first run outside capture
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step()
+    x0 = inputs.activations(T, cfg.H, seed=inputs.X_SEED + 1000 * rank, device=device)
+    run = StackRunner(layers, routers, x0, stream)
+    graph = run.graph
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -158,28 +297,10 @@ def run_native(args, rank, world):
     ms_per_step = ms / args.steps
     value = world * T * N_LAYERS * args.steps / (ms / 1e3)
 
-    # per-call timing of the FFN (the dominant kernels) and algorithmic bytes
+    # the dominant kernel: the expert FFN call of each layer, on the inputs the
+    # timed steps gave each layer, device-timed with the host kept ahead
     hbm, tf, peak_kind = peaks()
-    ffn_ms, ffn_bytes = [], []
-    with torch.cuda.stream(stream):
-        for l in range(N_LAYERS):
-            wr, bias = routers[l]
-            idx, w, _ = B.router_topk(ns[l], wr, bias, k)
-            off, srt, pos, act = B.bucketize(idx, cfg.E)
-            torch.cuda.synchronize()
-            touched = sorted(set(idx.cpu().numpy().reshape(-1).tolist()))
-            ffn_bytes.append(sum(layers[l].nbytes_expert(e) for e in touched) + layers[l].nbytes_expert(cfg.E))
-            # one call per layer: the previous layer's FFN (other weights) ran in between,
-            # so this layer's experts are not L2-resident
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            B.expert_ffn(layers[l], ns[l], k, off, srt, act, mode=B.FFN_AUTO)
-            b.record(stream)
-            b.synchronize()
-            ffn_ms.append(a.elapsed_time(b))
-    avg_ms = float(np.mean(ffn_ms))
-    avg_bytes = float(np.mean(ffn_bytes))
-    achieved = avg_bytes / (avg_ms / 1e3) / 1e9
+    fp = ffn_profile(layers, routers, run.ns[:N_LAYERS], stream)
 
     # end to end through the public API: pinned host input, eager calls, host output
     h_in = x0.cpu().pin_memory()
@@ -191,9 +312,9 @@ def run_native(args, rank, world):
                 torch.cuda.synchronize()
                 e0 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            xs[0].copy_(h_in, non_blocking=True)
-            step()
-            h_out.copy_(xs[N_LAYERS], non_blocking=True)
+            run.xs[0].copy_(h_in, non_blocking=True)
+            run.step()
+            h_out.copy_(run.xs[N_LAYERS], non_blocking=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -203,27 +324,65 @@ def run_native(args, rank, world):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_val = world * T * N_LAYERS / (e2e_ms / 1e3)
-    del graph
+    del graph, run
+
+    # the other workloads of the layer, reported beside the headline
+    extra = {}
+    if not args.headline_only:
+        extra = other_workloads(args, layers, routers, stream, rank)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "decode: 48 stacked MoE layers (H=2048, I=512, E=512, top-10 + 1 shared, "
+        "config": {"workload": f"decode: {N_LAYERS} stacked MoE layers (H=2048, I=512, E=512, top-10 + 1 shared, "
                                "shelves 128x8-bit/192x4-bit/192x3-bit, Zipf routing), 1 token per step per GPU",
                    "global_batch": world * T, "layers": N_LAYERS, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: ~1.37 GB of distinct expert weights touched per step",
-                   "graph": "one CUDA graph per step (48 x layer_forward)"},
-        "roofline": {"bound": "hbm", "kernel": "expert FFN (gate_up + down GEMV launches of one layer)",
-                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": None, "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": round(avg_bytes), "avg_launch_us": round(avg_ms * 1e3, 2)},
+                   "graph": f"one CUDA graph per step (rmsnorm + {N_LAYERS} x layer_forward)"},
+        "roofline": {"bound": "hbm", "kernel": "expert FFN call of one layer (counter clear + streaming GEMV)",
+                     "achieved": round(fp["gbs"], 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(fp["gbs"] / hbm, 4), "traffic": None, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": round(fp["bytes"]), "avg_launch_us": round(fp["ms"] * 1e3, 2)},
         "e2e": {"value": round(e2e_val, 1), "unit": UNIT,
                 "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2},
         "gpu_launches": args.steps * (N_LAYERS * KERNELS_PER_LAYER + 1),
         "clocks": clk.summary(),
     }
+    if extra:
+        line["workloads"] = extra
     return line
+
+
+def other_workloads(args, layers, routers, stream, rank):
+    """Decode with 8 tokens and the speculative-verify batch through the stack,
+    prefill of one layer, and the token sweep on single layers."""
+    cfg = inputs.DECODE
+    dev = torch.device("cuda", torch.cuda.current_device())
+    res = {}
+    n = len(layers)
+    for name, x0 in (("decode_T8", inputs.activations(8, cfg.H, seed=inputs.X_SEED + 1000 * rank + 8, device=dev)),
+                     ("verify_T5", inputs.correlated_activations(inputs.VERIFY_T, cfg.H,
+                                                                 seed=inputs.X_SEED + 1000 * rank, device=dev))):
+        run = StackRunner(layers, routers, x0, stream)
+        ms = run.time(args.steps, args.warmup)
+        res[name] = {"layer_tokens_per_s": round(x0.shape[0] * n / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+                     "layers": n, "tokens": x0.shape[0]}
+        del run
+    hbm, tf, _ = peaks()
+    pf = prefill_profile(layers[0], routers[0], stream)
+    res["prefill_T4096"] = {"layer_tokens_per_s": round(pf["T"] / (pf["layer_ms"] / 1e3), 1),
+                            "layer_ms": round(pf["layer_ms"], 4), "ffn_ms": round(pf["ffn_ms"], 4),
+                            "ffn_tflops": round(pf["tflops"], 1), "ffn_frac_of_bf16_peak": round(pf["tflops"] / tf, 4)}
+    sweep = []
+    for T in inputs.SWEEP_T:
+        xs = [inputs.activations(T, cfg.H, seed=inputs.X_SEED + 100 * l + T, device=dev) for l in range(n)]
+        fp = ffn_profile(layers, routers, xs, stream)
+        sweep.append({"T": T, "ffn_us": round(fp["ms"] * 1e3, 2), "gbs": round(fp["gbs"], 1),
+                      "frac_hbm": round(fp["gbs"] / hbm, 4), "tflops": round(fp["tflops"], 2),
+                      "frac_bf16": round(fp["tflops"] / tf, 4), "touched_mb": round(fp["bytes"] / 1e6, 2)})
+    res["sweep_one_layer_ffn"] = sweep
+    return res
 
 
 class OracleStack:
@@ -288,6 +447,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=inputs.N_STACK,
                     help="stack depth; the benchmark is defined at 48, fewer only for profiler captures")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+                    help="decode: the 48-layer one-token stack (default); prefill: one layer, 4096 tokens")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the secondary workloads (8-token decode, verify batch, prefill, sweep)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -321,9 +484,9 @@ def main():
         return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
-    line = run_native(args, rank, world)
+    line = run_native(args, rank, world) if args.workload == "decode" else run_prefill(args, rank, world)
     if rank == 0:
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and world == 1 and args.workload == "decode":
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line))
     if world > 1:

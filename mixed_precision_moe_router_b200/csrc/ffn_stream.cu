@@ -1,53 +1,119 @@
 // Tiered expert FFN, GEMV path: one persistent launch that streams every
-// touched expert's packed rows once through a shared-memory ring.
+// touched expert's packed rows once through a shared-memory ring and runs the
+// dot products on the tensor cores against up to 8 token columns at a time.
 //
 // [P1] "step 4: three shelves, all on the GPU": mul_mat_id runs each word
 // through its chosen experts, each shelf computes only the ids on it and the
 // shelf results add up; the decode kernel fuses gate, up and the activation.
 //
 // Design (B200):
-//  * Work is a list of tiles: for every active expert (any shelf) and the
-//    shared expert, I/8 gate_up tiles (8 gate rows + the 8 matching up rows)
-//    and H/64 down tiles (64 rows).  Each CTA takes a contiguous, byte-balanced
-//    share of the gate_up tiles and then of the down tiles, so 8-, 4- and
-//    3-bit experts spread evenly over the SMs.
-//  * One producer thread per CTA moves each tile's codes and scales into a
-//    4-6 stage shared-memory ring with 1-D bulk copies (cp.async.bulk) that
-//    complete on an mbarrier; 8 consumer warps dequantise from shared memory
-//    (w = d*q exact in fp32) and accumulate in fp32 against activations held
-//    in registers.
-//  * gate_up tiles write h = silu(g)*u (fp32) and count themselves done per
-//    expert; a down tile waits (bounded) for its expert's count before reading
-//    h, while its weights may already be in flight.  The grid is launched
-//    cooperatively so every CTA is resident and the waits always resolve.
+//  * Work is a list of tiles.  For every slot (an active expert whose token
+//    count is in (0, max_count], and the shared expert) there are gate_up
+//    tiles of 8R gate rows plus the 8R matching up rows, and down tiles of
+//    16R rows, with R the largest power of two <= 8 such that a tile holds at
+//    most 32K codes.  Each CTA takes a contiguous, cost-balanced share of the
+//    gate_up tiles and then of the down tiles, so 8-, 4- and 3-bit experts
+//    spread evenly over the SMs.
+//  * All 8 warps of a CTA stage the next tiles into a ring of shared-memory
+//    stages with 16-byte cp.async copies (commit / wait_group), so that copy
+//    issue is spread over 256 threads; rows land at a padded stride that
+//    makes the reads below bank-conflict free.
+//  * The 8 warps split a tile into R row subtiles x 8/R K slices.  For
+//    each 32-weight block a warp turns its codes into exact fp16 integers
+//    (|q| <= 127), multiplies them with fp16 activation fragments on the
+//    tensor cores (mma.sync m16n8k16: exact products, fp32 accumulation) and
+//    adds d * partial into fp32 accumulators.  The only roundings besides fp32
+//    accumulation are bf16 x -> fp16 (exact for |x| in [2^-14, 65504]) and the
+//    split of the fp32 intermediate h into two fp16 columns hi + lo (relative
+//    error <= 2^-22).  Dequantisation is paid once per tile for up to 8 tokens;
+//    more tokens take further passes over the resident tile.
+//  * K slices are summed in shared memory in a fixed order.  gate_up tiles
+//    write h = silu(g) * u and count themselves done per slot; a down tile
+//    waits (bounded) for its slot's count before reading h, while its weights
+//    may already be in flight.  The grid is launched cooperatively so every
+//    CTA is resident and the waits resolve.
 #include "common.cuh"
 #include "ffn.cuh"
 #include "sync.cuh"
 
 namespace moe {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kStreamThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kGuPairs = 16;                                 // gate/up row pairs per tile (2 per warp)
-constexpr int kDnRows = 64;                                  // down rows per tile
+constexpr int kWarps = 8;                          // compute warps
+constexpr int kThreads = kWarps * 32;
+constexpr int kProducerWarps = 2;                  // copy warps
+constexpr int kProducers = kProducerWarps * 32;
+constexpr int kBlockThreads = kThreads + kProducers;
+constexpr int kBarCompute = 1;                     // named barrier of the compute warps
 constexpr int kMaxStages = 6;
-constexpr int kMaxRegK = 2048;  // activations held in registers: K <= 2048
+constexpr int kStageBytes = 40 * 1024;
+constexpr int kMaxK = 2048;
 constexpr int kMaxSmemEntries = 2048;  // token-entry tables kept in shared memory up to this size
+constexpr int kTokPerPass = 8;         // gate_up token columns per pass over a resident tile
+constexpr int kRedBytes = kWarps * 32 * 4 * 4;
 
-__host__ __device__ __forceinline__ int row_bytes(int K, int bits) { return K * bits / 8; }
-__host__ __device__ __forceinline__ int gu_tile_bytes(int H, int bits) {
-    return 2 * kGuPairs * (row_bytes(H, bits) + H / 16);
+// ---------------------------------------------------------------------------
+// tile geometry
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int rows_pow2(int K) {
+    int R = 1;
+    while (R < 8 && 2 * R * K <= 2048) R *= 2;
+    return R;
 }
-__host__ __device__ __forceinline__ int dn_tile_bytes(int I, int bits) {
-    return kDnRows * (row_bytes(I, bits) + I / 16);
+
+// Stride of a code row in a stage: 8-bit reads (8 bytes per thread, 4 threads
+// per row) need the stride in words to be 8 or 24 mod 32; 4- and 3-bit reads
+// (at most 4 bytes) need 4 mod 8.  Strides stay multiples of 16 bytes.
+__host__ __device__ __forceinline__ int code_row_stride(int K, int bits) {
+    const int rb = K * bits / 8;
+    for (int p = 0; p < 128; p += 16) {
+        const int w = (rb + p) / 4;
+        if (bits == 8 ? (w % 32 == 8 || w % 32 == 24) : (w % 8 == 4)) return rb + p;
+    }
+    return rb;
 }
-// Work estimate used to balance tiles over CTAs: bytes moved plus a share for
-// the per-weight dequant/FMA work, which is the same for every precision.
-__host__ __device__ __forceinline__ long long gu_tile_cost(int H, int bits) {
-    return gu_tile_bytes(H, bits) + static_cast<long long>(2 * kGuPairs) * H / 2;
+
+struct Geo {
+    int K, R, rows;   // row subtiles and rows per tile
+    int rb, rs;       // code bytes per row, stage stride
+    int sb, ss;       // scale bytes per row, stage stride
+    bool row_scales;  // scales copied row by row (padded) or in one piece
+    int nb, bps;      // 32-weight blocks per row, blocks per K slice
+};
+
+__host__ __device__ __forceinline__ Geo geo(int K, int bits) {
+    Geo g;
+    g.K = K;
+    g.R = rows_pow2(K);
+    g.rows = 16 * g.R;
+    g.rb = K * bits / 8;
+    g.rs = code_row_stride(K, bits);
+    g.sb = K / 16;
+    g.row_scales = g.sb % 16 == 0 && g.sb >= 64;
+    g.ss = g.row_scales ? g.sb + 16 : g.sb;
+    g.nb = K / 32;
+    const int S = kWarps / g.R;
+    g.bps = ((g.nb + S - 1) / S + 1) & ~1;  // even, so blocks go in pairs
+    return g;
 }
-__host__ __device__ __forceinline__ long long dn_tile_cost(int I, int bits) {
-    return dn_tile_bytes(I, bits) + static_cast<long long>(kDnRows) * I / 2;
+
+__host__ __device__ __forceinline__ int stage_bytes(const Geo &g) { return g.rows * (g.rs + g.ss); }
+
+// x fragments in shared memory: [column][block][thread t][8 halves], with a
+// column stride that keeps the 16-byte reads of two columns in different banks.
+__host__ __device__ __forceinline__ int xf_col_stride(int K) { return (K / 32) * 64 + 64; }
+
+__host__ __device__ __forceinline__ int down_ntiles(int I) { return I <= 1024 ? 2 : 1; }
+
+__host__ __device__ __forceinline__ int xf_bytes(int H, int I) {
+    const int a = kTokPerPass * xf_col_stride(H);
+    const int b = 8 * down_ntiles(I) * xf_col_stride(I);
+    return a > b ? a : b;
+}
+
+// tokens of one pass: gate_up tiles use one column per token, down tiles two
+// (h = hi + lo) in n-tiles of 8 columns
+__host__ __device__ __forceinline__ int tokens_per_pass(int phase, int I) {
+    return phase == 0 ? kTokPerPass : 4 * down_ntiles(I);
 }
 
 struct SlotTabs {  // per expert slot, in shared memory
@@ -55,13 +121,12 @@ struct SlotTabs {  // per expert slot, in shared memory
     int *tok, *row;  // entries [first, first + count) of every slot: token and h/y row
 };
 
-// Shelf pointers of expert e, read from the kernel parameters with constant
-// indices only (no address of the parameter block is taken).
-struct ExpertPtrs {
-    const uint8_t *gq;
-    const uint16_t *gs;
-    const uint8_t *dq;
-    const uint16_t *ds;
+// Table base pointers of the shelves (index < n_tiers) and of the shared
+// expert (index n_tiers), copied from the parameters into shared memory so
+// that they can be indexed at run time.
+struct TierPtrs {
+    const uint8_t *gq, *gs, *dq, *ds;
+    int bits, first, n, pad;
 };
 
 __device__ __forceinline__ int expert_bits(const FfnParams &p, int e) {
@@ -75,158 +140,92 @@ __device__ __forceinline__ int expert_bits(const FfnParams &p, int e) {
     return b;
 }
 
-__device__ __forceinline__ ExpertPtrs expert_ptrs(const FfnParams &p, int e) {
-    const int H = p.w.H, I = p.w.I;
-    ExpertPtrs r{nullptr, nullptr, nullptr, nullptr};
-    if (e == p.E) {
-        r.gq = p.w.shared.gu_qs;
-        r.gs = p.w.shared.gu_scale;
-        r.dq = p.w.shared.dn_qs;
-        r.ds = p.w.shared.dn_scale;
-        return r;
-    }
-#pragma unroll
-    for (int i = 0; i < MOE_MAX_TIERS; ++i) {
-        if (i < p.w.n_tiers && e >= p.w.tiers[i].first_expert &&
-            e < p.w.tiers[i].first_expert + p.w.tiers[i].n_experts) {
-            const size_t j = static_cast<size_t>(e - p.w.tiers[i].first_expert);
-            const int b = p.w.tiers[i].bits;
-            r.gq = p.w.tiers[i].gu_qs + j * 2 * I * row_bytes(H, b);
-            r.gs = p.w.tiers[i].gu_scale + j * 2 * I * (H / 32);
-            r.dq = p.w.tiers[i].dn_qs + j * H * row_bytes(I, b);
-            r.ds = p.w.tiers[i].dn_scale + j * H * (I / 32);
-        }
-    }
-    return r;
+// Balancing weight of a tile: its bytes plus a per-weight share for the
+// dequantise-and-multiply work of each pass (3-bit codes take the most).
+__device__ __forceinline__ long long tile_cost(const FfnParams &p, int phase, int bits, int count) {
+    const int K = phase == 0 ? p.w.H : p.w.I;
+    const long long rows = 16 * rows_pow2(K);
+    const int tp = tokens_per_pass(phase, p.w.I);
+    const long long passes = (count + tp - 1) / tp;
+    return rows * (K * bits / 8 + K / 16) + passes * (rows * K / 3) * (bits == 3 ? 3 : 2);
 }
 
-// Calls f(phase, slot, tile) for this CTA's tiles, in order: its byte-balanced
-// share of all gate_up tiles (phase 0), then of all down tiles (phase 1).
-template <class F>
-__device__ __forceinline__ void for_each_tile(const FfnParams &p, const SlotTabs &st, int n_slots, F &&f) {
-    const int G = gridDim.x, c = blockIdx.x;
-    for (int phase = 0; phase < 2; ++phase) {
-        const int nt = phase == 0 ? p.w.I / kGuPairs : p.w.H / kDnRows;
-        long long total = 0;
-        for (int a = 0; a < n_slots; ++a)
-            total += static_cast<long long>(nt) *
-                     (phase == 0 ? gu_tile_cost(p.w.H, st.bits[a]) : dn_tile_cost(p.w.I, st.bits[a]));
-        const long long lo = total * c / G, hi = total * (c + 1) / G;
-        long long off = 0;
-        for (int a = 0; a < n_slots && off < hi; ++a) {
-            const long long tb = phase == 0 ? gu_tile_cost(p.w.H, st.bits[a]) : dn_tile_cost(p.w.I, st.bits[a]);
-            const long long end = off + nt * tb;
-            if (end > lo) {
-                const long long b0 = lo > off ? (lo - off + tb - 1) / tb : 0;
-                long long b1 = (hi - off + tb - 1) / tb;
-                if (b1 > nt) b1 = nt;
-                for (long long b = b0; b < b1; ++b) f(phase, a, static_cast<int>(b));
-            }
-            off = end;
-        }
-    }
+__device__ __forceinline__ int tiles_per_slot(const FfnParams &p, int phase) {
+    return phase == 0 ? p.w.I / (8 * rows_pow2(p.w.H)) : p.w.H / (16 * rows_pow2(p.w.I));
 }
 
-// ---------------------------------------------------------------------------
-// dot products of one 16-byte unit (shared memory) with activations in registers
-// ---------------------------------------------------------------------------
-template <int BITS> struct UnitW;
-template <> struct UnitW<8> { static constexpr int W = 16; };
-template <> struct UnitW<4> { static constexpr int W = 32; };
-template <> struct UnitW<3> { static constexpr int W = 64; };
+// Per-slot tile costs and inclusive prefix sums of the slots' total costs,
+// per phase, built once in the prologue (shared memory).
+struct Sched {
+    long long *tc0, *tc1;    // cost of one tile of each slot
+    long long *pre0, *pre1;  // inclusive prefix sums of the slots' total costs
+};
 
-template <int BITS>
-__device__ __forceinline__ float unit_dot(const uint8_t *qrow, const uint16_t *srow, int K, int u,
-                                          const float *a) {
-    if constexpr (BITS == 8) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(qrow + 16 * u);
-        const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
-        float p0 = 0.f, p1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float w[4];
-            s8x4_to_f32(wd[i], w);
-            p0 = fmaf(w[0], a[4 * i + 0], p0);
-            p1 = fmaf(w[1], a[4 * i + 1], p1);
-            p0 = fmaf(w[2], a[4 * i + 2], p0);
-            p1 = fmaf(w[3], a[4 * i + 3], p1);
-        }
-        return f16_bits_to_f32(srow[u >> 1]) * (p0 + p1);
-    } else if constexpr (BITS == 4) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(qrow + 16 * u);
-        const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
-        float p0 = 0.f, p1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float w[8];
-            u4x8_to_f32(wd[i], w);
-#pragma unroll
-            for (int m = 0; m < 8; m += 2) {
-                p0 = fmaf(w[m], a[8 * i + m], p0);
-                p1 = fmaf(w[m + 1], a[8 * i + m + 1], p1);
-            }
-        }
-        return f16_bits_to_f32(srow[u]) * (p0 + p1);
-    } else {
-        const uint4 lo = *reinterpret_cast<const uint4 *>(qrow + 16 * u);
-        const uint2 hi = *reinterpret_cast<const uint2 *>(qrow + K / 4 + 8 * u);
-        const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w};
-        const uint32_t hw[4] = {hi.x & 0xffffu, hi.x >> 16, hi.y & 0xffffu, hi.y >> 16};
-        float p[2] = {0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float w[16];
-            u3x16_to_f32(lw[i], hw[i], w);
-            float q0 = 0.f, q1 = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; m += 2) {
-                q0 = fmaf(w[m], a[16 * i + m], q0);
-                q1 = fmaf(w[m + 1], a[16 * i + m + 1], q1);
-            }
-            p[i >> 1] += q0 + q1;
-        }
-        return f16_bits_to_f32(srow[2 * u]) * p[0] + f16_bits_to_f32(srow[2 * u + 1]) * p[1];
-    }
+// floor(x / y) for 0 <= x < 2^52, 0 < y: a double quotient corrected to the
+// exact integer result (the 64-bit integer divide is a long routine).
+__device__ __forceinline__ long long div_floor(long long x, long long y) {
+    long long q = static_cast<long long>(static_cast<double>(x) / static_cast<double>(y));
+    while (q * y > x) --q;
+    while ((q + 1) * y <= x) ++q;
+    return q;
 }
 
-// Load the activations lane `lane` needs for a row of K weights at BITS:
-// unit u = lane + 32*j covers weights [W*u, W*u + W).  Source is bf16 (x) or
-// fp32 (h, read through L2 since other SMs wrote it).
-template <int BITS, int UPL>
-__device__ __forceinline__ void load_act_bf16(const uint16_t *row, int K, int lane, float *a) {
-    constexpr int W = UnitW<BITS>::W;
-    const int U = K / W;
-#pragma unroll
-    for (int j = 0; j < UPL; ++j) {
-        const int u = lane + 32 * j;
-        if (u < U) {
-#pragma unroll
-            for (int v = 0; v < W / 8; ++v) {
-                const uint4 q = *reinterpret_cast<const uint4 *>(row + W * u + 8 * v);
-                float *d = a + W * j + 8 * v;
-                d[0] = bf16lo(q.x); d[1] = bf16hi(q.x); d[2] = bf16lo(q.y); d[3] = bf16hi(q.y);
-                d[4] = bf16lo(q.z); d[5] = bf16hi(q.z); d[6] = bf16lo(q.w); d[7] = bf16hi(q.w);
-            }
+// This CTA's tiles, in order: its cost-balanced contiguous share of all
+// gate_up tiles (phase 0), then of all down tiles (phase 1).  phase == 2 once
+// the list is exhausted.
+struct TileIt {
+    int phase, a, b, b1;  // current tile: slot a, tile b; b1 ends this slot's range
+    long long lo, hi;     // this CTA's cost range in the current phase
+};
+
+__device__ __forceinline__ bool it_slot(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
+    const long long *pre = it.phase == 0 ? sc.pre0 : sc.pre1;
+    const long long *tc = it.phase == 0 ? sc.tc0 : sc.tc1;
+    const long long nt = tiles_per_slot(p, it.phase);
+    for (; it.a < n_slots; ++it.a) {
+        const long long tb = tc[it.a];
+        const long long off = pre[it.a] - nt * tb;
+        if (off >= it.hi) return false;
+        const long long b0 = it.lo > off ? div_floor(it.lo - off + tb - 1, tb) : 0;
+        long long b1 = div_floor(it.hi - off + tb - 1, tb);
+        if (b1 > nt) b1 = nt;
+        if (b0 < b1) {
+            it.b = static_cast<int>(b0);
+            it.b1 = static_cast<int>(b1);
+            return true;
         }
     }
+    return false;
 }
 
-template <int BITS, int UPL>
-__device__ __forceinline__ void load_act_f32(const float *row, int K, int lane, float *a) {
-    constexpr int W = UnitW<BITS>::W;
-    const int U = K / W;
-#pragma unroll
-    for (int j = 0; j < UPL; ++j) {
-        const int u = lane + 32 * j;
-        if (u < U) {
-#pragma unroll
-            for (int v = 0; v < W / 4; ++v) {
-                const float4 q = __ldcg(reinterpret_cast<const float4 *>(row + W * u + 4 * v));
-                float *d = a + W * j + 4 * v;
-                d[0] = q.x; d[1] = q.y; d[2] = q.z; d[3] = q.w;
-            }
-        }
+__device__ __forceinline__ bool it_phase(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it, int phase) {
+    it.phase = phase;
+    const long long *pre = phase == 0 ? sc.pre0 : sc.pre1;
+    const long long total = pre[n_slots - 1];
+    it.lo = div_floor(total * blockIdx.x, gridDim.x);
+    it.hi = div_floor(total * (blockIdx.x + 1), gridDim.x);
+    int a0 = 0, a1 = n_slots;  // first slot whose cost range ends after lo
+    while (a0 < a1) {
+        const int m = (a0 + a1) >> 1;
+        if (pre[m] > it.lo) a1 = m; else a0 = m + 1;
     }
+    it.a = a0;
+    return it_slot(p, sc, n_slots, it);
+}
+
+__device__ __forceinline__ void it_begin(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
+    it.phase = 2;
+    if (n_slots == 0) return;
+    if (!it_phase(p, sc, n_slots, it, 0) && !it_phase(p, sc, n_slots, it, 1)) it.phase = 2;
+}
+
+__device__ __forceinline__ void it_next(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
+    if (it.phase == 2) return;
+    if (++it.b < it.b1) return;
+    ++it.a;
+    if (it_slot(p, sc, n_slots, it)) return;
+    if (it.phase == 0 && it_phase(p, sc, n_slots, it, 1)) return;
+    it.phase = 2;
 }
 
 // token and output row of the n-th entry of slot a (tables built in the prologue)
@@ -245,319 +244,510 @@ __device__ __forceinline__ void slot_entry(const FfnParams &p, const SlotTabs &s
     }
 }
 
-// Sum each of N values over the 32 lanes with N-1 + log2(32/N) shuffles instead
-// of 5N: at every step each lane keeps half of its values and swaps the other
-// half.  On return lane l holds the full sum of value (l / (32 / N)) % N.
-template <int N>
-__device__ __forceinline__ float transpose_reduce(float (&v)[N]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int n = N, o = 16; n > 1; n >>= 1, o >>= 1) {
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < n / 2; ++i) {
-            const float send = upper ? v[i] : v[i + n / 2];
-            const float keep = upper ? v[i + n / 2] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-    }
-    float r = v[0];
-    constexpr int rest = 32 / N;  // lanes still holding partial sums of the same value
-#pragma unroll
-    for (int o = rest / 2; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
-    return r;
+// ---------------------------------------------------------------------------
+// Codes -> exact fp16 integers: four half2 pairs per row, block and thread.
+// A code c placed at mantissa bit s under the exponent of 2^(10-s) reads as
+// the half 2^(10-s) + c; subtracting 2^(10-s) + offset leaves q exactly.
+// Thread t owns weights 8t .. 8t+7 of each 32-weight block, paired as
+// (2p, 2p+1) for 8-bit codes and (p, p+4) for 4- and 3-bit codes, p = 0..3.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
 }
 
-// gate_up tile: warp w computes pairs i = 16*tile + 2*w + {0, 1} for every
-// token of the slot.  h is written with plain stores; the caller publishes it.
-template <int BITS, int UPL>
-__device__ __forceinline__ void consume_gu(const FfnParams &p, const SlotTabs &st, int a, int tile,
-                                           const uint8_t *stage, float *act, int &act_key) {
-    const int H = p.w.H, I = p.w.I;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int W = UnitW<BITS>::W;
-    const int U = H / W;
-    const int rb = row_bytes(H, BITS);
-    const int nsc = H / 32;
-    const uint8_t *q0 = stage + (2 * warp) * rb;                 // gate rows 2w, 2w+1
-    const uint8_t *q1 = stage + (kGuPairs + 2 * warp) * rb;      // up rows
-    const uint16_t *s0 = reinterpret_cast<const uint16_t *>(stage + 2 * kGuPairs * rb) + (2 * warp) * nsc;
-    const uint16_t *s1 = s0 + kGuPairs * nsc;
-    const int i0 = tile * kGuPairs + 2 * warp;
-    for (int n = 0; n < st.count[a]; ++n) {
-        int tok, row;
-        slot_entry(p, st, a, n, tok, row);
-        const int key = tok * 16 + BITS;
-        if (key != act_key) {
-            load_act_bf16<BITS, UPL>(p.x + static_cast<size_t>(tok) * H, H, lane, act);
-            act_key = key;
-        }
-        float v[4] = {0.f, 0.f, 0.f, 0.f};  // g(i0), g(i0+1), u(i0), u(i0+1)
-#pragma unroll
-        for (int j = 0; j < UPL; ++j) {
-            const int un = lane + 32 * j;
-            if (un < U) {
-                v[0] += unit_dot<BITS>(q0, s0, H, un, act + W * j);
-                v[1] += unit_dot<BITS>(q0 + rb, s0 + nsc, H, un, act + W * j);
-                v[2] += unit_dot<BITS>(q1, s1, H, un, act + W * j);
-                v[3] += unit_dot<BITS>(q1 + rb, s1 + nsc, H, un, act + W * j);
-            }
-        }
-        // lane l ends with value (l / 8) % 4: lanes 0 and 8 hold the two gates,
-        // 16 and 24 the two ups
-        const float r = transpose_reduce<4>(v);
-        const float up = __shfl_down_sync(0xffffffffu, r, 16);
-        if (lane == 0 || lane == 8) {
-            const int i = i0 + (lane >> 3);
-            p.h[static_cast<size_t>(row) * I + i] = r / (1.0f + expf(-r)) * up;
-        }
-    }
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
-// down tile: warp w computes rows 64*tile + 8*w + r (r < 8) for every token.
-template <int BITS, int UPL>
-__device__ __forceinline__ void consume_dn(const FfnParams &p, const SlotTabs &st, int a, int tile,
-                                           const uint8_t *stage, float *act, int &act_key) {
-    const int H = p.w.H, I = p.w.I;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int W = UnitW<BITS>::W;
-    const int U = I / W;
-    const int rb = row_bytes(I, BITS);
-    const uint16_t *sc = reinterpret_cast<const uint16_t *>(stage + kDnRows * rb);
-    constexpr int R = kDnRows / kConsumerWarps;
-    for (int n = 0; n < st.count[a]; ++n) {
-        int tok, row;
-        slot_entry(p, st, a, n, tok, row);
-        const int key = -(row * 16 + BITS) - 2;
-        if (key != act_key) {
-            load_act_f32<BITS, UPL>(p.h + static_cast<size_t>(row) * I, I, lane, act);
-            act_key = key;
-        }
-        float acc[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int lr = warp * R + r;
-            float v = 0.f;
-#pragma unroll
-            for (int j = 0; j < UPL; ++j) {
-                const int un = lane + 32 * j;
-                if (un < U) v += unit_dot<BITS>(stage + lr * rb, sc + lr * (I / 32), I, un, act + W * j);
-            }
-            acc[r] = v;
-        }
-        // lane l ends with the full sum of row (l / 4) % 8
-        const float res = transpose_reduce<R>(acc);
-        float *dst = row >= p.T * p.k ? p.y_shared + static_cast<size_t>(row - p.T * p.k) * H
-                                      : p.y_slots + static_cast<size_t>(row) * H;
-        if ((lane & 3) == 0) dst[tile * kDnRows + warp * R + (lane >> 2)] = res;
-    }
-}
-
-__device__ __forceinline__ int upl_of(int K, int bits) {
-    const int W = bits == 8 ? 16 : (bits == 4 ? 32 : 64);
-    const int U = K / W;
-    return (U + 31) / 32;
-}
-
-__device__ __forceinline__ void consume_tile(const FfnParams &p, const SlotTabs &st, int phase, int a, int tile,
-                             const uint8_t *stage, float *act, int &act_key) {
-    const int bits = st.bits[a];
-    if (phase == 0) {
-        const int upl = upl_of(p.w.H, bits);
-        if (bits == 8) {
-            if (upl <= 1) consume_gu<8, 1>(p, st, a, tile, stage, act, act_key);
-            else if (upl <= 2) consume_gu<8, 2>(p, st, a, tile, stage, act, act_key);
-            else consume_gu<8, 4>(p, st, a, tile, stage, act, act_key);
-        } else if (bits == 4) {
-            if (upl <= 1) consume_gu<4, 1>(p, st, a, tile, stage, act, act_key);
-            else consume_gu<4, 2>(p, st, a, tile, stage, act, act_key);
-        } else {
-            consume_gu<3, 1>(p, st, a, tile, stage, act, act_key);
-        }
+template <int BITS>
+__device__ __forceinline__ void dequant8(const uint8_t *row, int K, int b, int t, uint32_t (&P)[4]) {
+    if constexpr (BITS == 8) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(row + 32 * b + 8 * t);
+        const uint32_t u0 = w.x ^ 0x80808080u, u1 = w.y ^ 0x80808080u;  // c = q + 128
+        constexpr uint32_t kBias = 0x64806480u;                         // 1024 + 128
+        P[0] = hsub2(prmt(u0, 0x64646464u, 0x4140u), kBias);
+        P[1] = hsub2(prmt(u0, 0x64646464u, 0x4342u), kBias);
+        P[2] = hsub2(prmt(u1, 0x64646464u, 0x4140u), kBias);
+        P[3] = hsub2(prmt(u1, 0x64646464u, 0x4342u), kBias);
+    } else if constexpr (BITS == 4) {
+        // nibble i of the word at byte 16b + 4t is weight 8t + i (c = q + 8)
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(row + 16 * b + 4 * t);
+        const uint32_t v8 = v >> 8;
+        P[0] = hsub2((v & 0x000F000Fu) | 0x64006400u, 0x64086408u);   // 1024 + c - 1032
+        P[1] = hsub2((v & 0x00F000F0u) | 0x54005400u, 0x54805480u);   // 64 + c - 72
+        P[2] = hsub2((v8 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
+        P[3] = hsub2((v8 & 0x00F000F0u) | 0x54005400u, 0x54805480u);
     } else {
-        const int upl = upl_of(p.w.I, bits);
-        if (bits == 8) {
-            if (upl <= 1) consume_dn<8, 1>(p, st, a, tile, stage, act, act_key);
-            else if (upl <= 2) consume_dn<8, 2>(p, st, a, tile, stage, act, act_key);
-            else consume_dn<8, 4>(p, st, a, tile, stage, act, act_key);
-        } else if (bits == 4) {
-            if (upl <= 1) consume_dn<4, 1>(p, st, a, tile, stage, act, act_key);
-            else consume_dn<4, 2>(p, st, a, tile, stage, act, act_key);
-        } else {
-            consume_dn<3, 1>(p, st, a, tile, stage, act, act_key);
+        // low plane: bits 0-1 of weight 8t+i at bit 2i of the u16 at byte 8b+2t;
+        // high plane: bit 2 at bit i of byte K/4 + 4b + t (c = q + 4)
+        const uint32_t lo16 = *reinterpret_cast<const uint16_t *>(row + 8 * b + 2 * t);
+        const uint32_t hb = row[K / 4 + 4 * b + t];
+        const uint32_t X = prmt(lo16, 0u, 0x4140u);  // weights i and i+4 16 bits apart
+        const uint32_t Y = hb * 0x4004u;             // hb << 2 | hb << 14
+        P[0] = hsub2((X & 0x00030003u) | (Y & 0x00040004u) | 0x64006400u, 0x64046404u);           // 1024 + c - 1028
+        P[1] = hsub2((X & 0x000C000Cu) | ((Y << 1) & 0x00100010u) | 0x5C005C00u, 0x5C105C10u);  // 256 + c - 260
+        P[2] = hsub2((X & 0x00300030u) | ((Y << 2) & 0x00400040u) | 0x54005400u, 0x54405440u);  // 64 + c - 68
+        P[3] = hsub2((X & 0x00C000C0u) | ((Y << 3) & 0x01000100u) | 0x4C004C00u, 0x4D004D00u);  // 16 + c - 20
+    }
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// D = A B + D on one m16n8k16 tile (fp16 inputs, fp32 accumulation).
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float2 half2_to_float2(uint32_t v) {
+    return __half22float2(*reinterpret_cast<const __half2 *>(&v));
+}
+
+// One warp's share of a tile: stage rows rA (accumulator rows g) and rB (rows
+// g + 8), blocks [b0, b1), NT n-tiles of 8 columns.  acc[nt] follows the m16n8
+// accumulator layout: (row g, col 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
+template <int BITS, int NT>
+__device__ __forceinline__ void warp_tile(const uint8_t *stage, const Geo &G, int rA, int rB, int b0, int b1,
+                                          const uint8_t *xf, int cs, int ncol0, int ncol1, float (&acc)[2][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint8_t *qa = stage + rA * G.rs;
+    const uint8_t *qb = stage + rB * G.rs;
+    const uint8_t *sa = stage + G.rows * G.rs + rA * G.ss;
+    const uint8_t *sbr = stage + G.rows * G.rs + rB * G.ss;
+    const uint8_t *xg = xf + g * cs + t * 16;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+#pragma unroll 2
+    for (int b = b0; b < b1; b += 2) {
+        const float2 da = half2_to_float2(*reinterpret_cast<const uint32_t *>(sa + 2 * b));
+        const float2 db = half2_to_float2(*reinterpret_cast<const uint32_t *>(sbr + 2 * b));
+        uint32_t PA[2][4], PB[2][4];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+            dequant8<BITS>(qa, G.K, b + bb, t, PA[bb]);
+            dequant8<BITS>(qb, G.K, b + bb, t, PB[bb]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            uint4 X[2];
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                X[bb] = make_uint4(0u, 0u, 0u, 0u);
+                if (g < (nt == 0 ? ncol0 : ncol1))
+                    X[bb] = *reinterpret_cast<const uint4 *>(xg + nt * 8 * cs + (b + bb) * 64);
+            }
+            // four independent products: two k16 halves of two blocks
+            float c[4][4] = {};
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                mma16816(c[2 * bb], PA[bb][0], PB[bb][0], PA[bb][1], PB[bb][1], X[bb].x, X[bb].y);
+                mma16816(c[2 * bb + 1], PA[bb][2], PB[bb][2], PA[bb][3], PB[bb][3], X[bb].z, X[bb].w);
+            }
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                const float dA = bb ? da.y : da.x, dB = bb ? db.y : db.x;
+                acc[nt][0] = fmaf(dA, c[2 * bb][0] + c[2 * bb + 1][0], acc[nt][0]);
+                acc[nt][1] = fmaf(dA, c[2 * bb][1] + c[2 * bb + 1][1], acc[nt][1]);
+                acc[nt][2] = fmaf(dB, c[2 * bb][2] + c[2 * bb + 1][2], acc[nt][2]);
+                acc[nt][3] = fmaf(dB, c[2 * bb][3] + c[2 * bb + 1][3], acc[nt][3]);
+            }
         }
     }
+}
+
+// fp32 -> fp16 bits, noting values outside the fp16 range (or NaN)
+__device__ __forceinline__ uint16_t to_f16(float v, bool &bad) {
+    bad |= !(fabsf(v) <= 65504.f);
+    return __half_as_ushort(__float2half_rn(v));
+}
+
+__device__ __forceinline__ uint32_t pack_h2(uint16_t lo, uint16_t hi) {
+    return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// 8 consecutive values of a block (weights 8t .. 8t+7) in the pair order of
+// the codes, as 4 half2.
+__device__ __forceinline__ uint4 pack_frag(const uint16_t (&v)[8], int bits) {
+    uint4 r;
+    if (bits == 8) {
+        r.x = pack_h2(v[0], v[1]);
+        r.y = pack_h2(v[2], v[3]);
+        r.z = pack_h2(v[4], v[5]);
+        r.w = pack_h2(v[6], v[7]);
+    } else {
+        r.x = pack_h2(v[0], v[4]);
+        r.y = pack_h2(v[1], v[5]);
+        r.z = pack_h2(v[2], v[6]);
+        r.w = pack_h2(v[3], v[7]);
+    }
+    return r;
 }
 
 struct StreamSmem {
     uint8_t *stages;
-    uint64_t *full, *empty;
-    SlotTabs st;
+    uint8_t *xf;
+    float4 *red;
+    uint64_t *full, *empty;  // per stage: copies landed / stage consumed
     int *abort;
+    SlotTabs st;
+    Sched sc;
+    int *tier, *jloc;   // per slot: shelf index (n_tiers = shared) and index within the shelf
+    TierPtrs *tp;       // [MOE_MAX_TIERS + 1]
+    Geo *geo;           // [phase][8-, 4-, 3-bit]
 };
 
-// The persistent FFN kernel body; `n_slots` slots are described in st.
-__device__ __forceinline__ void ffn_stream_body(const FfnParams &p, StreamSmem &S, int n_slots, int nstages,
-                                int stage_bytes) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ int bits_idx(int bits) { return bits == 8 ? 0 : (bits == 4 ? 1 : 2); }
+
+// Stage the codes and scales of tile (phase, a, tile) into `dst`: producer
+// thread pt of kProducers copies its share of 16-byte chunks.
+__device__ __forceinline__ void issue_tile(const FfnParams &p, const StreamSmem &S, int phase, int a, int tile,
+                                           uint8_t *dst, int pt) {
     const int H = p.w.H, I = p.w.I;
-    if (warp == kConsumerWarps) {
-        // producer: one elected lane issues the bulk copies
-        if (lane != 0) return;
-        int i = 0;
-        for_each_tile(p, S.st, n_slots, [&](int phase, int a, int tile) {
-            if (*static_cast<volatile int *>(S.abort)) return;
-            const int s = i % nstages;
-            const uint32_t par = ((i / nstages) & 1) ^ 1;
-            if (!mbar_wait(&S.empty[s], par)) {
-                status_or(p.status, MOE_STATUS_TIMEOUT);
-                *static_cast<volatile int *>(S.abort) = 1;
-                return;
-            }
-            uint8_t *dst = S.stages + static_cast<size_t>(s) * stage_bytes;
-            const ExpertPtrs e = expert_ptrs(p, S.st.expert[a]);
-            const int bits = S.st.bits[a];
-            if (phase == 0) {
-                const int rb = row_bytes(H, bits);
-                const size_t r0 = static_cast<size_t>(tile) * kGuPairs;
-                const uint32_t qb = kGuPairs * rb, sb = kGuPairs * (H / 16);
-                mbar_expect_tx(&S.full[s], 2 * qb + 2 * sb);
-                bulk_g2s(dst, e.gq + r0 * rb, qb, &S.full[s]);
-                bulk_g2s(dst + qb, e.gq + (I + r0) * rb, qb, &S.full[s]);
-                bulk_g2s(dst + 2 * qb, e.gs + r0 * (H / 32), sb, &S.full[s]);
-                bulk_g2s(dst + 2 * qb + sb, e.gs + (I + r0) * (H / 32), sb, &S.full[s]);
-            } else {
-                const int rb = row_bytes(I, bits);
-                const size_t r0 = static_cast<size_t>(tile) * kDnRows;
-                const uint32_t qb = kDnRows * rb, sb = kDnRows * (I / 16);
-                mbar_expect_tx(&S.full[s], qb + sb);
-                bulk_g2s(dst, e.dq + r0 * rb, qb, &S.full[s]);
-                bulk_g2s(dst + qb, e.ds + r0 * (I / 32), sb, &S.full[s]);
-            }
-            ++i;
-        });
-        // drain: the last stages this thread filled must have landed before exit
-        for (int j = i - nstages < 0 ? 0 : i - nstages; j < i; ++j)
-            if (!mbar_wait(&S.full[j % nstages], (j / nstages) & 1)) status_or(p.status, MOE_STATUS_TIMEOUT);
-        return;
+    const int bits = S.st.bits[a];
+    const Geo &G = S.geo[phase * 3 + bits_idx(bits)];
+    const TierPtrs &T = S.tp[S.tier[a]];
+    const size_t j = static_cast<size_t>(S.jloc[a]);
+    const uint8_t *q, *sc;
+    size_t r_first, r_second;  // first matrix row of the tile's two row groups
+    int half;                  // rows in the first group
+    if (phase == 0) {
+        q = T.gq + j * 2 * I * G.rb;
+        sc = T.gs + j * 2 * I * G.sb;
+        r_first = static_cast<size_t>(tile) * 8 * G.R;  // gate pairs ...
+        r_second = I + r_first;                          // ... and their up rows
+        half = 8 * G.R;
+    } else {
+        q = T.dq + j * H * G.rb;
+        sc = T.ds + j * H * G.sb;
+        r_first = static_cast<size_t>(tile) * G.rows;
+        r_second = r_first + 8 * G.R;  // the same rows, contiguous
+        half = 8 * G.R;
     }
-    // consumers
-    float act[64];
-    int act_key = -1;
-    int i = 0;
-    // h of a slot is published (fence + count) once per warp when the warp
-    // leaves that slot: the count target is (gate_up tiles) x (consumer warps)
-    // contributions, each contribution counting its tiles.
-    int pend_slot = -1, pend_tiles = 0;
-    const int gu_done = (I / kGuPairs) * kConsumerWarps;
-    auto publish = [&]() {
-        if (pend_slot >= 0) {
-            __syncwarp();
-            if (lane == 0 || lane == 8) __threadfence();  // the two lanes that wrote h
-            __syncwarp();
-            if (lane == 0) atomicAdd(p.ctr + pend_slot, pend_tiles);
+    // codes: rows of rb bytes, cpr 16-byte chunks each; rps rows per sweep
+    {
+        const int cpr = G.rb / 16;
+        if (cpr >= kProducers) {
+            for (int r = 0; r < G.rows; ++r) {
+                const size_t mr = r < half ? r_first + r : r_second + (r - half);
+                for (int off = pt * 16; off < G.rb; off += kProducers * 16)
+                    cp_async16(dst + r * G.rs + off, q + mr * G.rb + off);
+            }
+        } else {
+            const int rps = kProducers / cpr;
+            const int r0 = pt / cpr, off = (pt - r0 * cpr) * 16;
+            if (r0 < rps)
+                for (int r = r0; r < G.rows; r += rps) {
+                    const size_t mr = r < half ? r_first + r : r_second + (r - half);
+                    cp_async16(dst + r * G.rs + off, q + mr * G.rb + off);
+                }
         }
-        pend_slot = -1;
-        pend_tiles = 0;
-    };
-    for_each_tile(p, S.st, n_slots, [&](int phase, int a, int tile) {
-        if (*static_cast<volatile int *>(S.abort)) return;
-        if (phase == 0 && a != pend_slot) publish();
-        if (phase == 1 && pend_slot >= 0) publish();
-        const int s = i % nstages;
-        const uint32_t par = (i / nstages) & 1;
-        bool ok = mbar_wait(&S.full[s], par);
-        if (phase == 1) {
-            int dep = 1;
-            if (lane == 0) dep = wait_geq(p.ctr + a, gu_done) ? 1 : 0;  // this expert's h is complete
-            ok = ok && __shfl_sync(0xffffffffu, dep, 0);
+    }
+    // scales: per row (padded stride) or each group of rows in one piece
+    uint8_t *dsc = dst + G.rows * G.rs;
+    if (G.row_scales) {
+        const int cpr = G.sb / 16, rps = kProducers / cpr;  // sb <= 128: cpr <= 8
+        const int r0 = pt / cpr, off = (pt - r0 * cpr) * 16;
+        if (r0 < rps)
+            for (int r = r0; r < G.rows; r += rps) {
+                const size_t mr = r < half ? r_first + r : r_second + (r - half);
+                cp_async16(dsc + r * G.ss + off, sc + mr * G.sb + off);
+            }
+    } else {
+        const int n = half * G.sb / 16;  // chunks per group
+        for (int c = pt; c < 2 * n; c += kProducers) {
+            const int grp = c >= n, cc = c - grp * n;
+            const size_t src = (grp ? r_second : r_first) * G.sb + cc * 16;
+            cp_async16(dsc + grp * half * G.sb + cc * 16, sc + src);
         }
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) {
-            if (lane == 0) status_or(p.status, MOE_STATUS_TIMEOUT);
-            *static_cast<volatile int *>(S.abort) = 1;
-            return;
-        }
-        consume_tile(p, S.st, phase, a, tile, S.stages + static_cast<size_t>(s) * stage_bytes, act, act_key);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[s]);
-        if (phase == 0) {
-            pend_slot = a;
-            ++pend_tiles;
-        }
-        ++i;
-    });
-    publish();
+    }
 }
 
-__global__ void __launch_bounds__(kStreamThreads, 1)
-ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
+
+// Arrive on bar once all of this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier of the compute warps that also ANDs a flag over them.
+__device__ __forceinline__ bool bar_and(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(ok ? 1u : 0u), "n"(kBarCompute), "n"(kThreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void bar_compute() { named_bar_sync(kBarCompute, kThreads); }
+
+
+// gate_up fragments of one pass: column n holds the token of entry pass*8 + n.
+__device__ __forceinline__ void build_xf_gu(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
+                                            int bits, uint8_t *xf, bool &bad) {
+    const int H = p.w.H, nb = H / 32, cs = xf_col_stride(H);
+    const int n_chunks = ntok * nb * 4;
+    for (int i = threadIdx.x; i < n_chunks; i += kThreads) {
+        const int n = i / (nb * 4), rem = i % (nb * 4);  // rem = 4 * block + t
+        int tok, row;
+        slot_entry(p, st, a, pass * kTokPerPass + n, tok, row);
+        const uint4 q = *reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(tok) * H + 8 * rem);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        uint16_t v[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[2 * j] = to_f16(bf16lo(w[j]), bad);
+            v[2 * j + 1] = to_f16(bf16hi(w[j]), bad);
+        }
+        *reinterpret_cast<uint4 *>(xf + n * cs + rem * 16) = pack_frag(v, bits);
+    }
+}
+
+// down fragments of one pass: in n-tile nt, column 2m holds hi and column
+// 2m + 1 lo of h for the token of entry pass*tp + 4nt + m.
+__device__ __forceinline__ void build_xf_dn(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
+                                            int bits, uint8_t *xf, bool &bad) {
+    const int I = p.w.I, nb = I / 32, cs = xf_col_stride(I);
+    const int tp = tokens_per_pass(1, I);
+    const int n_chunks = ntok * nb * 4;
+    for (int i = threadIdx.x; i < n_chunks; i += kThreads) {
+        const int n = i / (nb * 4), rem = i % (nb * 4);
+        int tok, row;
+        slot_entry(p, st, a, pass * tp + n, tok, row);
+        const float *src = p.h + static_cast<size_t>(row) * I + 8 * rem;
+        const float4 f0 = __ldcg(reinterpret_cast<const float4 *>(src));
+        const float4 f1 = __ldcg(reinterpret_cast<const float4 *>(src + 4));
+        const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+        uint16_t hi[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            hi[j] = to_f16(f[j], bad);
+            lo[j] = __half_as_ushort(__float2half_rn(f[j] - __half2float(__ushort_as_half(hi[j]))));
+        }
+        const int col = (n >> 2) * 8 + 2 * (n & 3);
+        *reinterpret_cast<uint4 *>(xf + col * cs + rem * 16) = pack_frag(hi, bits);
+        *reinterpret_cast<uint4 *>(xf + (col + 1) * cs + rem * 16) = pack_frag(lo, bits);
+    }
+}
+
+// This warp's partial sums of the resident tile, to red[warp][lane].
+template <int BITS>
+__device__ __forceinline__ void compute_tile(const FfnParams &p, const Geo &G, int phase, const uint8_t *stage,
+                                             const uint8_t *xf, int ntok, float4 *red) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = warp % G.R, s = warp / G.R;
+    const int b0 = min(G.nb, s * G.bps), b1 = min(G.nb, (s + 1) * G.bps);
+    const int cs = xf_col_stride(G.K);
+    const int g = lane >> 2;
+    float acc[2][4];
+    if (phase == 0) {
+        warp_tile<BITS, 1>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs, ntok, 0, acc);
+        red[warp * 32 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+    } else {
+        const int nc0 = 2 * max(0, min(4, ntok)), nc1 = 2 * max(0, min(4, ntok - 4));
+        if (down_ntiles(p.w.I) == 2)
+            warp_tile<BITS, 2>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1, acc);
+        else
+            warp_tile<BITS, 1>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1, acc);
+        // hi + lo columns of each token
+        red[warp * 32 + lane] =
+            make_float4(acc[0][0] + acc[0][1], acc[0][2] + acc[0][3], acc[1][0] + acc[1][1], acc[1][2] + acc[1][3]);
+    }
+}
+
+// K slices summed in a fixed order; gate_up -> h = silu(g) * u, down -> y.
+__device__ __forceinline__ void epilogue(const FfnParams &p, const SlotTabs &st, int phase, int a, int tile,
+                                         int pass, int ntok, const float4 *red) {
+    const int K = phase == 0 ? p.w.H : p.w.I;
+    const int R = rows_pow2(K), S = kWarps / R;
+    const float *rf = reinterpret_cast<const float *>(red);
+    if (phase == 0) {
+        const int I = p.w.I;
+        const int n_out = R * 8 * ntok;
+        for (int o = threadIdx.x; o < n_out; o += kThreads) {
+            const int n = o % ntok, rg = o / ntok, g = rg % 8, r = rg / 8;
+            const int lane = 4 * g + (n >> 1), sub = n & 1;
+            float gate = 0.f, up = 0.f;
+            for (int s = 0; s < S; ++s) {
+                const float *v = rf + ((r + R * s) * 32 + lane) * 4;
+                gate += v[sub];
+                up += v[2 + sub];
+            }
+            int tok, row;
+            slot_entry(p, st, a, pass * kTokPerPass + n, tok, row);
+            p.h[static_cast<size_t>(row) * I + tile * 8 * R + 8 * r + g] = gate / (1.0f + expf(-gate)) * up;
+        }
+    } else {
+        const int H = p.w.H, tp = tokens_per_pass(1, p.w.I);
+        const int n_out = R * 16 * ntok;
+        for (int o = threadIdx.x; o < n_out; o += kThreads) {
+            const int rr = o % (R * 16), n = o / (R * 16);
+            const int r = rr / 16, row16 = rr % 16;
+            const int lane = 4 * (row16 % 8) + (n & 3), idx = 2 * (n >> 2) + row16 / 8;
+            float v = 0.f;
+            for (int s = 0; s < S; ++s) v += rf[((r + R * s) * 32 + lane) * 4 + idx];
+            int tok, row;
+            slot_entry(p, st, a, pass * tp + n, tok, row);
+            float *dst = row >= p.T * p.k ? p.y_shared + static_cast<size_t>(row - p.T * p.k) * H
+                                          : p.y_slots + static_cast<size_t>(row) * H;
+            dst[tile * 16 * R + rr] = v;
+        }
+    }
+}
+
+// The persistent FFN kernel body; `n_slots` slots are described in S.
+__device__ __forceinline__ void ffn_stream_body(const FfnParams &p, StreamSmem &S, int n_slots, int nstages) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int I = p.w.I;
+    if (warp >= kWarps) {
+        // producer warps: stage the CTA's tiles in order; every producer
+        // thread arrives on the stage's full barrier once its copies landed
+        const int pt = threadIdx.x - kThreads;
+        TileIt pf;
+        it_begin(p, S.sc, n_slots, pf);
+        for (int i = 0; pf.phase < 2; ++i, it_next(p, S.sc, n_slots, pf)) {
+            if (*static_cast<volatile int *>(S.abort)) break;
+            const int s = i % nstages;
+            if (!mbar_wait(&S.empty[s], ((i / nstages) & 1) ^ 1)) {
+                status_or(p.status, MOE_STATUS_TIMEOUT);
+                *static_cast<volatile int *>(S.abort) = 1;
+                break;
+            }
+            issue_tile(p, S, pf.phase, pf.a, pf.b, S.stages + static_cast<size_t>(s) * kStageBytes, pt);
+            cp_async_arrive(&S.full[s]);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
+    // compute warps: every branch below depends only on values that are the
+    // same in all of them, so they pass the same barriers in the same order
+    const int gu_tiles = tiles_per_slot(p, 0);
+    TileIt it;
+    it_begin(p, S.sc, n_slots, it);
+    int xf_key = -1;      // (slot, phase, pass) whose fragments xf holds
+    int ready_slot = -1;  // a slot whose h is known to be complete
+    int pend_tiles = 0;   // gate_up tiles of the current slot not yet counted
+    bool bad = false;
+    for (int i = 0; it.phase < 2; ++i) {
+        const int phase = it.phase, a = it.a, tile = it.b;
+        const int s = i % nstages;
+        bool ok = mbar_wait(&S.full[s], (i / nstages) & 1);
+        // one thread polls the slot's gate_up count (with backoff, so that
+        // pollers do not crowd the counters' L2 slice); the barrier passes
+        // the result on and orders every thread's reads of h after it
+        if (phase == 1 && a != ready_slot && threadIdx.x == 0) ok = ok && wait_geq_backoff(p.ctr + a, gu_tiles);
+        if (!bar_and(ok)) {
+            if (threadIdx.x == 0) {
+                status_or(p.status, MOE_STATUS_TIMEOUT);
+                *static_cast<volatile int *>(S.abort) = 1;
+            }
+            break;
+        }
+        if (phase == 1) ready_slot = a;
+        const uint8_t *stage = S.stages + static_cast<size_t>(s) * kStageBytes;
+        const int bits = S.st.bits[a], cnt = S.st.count[a];
+        const Geo &G = S.geo[phase * 3 + bits_idx(bits)];
+        const int tp = tokens_per_pass(phase, I);
+        const int np = (cnt + tp - 1) / tp;
+        for (int pass = 0; pass < np; ++pass) {
+            const int ntok = min(tp, cnt - pass * tp);
+            const int key = (a * 2 + phase) * 65536 + pass;
+            if (key != xf_key) {  // the last readers of xf passed a barrier since
+                if (phase == 0)
+                    build_xf_gu(p, S.st, a, pass, ntok, bits, S.xf, bad);
+                else
+                    build_xf_dn(p, S.st, a, pass, ntok, bits, S.xf, bad);
+                xf_key = key;
+                bar_compute();
+            }
+            if (bits == 8)
+                compute_tile<8>(p, G, phase, stage, S.xf, ntok, S.red);
+            else if (bits == 4)
+                compute_tile<4>(p, G, phase, stage, S.xf, ntok, S.red);
+            else
+                compute_tile<3>(p, G, phase, stage, S.xf, ntok, S.red);
+            if (pass == np - 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.empty[s]);  // this warp is done with the stage
+            }
+            bar_compute();
+            epilogue(p, S.st, phase, a, tile, pass, ntok, S.red);
+            if (pass + 1 < np) bar_compute();  // red is written again by the next pass
+        }
+        it_next(p, S.sc, n_slots, it);
+        if (phase == 0) {
+            // when this CTA leaves the slot, count its gate_up tiles of it:
+            // after every thread's h writes (barrier) and a fence, and before
+            // this CTA waits on any other slot's count
+            ++pend_tiles;
+            if (it.phase != 0 || it.a != a) {
+                bar_compute();
+                if (threadIdx.x == 0) {
+                    __threadfence();
+                    atomicAdd(p.ctr + a, pend_tiles);
+                }
+                pend_tiles = 0;
+            }
+        }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(p.status, MOE_STATUS_FP16_RANGE);
+}
+
+__global__ void __launch_bounds__(kBlockThreads, 1)
+ffn_stream_kernel(const FfnParams p, int nstages) {
     extern __shared__ __align__(1024) uint8_t smem[];
     StreamSmem S;
     S.stages = smem;
-    uint8_t *tail = smem + static_cast<size_t>(nstages) * stage_bytes;
-    S.full = reinterpret_cast<uint64_t *>(tail);
+    S.xf = smem + static_cast<size_t>(nstages) * kStageBytes;
+    S.red = reinterpret_cast<float4 *>(S.xf + xf_bytes(p.w.H, p.w.I));
+    S.full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(S.red) + kRedBytes);
     S.empty = S.full + kMaxStages;
-    S.abort = reinterpret_cast<int *>(S.empty + kMaxStages);
-    int *tabs = S.abort + 4;
+    S.tp = reinterpret_cast<TierPtrs *>(S.empty + kMaxStages);
+    S.geo = reinterpret_cast<Geo *>(S.tp + MOE_MAX_TIERS + 1);
+    S.abort = reinterpret_cast<int *>(S.geo + 6);
+    int *tabs = S.abort + 2;
     const int max_slots = p.max_active + 1;
     S.st.expert = tabs;
     S.st.bits = tabs + max_slots;
     S.st.count = tabs + 2 * max_slots;
     S.st.first = tabs + 3 * max_slots;
+    S.tier = tabs + 4 * max_slots;
+    S.jloc = tabs + 5 * max_slots;
     // entry tables in shared memory when they fit, else read from global
     const int n_ent = p.T * p.k + p.T;
     const bool ent_smem = n_ent <= kMaxSmemEntries;
-    S.st.tok = ent_smem ? tabs + 4 * max_slots : nullptr;
+    S.st.tok = ent_smem ? tabs + 6 * max_slots : nullptr;
     S.st.row = ent_smem ? S.st.tok + n_ent : nullptr;
-    // slot table: active routed experts with work for this path (compacted),
-    // then the shared expert
-    __shared__ int n_keep;
-    if (threadIdx.x == 0) n_keep = 0;
-    __syncthreads();
-    const int n_active_all = min(p.active[0], p.max_active);
-    for (int a0 = 0; a0 < n_active_all; a0 += blockDim.x) {
-        const int a = a0 + threadIdx.x;
-        int e = -1, f = 0, cnt = 0;
-        if (a < n_active_all) {
-            e = p.active[1 + a];
-            if (e >= 0 && e < p.E) {
-                f = p.offsets[e];
-                cnt = p.offsets[e + 1] - f;
-            }
-        }
-        const bool keep = a < n_active_all && e >= 0 && e < p.E && cnt > 0 && cnt <= p.max_count;
-        // order-preserving compaction within this block-wide step
-        const unsigned m = __ballot_sync(0xffffffffu, keep);
-        __shared__ int warp_base[kStreamThreads / 32];
-        if ((threadIdx.x & 31) == 0) warp_base[threadIdx.x >> 5] = __popc(m);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int run = n_keep;
-            for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
-                const int c = warp_base[w];
-                warp_base[w] = run;
-                run += c;
-            }
-            n_keep = run;
-        }
-        __syncthreads();
-        if (keep) {
-            const int pos = warp_base[threadIdx.x >> 5] + __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
-            S.st.expert[pos] = e;
-            S.st.bits[pos] = expert_bits(p, e);
-            S.st.first[pos] = f;
-            S.st.count[pos] = cnt;
-        }
-        __syncthreads();
-    }
-    const int n_active = n_keep;
-    // entries: routed slots in sorted order (first = expert offset), then the
-    // shared expert's T tokens at [T*k, T*k + T)
+    // 8-byte aligned: every table before it has an even number of ints
+    long long *sched = reinterpret_cast<long long *>(tabs + 6 * max_slots + (ent_smem ? 2 * n_ent : 0));
+    S.sc.tc0 = sched;
+    S.sc.tc1 = sched + max_slots;
+    S.sc.pre0 = sched + 2 * max_slots;
+    S.sc.pre1 = sched + 3 * max_slots;
+    // copies of the routing tables: active list and expert offsets
+    int *act_s = reinterpret_cast<int *>(sched + 4 * max_slots);
+    int *off_s = act_s + max_slots;
+    // one round of independent global loads fills every table below
     const int S_ = p.T * p.k;
-    const int n_routed = min(p.offsets[p.E], S_);
+    for (int i = threadIdx.x; i < max_slots; i += blockDim.x) act_s[i] = p.active[i];
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) off_s[e] = p.offsets[e];
     if (ent_smem) {
-        for (int j = threadIdx.x; j < n_routed; j += blockDim.x) {
+        for (int j = threadIdx.x; j < S_; j += blockDim.x) {
             const int sl = p.sorted[j];
             const bool okj = sl >= 0 && sl < S_;
             S.st.tok[j] = okj ? sl / p.k : 0;
@@ -568,41 +758,143 @@ ffn_stream_kernel(const FfnParams p, int nstages, int stage_bytes) {
             S.st.row[S_ + t] = S_ + t;
         }
     }
+    // shelf table pointers (constant-index reads of the parameters), tile
+    // geometry of each phase and precision, and the stage barriers
     if (threadIdx.x == 0) {
-        if (p.has_shared && p.T <= p.max_count) {
-            S.st.expert[n_active] = p.E;
-            S.st.bits[n_active] = p.w.shared.bits;
-            S.st.first[n_active] = S_;
-            S.st.count[n_active] = p.T;
+#pragma unroll
+        for (int t = 0; t < MOE_MAX_TIERS; ++t) {
+            if (t < p.w.n_tiers) {
+                S.tp[t].gq = p.w.tiers[t].gu_qs;
+                S.tp[t].gs = reinterpret_cast<const uint8_t *>(p.w.tiers[t].gu_scale);
+                S.tp[t].dq = p.w.tiers[t].dn_qs;
+                S.tp[t].ds = reinterpret_cast<const uint8_t *>(p.w.tiers[t].dn_scale);
+                S.tp[t].bits = p.w.tiers[t].bits;
+                S.tp[t].first = p.w.tiers[t].first_expert;
+                S.tp[t].n = p.w.tiers[t].n_experts;
+            }
         }
-        for (int s = 0; s < nstages; ++s) {
-            mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], kConsumerWarps);
+        const int t = p.w.n_tiers;
+        S.tp[t].gq = p.w.shared.gu_qs;
+        S.tp[t].gs = reinterpret_cast<const uint8_t *>(p.w.shared.gu_scale);
+        S.tp[t].dq = p.w.shared.dn_qs;
+        S.tp[t].ds = reinterpret_cast<const uint8_t *>(p.w.shared.dn_scale);
+        S.tp[t].bits = p.w.shared.bits;
+        S.tp[t].first = p.E;
+        S.tp[t].n = 1;
+        for (int st = 0; st < nstages; ++st) {
+            mbar_init(&S.full[st], kProducers);  // one arrival per producer thread
+            mbar_init(&S.empty[st], kWarps);     // one per compute warp
         }
         *S.abort = 0;
         mbar_fence_init();
     }
+    if (threadIdx.x < 6) {
+        const int phase = threadIdx.x / 3, bi = threadIdx.x % 3;
+        S.geo[threadIdx.x] = geo(phase == 0 ? p.w.H : p.w.I, bi == 0 ? 8 : (bi == 1 ? 4 : 3));
+    }
+    // slot table: active routed experts with work for this path (compacted),
+    // then the shared expert
+    __shared__ int n_keep;
+    __shared__ int warp_base[kBlockThreads / 32];
+    if (threadIdx.x == 0) n_keep = 0;
     __syncthreads();
-    const int n_slots = n_active + (p.has_shared && p.T <= p.max_count ? 1 : 0);
-    ffn_stream_body(p, S, n_slots, nstages, stage_bytes);
+    const int n_active_all = min(act_s[0], p.max_active);
+    for (int a0 = 0; a0 < n_active_all; a0 += blockDim.x) {
+        const int a = a0 + threadIdx.x;
+        int e = -1, f = 0, cnt = 0;
+        if (a < n_active_all) {
+            e = act_s[1 + a];
+            if (e >= 0 && e < p.E) {
+                f = off_s[e];
+                cnt = off_s[e + 1] - f;
+            }
+        }
+        const bool keep = a < n_active_all && e >= 0 && e < p.E && cnt > 0 && cnt <= p.max_count;
+        // order-preserving compaction within this block-wide step
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if ((threadIdx.x & 31) == 0) warp_base[threadIdx.x >> 5] = __popc(m);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int run = n_keep;
+            for (int w = 0; w < kBlockThreads / 32; ++w) {
+                const int c = warp_base[w];
+                warp_base[w] = run;
+                run += c;
+            }
+            n_keep = run;
+        }
+        __syncthreads();
+        if (keep) {
+            const int pos = warp_base[threadIdx.x >> 5] + __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
+            int ti = 0;  // the shelf holding e (shelves cover [0, E) without overlap)
+            for (int t = 0; t < p.w.n_tiers; ++t)
+                if (e >= S.tp[t].first && e - S.tp[t].first < S.tp[t].n) ti = t;
+            S.st.expert[pos] = e;
+            S.st.bits[pos] = S.tp[ti].bits;
+            S.st.first[pos] = f;
+            S.st.count[pos] = cnt;
+            S.tier[pos] = ti;
+            S.jloc[pos] = e - S.tp[ti].first;
+        }
+        __syncthreads();
+    }
+    const int n_active = n_keep;
+    const bool shared_here = p.has_shared && p.T <= p.max_count;
+    if (threadIdx.x == 0 && shared_here) {
+        S.st.expert[n_active] = p.E;
+        S.st.bits[n_active] = p.w.shared.bits;
+        S.st.first[n_active] = S_;
+        S.st.count[n_active] = p.T;
+        S.tier[n_active] = p.w.n_tiers;
+        S.jloc[n_active] = 0;
+    }
+    __syncthreads();
+    const int n_slots = n_active + (shared_here ? 1 : 0);
+    // schedule: tile costs per slot and phase, and their prefix sums (warp 0)
+    for (int a = threadIdx.x; a < n_slots; a += blockDim.x) {
+        S.sc.tc0[a] = tile_cost(p, 0, S.st.bits[a], S.st.count[a]);
+        S.sc.tc1[a] = tile_cost(p, 1, S.st.bits[a], S.st.count[a]);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        for (int phase = 0; phase < 2; ++phase) {
+            const long long nt = tiles_per_slot(p, phase);
+            long long run = 0;
+            for (int a0 = 0; a0 < n_slots; a0 += 32) {
+                const int a = a0 + lane;
+                long long v = a < n_slots ? nt * (phase == 0 ? S.sc.tc0 : S.sc.tc1)[a] : 0;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const long long u = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += u;
+                }
+                if (a < n_slots) (phase == 0 ? S.sc.pre0 : S.sc.pre1)[a] = run + v;
+                run += __shfl_sync(0xffffffffu, v, 31);
+            }
+        }
+    }
+    __syncthreads();
+    ffn_stream_body(p, S, n_slots, nstages);
 }
 
 }  // namespace moe
 
-size_t moe_ffn_stream_smem(int H, int I, int max_slots, int n_ent, int *nstages, int *stage_bytes) {
-    int sb = moe::gu_tile_bytes(H, 8);
-    const int d = moe::dn_tile_bytes(I, 8);
-    if (d > sb) sb = d;
-    sb = (sb + 1023) & ~1023;
+// Shared memory of one CTA: the stage ring, x fragments, K-slice partials,
+// shelf and geometry tables, and the slot/entry/schedule tables.  Returns the
+// byte count and the number of stages that fit in the budget.
+size_t moe_ffn_stream_smem(int H, int I, int max_slots, int n_ent, int *nstages) {
     const size_t ent = n_ent <= moe::kMaxSmemEntries ? 2 * sizeof(int) * static_cast<size_t>(n_ent) : 0;
-    const size_t tail =
-        2 * moe::kMaxStages * sizeof(uint64_t) + 16 + 4 * sizeof(int) * static_cast<size_t>(max_slots) + ent;
+    const size_t fixed = static_cast<size_t>(moe::xf_bytes(H, I)) + moe::kRedBytes +
+                         2 * moe::kMaxStages * sizeof(uint64_t) + (MOE_MAX_TIERS + 1) * sizeof(moe::TierPtrs) +
+                         6 * sizeof(moe::Geo) + 8 + 6 * sizeof(int) * static_cast<size_t>(max_slots) + ent +
+                         4 * sizeof(long long) * static_cast<size_t>(max_slots) +
+                         sizeof(int) * (static_cast<size_t>(max_slots) + MOE_MAX_EXPERTS + 1) + 16;
     const size_t budget = 220 * 1024;
-    int ns = static_cast<int>((budget - tail) / sb);
+    int ns = fixed < budget ? static_cast<int>((budget - fixed) / moe::kStageBytes) : 0;
     if (ns > moe::kMaxStages) ns = moe::kMaxStages;
     *nstages = ns;
-    *stage_bytes = sb;
-    return static_cast<size_t>(ns) * sb + tail;
+    return static_cast<size_t>(ns) * moe::kStageBytes + fixed;
 }
 
 cudaError_t moe_configure_ffn_stream() {
@@ -612,14 +904,13 @@ cudaError_t moe_configure_ffn_stream() {
 }
 
 bool moe_ffn_stream_supported(int H, int I) {
-    return H <= moe::kMaxRegK && I <= moe::kMaxRegK && H % 128 == 0 && I % 128 == 0;
+    return H <= moe::kMaxK && I <= moe::kMaxK && H % 128 == 0 && I % 128 == 0;
 }
 
 // counters (int[max_active + 1]) must be zero on entry; the caller clears them.
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
-    int nstages = 0, stage_bytes = 0;
-    const size_t smem =
-        moe_ffn_stream_smem(p.w.H, p.w.I, p.max_active + 1, p.T * p.k + p.T, &nstages, &stage_bytes);
+    int nstages = 0;
+    const size_t smem = moe_ffn_stream_smem(p.w.H, p.w.I, p.max_active + 1, p.T * p.k + p.T, &nstages);
     if (nstages < 2) return cudaErrorInvalidConfiguration;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -627,7 +918,7 @@ cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
-    cfg.blockDim = dim3(moe::kStreamThreads);
+    cfg.blockDim = dim3(moe::kBlockThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -635,5 +926,5 @@ cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, nstages, stage_bytes);
+    return cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, nstages);
 }

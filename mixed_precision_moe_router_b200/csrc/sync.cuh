@@ -83,6 +83,19 @@ __device__ __forceinline__ bool wait_geq(const int *ctr, int target) {
     return true;
 }
 
+// As wait_geq, sleeping 32 ns, 64 ns, ... up to 1 us between polls.
+__device__ __forceinline__ bool wait_geq_backoff(const int *ctr, int target) {
+    if (ld_acquire(ctr) >= target) return true;
+    const long long t0 = clock64();
+    unsigned ns = 32;
+    while (ld_acquire(ctr) < target) {
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+        __nanosleep(ns);
+        if (ns < 1024) ns *= 2;
+    }
+    return true;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
