@@ -140,14 +140,16 @@ __device__ __forceinline__ int expert_bits(const FfnParams &p, int e) {
     return b;
 }
 
-// Balancing weight of a tile: its bytes plus a per-weight share for the
+// Balancing weight of a tile: a fixed share for the per-tile work (waits,
+// barriers, epilogue), its bytes, and a per-weight share for the
 // dequantise-and-multiply work of each pass (3-bit codes take the most).
+constexpr long long kTileFixedCost = 65536;
 __device__ __forceinline__ long long tile_cost(const FfnParams &p, int phase, int bits, int count) {
     const int K = phase == 0 ? p.w.H : p.w.I;
     const long long rows = 16 * rows_pow2(K);
     const int tp = tokens_per_pass(phase, p.w.I);
     const long long passes = (count + tp - 1) / tp;
-    return rows * (K * bits / 8 + K / 16) + passes * (rows * K / 3) * (bits == 3 ? 3 : 2);
+    return kTileFixedCost + rows * (K * bits / 8 + K / 16) + passes * (rows * K / 3) * (bits == 3 ? 3 : 2);
 }
 
 __device__ __forceinline__ int tiles_per_slot(const FfnParams &p, int phase) {
@@ -792,89 +794,78 @@ ffn_stream_kernel(const FfnParams p, int nstages) {
         const int phase = threadIdx.x / 3, bi = threadIdx.x % 3;
         S.geo[threadIdx.x] = geo(phase == 0 ? p.w.H : p.w.I, bi == 0 ? 8 : (bi == 1 ? 4 : 3));
     }
-    // slot table: active routed experts with work for this path (compacted),
-    // then the shared expert
+    __syncthreads();
+    // slot table: active routed experts with work for this path, compacted in
+    // order by warp 0 (no block-wide barrier per step), then the shared
+    // expert; then the schedule (unit costs and their prefix sums)
     __shared__ int n_keep;
-    __shared__ int warp_base[kBlockThreads / 32];
-    if (threadIdx.x == 0) n_keep = 0;
-    __syncthreads();
-    const int n_active_all = min(act_s[0], p.max_active);
-    for (int a0 = 0; a0 < n_active_all; a0 += blockDim.x) {
-        const int a = a0 + threadIdx.x;
-        int e = -1, f = 0, cnt = 0;
-        if (a < n_active_all) {
-            e = act_s[1 + a];
-            if (e >= 0 && e < p.E) {
-                f = off_s[e];
-                cnt = off_s[e + 1] - f;
-            }
-        }
-        const bool keep = a < n_active_all && e >= 0 && e < p.E && cnt > 0 && cnt <= p.max_count;
-        // order-preserving compaction within this block-wide step
-        const unsigned m = __ballot_sync(0xffffffffu, keep);
-        if ((threadIdx.x & 31) == 0) warp_base[threadIdx.x >> 5] = __popc(m);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int run = n_keep;
-            for (int w = 0; w < kBlockThreads / 32; ++w) {
-                const int c = warp_base[w];
-                warp_base[w] = run;
-                run += c;
-            }
-            n_keep = run;
-        }
-        __syncthreads();
-        if (keep) {
-            const int pos = warp_base[threadIdx.x >> 5] + __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
-            int ti = 0;  // the shelf holding e (shelves cover [0, E) without overlap)
-            for (int t = 0; t < p.w.n_tiers; ++t)
-                if (e >= S.tp[t].first && e - S.tp[t].first < S.tp[t].n) ti = t;
-            S.st.expert[pos] = e;
-            S.st.bits[pos] = S.tp[ti].bits;
-            S.st.first[pos] = f;
-            S.st.count[pos] = cnt;
-            S.tier[pos] = ti;
-            S.jloc[pos] = e - S.tp[ti].first;
-        }
-        __syncthreads();
-    }
-    const int n_active = n_keep;
-    const bool shared_here = p.has_shared && p.T <= p.max_count;
-    if (threadIdx.x == 0 && shared_here) {
-        S.st.expert[n_active] = p.E;
-        S.st.bits[n_active] = p.w.shared.bits;
-        S.st.first[n_active] = S_;
-        S.st.count[n_active] = p.T;
-        S.tier[n_active] = p.w.n_tiers;
-        S.jloc[n_active] = 0;
-    }
-    __syncthreads();
-    const int n_slots = n_active + (shared_here ? 1 : 0);
-    // schedule: tile costs per slot and phase, and their prefix sums (warp 0)
-    for (int a = threadIdx.x; a < n_slots; a += blockDim.x) {
-        S.sc.tc0[a] = tile_cost(p, 0, S.st.bits[a], S.st.count[a]);
-        S.sc.tc1[a] = tile_cost(p, 1, S.st.bits[a], S.st.count[a]);
-    }
-    __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
+        const int n_active_all = min(act_s[0], p.max_active);
+        int run = 0;
+        for (int a0 = 0; a0 < n_active_all; a0 += 32) {
+            const int a = a0 + lane;
+            int e = -1, f = 0, cnt = 0;
+            if (a < n_active_all) {
+                e = act_s[1 + a];
+                if (e >= 0 && e < p.E) {
+                    f = off_s[e];
+                    cnt = off_s[e + 1] - f;
+                }
+            }
+            const bool keep = a < n_active_all && e >= 0 && e < p.E && cnt > 0 && cnt <= p.max_count;
+            const unsigned m = __ballot_sync(0xffffffffu, keep);
+            if (keep) {
+                const int pos = run + __popc(m & ((1u << lane) - 1u));
+                int ti = 0;  // the shelf holding e (shelves cover [0, E) without overlap)
+                for (int t = 0; t < p.w.n_tiers; ++t)
+                    if (e >= S.tp[t].first && e - S.tp[t].first < S.tp[t].n) ti = t;
+                S.st.expert[pos] = e;
+                S.st.bits[pos] = S.tp[ti].bits;
+                S.st.first[pos] = f;
+                S.st.count[pos] = cnt;
+                S.tier[pos] = ti;
+                S.jloc[pos] = e - S.tp[ti].first;
+            }
+            run += __popc(m);
+        }
+        const bool shared_here = p.has_shared && p.T <= p.max_count;
+        if (lane == 0 && shared_here) {
+            S.st.expert[run] = p.E;
+            S.st.bits[run] = p.w.shared.bits;
+            S.st.first[run] = S_;
+            S.st.count[run] = p.T;
+            S.tier[run] = p.w.n_tiers;
+            S.jloc[run] = 0;
+        }
+        const int ns = run + (shared_here ? 1 : 0);
+        if (lane == 0) n_keep = ns;
+        __syncwarp();
         for (int phase = 0; phase < 2; ++phase) {
             const long long nt = tiles_per_slot(p, phase);
-            long long run = 0;
-            for (int a0 = 0; a0 < n_slots; a0 += 32) {
+            long long *tc = phase == 0 ? S.sc.tc0 : S.sc.tc1;
+            long long *pre = phase == 0 ? S.sc.pre0 : S.sc.pre1;
+            long long base = 0;
+            for (int a0 = 0; a0 < ns; a0 += 32) {
                 const int a = a0 + lane;
-                long long v = a < n_slots ? nt * (phase == 0 ? S.sc.tc0 : S.sc.tc1)[a] : 0;
+                long long v = 0;
+                if (a < ns) {
+                    const long long c = tile_cost(p, phase, S.st.bits[a], S.st.count[a]);
+                    tc[a] = c;
+                    v = nt * c;
+                }
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const long long u = __shfl_up_sync(0xffffffffu, v, o);
                     if (lane >= o) v += u;
                 }
-                if (a < n_slots) (phase == 0 ? S.sc.pre0 : S.sc.pre1)[a] = run + v;
-                run += __shfl_sync(0xffffffffu, v, 31);
+                if (a < ns) pre[a] = base + v;
+                base += __shfl_sync(0xffffffffu, v, 31);
             }
         }
     }
     __syncthreads();
+    const int n_slots = n_keep;
     ffn_stream_body(p, S, n_slots, nstages);
 }
 
