@@ -37,6 +37,12 @@ UNIT = "layer-tokens/s"
 N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
 KERNELS_PER_LAYER = 5  # router logits, top-k, bucketize, streaming FFN, combine (+1 rmsnorm per step)
 
+# DRAM bytes (read + write) per launch measured by ncu for the kernel versions
+# in this tree (profiles/ffn_stream_decode_T1.md, profiles/ffn_gemm_prefill_T4096.md);
+# to be re-measured whenever those kernels change.
+DECODE_FFN_TRAFFIC = 28.6e6   # streaming FFN kernel, one decode token, mean of 2 launches
+PREFILL_FFN_TRAFFIC = 1.519e9  # the gate_up and down GEMM launches of one 4096-token call
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -253,7 +259,7 @@ def run_prefill(args, rank, world):
                    "l2": "inputs larger than L2: every expert of the layer (~0.6 GB) is read each step"},
         "roofline": {"bound": "tensor", "kernel": "expert FFN call (f16 staging + gate_up GEMM + down GEMM)",
                      "achieved": round(pf["tflops"], 1), "peak": tf, "unit": "TFLOP/s",
-                     "frac": round(pf["tflops"] / tf, 4), "traffic": None, "peak_kind": peak_kind + " burst",
+                     "frac": round(pf["tflops"] / tf, 4), "traffic": PREFILL_FFN_TRAFFIC, "peak_kind": peak_kind + " burst",
                      "algorithmic_flops_per_launch": pf["flops"], "avg_launch_us": round(pf["ffn_ms"] * 1e3, 1)},
         "gpu_launches": max(args.steps, 3) * 8,
         "clocks": clk.summary(),
@@ -342,7 +348,7 @@ def run_native(args, rank, world):
                    "graph": f"one CUDA graph per step (rmsnorm + {N_LAYERS} x layer_forward)"},
         "roofline": {"bound": "hbm", "kernel": "expert FFN call of one layer (counter clear + streaming GEMV)",
                      "achieved": round(fp["gbs"], 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(fp["gbs"] / hbm, 4), "traffic": None, "peak_kind": peak_kind,
+                     "frac": round(fp["gbs"] / hbm, 4), "traffic": DECODE_FFN_TRAFFIC, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": round(fp["bytes"]), "avg_launch_us": round(fp["ms"] * 1e3, 2)},
         "e2e": {"value": round(e2e_val, 1), "unit": UNIT,
                 "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2},
