@@ -123,7 +123,7 @@ typedef struct moe_layer_weights {
 
 /* FFN execution path */
 #define MOE_FFN_AUTO 0 /* per expert: GEMV below the token threshold, GEMM above */
-#define MOE_FFN_GEMV 1 /* every expert through the CUDA-core GEMV */
+#define MOE_FFN_GEMV 1 /* every expert through the streaming GEMV (mma.sync tiles) */
 #define MOE_FFN_GEMM 2 /* every expert through the tcgen05 GEMM */
 
 /* Description of the most recent error on the calling host thread. */
@@ -201,10 +201,12 @@ int moe_bucketize(const int32_t *topk_idx, int32_t T, int32_t k, int32_t E,
  *   g = W_gate[e] x[t], u = W_up[e] x[t], h = silu(g) * u, y = W_down[e] h
  *   y_slots  fp32 [T*k][H]  (row s = t*k+j)
  *   y_shared fp32 [T][H]    (NULL iff the layer has no shared expert)
- * `mode` is MOE_FFN_AUTO / _GEMV / _GEMM.  The GEMV path dequantises to fp32
- * (exact) and accumulates in fp32; the GEMM path stages w, x and h in fp16 and
- * accumulates in fp32 (tcgen05), reporting MOE_STATUS_FP16_RANGE if x or h
- * leaves the fp16 range.
+ * `mode` is MOE_FFN_AUTO / _GEMV / _GEMM.  The GEMV path multiplies exact
+ * integer codes with fp16 x (exact for bf16 magnitudes in [2^-14, 65504]) and
+ * with h split into fp16 hi + lo, accumulates in fp32 and applies each block's
+ * scale in fp32; the GEMM path stages d*q, x and h in fp16 and accumulates in
+ * fp32 (tcgen05).  Both report MOE_STATUS_FP16_RANGE if x or h leaves the fp16
+ * range.  AUTO sends experts with at least 8 tokens to the GEMM path.
  * workspace: moe_ffn_workspace_size() bytes.
  */
 size_t moe_ffn_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k,
