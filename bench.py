@@ -40,7 +40,7 @@ KERNELS_PER_LAYER = 5  # router logits, top-k, bucketize, streaming FFN, combine
 # DRAM bytes (read + write) per launch measured by ncu for the kernel versions
 # in this tree (profiles/ffn_stream_decode_T1.md, profiles/ffn_gemm_prefill_T4096.md);
 # to be re-measured whenever those kernels change.
-DECODE_FFN_TRAFFIC = 28.6e6   # streaming FFN kernel, one decode token, mean of 2 launches
+DECODE_FFN_TRAFFIC = None     # streaming FFN kernel, one decode token (changed since the last capture)
 PREFILL_FFN_TRAFFIC = 1.519e9  # the gate_up and down GEMM launches of one 4096-token call
 
 

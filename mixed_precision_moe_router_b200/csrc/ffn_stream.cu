@@ -14,11 +14,13 @@
 //    most 32K codes.  Each CTA takes a contiguous, cost-balanced share of the
 //    gate_up tiles and then of the down tiles, so 8-, 4- and 3-bit experts
 //    spread evenly over the SMs.
-//  * All 8 warps of a CTA stage the next tiles into a ring of shared-memory
-//    stages with 16-byte cp.async copies (commit / wait_group), so that copy
-//    issue is spread over 256 threads; rows land at a padded stride that
-//    makes the reads below bank-conflict free.
-//  * The 8 warps split a tile into R row subtiles x 8/R K slices.  For
+//  * One producer thread moves each tile into a stage of a shared-memory ring
+//    with TMA tensor copies (cp.async.bulk.tensor) that complete on the
+//    stage's mbarrier: one copy per 128-byte column chunk of the tile (8R gate
+//    rows and their 8R up rows in one 4-D box), plus one for the scales.  The
+//    copies store the tile with the TMA swizzle, which makes the fragment
+//    reads below bank-conflict free.
+//  * 8 compute warps split a tile into R row subtiles x 8/R K slices.  For
 //    each 32-weight block a warp turns its codes into exact fp16 integers
 //    (|q| <= 127), multiplies them with fp16 activation fragments on the
 //    tensor cores (mma.sync m16n8k16: exact products, fp32 accumulation) and
@@ -32,6 +34,12 @@
 //    waits (bounded) for its slot's count before reading h, while its weights
 //    may already be in flight.  The grid is launched cooperatively so every
 //    CTA is resident and the waits resolve.
+#include <cuda.h>
+
+#include <cstring>
+#include <map>
+#include <mutex>
+
 #include "common.cuh"
 #include "ffn.cuh"
 #include "sync.cuh"
@@ -40,9 +48,7 @@ namespace moe {
 
 constexpr int kWarps = 8;                          // compute warps
 constexpr int kThreads = kWarps * 32;
-constexpr int kProducerWarps = 2;                  // copy warps
-constexpr int kProducers = kProducerWarps * 32;
-constexpr int kBlockThreads = kThreads + kProducers;
+constexpr int kBlockThreads = kThreads + 32;       // + one producer warp (one thread issues)
 constexpr int kBarCompute = 1;                     // named barrier of the compute warps
 constexpr int kMaxStages = 6;
 constexpr int kStageBytes = 40 * 1024;
@@ -60,24 +66,19 @@ __host__ __device__ __forceinline__ int rows_pow2(int K) {
     return R;
 }
 
-// Stride of a code row in a stage: 8-bit reads (8 bytes per thread, 4 threads
-// per row) need the stride in words to be 8 or 24 mod 32; 4- and 3-bit reads
-// (at most 4 bytes) need 4 mod 8.  Strides stay multiples of 16 bytes.
-__host__ __device__ __forceinline__ int code_row_stride(int K, int bits) {
-    const int rb = K * bits / 8;
-    for (int p = 0; p < 128; p += 16) {
-        const int w = (rb + p) / 4;
-        if (bits == 8 ? (w % 32 == 8 || w % 32 == 24) : (w % 8 == 4)) return rb + p;
-    }
-    return rb;
+// Swizzle width of a row of `bytes` bytes: the largest of 128, 64 and 32 that
+// divides it (its 16-byte chunks are permuted within that span), else 16 (no
+// swizzle).
+__host__ __device__ __forceinline__ int swizzle_width(int bytes) {
+    return bytes % 128 == 0 ? 128 : (bytes % 64 == 0 ? 64 : (bytes % 32 == 0 ? 32 : 16));
 }
 
 struct Geo {
-    int K, R, rows;   // row subtiles and rows per tile
-    int rb, rs;       // code bytes per row, stage stride
-    int sb, ss;       // scale bytes per row, stage stride
-    bool row_scales;  // scales copied row by row (padded) or in one piece
-    int nb, bps;      // 32-weight blocks per row, blocks per K slice
+    int K, R, rows;  // row subtiles and rows per tile
+    int rb, sb;      // code and scale bytes per row
+    int W, lw;       // code swizzle width (and log2): the tile is stored as column chunks of W bytes
+    int Ws;          // scale swizzle width, 0 when the scales come as plain bulk copies
+    int nb, bps;     // 32-weight blocks per row, blocks per K slice
 };
 
 __host__ __device__ __forceinline__ Geo geo(int K, int bits) {
@@ -86,17 +87,32 @@ __host__ __device__ __forceinline__ Geo geo(int K, int bits) {
     g.R = rows_pow2(K);
     g.rows = 16 * g.R;
     g.rb = K * bits / 8;
-    g.rs = code_row_stride(K, bits);
     g.sb = K / 16;
-    g.row_scales = g.sb % 16 == 0 && g.sb >= 64;
-    g.ss = g.row_scales ? g.sb + 16 : g.sb;
+    g.W = swizzle_width(g.rb);
+    g.lw = g.W == 128 ? 7 : (g.W == 64 ? 6 : (g.W == 32 ? 5 : 4));
+    // the scale box is a whole row: swizzled only when the row is 32, 64 or 128 bytes
+    g.Ws = g.sb % 16 != 0 ? 0 : ((g.sb == 32 || g.sb == 64 || g.sb == 128) ? g.sb : 16);
     g.nb = K / 32;
     const int S = kWarps / g.R;
     g.bps = ((g.nb + S - 1) / S + 1) & ~1;  // even, so blocks go in pairs
     return g;
 }
 
-__host__ __device__ __forceinline__ int stage_bytes(const Geo &g) { return g.rows * (g.rs + g.ss); }
+__host__ __device__ __forceinline__ int stage_bytes(const Geo &g) { return g.rows * (g.rb + g.sb); }
+
+// XOR that the TMA swizzle of width W applies to the 16-byte chunk index of
+// row r of a box (boxes start on a swizzle-atom boundary and hold a multiple
+// of 8 rows)
+__device__ __forceinline__ int swz(int r, int W) {
+    return W == 128 ? (r & 7) << 4 : (W == 64 ? ((r >> 1) & 3) << 4 : (W == 32 ? ((r >> 2) & 1) << 4 : 0));
+}
+
+// Byte offset of byte o of row r in a tile of `rows` rows stored as column
+// chunks of W bytes with the TMA swizzle (xr = swz(r, W)).
+__device__ __forceinline__ int tile_off(int o, int r, const Geo &G, int xr) {
+    return (o >> G.lw) * (G.rows << G.lw) + (r << G.lw) + ((o & (G.W - 1)) ^ xr);
+}
+
 
 // x fragments in shared memory: [column][block][thread t][8 halves], with a
 // column stride that keeps the 16-byte reads of two columns in different banks.
@@ -266,9 +282,10 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
 }
 
 template <int BITS>
-__device__ __forceinline__ void dequant8(const uint8_t *row, int K, int b, int t, uint32_t (&P)[4]) {
+__device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int r, int xr, int b, int t,
+                                         uint32_t (&P)[4]) {
     if constexpr (BITS == 8) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(row + 32 * b + 8 * t);
+        const uint2 w = *reinterpret_cast<const uint2 *>(tile + tile_off(32 * b + 8 * t, r, G, xr));
         const uint32_t u0 = w.x ^ 0x80808080u, u1 = w.y ^ 0x80808080u;  // c = q + 128
         constexpr uint32_t kBias = 0x64806480u;                         // 1024 + 128
         P[0] = hsub2(prmt(u0, 0x64646464u, 0x4140u), kBias);
@@ -277,7 +294,7 @@ __device__ __forceinline__ void dequant8(const uint8_t *row, int K, int b, int t
         P[3] = hsub2(prmt(u1, 0x64646464u, 0x4342u), kBias);
     } else if constexpr (BITS == 4) {
         // nibble i of the word at byte 16b + 4t is weight 8t + i (c = q + 8)
-        const uint32_t v = *reinterpret_cast<const uint32_t *>(row + 16 * b + 4 * t);
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(tile + tile_off(16 * b + 4 * t, r, G, xr));
         const uint32_t v8 = v >> 8;
         P[0] = hsub2((v & 0x000F000Fu) | 0x64006400u, 0x64086408u);   // 1024 + c - 1032
         P[1] = hsub2((v & 0x00F000F0u) | 0x54005400u, 0x54805480u);   // 64 + c - 72
@@ -286,8 +303,8 @@ __device__ __forceinline__ void dequant8(const uint8_t *row, int K, int b, int t
     } else {
         // low plane: bits 0-1 of weight 8t+i at bit 2i of the u16 at byte 8b+2t;
         // high plane: bit 2 at bit i of byte K/4 + 4b + t (c = q + 4)
-        const uint32_t lo16 = *reinterpret_cast<const uint16_t *>(row + 8 * b + 2 * t);
-        const uint32_t hb = row[K / 4 + 4 * b + t];
+        const uint32_t lo16 = *reinterpret_cast<const uint16_t *>(tile + tile_off(8 * b + 2 * t, r, G, xr));
+        const uint32_t hb = tile[tile_off(G.K / 4 + 4 * b + t, r, G, xr)];
         const uint32_t X = prmt(lo16, 0u, 0x4140u);  // weights i and i+4 16 bits apart
         const uint32_t Y = hb * 0x4004u;             // hb << 2 | hb << 14
         P[0] = hsub2((X & 0x00030003u) | (Y & 0x00040004u) | 0x64006400u, 0x64046404u);           // 1024 + c - 1028
@@ -295,10 +312,6 @@ __device__ __forceinline__ void dequant8(const uint8_t *row, int K, int b, int t
         P[2] = hsub2((X & 0x00300030u) | ((Y << 2) & 0x00400040u) | 0x54005400u, 0x54405440u);  // 64 + c - 68
         P[3] = hsub2((X & 0x00C000C0u) | ((Y << 3) & 0x01000100u) | 0x4C004C00u, 0x4D004D00u);  // 16 + c - 20
     }
-}
-
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
 // D = A B + D on one m16n8k16 tile (fp16 inputs, fp32 accumulation).
@@ -322,10 +335,10 @@ template <int BITS, int NT>
 __device__ __forceinline__ void warp_tile(const uint8_t *stage, const Geo &G, int rA, int rB, int b0, int b1,
                                           const uint8_t *xf, int cs, int ncol0, int ncol1, float (&acc)[2][4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const uint8_t *qa = stage + rA * G.rs;
-    const uint8_t *qb = stage + rB * G.rs;
-    const uint8_t *sa = stage + G.rows * G.rs + rA * G.ss;
-    const uint8_t *sbr = stage + G.rows * G.rs + rB * G.ss;
+    const int xa = swz(rA, G.W), xb = swz(rB, G.W);
+    // scales: [row][sb] after the codes, swizzled at width Ws (or plain)
+    const uint8_t *scl = stage + G.rows * G.rb;
+    const int sxa = G.Ws ? swz(rA, G.Ws) : 0, sxb = G.Ws ? swz(rB, G.Ws) : 0;
     const uint8_t *xg = xf + g * cs + t * 16;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -333,13 +346,13 @@ __device__ __forceinline__ void warp_tile(const uint8_t *stage, const Geo &G, in
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
 #pragma unroll 2
     for (int b = b0; b < b1; b += 2) {
-        const float2 da = half2_to_float2(*reinterpret_cast<const uint32_t *>(sa + 2 * b));
-        const float2 db = half2_to_float2(*reinterpret_cast<const uint32_t *>(sbr + 2 * b));
+        const float2 da = half2_to_float2(*reinterpret_cast<const uint32_t *>(scl + rA * G.sb + ((2 * b) ^ sxa)));
+        const float2 db = half2_to_float2(*reinterpret_cast<const uint32_t *>(scl + rB * G.sb + ((2 * b) ^ sxb)));
         uint32_t PA[2][4], PB[2][4];
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
-            dequant8<BITS>(qa, G.K, b + bb, t, PA[bb]);
-            dequant8<BITS>(qb, G.K, b + bb, t, PB[bb]);
+            dequant8<BITS>(stage, G, rA, xa, b + bb, t, PA[bb]);
+            dequant8<BITS>(stage, G, rB, xb, b + bb, t, PB[bb]);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -412,74 +425,66 @@ struct StreamSmem {
 
 __device__ __forceinline__ int bits_idx(int bits) { return bits == 8 ? 0 : (bits == 4 ? 1 : 2); }
 
-// Stage the codes and scales of tile (phase, a, tile) into `dst`: producer
-// thread pt of kProducers copies its share of 16-byte chunks.
-__device__ __forceinline__ void issue_tile(const FfnParams &p, const StreamSmem &S, int phase, int a, int tile,
-                                           uint8_t *dst, int pt) {
-    const int H = p.w.H, I = p.w.I;
-    const int bits = S.st.bits[a];
-    const Geo &G = S.geo[phase * 3 + bits_idx(bits)];
-    const TierPtrs &T = S.tp[S.tier[a]];
-    const size_t j = static_cast<size_t>(S.jloc[a]);
-    const uint8_t *q, *sc;
-    size_t r_first, r_second;  // first matrix row of the tile's two row groups
-    int half;                  // rows in the first group
-    if (phase == 0) {
-        q = T.gq + j * 2 * I * G.rb;
-        sc = T.gs + j * 2 * I * G.sb;
-        r_first = static_cast<size_t>(tile) * 8 * G.R;  // gate pairs ...
-        r_second = I + r_first;                          // ... and their up rows
-        half = 8 * G.R;
-    } else {
-        q = T.dq + j * H * G.rb;
-        sc = T.ds + j * H * G.sb;
-        r_first = static_cast<size_t>(tile) * G.rows;
-        r_second = r_first + 8 * G.R;  // the same rows, contiguous
-        half = 8 * G.R;
-    }
-    // codes: rows of rb bytes, cpr 16-byte chunks each; rps rows per sweep
-    {
-        const int cpr = G.rb / 16;
-        if (cpr >= kProducers) {
-            for (int r = 0; r < G.rows; ++r) {
-                const size_t mr = r < half ? r_first + r : r_second + (r - half);
-                for (int off = pt * 16; off < G.rb; off += kProducers * 16)
-                    cp_async16(dst + r * G.rs + off, q + mr * G.rb + off);
-            }
-        } else {
-            const int rps = kProducers / cpr;
-            const int r0 = pt / cpr, off = (pt - r0 * cpr) * 16;
-            if (r0 < rps)
-                for (int r = r0; r < G.rows; r += rps) {
-                    const size_t mr = r < half ? r_first + r : r_second + (r - half);
-                    cp_async16(dst + r * G.rs + off, q + mr * G.rb + off);
-                }
-        }
-    }
-    // scales: per row (padded stride) or each group of rows in one piece
-    uint8_t *dsc = dst + G.rows * G.rs;
-    if (G.row_scales) {
-        const int cpr = G.sb / 16, rps = kProducers / cpr;  // sb <= 128: cpr <= 8
-        const int r0 = pt / cpr, off = (pt - r0 * cpr) * 16;
-        if (r0 < rps)
-            for (int r = r0; r < G.rows; r += rps) {
-                const size_t mr = r < half ? r_first + r : r_second + (r - half);
-                cp_async16(dsc + r * G.ss + off, sc + mr * G.sb + off);
-            }
-    } else {
-        const int n = half * G.sb / 16;  // chunks per group
-        for (int c = pt; c < 2 * n; c += kProducers) {
-            const int grp = c >= n, cc = c - grp * n;
-            const size_t src = (grp ? r_second : r_first) * G.sb + cc * 16;
-            cp_async16(dsc + grp * half * G.sb + cc * 16, sc + src);
-        }
-    }
+// Tensor maps of the shelf tables (index < n_tiers) and of the shared expert
+// (index n_tiers), built on the host:
+//   gq: 4-D [expert][gate|up][I][rb_H] bytes, box {W_H, 8R, 2, 1}
+//   gs: 4-D [expert][gate|up][I][sb_H] bytes, box {sb_H, 8R, 2, 1}
+//   dq: 3-D [expert][H][rb_I], box {W_I, 16R, 1};  ds: 3-D [expert][H][sb_I]
+// each stored with the swizzle of its inner box width.
+struct StreamMaps {
+    CUtensorMap gq[MOE_MAX_TIERS + 1], gs[MOE_MAX_TIERS + 1];
+    CUtensorMap dq[MOE_MAX_TIERS + 1], ds[MOE_MAX_TIERS + 1];
+};
+
+__device__ __forceinline__ void tma_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
 }
 
+__device__ __forceinline__ void tma_4d(void *dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                       uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
 
-// Arrive on bar once all of this thread's earlier cp.async copies have landed.
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Stage the codes and scales of tile (phase, a, tile) into `dst`, completing
+// on `bar`: a gate_up tile is its 8R gate rows and the matching 8R up rows, a
+// down tile 16R consecutive rows; codes as column chunks of W bytes.
+__device__ __forceinline__ void issue_tile(const FfnParams &p, const StreamMaps &M, const StreamSmem &S, int phase,
+                                           int a, int tile, uint8_t *dst, uint64_t *bar) {
+    const int I = p.w.I;
+    const Geo &G = S.geo[phase * 3 + bits_idx(S.st.bits[a])];
+    const int ti = S.tier[a], j = S.jloc[a];
+    const TierPtrs &T = S.tp[ti];
+    uint8_t *dsc = dst + G.rows * G.rb;
+    const int chunk = G.rows << G.lw;  // bytes of one column chunk of the tile
+    mbar_expect_tx(bar, static_cast<uint32_t>(G.rows) * (G.rb + G.sb));
+    if (phase == 0) {
+        const int half = 8 * G.R, P = tile * half;
+        for (int c = 0; c * G.W < G.rb; ++c) tma_4d(dst + c * chunk, &M.gq[ti], c * G.W, P, 0, j, bar);
+        if (G.Ws) {
+            tma_4d(dsc, &M.gs[ti], 0, P, 0, j, bar);
+        } else {
+            const uint8_t *sc = T.gs + static_cast<size_t>(j) * 2 * I * G.sb;
+            bulk_g2s(dsc, sc + static_cast<size_t>(P) * G.sb, half * G.sb, bar);
+            bulk_g2s(dsc + half * G.sb, sc + static_cast<size_t>(I + P) * G.sb, half * G.sb, bar);
+        }
+    } else {
+        const int Q = tile * G.rows;
+        for (int c = 0; c * G.W < G.rb; ++c) tma_3d(dst + c * chunk, &M.dq[ti], c * G.W, Q, j, bar);
+        if (G.Ws) {
+            tma_3d(dsc, &M.ds[ti], 0, Q, j, bar);
+        } else {
+            const uint8_t *sc = T.ds + static_cast<size_t>(j) * p.w.H * G.sb;
+            bulk_g2s(dsc, sc + static_cast<size_t>(Q) * G.sb, G.rows * G.sb, bar);
+        }
+    }
 }
 
 // Barrier of the compute warps that also ANDs a flag over them.
@@ -613,16 +618,17 @@ __device__ __forceinline__ void epilogue(const FfnParams &p, const SlotTabs &st,
 }
 
 // The persistent FFN kernel body; `n_slots` slots are described in S.
-__device__ __forceinline__ void ffn_stream_body(const FfnParams &p, StreamSmem &S, int n_slots, int nstages) {
+__device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const StreamMaps &M, StreamSmem &S, int n_slots,
+                                                int nstages) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int I = p.w.I;
     if (warp >= kWarps) {
-        // producer warps: stage the CTA's tiles in order; every producer
-        // thread arrives on the stage's full barrier once its copies landed
-        const int pt = threadIdx.x - kThreads;
+        // producer: one thread stages the CTA's tiles in order
+        if (lane != 0) return;
         TileIt pf;
         it_begin(p, S.sc, n_slots, pf);
-        for (int i = 0; pf.phase < 2; ++i, it_next(p, S.sc, n_slots, pf)) {
+        int i = 0;
+        for (; pf.phase < 2; ++i, it_next(p, S.sc, n_slots, pf)) {
             if (*static_cast<volatile int *>(S.abort)) break;
             const int s = i % nstages;
             if (!mbar_wait(&S.empty[s], ((i / nstages) & 1) ^ 1)) {
@@ -630,10 +636,11 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, StreamSmem &
                 *static_cast<volatile int *>(S.abort) = 1;
                 break;
             }
-            issue_tile(p, S, pf.phase, pf.a, pf.b, S.stages + static_cast<size_t>(s) * kStageBytes, pt);
-            cp_async_arrive(&S.full[s]);
+            issue_tile(p, M, S, pf.phase, pf.a, pf.b, S.stages + static_cast<size_t>(s) * kStageBytes, &S.full[s]);
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
+        // the copies still in flight must land before the CTA exits
+        for (int k = i - nstages < 0 ? 0 : i - nstages; k < i; ++k)
+            if (!mbar_wait(&S.full[k % nstages], (k / nstages) & 1)) status_or(p.status, MOE_STATUS_TIMEOUT);
         return;
     }
     // compute warps: every branch below depends only on values that are the
@@ -711,7 +718,7 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, StreamSmem &
 }
 
 __global__ void __launch_bounds__(kBlockThreads, 1)
-ffn_stream_kernel(const FfnParams p, int nstages) {
+ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ StreamMaps M, int nstages) {
     extern __shared__ __align__(1024) uint8_t smem[];
     StreamSmem S;
     S.stages = smem;
@@ -784,7 +791,7 @@ ffn_stream_kernel(const FfnParams p, int nstages) {
         S.tp[t].first = p.E;
         S.tp[t].n = 1;
         for (int st = 0; st < nstages; ++st) {
-            mbar_init(&S.full[st], kProducers);  // one arrival per producer thread
+            mbar_init(&S.full[st], 1);  // the producer's expect_tx arrival
             mbar_init(&S.empty[st], kWarps);     // one per compute warp
         }
         *S.abort = 0;
@@ -866,7 +873,7 @@ ffn_stream_kernel(const FfnParams p, int nstages) {
     }
     __syncthreads();
     const int n_slots = n_keep;
-    ffn_stream_body(p, S, n_slots, nstages);
+    ffn_stream_body(p, M, S, n_slots, nstages);
 }
 
 }  // namespace moe
@@ -898,6 +905,107 @@ bool moe_ffn_stream_supported(int H, int I) {
     return H <= moe::kMaxK && I <= moe::kMaxK && H % 128 == 0 && I % 128 == 0;
 }
 
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_tiled() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(ptr);
+    });
+    return fn;
+}
+
+CUtensorMapSwizzle swizzle_mode(int w) {
+    return w == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                    : (w == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : (w == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE));
+}
+
+// A byte tensor map: dims[0] contiguous bytes, dims[i] at strides[i-1] bytes.
+// Maps depend only on these arguments, so they are cached by them (a table
+// freed and reallocated at the same address with the same shape maps the
+// same way).
+struct MapKey {
+    const void *ptr;
+    int rank, sw;
+    uint64_t dims[4], strides[3];
+    uint32_t box[4];
+    bool operator<(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) < 0; }
+};
+
+std::mutex g_map_mu;
+std::map<MapKey, CUtensorMap> g_maps;
+
+bool byte_map(CUtensorMap *out, const void *ptr, int rank, const uint64_t *dims, const uint64_t *strides,
+              const uint32_t *box, int sw) {
+    MapKey key;
+    std::memset(&key, 0, sizeof(key));
+    key.ptr = ptr;
+    key.rank = rank;
+    key.sw = sw;
+    for (int i = 0; i < rank; ++i) key.dims[i] = dims[i], key.box[i] = box[i];
+    for (int i = 0; i + 1 < rank; ++i) key.strides[i] = strides[i];
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+        *out = it->second;
+        return true;
+    }
+    const EncodeTiled fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (fn(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void *>(ptr), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_mode(sw), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    if (g_maps.size() > 4096) g_maps.clear();
+    g_maps.emplace(key, *out);
+    return true;
+}
+
+// Maps of one shelf (or of the shared expert) at table index t.
+bool shelf_maps(moe::StreamMaps &M, int t, const moe_tier &tier, int H, int I) {
+    const uint64_t n = static_cast<uint64_t>(tier.n_experts);
+    const moe::Geo g0 = moe::geo(H, tier.bits), g1 = moe::geo(I, tier.bits);
+    {
+        const uint64_t dims[4] = {static_cast<uint64_t>(g0.rb), static_cast<uint64_t>(I), 2, n};
+        const uint64_t str[3] = {static_cast<uint64_t>(g0.rb), static_cast<uint64_t>(I) * g0.rb,
+                                 2ull * I * g0.rb};
+        const uint32_t box[4] = {static_cast<uint32_t>(g0.W), static_cast<uint32_t>(8 * g0.R), 2, 1};
+        if (!byte_map(&M.gq[t], tier.gu_qs, 4, dims, str, box, g0.W)) return false;
+    }
+    if (g0.Ws) {
+        const uint64_t dims[4] = {static_cast<uint64_t>(g0.sb), static_cast<uint64_t>(I), 2, n};
+        const uint64_t str[3] = {static_cast<uint64_t>(g0.sb), static_cast<uint64_t>(I) * g0.sb,
+                                 2ull * I * g0.sb};
+        const uint32_t box[4] = {static_cast<uint32_t>(g0.sb), static_cast<uint32_t>(8 * g0.R), 2, 1};
+        if (!byte_map(&M.gs[t], tier.gu_scale, 4, dims, str, box, g0.Ws)) return false;
+    }
+    {
+        const uint64_t dims[3] = {static_cast<uint64_t>(g1.rb), static_cast<uint64_t>(H), n};
+        const uint64_t str[2] = {static_cast<uint64_t>(g1.rb), static_cast<uint64_t>(H) * g1.rb};
+        const uint32_t box[3] = {static_cast<uint32_t>(g1.W), static_cast<uint32_t>(g1.rows), 1};
+        if (!byte_map(&M.dq[t], tier.dn_qs, 3, dims, str, box, g1.W)) return false;
+    }
+    if (g1.Ws) {
+        const uint64_t dims[3] = {static_cast<uint64_t>(g1.sb), static_cast<uint64_t>(H), n};
+        const uint64_t str[2] = {static_cast<uint64_t>(g1.sb), static_cast<uint64_t>(H) * g1.sb};
+        const uint32_t box[3] = {static_cast<uint32_t>(g1.sb), static_cast<uint32_t>(g1.rows), 1};
+        if (!byte_map(&M.ds[t], tier.dn_scale, 3, dims, str, box, g1.Ws)) return false;
+    }
+    return true;
+}
+
+}  // namespace
+
 // counters (int[max_active + 1]) must be zero on entry; the caller clears them.
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     int nstages = 0;
@@ -917,5 +1025,10 @@ cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, nstages);
+    moe::StreamMaps M;
+    std::memset(&M, 0, sizeof(M));
+    for (int t = 0; t < p.w.n_tiers; ++t)
+        if (!shelf_maps(M, t, p.w.tiers[t], p.w.H, p.w.I)) return cudaErrorInvalidValue;
+    if (p.has_shared && !shelf_maps(M, p.w.n_tiers, p.w.shared, p.w.H, p.w.I)) return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, M, nstages);
 }
