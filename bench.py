@@ -35,7 +35,7 @@ from mixed_precision_moe_router_b200 import inputs  # noqa: E402
 METRIC = "MoE-layer tokens/s; decode expert-weight GB/s vs HBM peak; prefill TFLOP/s"
 UNIT = "layer-tokens/s"
 N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
-KERNELS_PER_LAYER = 5  # router logits, top-k, bucketize, streaming FFN, combine (+1 rmsnorm per step)
+KERNELS_PER_LAYER = 3  # fused routing, streaming FFN, combine (+1 rmsnorm per step)
 
 # DRAM bytes (read + write) per launch measured by ncu for the kernel versions
 # in this tree (profiles/ffn_stream_decode_T1.md, profiles/ffn_gemm_prefill_T4096.md);

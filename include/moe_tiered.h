@@ -193,6 +193,29 @@ int moe_bucketize(const int32_t *topk_idx, int32_t T, int32_t k, int32_t E,
                   int32_t *active, int32_t *status, moe_stream_t stream);
 
 /*
+ * moe_route: moe_router_topk followed by moe_bucketize ([P1] "a small
+ * dictionary", "the four bugs, briefly"), with the same outputs bit for bit.
+ * A batch of at most 16 tokens (whose bf16 rows fit in 200 KB of shared
+ * memory) takes one fused kernel: every CTA computes the logits of 8 experts
+ * and the CTA that finishes last ranks every token and groups the T*k slots;
+ * larger batches run the two calls' kernels.
+ *   outputs: topk_idx, topk_w as in moe_router_topk; expert_offsets,
+ *            sorted_slot, slot_pos, active, status as in moe_bucketize
+ *   workspace: moe_route_workspace_size() bytes, 16-byte aligned: the logits
+ *            and a counter that the call clears with a memset and the fused
+ *            kernel leaves at zero.  Calls sharing a workspace must not
+ *            overlap on the GPU (issue them on one stream).
+ * Limits: those of moe_router_topk and moe_bucketize.  T == 0 writes the
+ * empty grouping (expert_offsets all 0, active[0] = 0).
+ */
+size_t moe_route_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
+int moe_route(const uint16_t *x, const uint16_t *w_router, const float *bias,
+              int32_t T, int32_t H, int32_t E, int32_t k, int32_t *topk_idx,
+              float *topk_w, int32_t *expert_offsets, int32_t *sorted_slot,
+              int32_t *slot_pos, int32_t *active, int32_t *status, void *workspace,
+              size_t workspace_bytes, moe_stream_t stream);
+
+/*
  * moe_expert_ffn_tiered: the tiered SwiGLU expert FFN ([P1] "step 4":
  * mul_mat_id takes an id range, each shelf computes only the ids on it, and
  * the shelf results add up; the decode path fuses gate, up and activation).
@@ -276,8 +299,9 @@ int moe_combine(const float *y_slots, const float *y_shared, const float *topk_w
 int moe_rmsnorm(const uint16_t *x, int32_t T, int32_t H, uint16_t *n, moe_stream_t stream);
 
 /*
- * moe_layer_forward: router -> bucketize -> tiered FFN -> combine, with every
- * intermediate in `workspace` (moe_layer_workspace_size() bytes).
+ * moe_layer_forward: moe_route -> tiered FFN -> combine, with every
+ * intermediate in `workspace` (moe_layer_workspace_size() bytes).  The routing
+ * kernel also clears the FFN's counters, so the FFN needs no memset of its own.
  *   x bf16 [T][H] (the layer input); w_router bf16 [E][H]; bias fp32 [E] or NULL
  *   out bf16 [T][H]; with residual != NULL also x_next and x_next_norm as in
  *   moe_combine (in a stack: x = the normalised stream, residual = the stream).

@@ -52,6 +52,9 @@ SIGNATURES = [
                                 c_size, c_vp]),
     ("moe_topk_softmax", c_i32, [c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
     ("moe_bucketize", c_i32, [c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    ("moe_route_workspace_size", c_size, [c_i32, c_i32, c_i32, c_i32]),
+    ("moe_route", c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                          c_vp, c_vp, c_size, c_vp]),
     ("moe_ffn_workspace_size", c_size, [ctypes.POINTER(LayerWeights), c_i32, c_i32, c_i32]),
     ("moe_expert_ffn_tiered", c_i32, [ctypes.POINTER(LayerWeights), c_vp, c_i32, c_i32, c_vp, c_vp, c_vp,
                                       c_vp, c_vp, c_vp, c_size, c_i32, c_vp, c_vp]),
@@ -267,6 +270,33 @@ def bucketize(topk_idx, E, status=None):
     _check(lib().moe_bucketize(_ptr(topk_idx), T, k, E, _ptr(offsets), _ptr(sorted_slot), _ptr(slot_pos),
                                _ptr(active), _ptr(status), _stream()))
     return offsets, sorted_slot[: T * k], slot_pos[: T * k], active
+
+
+def route(x, w_router, bias, k, status=None, workspace=None):
+    """moe_route: the router's top-k and the token -> expert grouping in one
+    call.  Returns (topk_idx, topk_w, offsets, sorted_slot, slot_pos, active).
+    A caller-owned `workspace` (uint8, moe_route_workspace_size bytes) may be
+    reused across calls on one stream."""
+    _need(x, torch.bfloat16, name="x")
+    _need(w_router, torch.bfloat16, name="w_router")
+    T, H = x.shape
+    E = w_router.shape[0]
+    dev = x.device
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    idx = torch.empty(max(T, 1), k, dtype=torch.int32, device=dev)
+    w = torch.empty(max(T, 1), k, dtype=torch.float32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sorted_slot = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    slot_pos = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    active = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    nws = int(lib().moe_route_workspace_size(T, H, E, k))
+    if workspace is None:
+        workspace = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+    _check(lib().moe_route(_ptr(x), _ptr(w_router), _ptr(bias), T, H, E, k, _ptr(idx), _ptr(w), _ptr(offsets),
+                           _ptr(sorted_slot), _ptr(slot_pos), _ptr(active), _ptr(status), _ptr(workspace),
+                           workspace.numel(), _stream()))
+    return idx[:T], w[:T], offsets, sorted_slot[: T * k], slot_pos[: T * k], active
 
 
 def expert_ffn(layer, x, k, offsets, sorted_slot, active, mode=FFN_AUTO, status=None):

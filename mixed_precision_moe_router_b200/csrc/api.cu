@@ -17,6 +17,11 @@ cudaError_t moe_configure_router();
 cudaError_t moe_launch_router_logits(const uint16_t *, const uint16_t *, const float *, int, int, int, float *,
                                      cudaStream_t);
 cudaError_t moe_launch_topk(const float *, int, int, int, int32_t *, float *, cudaStream_t);
+cudaError_t moe_configure_route_small();
+bool moe_route_small_supported(int T, int H, int E, int k);
+cudaError_t moe_launch_route_small(const uint16_t *, const uint16_t *, const float *, int, int, int, int, float *,
+                                   int32_t *, float *, int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, int *,
+                                   int *, int, cudaStream_t);
 bool moe_router_gemm_supported(int T, int H, int E);
 cudaError_t moe_launch_router_gemm(const uint16_t *, const uint16_t *, const float *, int, int, int, float *,
                                    cudaStream_t);
@@ -71,6 +76,7 @@ int ensure_configured() {
     if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d", dev);
     std::call_once(g_dev_once[dev], [dev]() {
         cudaError_t r = moe_configure_router();
+        if (r == cudaSuccess) r = moe_configure_route_small();
         if (r == cudaSuccess) r = moe_configure_bucketize();
         if (r == cudaSuccess) r = moe_configure_ffn_stream();
         if (r == cudaSuccess) r = moe_configure_ffn_gemm();
@@ -288,10 +294,26 @@ size_t moe_ffn_workspace_size(const moe_layer_weights *w, int32_t T, int32_t k, 
     return ffn_ws_bytes(w, T, k, mode);
 }
 
-int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t k,
-                          const int32_t *expert_offsets, const int32_t *sorted_slot, const int32_t *active,
-                          float *y_slots, float *y_shared, void *workspace, size_t workspace_bytes, int32_t mode,
-                          int32_t *status, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The GEMV path's per-slot counters inside an FFN workspace (NULL when the
+// mode does not use that path); *n = how many ints the kernel reads.
+int *gemv_counters(const moe_layer_weights *w, int T, int k, int mode, void *workspace, int *n) {
+    *n = 0;
+    if (!uses_gemv(mode) || !workspace) return nullptr;
+    const size_t hb = align_up((static_cast<size_t>(T) * k + T) * w->I * sizeof(float));
+    const long ma = static_cast<long>(T) * k;
+    *n = static_cast<int>(ma < w->E ? ma : w->E) + 1;
+    return reinterpret_cast<int *>(static_cast<char *>(workspace) + hb);
+}
+
+// moe_expert_ffn_tiered; counters_clear: the GEMV counters are known to be
+// zero already (cleared by an earlier kernel on the stream), so no memset.
+int expert_ffn(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t k, const int32_t *expert_offsets,
+               const int32_t *sorted_slot, const int32_t *active, float *y_slots, float *y_shared, void *workspace,
+               size_t workspace_bytes, int32_t mode, int32_t *status, moe_stream_t stream, bool counters_clear) {
     int r = check_weights(w);
     if (r) return r;
     r = check_k(T, w->E, k);
@@ -322,10 +344,10 @@ int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t
     const bool gemm = uses_gemm(mode, T);
     const int split = mode == MOE_FFN_GEMM ? 1 : kGemmMinTokens;  // GEMM takes experts with >= split tokens
     if (uses_gemv(mode)) {
-        const size_t hb = align_up((static_cast<size_t>(T) * k + T) * w->I * sizeof(float));
-        p.ctr = reinterpret_cast<int *>(ws + hb);
+        int n_ctr = 0;
+        p.ctr = gemv_counters(w, T, k, mode, workspace, &n_ctr);
         p.max_count = gemm ? split - 1 : 0x7fffffff;
-        e = cudaMemsetAsync(p.ctr, 0, ffn_ctr_bytes(w, T, k), s);
+        if (!counters_clear) e = cudaMemsetAsync(p.ctr, 0, ffn_ctr_bytes(w, T, k), s);
         if (e == cudaSuccess) e = moe_launch_ffn_stream(p, s);
     }
     if (e == cudaSuccess && gemm) {
@@ -333,6 +355,76 @@ int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t
         e = moe_launch_ffn_gemm(p, gws, 0, s, split);
     }
     return e == cudaSuccess ? ok() : cuda_fail(e, "ffn launch");
+}
+
+size_t route_ws_bytes(int T, int E) { return align_up(static_cast<size_t>(T) * E * sizeof(float)) + 256; }
+
+// moe_route; clear/n_clear: ints the fused kernel zeroes on its way out (the
+// next kernel's counters), or a memset when the batch takes the separate
+// kernels.
+int route(const uint16_t *x, const uint16_t *w_router, const float *bias, int32_t T, int32_t H, int32_t E, int32_t k,
+          int32_t *topk_idx, float *topk_w, int32_t *expert_offsets, int32_t *sorted_slot, int32_t *slot_pos,
+          int32_t *active, int32_t *status, void *workspace, size_t workspace_bytes, moe_stream_t stream, int *clear,
+          int n_clear) {
+    int r = check_k(T, E, k);
+    if (r) return r;
+    if (H <= 0 || H % 64 != 0 || H > 16384) return fail(MOE_ERR_INVALID_ARG, "H = %d must be a multiple of 64 in (0, 16384]", H);
+    if (!expert_offsets || !active) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (T > 0 && (!x || !w_router || !topk_idx || !topk_w || !sorted_slot || !slot_pos))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (T > 0 && (!aligned16(x) || !aligned16(w_router))) return fail(MOE_ERR_INVALID_ARG, "x / w_router not 16-byte aligned");
+    const size_t need = route_ws_bytes(T, E);
+    if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "route workspace needs %zu bytes", need);
+    if (!aligned16(workspace)) return fail(MOE_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    r = ensure_configured();
+    if (r) return r;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float *logits = static_cast<float *>(workspace);
+    int *ticket = reinterpret_cast<int *>(static_cast<char *>(workspace) + need - 256);
+    cudaError_t e = cudaSuccess;
+    if (moe_route_small_supported(T, H, E, k)) {
+        e = cudaMemsetAsync(ticket, 0, sizeof(int), s);
+        if (e == cudaSuccess)
+            e = moe_launch_route_small(x, w_router, bias, T, H, E, k, logits, topk_idx, topk_w, expert_offsets,
+                                       sorted_slot, slot_pos, active, status, ticket, clear, n_clear, s);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "route launch");
+    }
+    r = moe_router_topk(x, w_router, bias, T, H, E, k, logits, topk_idx, topk_w, nullptr, 0, stream);
+    if (r) return r;
+    r = moe_bucketize(topk_idx, T, k, E, expert_offsets, sorted_slot, slot_pos, active, status, stream);
+    if (r) return r;
+    if (n_clear > 0) {
+        e = cudaMemsetAsync(clear, 0, static_cast<size_t>(n_clear) * sizeof(int), s);
+        if (e != cudaSuccess) return cuda_fail(e, "memset");
+    }
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t k,
+                          const int32_t *expert_offsets, const int32_t *sorted_slot, const int32_t *active,
+                          float *y_slots, float *y_shared, void *workspace, size_t workspace_bytes, int32_t mode,
+                          int32_t *status, moe_stream_t stream) {
+    return expert_ffn(w, x, T, k, expert_offsets, sorted_slot, active, y_slots, y_shared, workspace, workspace_bytes,
+                      mode, status, stream, false);
+}
+
+size_t moe_route_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k) {
+    (void)H;
+    (void)k;
+    if (T < 0 || E <= 0) return 0;
+    return route_ws_bytes(T, E);
+}
+
+int moe_route(const uint16_t *x, const uint16_t *w_router, const float *bias, int32_t T, int32_t H, int32_t E,
+              int32_t k, int32_t *topk_idx, float *topk_w, int32_t *expert_offsets, int32_t *sorted_slot,
+              int32_t *slot_pos, int32_t *active, int32_t *status, void *workspace, size_t workspace_bytes,
+              moe_stream_t stream) {
+    return route(x, w_router, bias, T, H, E, k, topk_idx, topk_w, expert_offsets, sorted_slot, slot_pos, active,
+                 status, workspace, workspace_bytes, stream, nullptr, 0);
 }
 
 int moe_combine(const float *y_slots, const float *y_shared, const float *topk_w, int32_t T, int32_t k, int32_t H,
@@ -365,7 +457,8 @@ int moe_rmsnorm(const uint16_t *x, int32_t T, int32_t H, uint16_t *n, moe_stream
 
 namespace {
 struct LayerWs {
-    float *logits;
+    void *route_ws;  // logits and the fused router's ticket
+    size_t route_bytes;
     int32_t *idx;
     float *tw;
     int32_t *offsets, *sorted, *pos, *active;
@@ -384,7 +477,8 @@ LayerWs carve(const moe_layer_weights *w, int T, int k, int mode, char *base) {
         return p;
     };
     const size_t S = static_cast<size_t>(T) * k;
-    L.logits = reinterpret_cast<float *>(take(static_cast<size_t>(T) * w->E * sizeof(float)));
+    L.route_bytes = route_ws_bytes(T, w->E);
+    L.route_ws = take(L.route_bytes);
     L.idx = reinterpret_cast<int32_t *>(take(S * sizeof(int32_t)));
     L.tw = reinterpret_cast<float *>(take(S * sizeof(float)));
     L.offsets = reinterpret_cast<int32_t *>(take((w->E + 1) * sizeof(int32_t)));
@@ -418,13 +512,14 @@ int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router, cons
     if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "layer workspace needs %zu bytes", need);
     if (!aligned16(workspace)) return fail(MOE_ERR_INVALID_ARG, "workspace not 16-byte aligned");
     LayerWs L = carve(w, T, k, mode, static_cast<char *>(workspace));
-    r = moe_router_topk(x, w_router, bias, T, w->H, w->E, k, L.logits, L.idx, L.tw, nullptr, 0, stream);
+    // the routing kernel also zeroes the FFN's GEMV counters on its way out
+    int n_ctr = 0;
+    int *ctr = gemv_counters(w, T, k, mode, L.ffn_ws, &n_ctr);
+    r = route(x, w_router, bias, T, w->H, w->E, k, L.idx, L.tw, L.offsets, L.sorted, L.pos, L.active, status,
+              L.route_ws, L.route_bytes, stream, ctr, n_ctr);
     if (r) return r;
-    r = moe_bucketize(L.idx, T, k, w->E, L.offsets, L.sorted, L.pos, L.active, status, stream);
-    if (r) return r;
-    r = moe_expert_ffn_tiered(w, x, T, k, L.offsets, L.sorted, L.active, L.y_slots,
-                              w->shared.n_experts == 1 ? L.y_shared : nullptr, L.ffn_ws, L.ffn_bytes, mode, status,
-                              stream);
+    r = expert_ffn(w, x, T, k, L.offsets, L.sorted, L.active, L.y_slots, w->shared.n_experts == 1 ? L.y_shared : nullptr,
+                   L.ffn_ws, L.ffn_bytes, mode, status, stream, true);
     if (r) return r;
     return moe_combine(L.y_slots, w->shared.n_experts == 1 ? L.y_shared : nullptr, L.tw, T, k, w->H, residual, out,
                        x_next, x_next_norm, stream);

@@ -8,7 +8,7 @@
 
 namespace moe {
 
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 512;
 
 __device__ __forceinline__ float block_sum(float v, float *red) {
     v = warp_sum(v);
@@ -31,26 +31,43 @@ __device__ __forceinline__ uint2 pack4(uint16_t a, uint16_t b, uint16_t c, uint1
                       static_cast<uint32_t>(c) | (static_cast<uint32_t>(d) << 16));
 }
 
+__device__ __forceinline__ void fma4(float4 &a, float w, const float4 &v) {
+    a.x = fmaf(w, v.x, a.x);
+    a.y = fmaf(w, v.y, a.y);
+    a.z = fmaf(w, v.z, a.z);
+    a.w = fmaf(w, v.w, a.w);
+}
+
 // One CTA per token; each thread owns 4-element chunks c = threadIdx.x + i*blockDim.
+// The k slot rows are read four at a time (independent loads in flight) and
+// added in slot order j = 0 .. k-1.
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const float *__restrict__ y, const float *__restrict__ ysh, const float *__restrict__ w,
                int T, int k, int H, const uint16_t *__restrict__ res, uint16_t *__restrict__ out,
                uint16_t *__restrict__ xnext, uint16_t *__restrict__ nnext, float eps) {
     __shared__ float red[32];
+    __shared__ float ws[MOE_MAX_TOPK];
     const int t = blockIdx.x;
     const int chunks = H / 4;
     const size_t row = static_cast<size_t>(t) * H;
+    if (threadIdx.x < k) ws[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
+    __syncthreads();
+    const float4 *yt = reinterpret_cast<const float4 *>(y + static_cast<size_t>(t) * k * H);
     float ss = 0.f;
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const float wj = w[static_cast<size_t>(t) * k + j];
-            const float4 v = reinterpret_cast<const float4 *>(y + (static_cast<size_t>(t) * k + j) * H)[c];
-            a.x = fmaf(wj, v.x, a.x);
-            a.y = fmaf(wj, v.y, a.y);
-            a.z = fmaf(wj, v.z, a.z);
-            a.w = fmaf(wj, v.w, a.w);
+        int j = 0;
+        for (; j + 4 <= k; j += 4) {
+            const float4 v0 = yt[static_cast<size_t>(j) * chunks + c];
+            const float4 v1 = yt[static_cast<size_t>(j + 1) * chunks + c];
+            const float4 v2 = yt[static_cast<size_t>(j + 2) * chunks + c];
+            const float4 v3 = yt[static_cast<size_t>(j + 3) * chunks + c];
+            fma4(a, ws[j], v0);
+            fma4(a, ws[j + 1], v1);
+            fma4(a, ws[j + 2], v2);
+            fma4(a, ws[j + 3], v3);
         }
+        for (; j < k; ++j) fma4(a, ws[j], yt[static_cast<size_t>(j) * chunks + c]);
         if (ysh) {
             const float4 v = reinterpret_cast<const float4 *>(ysh + row)[c];
             a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;

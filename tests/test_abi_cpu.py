@@ -116,3 +116,33 @@ def test_layer_workspace_sizes_grow_with_tokens():
     b = L.moe_layer_workspace_size(ctypes.byref(d), 4096, 10, 0)
     assert 0 < a < b
     assert b >= 4096 * 10 * 2048 * 4
+
+
+def _route(T=1, H=2048, E=512, k=10, ws=1 << 20, x=0x20000, wsp=0x40000):
+    L = B.lib()
+    p = ctypes.c_void_p(0x30000)
+    return L.moe_route(ctypes.c_void_p(x), p, None, T, H, E, k, p, p, p, p, p, p, None,
+                       ctypes.c_void_p(wsp) if wsp else None, ws, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), B.MOE_ERR_INVALID_ARG),
+    (dict(k=33, E=64), B.MOE_ERR_INVALID_ARG),          # k > MOE_MAX_TOPK
+    (dict(E=1025), B.MOE_ERR_INVALID_ARG),
+    (dict(H=100), B.MOE_ERR_INVALID_ARG),               # H % 64
+    (dict(x=0x20008), B.MOE_ERR_INVALID_ARG),           # misaligned x
+    (dict(ws=16), B.MOE_ERR_WORKSPACE),                 # smaller than logits + counter
+    (dict(wsp=0), B.MOE_ERR_WORKSPACE),
+    (dict(wsp=0x40008), B.MOE_ERR_INVALID_ARG),         # misaligned workspace
+])
+def test_route_rejects_bad_arguments(kw, code):
+    assert _route(**kw) == code
+    assert B.lib().moe_last_error()
+
+
+def test_route_workspace_size():
+    L = B.lib()
+    # fp32 logits [T][E] (256-byte aligned) plus 256 bytes for the counter
+    assert L.moe_route_workspace_size(1, 2048, 512, 10) == 2048 + 256
+    assert L.moe_route_workspace_size(3, 2048, 100, 10) == 1280 + 256
+    assert L.moe_route_workspace_size(0, 2048, 512, 10) == 256
