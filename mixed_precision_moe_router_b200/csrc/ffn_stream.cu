@@ -13,13 +13,18 @@
 //    16R rows, with R the largest power of two <= 8 such that a tile holds at
 //    most 32K codes.  Each CTA takes a contiguous, cost-balanced share of the
 //    gate_up tiles and then of the down tiles, so 8-, 4- and 3-bit experts
-//    spread evenly over the SMs.
-//  * One producer thread moves each tile into a stage of a shared-memory ring
+//    spread evenly over the SMs.  The prologue turns that share into a tile
+//    range per slot, so walking the list is integer increments.
+//  * Two consumer groups of 8 warps take alternate tiles of the CTA's list,
+//    so one group's barriers, epilogue and waits overlap the other's
+//    arithmetic.  Each group stages its own tiles into a shared-memory ring
 //    with TMA tensor copies (cp.async.bulk.tensor) that complete on the
-//    stage's mbarrier: one copy per 128-byte column chunk of the tile (8R gate
-//    rows and their 8R up rows in one 4-D box), plus one for the scales.  The
-//    copies store the tile with the TMA swizzle, which makes the fragment
-//    reads below bank-conflict free.
+//    stage's mbarrier.  A gate_up tile is one 5-D copy when its rows are
+//    whole 128-byte lines: [gate|up][8R rows][lines, padded to an odd count
+//    with zero-filled out-of-range lines][128 bytes]; otherwise, and for down
+//    tiles, one copy per 128-byte column chunk.  Either way the copies store
+//    the tile with the TMA swizzle, which makes the fragment reads below
+//    bank-conflict free, and one more copy brings the scales.
 //  * 8 compute warps split a tile into R row subtiles x 8/R K slices.  For
 //    each 32-weight block a warp turns its codes into exact fp16 integers
 //    (|q| <= 127), multiplies them with fp16 activation fragments on the
@@ -46,10 +51,11 @@
 
 namespace moe {
 
-constexpr int kWarps = 8;                          // compute warps
-constexpr int kThreads = kWarps * 32;
-constexpr int kBlockThreads = kThreads + 32;       // + one producer warp (one thread issues)
-constexpr int kBarCompute = 1;                     // named barrier of the compute warps
+constexpr int kWarps = 8;                          // compute warps of a group (they split a tile)
+constexpr int kThreads = kWarps * 32;              // threads of a group
+constexpr int kGroups = 2;                         // consumer groups, taking alternate tiles
+constexpr int kBlockThreads = kGroups * kThreads;
+constexpr int kBarGroup0 = 1;                      // named barrier of group g: kBarGroup0 + g
 constexpr int kMaxStages = 6;
 constexpr int kStageBytes = 40 * 1024;
 constexpr int kMaxK = 2048;
@@ -79,6 +85,8 @@ struct Geo {
     int W, lw;       // code swizzle width (and log2): the tile is stored as column chunks of W bytes
     int Ws;          // scale swizzle width, 0 when the scales come as plain bulk copies
     int nb, bps;     // 32-weight blocks per row, blocks per K slice
+    int pad, nc1;    // padded row-major layout (one 5-D copy per tile): 128-byte lines per row
+    int cb;          // code bytes of a staged tile (the scales follow)
 };
 
 __host__ __device__ __forceinline__ Geo geo(int K, int bits) {
@@ -95,10 +103,32 @@ __host__ __device__ __forceinline__ Geo geo(int K, int bits) {
     g.nb = K / 32;
     const int S = kWarps / g.R;
     g.bps = ((g.nb + S - 1) / S + 1) & ~1;  // even, so blocks go in pairs
+    g.pad = 0;
+    g.nc1 = 0;
+    g.cb = g.rows * g.rb;
     return g;
 }
 
-__host__ __device__ __forceinline__ int stage_bytes(const Geo &g) { return g.rows * (g.rb + g.sb); }
+// gate_up tiles: when the rows are whole 128-byte lines and the padded tile
+// fits a stage, one 5-D copy stages the whole tile.  Each row then takes nc1
+// lines: its rb / 128 lines plus one or two out-of-range lines (zero-filled,
+// no memory traffic) so that nc1 is odd; the 128-byte swizzle then puts the 8
+// rows an mma reads at one offset into 8 different 16-byte bank groups.
+__host__ __device__ __forceinline__ Geo geo_gu(int K, int bits) {
+    Geo g = geo(K, bits);
+    if (g.W == 128) {
+        const int n = g.rb / 128;
+        const int nc1 = n + 1 + (n & 1);
+        if (nc1 <= 256 && g.rows * (nc1 * 128 + g.sb) <= kStageBytes) {
+            g.pad = 1;
+            g.nc1 = nc1;
+            g.cb = g.rows * nc1 * 128;
+        }
+    }
+    return g;
+}
+
+__host__ __device__ __forceinline__ int stage_bytes(const Geo &g) { return g.cb + g.rows * g.sb; }
 
 // XOR that the TMA swizzle of width W applies to the 16-byte chunk index of
 // row r of a box (boxes start on a swizzle-atom boundary and hold a multiple
@@ -107,10 +137,25 @@ __device__ __forceinline__ int swz(int r, int W) {
     return W == 128 ? (r & 7) << 4 : (W == 64 ? ((r >> 1) & 3) << 4 : (W == 32 ? ((r >> 2) & 1) << 4 : 0));
 }
 
-// Byte offset of byte o of row r in a tile of `rows` rows stored as column
-// chunks of W bytes with the TMA swizzle (xr = swz(r, W)).
+// Byte offset of byte o of row r in a staged tile.  Column-chunk layout: the
+// tile is stored as column chunks of W bytes with the TMA swizzle (xr =
+// swz(r, W)).  Padded layout: row r starts at 128-byte line xr = r * nc1 and
+// the swizzle permutes the 16-byte units of line L by L mod 8.
+template <bool PAD>
 __device__ __forceinline__ int tile_off(int o, int r, const Geo &G, int xr) {
-    return (o >> G.lw) * (G.rows << G.lw) + (r << G.lw) + ((o & (G.W - 1)) ^ xr);
+    if constexpr (PAD) {
+        const int line = xr + (o >> 7);
+        return (line << 7) + ((o & 127) ^ ((line & 7) << 4));
+    } else {
+        return (o >> G.lw) * (G.rows << G.lw) + (r << G.lw) + ((o & (G.W - 1)) ^ xr);
+    }
+}
+
+// xr of row r for tile_off
+template <bool PAD>
+__device__ __forceinline__ int row_x(int r, const Geo &G) {
+    if constexpr (PAD) return r * G.nc1;
+    else return swz(r, G.W);
 }
 
 
@@ -120,11 +165,22 @@ __host__ __device__ __forceinline__ int xf_col_stride(int K) { return (K / 32) *
 
 __host__ __device__ __forceinline__ int down_ntiles(int I) { return I <= 1024 ? 2 : 1; }
 
-__host__ __device__ __forceinline__ int xf_bytes(int H, int I) {
-    const int a = kTokPerPass * xf_col_stride(H);
-    const int b = 8 * down_ntiles(I) * xf_col_stride(I);
-    return a > b ? a : b;
+// Fragment columns a pass can use with at most T tokens: gate_up one per
+// token (up to 8), down hi + lo per token in n-tiles of 8 (column 8*(n/4) +
+// 2*(n%4) + 1 is the last one written for token n).
+__host__ __device__ __forceinline__ int xf_bytes(int H, int I, int T) {
+    const int cg = T < kTokPerPass ? T : kTokPerPass;
+    const int nd = T < 4 * down_ntiles(I) ? T : 4 * down_ntiles(I);
+    const int cd = nd <= 4 ? 2 * nd : 8 + 2 * (nd - 4);
+    const int a = cg * xf_col_stride(H);
+    const int b = cd * xf_col_stride(I);
+    const int m = a > b ? a : b;
+    return (m + 127) & ~127;
 }
+
+// Thread index within its consumer group, and the group.
+__device__ __forceinline__ int gtid() { return threadIdx.x & (kThreads - 1); }
+__device__ __forceinline__ int group_of_thread() { return threadIdx.x / kThreads; }
 
 // tokens of one pass: gate_up tiles use one column per token, down tiles two
 // (h = hi + lo) in n-tiles of 8 columns
@@ -177,6 +233,8 @@ __device__ __forceinline__ int tiles_per_slot(const FfnParams &p, int phase) {
 struct Sched {
     long long *tc0, *tc1;    // cost of one tile of each slot
     long long *pre0, *pre1;  // inclusive prefix sums of the slots' total costs
+    int2 *rng0, *rng1;       // per slot: this CTA's tiles of it, [b0, b1)
+    int *fl;                 // per phase: first and last slot with tiles in this CTA (last < first: none)
 };
 
 // floor(x / y) for 0 <= x < 2^52, 0 < y: a double quotient corrected to the
@@ -190,59 +248,57 @@ __device__ __forceinline__ long long div_floor(long long x, long long y) {
 
 // This CTA's tiles, in order: its cost-balanced contiguous share of all
 // gate_up tiles (phase 0), then of all down tiles (phase 1).  phase == 2 once
-// the list is exhausted.
+// the list is exhausted.  The per-slot tile ranges are computed once in the
+// prologue, so stepping is a few integer operations.
 struct TileIt {
     int phase, a, b, b1;  // current tile: slot a, tile b; b1 ends this slot's range
-    long long lo, hi;     // this CTA's cost range in the current phase
 };
 
-__device__ __forceinline__ bool it_slot(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
-    const long long *pre = it.phase == 0 ? sc.pre0 : sc.pre1;
-    const long long *tc = it.phase == 0 ? sc.tc0 : sc.tc1;
-    const long long nt = tiles_per_slot(p, it.phase);
-    for (; it.a < n_slots; ++it.a) {
-        const long long tb = tc[it.a];
-        const long long off = pre[it.a] - nt * tb;
-        if (off >= it.hi) return false;
-        const long long b0 = it.lo > off ? div_floor(it.lo - off + tb - 1, tb) : 0;
-        long long b1 = div_floor(it.hi - off + tb - 1, tb);
-        if (b1 > nt) b1 = nt;
-        if (b0 < b1) {
-            it.b = static_cast<int>(b0);
-            it.b1 = static_cast<int>(b1);
-            return true;
-        }
-    }
-    return false;
+// Tiles of a slot (nt tiles of cost tb) that start before cost offset x from
+// the slot's start: ceil(x / tb) clamped to [0, nt].  A float quotient
+// corrected to the exact integer (the quotient is below nt <= 256 here).
+__device__ __forceinline__ int tiles_before(long long x, long long tb, int nt) {
+    if (x <= 0) return 0;
+    if (x >= nt * tb) return nt;
+    long long q = static_cast<long long>(__fdividef(static_cast<float>(x), static_cast<float>(tb)));
+    while (q * tb < x) ++q;
+    while (q > 0 && (q - 1) * tb >= x) --q;
+    return static_cast<int>(q);
 }
 
-__device__ __forceinline__ bool it_phase(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it, int phase) {
+__device__ __forceinline__ bool it_enter(const Sched &sc, TileIt &it, int phase) {
+    const int f = sc.fl[2 * phase], l = sc.fl[2 * phase + 1];
+    if (f > l) return false;
+    const int2 r = (phase == 0 ? sc.rng0 : sc.rng1)[f];
     it.phase = phase;
-    const long long *pre = phase == 0 ? sc.pre0 : sc.pre1;
-    const long long total = pre[n_slots - 1];
-    it.lo = div_floor(total * blockIdx.x, gridDim.x);
-    it.hi = div_floor(total * (blockIdx.x + 1), gridDim.x);
-    int a0 = 0, a1 = n_slots;  // first slot whose cost range ends after lo
-    while (a0 < a1) {
-        const int m = (a0 + a1) >> 1;
-        if (pre[m] > it.lo) a1 = m; else a0 = m + 1;
-    }
-    it.a = a0;
-    return it_slot(p, sc, n_slots, it);
+    it.a = f;
+    it.b = r.x;
+    it.b1 = r.y;
+    return true;
 }
 
 __device__ __forceinline__ void it_begin(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
+    (void)p;
     it.phase = 2;
     if (n_slots == 0) return;
-    if (!it_phase(p, sc, n_slots, it, 0) && !it_phase(p, sc, n_slots, it, 1)) it.phase = 2;
+    if (!it_enter(sc, it, 0) && !it_enter(sc, it, 1)) it.phase = 2;
 }
 
+// Slots strictly between a phase's first and last slot lie wholly inside the
+// CTA's contiguous cost range, so each of them has tiles here.
 __device__ __forceinline__ void it_next(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
+    (void)p;
+    (void)n_slots;
     if (it.phase == 2) return;
     if (++it.b < it.b1) return;
-    ++it.a;
-    if (it_slot(p, sc, n_slots, it)) return;
-    if (it.phase == 0 && it_phase(p, sc, n_slots, it, 1)) return;
+    if (it.a < sc.fl[2 * it.phase + 1]) {
+        ++it.a;
+        const int2 r = (it.phase == 0 ? sc.rng0 : sc.rng1)[it.a];
+        it.b = r.x;
+        it.b1 = r.y;
+        return;
+    }
+    if (it.phase == 0 && it_enter(sc, it, 1)) return;
     it.phase = 2;
 }
 
@@ -281,11 +337,11 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
     return d;
 }
 
-template <int BITS>
+template <int BITS, bool PAD>
 __device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int r, int xr, int b, int t,
                                          uint32_t (&P)[4]) {
     if constexpr (BITS == 8) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(tile + tile_off(32 * b + 8 * t, r, G, xr));
+        const uint2 w = *reinterpret_cast<const uint2 *>(tile + tile_off<PAD>(32 * b + 8 * t, r, G, xr));
         const uint32_t u0 = w.x ^ 0x80808080u, u1 = w.y ^ 0x80808080u;  // c = q + 128
         constexpr uint32_t kBias = 0x64806480u;                         // 1024 + 128
         P[0] = hsub2(prmt(u0, 0x64646464u, 0x4140u), kBias);
@@ -294,7 +350,7 @@ __device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int 
         P[3] = hsub2(prmt(u1, 0x64646464u, 0x4342u), kBias);
     } else if constexpr (BITS == 4) {
         // nibble i of the word at byte 16b + 4t is weight 8t + i (c = q + 8)
-        const uint32_t v = *reinterpret_cast<const uint32_t *>(tile + tile_off(16 * b + 4 * t, r, G, xr));
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(tile + tile_off<PAD>(16 * b + 4 * t, r, G, xr));
         const uint32_t v8 = v >> 8;
         P[0] = hsub2((v & 0x000F000Fu) | 0x64006400u, 0x64086408u);   // 1024 + c - 1032
         P[1] = hsub2((v & 0x00F000F0u) | 0x54005400u, 0x54805480u);   // 64 + c - 72
@@ -303,8 +359,8 @@ __device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int 
     } else {
         // low plane: bits 0-1 of weight 8t+i at bit 2i of the u16 at byte 8b+2t;
         // high plane: bit 2 at bit i of byte K/4 + 4b + t (c = q + 4)
-        const uint32_t lo16 = *reinterpret_cast<const uint16_t *>(tile + tile_off(8 * b + 2 * t, r, G, xr));
-        const uint32_t hb = tile[tile_off(G.K / 4 + 4 * b + t, r, G, xr)];
+        const uint32_t lo16 = *reinterpret_cast<const uint16_t *>(tile + tile_off<PAD>(8 * b + 2 * t, r, G, xr));
+        const uint32_t hb = tile[tile_off<PAD>(G.K / 4 + 4 * b + t, r, G, xr)];
         const uint32_t X = prmt(lo16, 0u, 0x4140u);  // weights i and i+4 16 bits apart
         const uint32_t Y = hb * 0x4004u;             // hb << 2 | hb << 14
         P[0] = hsub2((X & 0x00030003u) | (Y & 0x00040004u) | 0x64006400u, 0x64046404u);           // 1024 + c - 1028
@@ -331,13 +387,19 @@ __device__ __forceinline__ float2 half2_to_float2(uint32_t v) {
 // One warp's share of a tile: stage rows rA (accumulator rows g) and rB (rows
 // g + 8), blocks [b0, b1), NT n-tiles of 8 columns.  acc[nt] follows the m16n8
 // accumulator layout: (row g, col 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
-template <int BITS, int NT>
-__device__ __forceinline__ void warp_tile(const uint8_t *stage, const Geo &G, int rA, int rB, int b0, int b1,
-                                          const uint8_t *xf, int cs, int ncol0, int ncol1, float (&acc)[2][4]) {
+struct TileAcc {
+    float acc[2][4];
+};
+
+template <int BITS, int NT, bool PAD>
+__device__ __forceinline__ TileAcc warp_tile(const uint8_t *stage, const Geo G, int rA, int rB, int b0, int b1,
+                                          const uint8_t *xf, int cs, int ncol0, int ncol1) {
+    TileAcc out;
+    float (&acc)[2][4] = out.acc;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int xa = swz(rA, G.W), xb = swz(rB, G.W);
+    const int xa = row_x<PAD>(rA, G), xb = row_x<PAD>(rB, G);
     // scales: [row][sb] after the codes, swizzled at width Ws (or plain)
-    const uint8_t *scl = stage + G.rows * G.rb;
+    const uint8_t *scl = stage + G.cb;
     const int sxa = G.Ws ? swz(rA, G.Ws) : 0, sxb = G.Ws ? swz(rB, G.Ws) : 0;
     const uint8_t *xg = xf + g * cs + t * 16;
 #pragma unroll
@@ -351,8 +413,8 @@ __device__ __forceinline__ void warp_tile(const uint8_t *stage, const Geo &G, in
         uint32_t PA[2][4], PB[2][4];
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
-            dequant8<BITS>(stage, G, rA, xa, b + bb, t, PA[bb]);
-            dequant8<BITS>(stage, G, rB, xb, b + bb, t, PB[bb]);
+            dequant8<BITS, PAD>(stage, G, rA, xa, b + bb, t, PA[bb]);
+            dequant8<BITS, PAD>(stage, G, rB, xb, b + bb, t, PB[bb]);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -380,6 +442,7 @@ __device__ __forceinline__ void warp_tile(const uint8_t *stage, const Geo &G, in
             }
         }
     }
+    return out;
 }
 
 // fp32 -> fp16 bits, noting values outside the fp16 range (or NaN)
@@ -412,10 +475,14 @@ __device__ __forceinline__ uint4 pack_frag(const uint16_t (&v)[8], int bits) {
 
 struct StreamSmem {
     uint8_t *stages;
-    uint8_t *xf;
-    float4 *red;
-    uint64_t *full, *empty;  // per stage: copies landed / stage consumed
+    uint8_t *xf;             // [kGroups][xf_size]
+    int xf_size;
+    float4 *red;             // [kGroups][kWarps * 32]
+    uint64_t *full;          // per stage: copies landed
     int *abort;
+    // per group: how many of its tiles (g, g + 2, ...) are staged, and the
+    // iterator at the next one to stage
+    struct Ahead { TileIt it; int n; } *ahead;
     SlotTabs st;
     Sched sc;
     int *tier, *jloc;   // per slot: shelf index (n_tiers = shared) and index within the shelf
@@ -453,6 +520,15 @@ __device__ __forceinline__ void tma_4d(void *dst, const CUtensorMap *map, int x,
         : "memory");
 }
 
+__device__ __forceinline__ void tma_5d(void *dst, const CUtensorMap *map, int x, int y, int z, int w, int v,
+                                       uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Stage the codes and scales of tile (phase, a, tile) into `dst`, completing
 // on `bar`: a gate_up tile is its 8R gate rows and the matching 8R up rows, a
 // down tile 16R consecutive rows; codes as column chunks of W bytes.
@@ -462,12 +538,15 @@ __device__ __forceinline__ void issue_tile(const FfnParams &p, const StreamMaps 
     const Geo &G = S.geo[phase * 3 + bits_idx(S.st.bits[a])];
     const int ti = S.tier[a], j = S.jloc[a];
     const TierPtrs &T = S.tp[ti];
-    uint8_t *dsc = dst + G.rows * G.rb;
+    uint8_t *dsc = dst + G.cb;
     const int chunk = G.rows << G.lw;  // bytes of one column chunk of the tile
-    mbar_expect_tx(bar, static_cast<uint32_t>(G.rows) * (G.rb + G.sb));
+    mbar_expect_tx(bar, static_cast<uint32_t>(stage_bytes(G)));
     if (phase == 0) {
         const int half = 8 * G.R, P = tile * half;
-        for (int c = 0; c * G.W < G.rb; ++c) tma_4d(dst + c * chunk, &M.gq[ti], c * G.W, P, 0, j, bar);
+        if (G.pad)  // one box: [gate|up][8R rows][nc1 lines][128 bytes]
+            tma_5d(dst, &M.gq[ti], 0, 0, P, 0, j, bar);
+        else
+            for (int c = 0; c * G.W < G.rb; ++c) tma_4d(dst + c * chunk, &M.gq[ti], c * G.W, P, 0, j, bar);
         if (G.Ws) {
             tma_4d(dsc, &M.gs[ti], 0, P, 0, j, bar);
         } else {
@@ -487,7 +566,7 @@ __device__ __forceinline__ void issue_tile(const FfnParams &p, const StreamMaps 
     }
 }
 
-// Barrier of the compute warps that also ANDs a flag over them.
+// Barrier of one consumer group that also ANDs a flag over it.
 __device__ __forceinline__ bool bar_and(bool ok) {
     uint32_t r;
     asm volatile(
@@ -496,20 +575,21 @@ __device__ __forceinline__ bool bar_and(bool ok) {
         "bar.red.and.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(ok ? 1u : 0u), "n"(kBarCompute), "n"(kThreads)
+        : "r"(ok ? 1u : 0u), "r"(kBarGroup0 + group_of_thread()), "n"(kThreads)
         : "memory");
     return r != 0;
 }
 
-__device__ __forceinline__ void bar_compute() { named_bar_sync(kBarCompute, kThreads); }
+__device__ __forceinline__ void bar_compute() { named_bar_sync(kBarGroup0 + group_of_thread(), kThreads); }
 
 
 // gate_up fragments of one pass: column n holds the token of entry pass*8 + n.
-__device__ __forceinline__ void build_xf_gu(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
-                                            int bits, uint8_t *xf, bool &bad) {
+__device__ __forceinline__ bool build_xf_gu(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
+                                         int bits, uint8_t *xf) {
+    bool bad = false;
     const int H = p.w.H, nb = H / 32, cs = xf_col_stride(H);
     const int n_chunks = ntok * nb * 4;
-    for (int i = threadIdx.x; i < n_chunks; i += kThreads) {
+    for (int i = gtid(); i < n_chunks; i += kThreads) {
         const int n = i / (nb * 4), rem = i % (nb * 4);  // rem = 4 * block + t
         int tok, row;
         slot_entry(p, st, a, pass * kTokPerPass + n, tok, row);
@@ -523,16 +603,18 @@ __device__ __forceinline__ void build_xf_gu(const FfnParams &p, const SlotTabs &
         }
         *reinterpret_cast<uint4 *>(xf + n * cs + rem * 16) = pack_frag(v, bits);
     }
+    return bad;
 }
 
 // down fragments of one pass: in n-tile nt, column 2m holds hi and column
 // 2m + 1 lo of h for the token of entry pass*tp + 4nt + m.
-__device__ __forceinline__ void build_xf_dn(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
-                                            int bits, uint8_t *xf, bool &bad) {
+__device__ __forceinline__ bool build_xf_dn(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
+                                         int bits, uint8_t *xf) {
+    bool bad = false;
     const int I = p.w.I, nb = I / 32, cs = xf_col_stride(I);
     const int tp = tokens_per_pass(1, I);
     const int n_chunks = ntok * nb * 4;
-    for (int i = threadIdx.x; i < n_chunks; i += kThreads) {
+    for (int i = gtid(); i < n_chunks; i += kThreads) {
         const int n = i / (nb * 4), rem = i % (nb * 4);
         int tok, row;
         slot_entry(p, st, a, pass * tp + n, tok, row);
@@ -550,27 +632,29 @@ __device__ __forceinline__ void build_xf_dn(const FfnParams &p, const SlotTabs &
         *reinterpret_cast<uint4 *>(xf + col * cs + rem * 16) = pack_frag(hi, bits);
         *reinterpret_cast<uint4 *>(xf + (col + 1) * cs + rem * 16) = pack_frag(lo, bits);
     }
+    return bad;
 }
 
 // This warp's partial sums of the resident tile, to red[warp][lane].
 template <int BITS>
 __device__ __forceinline__ void compute_tile(const FfnParams &p, const Geo &G, int phase, const uint8_t *stage,
                                              const uint8_t *xf, int ntok, float4 *red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = gtid() >> 5, lane = threadIdx.x & 31;
     const int r = warp % G.R, s = warp / G.R;
     const int b0 = min(G.nb, s * G.bps), b1 = min(G.nb, (s + 1) * G.bps);
     const int cs = xf_col_stride(G.K);
     const int g = lane >> 2;
-    float acc[2][4];
     if (phase == 0) {
-        warp_tile<BITS, 1>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs, ntok, 0, acc);
+        const TileAcc t = G.pad ? warp_tile<BITS, 1, true>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs, ntok, 0)
+                                : warp_tile<BITS, 1, false>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs, ntok, 0);
+        const float(&acc)[2][4] = t.acc;
         red[warp * 32 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
     } else {
         const int nc0 = 2 * max(0, min(4, ntok)), nc1 = 2 * max(0, min(4, ntok - 4));
-        if (down_ntiles(p.w.I) == 2)
-            warp_tile<BITS, 2>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1, acc);
-        else
-            warp_tile<BITS, 1>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1, acc);
+        const TileAcc t = down_ntiles(p.w.I) == 2
+                              ? warp_tile<BITS, 2, false>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1)
+                              : warp_tile<BITS, 1, false>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1);
+        const float(&acc)[2][4] = t.acc;
         // hi + lo columns of each token
         red[warp * 32 + lane] =
             make_float4(acc[0][0] + acc[0][1], acc[0][2] + acc[0][3], acc[1][0] + acc[1][1], acc[1][2] + acc[1][3]);
@@ -586,7 +670,7 @@ __device__ __forceinline__ void epilogue(const FfnParams &p, const SlotTabs &st,
     if (phase == 0) {
         const int I = p.w.I;
         const int n_out = R * 8 * ntok;
-        for (int o = threadIdx.x; o < n_out; o += kThreads) {
+        for (int o = gtid(); o < n_out; o += kThreads) {
             const int n = o % ntok, rg = o / ntok, g = rg % 8, r = rg / 8;
             const int lane = 4 * g + (n >> 1), sub = n & 1;
             float gate = 0.f, up = 0.f;
@@ -602,7 +686,7 @@ __device__ __forceinline__ void epilogue(const FfnParams &p, const SlotTabs &st,
     } else {
         const int H = p.w.H, tp = tokens_per_pass(1, p.w.I);
         const int n_out = R * 16 * ntok;
-        for (int o = threadIdx.x; o < n_out; o += kThreads) {
+        for (int o = gtid(); o < n_out; o += kThreads) {
             const int rr = o % (R * 16), n = o / (R * 16);
             const int r = rr / 16, row16 = rr % 16;
             const int lane = 4 * (row16 % 8) + (n & 3), idx = 2 * (n >> 2) + row16 / 8;
@@ -617,56 +701,67 @@ __device__ __forceinline__ void epilogue(const FfnParams &p, const SlotTabs &st,
     }
 }
 
+// Advance an iterator by `n` tiles.
+__device__ __forceinline__ void it_skip(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it, int n) {
+    for (int k = 0; k < n; ++k) it_next(p, sc, n_slots, it);
+}
+
 // The persistent FFN kernel body; `n_slots` slots are described in S.
+//
+// Two consumer groups of 8 warps take alternate tiles of the CTA's list
+// (group g: tiles g, g + 2, ...), so one group's barriers, epilogue and
+// dependency waits overlap the other's dequantise-and-multiply.  Tile i lives
+// in stage i % nstages; nstages is even, so a stage always serves the same
+// group.  The first nstages tiles are staged in the prologue; afterwards a
+// group stages its tile i + nstages as soon as its barrier after the last
+// pass over tile i shows the stage drained.  A group therefore never waits
+// on copies the other group issues, and a group waiting on another slot's
+// gate_up count cannot hold back the tiles that produce that count.
 __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const StreamMaps &M, StreamSmem &S, int n_slots,
                                                 int nstages) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = group_of_thread(), gt = gtid(), lane = threadIdx.x & 31;
     const int I = p.w.I;
-    if (warp >= kWarps) {
-        // producer: one thread stages the CTA's tiles in order
-        if (lane != 0) return;
-        TileIt pf;
-        it_begin(p, S.sc, n_slots, pf);
-        int i = 0;
-        for (; pf.phase < 2; ++i, it_next(p, S.sc, n_slots, pf)) {
-            if (*static_cast<volatile int *>(S.abort)) break;
-            const int s = i % nstages;
-            if (!mbar_wait(&S.empty[s], ((i / nstages) & 1) ^ 1)) {
-                status_or(p.status, MOE_STATUS_TIMEOUT);
-                *static_cast<volatile int *>(S.abort) = 1;
-                break;
-            }
-            issue_tile(p, M, S, pf.phase, pf.a, pf.b, S.stages + static_cast<size_t>(s) * kStageBytes, &S.full[s]);
-        }
-        // the copies still in flight must land before the CTA exits
-        for (int k = i - nstages < 0 ? 0 : i - nstages; k < i; ++k)
-            if (!mbar_wait(&S.full[k % nstages], (k / nstages) & 1)) status_or(p.status, MOE_STATUS_TIMEOUT);
-        return;
-    }
-    // compute warps: every branch below depends only on values that are the
-    // same in all of them, so they pass the same barriers in the same order
+    uint8_t *xf = S.xf + grp * S.xf_size;
+    float4 *red = S.red + grp * kWarps * 32;
     const int gu_tiles = tiles_per_slot(p, 0);
     TileIt it;
     it_begin(p, S.sc, n_slots, it);
+    it_skip(p, S.sc, n_slots, it, grp);
+    if (gt == 0) {
+        // the group leader stages the group's first nstages / 2 tiles
+        StreamSmem::Ahead &ah = S.ahead[grp];
+        ah.it = it;
+        ah.n = 0;
+        while (ah.n < nstages / kGroups && ah.it.phase < 2) {
+            const int k = grp + kGroups * ah.n;
+            issue_tile(p, M, S, ah.it.phase, ah.it.a, ah.it.b, S.stages + static_cast<size_t>(k) * kStageBytes,
+                       &S.full[k]);
+            it_skip(p, S.sc, n_slots, ah.it, kGroups);
+            ++ah.n;
+        }
+    }
     int xf_key = -1;      // (slot, phase, pass) whose fragments xf holds
     int ready_slot = -1;  // a slot whose h is known to be complete
     int pend_tiles = 0;   // gate_up tiles of the current slot not yet counted
+    int consumed = 0;     // this group's tiles whose copies have landed
     bool bad = false;
-    for (int i = 0; it.phase < 2; ++i) {
+    int i = grp;
+    for (; it.phase < 2; i += kGroups) {
         const int phase = it.phase, a = it.a, tile = it.b;
         const int s = i % nstages;
         bool ok = mbar_wait(&S.full[s], (i / nstages) & 1);
         // one thread polls the slot's gate_up count (with backoff, so that
         // pollers do not crowd the counters' L2 slice); the barrier passes
         // the result on and orders every thread's reads of h after it
-        if (phase == 1 && a != ready_slot && threadIdx.x == 0) ok = ok && wait_geq_backoff(p.ctr + a, gu_tiles);
-        if (!bar_and(ok)) {
-            if (threadIdx.x == 0) {
+        if (phase == 1 && a != ready_slot && gt == 0) ok = ok && wait_geq_backoff(p.ctr + a, gu_tiles);
+        if (!bar_and(ok && !*static_cast<volatile int *>(S.abort))) {
+            if (gt == 0) {
                 status_or(p.status, MOE_STATUS_TIMEOUT);
                 *static_cast<volatile int *>(S.abort) = 1;
             }
             break;
         }
+        ++consumed;
         if (phase == 1) ready_slot = a;
         const uint8_t *stage = S.stages + static_cast<size_t>(s) * kStageBytes;
         const int bits = S.st.bits[a], cnt = S.st.count[a];
@@ -677,36 +772,42 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const Stream
             const int ntok = min(tp, cnt - pass * tp);
             const int key = (a * 2 + phase) * 65536 + pass;
             if (key != xf_key) {  // the last readers of xf passed a barrier since
-                if (phase == 0)
-                    build_xf_gu(p, S.st, a, pass, ntok, bits, S.xf, bad);
-                else
-                    build_xf_dn(p, S.st, a, pass, ntok, bits, S.xf, bad);
+                bad |= phase == 0 ? build_xf_gu(p, S.st, a, pass, ntok, bits, xf)
+                                  : build_xf_dn(p, S.st, a, pass, ntok, bits, xf);
                 xf_key = key;
                 bar_compute();
             }
             if (bits == 8)
-                compute_tile<8>(p, G, phase, stage, S.xf, ntok, S.red);
+                compute_tile<8>(p, G, phase, stage, xf, ntok, red);
             else if (bits == 4)
-                compute_tile<4>(p, G, phase, stage, S.xf, ntok, S.red);
+                compute_tile<4>(p, G, phase, stage, xf, ntok, red);
             else
-                compute_tile<3>(p, G, phase, stage, S.xf, ntok, S.red);
-            if (pass == np - 1) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.empty[s]);  // this warp is done with the stage
-            }
+                compute_tile<3>(p, G, phase, stage, xf, ntok, red);
             bar_compute();
-            epilogue(p, S.st, phase, a, tile, pass, ntok, S.red);
+            if (pass == np - 1 && gt == 0) {
+                // every warp of the group is past its reads of the stage:
+                // stage this group's tile i + nstages into it
+                StreamSmem::Ahead &ah = S.ahead[grp];
+                if (ah.it.phase < 2) {
+                    const int k = grp + kGroups * ah.n;  // == i + nstages
+                    issue_tile(p, M, S, ah.it.phase, ah.it.a, ah.it.b,
+                               S.stages + static_cast<size_t>(k % nstages) * kStageBytes, &S.full[k % nstages]);
+                    it_skip(p, S.sc, n_slots, ah.it, kGroups);
+                    ++ah.n;
+                }
+            }
+            epilogue(p, S.st, phase, a, tile, pass, ntok, red);
             if (pass + 1 < np) bar_compute();  // red is written again by the next pass
         }
-        it_next(p, S.sc, n_slots, it);
+        it_skip(p, S.sc, n_slots, it, kGroups);
         if (phase == 0) {
-            // when this CTA leaves the slot, count its gate_up tiles of it:
+            // when this group leaves the slot, count its gate_up tiles of it:
             // after every thread's h writes (barrier) and a fence, and before
-            // this CTA waits on any other slot's count
+            // this group waits on any other slot's count
             ++pend_tiles;
             if (it.phase != 0 || it.a != a) {
                 bar_compute();
-                if (threadIdx.x == 0) {
+                if (gt == 0) {
                     __threadfence();
                     atomicAdd(p.ctr + a, pend_tiles);
                 }
@@ -715,6 +816,14 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const Stream
         }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(p.status, MOE_STATUS_FP16_RANGE);
+    // after an abort, copies this group staged but never consumed must land
+    // before the CTA exits (on a normal exit there are none)
+    if (gt == 0) {
+        for (int m = consumed; m < S.ahead[grp].n; ++m) {
+            const int k = grp + kGroups * m;
+            if (!mbar_wait(&S.full[k % nstages], (k / nstages) & 1)) status_or(p.status, MOE_STATUS_TIMEOUT);
+        }
+    }
 }
 
 __global__ void __launch_bounds__(kBlockThreads, 1)
@@ -722,11 +831,12 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     extern __shared__ __align__(1024) uint8_t smem[];
     StreamSmem S;
     S.stages = smem;
+    S.xf_size = xf_bytes(p.w.H, p.w.I, p.T);
     S.xf = smem + static_cast<size_t>(nstages) * kStageBytes;
-    S.red = reinterpret_cast<float4 *>(S.xf + xf_bytes(p.w.H, p.w.I));
-    S.full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(S.red) + kRedBytes);
-    S.empty = S.full + kMaxStages;
-    S.tp = reinterpret_cast<TierPtrs *>(S.empty + kMaxStages);
+    S.red = reinterpret_cast<float4 *>(S.xf + kGroups * S.xf_size);
+    S.full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(S.red) + kGroups * kRedBytes);
+    S.ahead = reinterpret_cast<StreamSmem::Ahead *>(S.full + kMaxStages);
+    S.tp = reinterpret_cast<TierPtrs *>(S.ahead + kGroups);
     S.geo = reinterpret_cast<Geo *>(S.tp + MOE_MAX_TIERS + 1);
     S.abort = reinterpret_cast<int *>(S.geo + 6);
     int *tabs = S.abort + 2;
@@ -748,8 +858,11 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     S.sc.tc1 = sched + max_slots;
     S.sc.pre0 = sched + 2 * max_slots;
     S.sc.pre1 = sched + 3 * max_slots;
+    S.sc.rng0 = reinterpret_cast<int2 *>(sched + 4 * max_slots);
+    S.sc.rng1 = S.sc.rng0 + max_slots;
+    S.sc.fl = reinterpret_cast<int *>(S.sc.rng1 + max_slots);
     // copies of the routing tables: active list and expert offsets
-    int *act_s = reinterpret_cast<int *>(sched + 4 * max_slots);
+    int *act_s = S.sc.fl + 4;
     int *off_s = act_s + max_slots;
     // one round of independent global loads fills every table below
     const int S_ = p.T * p.k;
@@ -790,16 +903,14 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
         S.tp[t].bits = p.w.shared.bits;
         S.tp[t].first = p.E;
         S.tp[t].n = 1;
-        for (int st = 0; st < nstages; ++st) {
-            mbar_init(&S.full[st], 1);  // the producer's expect_tx arrival
-            mbar_init(&S.empty[st], kWarps);     // one per compute warp
-        }
+        for (int st = 0; st < nstages; ++st) mbar_init(&S.full[st], 1);  // the stager's expect_tx arrival
         *S.abort = 0;
         mbar_fence_init();
     }
     if (threadIdx.x < 6) {
         const int phase = threadIdx.x / 3, bi = threadIdx.x % 3;
-        S.geo[threadIdx.x] = geo(phase == 0 ? p.w.H : p.w.I, bi == 0 ? 8 : (bi == 1 ? 4 : 3));
+        const int bits = bi == 0 ? 8 : (bi == 1 ? 4 : 3);
+        S.geo[threadIdx.x] = phase == 0 ? geo_gu(p.w.H, bits) : geo(p.w.I, bits);
     }
     __syncthreads();
     // slot table: active routed experts with work for this path, compacted in
@@ -869,6 +980,32 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
                 if (a < ns) pre[a] = base + v;
                 base += __shfl_sync(0xffffffffu, v, 31);
             }
+            // this CTA's contiguous share [lo, hi) of the phase's total cost,
+            // and each slot's tiles whose start falls in it
+            const long long lo = div_floor(base * blockIdx.x, gridDim.x);
+            const long long hi = div_floor(base * (blockIdx.x + 1), gridDim.x);
+            int2 *rng = phase == 0 ? S.sc.rng0 : S.sc.rng1;
+            int first = 0x7fffffff, last = -1;
+            for (int a0 = 0; a0 < ns; a0 += 32) {
+                const int a = a0 + lane;
+                bool has = false;
+                if (a < ns) {
+                    const long long tb = tc[a], off = pre[a] - nt * tb;
+                    const int b0 = tiles_before(lo - off, tb, static_cast<int>(nt));
+                    const int b1 = tiles_before(hi - off, tb, static_cast<int>(nt));
+                    rng[a] = make_int2(b0, b1);
+                    has = b0 < b1;
+                }
+                const unsigned m = __ballot_sync(0xffffffffu, has);
+                if (m) {
+                    first = min(first, a0 + __ffs(m) - 1);
+                    last = max(last, a0 + 31 - __clz(m));
+                }
+            }
+            if (lane == 0) {
+                S.sc.fl[2 * phase] = first;
+                S.sc.fl[2 * phase + 1] = last;
+            }
         }
     }
     __syncthreads();
@@ -878,19 +1015,23 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
 
 }  // namespace moe
 
-// Shared memory of one CTA: the stage ring, x fragments, K-slice partials,
-// shelf and geometry tables, and the slot/entry/schedule tables.  Returns the
-// byte count and the number of stages that fit in the budget.
-size_t moe_ffn_stream_smem(int H, int I, int max_slots, int n_ent, int *nstages) {
+// Shared memory of one CTA: the stage ring, each group's x fragments and
+// K-slice partials, shelf and geometry tables, and the slot/entry/schedule
+// tables.  Returns the byte count and the number of stages that fit in the
+// budget (even: each stage serves one group).
+size_t moe_ffn_stream_smem(int H, int I, int T, int max_slots, int n_ent, int *nstages) {
     const size_t ent = n_ent <= moe::kMaxSmemEntries ? 2 * sizeof(int) * static_cast<size_t>(n_ent) : 0;
-    const size_t fixed = static_cast<size_t>(moe::xf_bytes(H, I)) + moe::kRedBytes +
-                         2 * moe::kMaxStages * sizeof(uint64_t) + (MOE_MAX_TIERS + 1) * sizeof(moe::TierPtrs) +
+    const size_t fixed = moe::kGroups * (static_cast<size_t>(moe::xf_bytes(H, I, T)) + moe::kRedBytes) +
+                         moe::kMaxStages * sizeof(uint64_t) + moe::kGroups * sizeof(moe::StreamSmem::Ahead) +
+                         (MOE_MAX_TIERS + 1) * sizeof(moe::TierPtrs) +
                          6 * sizeof(moe::Geo) + 8 + 6 * sizeof(int) * static_cast<size_t>(max_slots) + ent +
                          4 * sizeof(long long) * static_cast<size_t>(max_slots) +
+                         2 * sizeof(int2) * static_cast<size_t>(max_slots) + 4 * sizeof(int) +
                          sizeof(int) * (static_cast<size_t>(max_slots) + MOE_MAX_EXPERTS + 1) + 16;
     const size_t budget = 220 * 1024;
     int ns = fixed < budget ? static_cast<int>((budget - fixed) / moe::kStageBytes) : 0;
     if (ns > moe::kMaxStages) ns = moe::kMaxStages;
+    ns &= ~(moe::kGroups - 1);
     *nstages = ns;
     return static_cast<size_t>(ns) * moe::kStageBytes + fixed;
 }
@@ -936,8 +1077,8 @@ CUtensorMapSwizzle swizzle_mode(int w) {
 struct MapKey {
     const void *ptr;
     int rank, sw;
-    uint64_t dims[4], strides[3];
-    uint32_t box[4];
+    uint64_t dims[5], strides[4];
+    uint32_t box[5];
     bool operator<(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) < 0; }
 };
 
@@ -961,7 +1102,7 @@ bool byte_map(CUtensorMap *out, const void *ptr, int rank, const uint64_t *dims,
     }
     const EncodeTiled fn = encode_tiled();
     if (!fn) return false;
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     if (fn(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void *>(ptr), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_mode(sw), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -974,8 +1115,15 @@ bool byte_map(CUtensorMap *out, const void *ptr, int rank, const uint64_t *dims,
 // Maps of one shelf (or of the shared expert) at table index t.
 bool shelf_maps(moe::StreamMaps &M, int t, const moe_tier &tier, int H, int I) {
     const uint64_t n = static_cast<uint64_t>(tier.n_experts);
-    const moe::Geo g0 = moe::geo(H, tier.bits), g1 = moe::geo(I, tier.bits);
-    {
+    const moe::Geo g0 = moe::geo_gu(H, tier.bits), g1 = moe::geo(I, tier.bits);
+    if (g0.pad) {
+        // [expert][gate|up][row][line][128 bytes], box {128, nc1, 8R, 2, 1}
+        const uint64_t dims[5] = {128, static_cast<uint64_t>(g0.rb / 128), static_cast<uint64_t>(I), 2, n};
+        const uint64_t str[4] = {128, static_cast<uint64_t>(g0.rb), static_cast<uint64_t>(I) * g0.rb,
+                                 2ull * I * g0.rb};
+        const uint32_t box[5] = {128, static_cast<uint32_t>(g0.nc1), static_cast<uint32_t>(8 * g0.R), 2, 1};
+        if (!byte_map(&M.gq[t], tier.gu_qs, 5, dims, str, box, 128)) return false;
+    } else {
         const uint64_t dims[4] = {static_cast<uint64_t>(g0.rb), static_cast<uint64_t>(I), 2, n};
         const uint64_t str[3] = {static_cast<uint64_t>(g0.rb), static_cast<uint64_t>(I) * g0.rb,
                                  2ull * I * g0.rb};
@@ -1009,8 +1157,8 @@ bool shelf_maps(moe::StreamMaps &M, int t, const moe_tier &tier, int H, int I) {
 // counters (int[max_active + 1]) must be zero on entry; the caller clears them.
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     int nstages = 0;
-    const size_t smem = moe_ffn_stream_smem(p.w.H, p.w.I, p.max_active + 1, p.T * p.k + p.T, &nstages);
-    if (nstages < 2) return cudaErrorInvalidConfiguration;
+    const size_t smem = moe_ffn_stream_smem(p.w.H, p.w.I, p.T, p.max_active + 1, p.T * p.k + p.T, &nstages);
+    if (nstages < moe::kGroups) return cudaErrorInvalidConfiguration;
     int dev = 0;
     cudaGetDevice(&dev);
     int sms = 0;
