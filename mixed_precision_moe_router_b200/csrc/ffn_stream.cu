@@ -56,6 +56,8 @@ constexpr int kThreads = kWarps * 32;              // threads of a group
 constexpr int kGroups = 2;                         // consumer groups, taking alternate tiles
 constexpr int kBlockThreads = kGroups * kThreads;
 constexpr int kBarGroup0 = 1;                      // named barrier of group g: kBarGroup0 + g
+constexpr int kStager = 32;  // the thread of a group that stages its tiles: lane 0 of its second
+                             // warp, so the staging overlaps the epilogue (low threads first)
 constexpr int kMaxStages = 6;
 constexpr int kStageBytes = 40 * 1024;
 constexpr int kMaxK = 2048;
@@ -727,8 +729,8 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const Stream
     TileIt it;
     it_begin(p, S.sc, n_slots, it);
     it_skip(p, S.sc, n_slots, it, grp);
-    if (gt == 0) {
-        // the group leader stages the group's first nstages / 2 tiles
+    if (gt == kStager) {
+        // the group's stager stages its first nstages / 2 tiles
         StreamSmem::Ahead &ah = S.ahead[grp];
         ah.it = it;
         ah.n = 0;
@@ -749,6 +751,17 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const Stream
     for (; it.phase < 2; i += kGroups) {
         const int phase = it.phase, a = it.a, tile = it.b;
         const int s = i % nstages;
+        if (phase == 0) {
+            // gate_up fragments of the first pass do not depend on the tile:
+            // build them while its copies are in flight (every reader of the
+            // old fragments is past the previous tile's barriers, and the
+            // barrier below orders these writes before the reads)
+            const int key0 = (a * 2) * 65536;
+            if (key0 != xf_key) {
+                bad |= build_xf_gu(p, S.st, a, 0, min(kTokPerPass, S.st.count[a]), S.st.bits[a], xf);
+                xf_key = key0;
+            }
+        }
         bool ok = mbar_wait(&S.full[s], (i / nstages) & 1);
         // one thread polls the slot's gate_up count (with backoff, so that
         // pollers do not crowd the counters' L2 slice); the barrier passes
@@ -784,7 +797,7 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const Stream
             else
                 compute_tile<3>(p, G, phase, stage, xf, ntok, red);
             bar_compute();
-            if (pass == np - 1 && gt == 0) {
+            if (pass == np - 1 && gt == kStager) {
                 // every warp of the group is past its reads of the stage:
                 // stage this group's tile i + nstages into it
                 StreamSmem::Ahead &ah = S.ahead[grp];
@@ -818,7 +831,7 @@ __device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const Stream
     if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(p.status, MOE_STATUS_FP16_RANGE);
     // after an abort, copies this group staged but never consumed must land
     // before the CTA exits (on a normal exit there are none)
-    if (gt == 0) {
+    if (gt == kStager) {
         for (int m = consumed; m < S.ahead[grp].n; ++m) {
             const int k = grp + kGroups * m;
             if (!mbar_wait(&S.full[k % nstages], (k / nstages) & 1)) status_or(p.status, MOE_STATUS_TIMEOUT);
@@ -958,8 +971,13 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
         }
         const int ns = run + (shared_here ? 1 : 0);
         if (lane == 0) n_keep = ns;
-        __syncwarp();
-        for (int phase = 0; phase < 2; ++phase) {
+    }
+    __syncthreads();
+    // the schedule: warp 0 for the gate_up tiles, warp 1 for the down tiles
+    if (threadIdx.x < 64) {
+        const int lane = threadIdx.x & 31, phase = threadIdx.x >> 5;
+        const int ns = n_keep;
+        {
             const long long nt = tiles_per_slot(p, phase);
             long long *tc = phase == 0 ? S.sc.tc0 : S.sc.tc1;
             long long *pre = phase == 0 ? S.sc.pre0 : S.sc.pre1;
