@@ -40,7 +40,7 @@ KERNELS_PER_LAYER = 3  # fused routing, streaming FFN, combine (+1 rmsnorm per s
 # DRAM bytes (read + write) per launch measured by ncu for the kernel versions
 # in this tree (profiles/ffn_stream_decode_T1.md, profiles/ffn_gemm_prefill_T4096.md);
 # to be re-measured whenever those kernels change.
-DECODE_FFN_TRAFFIC = 28.65e6  # streaming FFN kernel, one decode token: mean DRAM bytes of 2 captured launches
+DECODE_FFN_TRAFFIC = 28.80e6  # streaming FFN kernel, one decode token: mean DRAM bytes of 2 captured launches
 PREFILL_FFN_TRAFFIC = 1.519e9  # the gate_up and down GEMM launches of one 4096-token call
 
 
