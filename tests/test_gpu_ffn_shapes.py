@@ -1,0 +1,58 @@
+"""The streaming expert FFN (GEMV mode) against the oracle on layer shapes
+that select each tile layout and schedule the kernel has.
+
+- gate_up tiles staged as one padded 5-D copy (rows of whole 128-byte lines:
+  H = 2048 and H = 1024 at every precision) and as one copy per column chunk
+  (H = 256);
+- down tiles of 16R rows with R = 8 (I = 128), R = 4 (I = 512) and R = 2
+  (I = 1024);
+- few tiles per CTA (16 experts) and many (512 experts at T = 8), so that the
+  stage ring wraps around and both consumer groups take several tiles of
+  several slots.
+The per-slot outputs must match the oracle's expert FFN to 1e-5 relative L2
+(the GEMV path's products are exact and its only roundings are x -> fp16 and
+the hi + lo split of h).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixed_precision_moe_router_b200 import binding as B
+from mixed_precision_moe_router_b200 import inputs
+from mixed_precision_moe_router_b200.inputs import LayerConfig
+from tests import helpers as Hh
+
+DEV = "cuda"
+
+SHAPES = {
+    "H256_I1024_many_tiles": (LayerConfig("s1", H=256, I=1024, E=64, k=10, tiers=((8, 16), (4, 24), (3, 24))), 8),
+    "H2048_I128_few_tiles": (LayerConfig("s2", H=2048, I=128, E=16, k=2, tiers=((8, 4), (4, 6), (3, 6))), 1),
+    "H2048_I128_E512": (LayerConfig("s3", H=2048, I=128, E=512, k=10, tiers=((8, 128), (4, 192), (3, 192))), 1),
+    "H1024_I512_E512": (LayerConfig("s4", H=1024, I=512, E=512, k=10, tiers=((8, 128), (4, 192), (3, 192))), 1),
+    "H2048_I512_T8": (inputs.DECODE, 8),
+}
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_streaming_ffn_shapes_match_oracle(name):
+    cfg, T = SHAPES[name]
+    seed = 1234
+    layer = B.build_layer(cfg, seed, DEV)
+    x = inputs.activations(T, cfg.H, seed=seed, device=DEV)
+    ids = torch.stack([torch.randperm(cfg.E, generator=torch.Generator().manual_seed(t))[: cfg.k]
+                       for t in range(T)]).to(torch.int32).to(DEV)
+    off, srt, pos, act = B.bucketize(ids, cfg.E)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y, ysh = B.expert_ffn(layer, x, cfg.k, off, srt, act, mode=B.FFN_GEMV, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ox = Hh.OracleExperts(cfg, seed, DEV)
+    xn = x.float().cpu().numpy()
+    idn = ids.cpu().numpy().reshape(-1)
+    exp = np.stack([oracle.expert_ffn(xn[s // cfg.k: s // cfg.k + 1], *ox(int(idn[s])))[0]
+                    for s in range(T * cfg.k)])
+    assert Hh.rel_l2(y.cpu().numpy(), exp) < 1e-5
+    esh = oracle.expert_ffn(xn, *ox.shared())
+    assert Hh.rel_l2(ysh.cpu().numpy(), esh) < 1e-5
