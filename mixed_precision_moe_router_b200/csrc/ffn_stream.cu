@@ -203,17 +203,6 @@ struct TierPtrs {
     int bits, first, n, pad;
 };
 
-__device__ __forceinline__ int expert_bits(const FfnParams &p, int e) {
-    if (e == p.E) return p.w.shared.bits;
-    int b = 0;
-#pragma unroll
-    for (int i = 0; i < MOE_MAX_TIERS; ++i)
-        if (i < p.w.n_tiers && e >= p.w.tiers[i].first_expert &&
-            e < p.w.tiers[i].first_expert + p.w.tiers[i].n_experts)
-            b = p.w.tiers[i].bits;
-    return b;
-}
-
 // Balancing weight of a tile: a fixed share for the per-tile work (waits,
 // barriers, epilogue), its bytes, and a per-weight share for the
 // dequantise-and-multiply work of each pass (3-bit codes take the most).

@@ -72,18 +72,8 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
     return v;
 }
 
-// Spin until *ctr >= target (acquire); false on timeout.
-__device__ __forceinline__ bool wait_geq(const int *ctr, int target) {
-    if (ld_acquire(ctr) >= target) return true;
-    const long long t0 = clock64();
-    while (ld_acquire(ctr) < target) {
-        if (clock64() - t0 > kWaitLimitCycles) return false;
-        __nanosleep(64);
-    }
-    return true;
-}
-
-// As wait_geq, sleeping 32 ns, 64 ns, ... up to 1 us between polls.
+// Spin until *ctr >= target (acquire), sleeping 32 ns, 64 ns, ... up to 1 us
+// between polls; false on timeout.
 __device__ __forceinline__ bool wait_geq_backoff(const int *ctr, int target) {
     if (ld_acquire(ctr) >= target) return true;
     const long long t0 = clock64();
