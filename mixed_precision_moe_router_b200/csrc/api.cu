@@ -31,6 +31,7 @@ cudaError_t moe_launch_bucketize(const int32_t *, int, int, int32_t *, int32_t *
 cudaError_t moe_configure_ffn_stream();
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &, cudaStream_t);
 bool moe_ffn_stream_supported(int H, int I);
+bool moe_ffn_stream_fits(int H, int I, int T, int max_slots, int n_ent);
 cudaError_t moe_configure_ffn_gemm();
 cudaError_t moe_launch_ffn_gemm(const moe::FfnParams &, void *ws, size_t ws_bytes, cudaStream_t, int min_count);
 bool moe_ffn_gemm_supported(int H, int I);
@@ -334,6 +335,13 @@ int expert_ffn(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t
     if (r) return r;
     if (uses_gemv(mode) && !moe_ffn_stream_supported(w->H, w->I))
         return fail(MOE_ERR_UNSUPPORTED, "GEMV path supports H, I <= 2048");
+    if (uses_gemv(mode)) {
+        const long ma = static_cast<long>(T) * k;
+        const int max_slots = static_cast<int>(ma < w->E ? ma : w->E) + 1;
+        if (!moe_ffn_stream_fits(w->H, w->I, T, max_slots, T * k + T))
+            return fail(MOE_ERR_UNSUPPORTED, "GEMV path: shared memory for T = %d, k = %d leaves fewer than 2 stages",
+                        T, k);
+    }
     if (uses_gemm(mode, T) && !moe_ffn_gemm_supported(w->H, w->I))
         return fail(MOE_ERR_UNSUPPORTED, "GEMM path needs H %% 128 == 0 and I %% 64 == 0");
     char *ws = static_cast<char *>(workspace);

@@ -855,16 +855,20 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     S.st.tok = ent_smem ? tabs + 6 * max_slots : nullptr;
     S.st.row = ent_smem ? S.st.tok + n_ent : nullptr;
     // 8-byte aligned: every table before it has an even number of ints
-    long long *sched = reinterpret_cast<long long *>(tabs + 6 * max_slots + (ent_smem ? 2 * n_ent : 0));
+    S.sc.rng0 = reinterpret_cast<int2 *>(tabs + 6 * max_slots + (ent_smem ? 2 * n_ent : 0));
+    S.sc.rng1 = S.sc.rng0 + max_slots;
+    S.sc.fl = reinterpret_cast<int *>(S.sc.rng1 + max_slots);
+    // Tables the prologue alone uses live in the stage ring, which no copy
+    // touches before the prologue's last barrier (the ring holds at least two
+    // 40 KB stages; these take at most 36 * 1025 + 4 * 1025 bytes): the tile
+    // costs and prefix sums, and copies of the active list and the expert
+    // offsets.
+    long long *sched = reinterpret_cast<long long *>(S.stages);
     S.sc.tc0 = sched;
     S.sc.tc1 = sched + max_slots;
     S.sc.pre0 = sched + 2 * max_slots;
     S.sc.pre1 = sched + 3 * max_slots;
-    S.sc.rng0 = reinterpret_cast<int2 *>(sched + 4 * max_slots);
-    S.sc.rng1 = S.sc.rng0 + max_slots;
-    S.sc.fl = reinterpret_cast<int *>(S.sc.rng1 + max_slots);
-    // copies of the routing tables: active list and expert offsets
-    int *act_s = S.sc.fl + 4;
+    int *act_s = reinterpret_cast<int *>(sched + 4 * max_slots);
     int *off_s = act_s + max_slots;
     // one round of independent global loads fills every table below
     const int S_ = p.T * p.k;
@@ -1015,6 +1019,9 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
             }
         }
     }
+    // the prologue's tables in the stage ring are overwritten by TMA copies
+    // from here on: order this thread's generic accesses before them
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     const int n_slots = n_keep;
     ffn_stream_body(p, M, S, n_slots, nstages);
@@ -1032,9 +1039,7 @@ size_t moe_ffn_stream_smem(int H, int I, int T, int max_slots, int n_ent, int *n
                          moe::kMaxStages * sizeof(uint64_t) + moe::kGroups * sizeof(moe::StreamSmem::Ahead) +
                          (MOE_MAX_TIERS + 1) * sizeof(moe::TierPtrs) +
                          6 * sizeof(moe::Geo) + 8 + 6 * sizeof(int) * static_cast<size_t>(max_slots) + ent +
-                         4 * sizeof(long long) * static_cast<size_t>(max_slots) +
-                         2 * sizeof(int2) * static_cast<size_t>(max_slots) + 4 * sizeof(int) +
-                         sizeof(int) * (static_cast<size_t>(max_slots) + MOE_MAX_EXPERTS + 1) + 16;
+                         2 * sizeof(int2) * static_cast<size_t>(max_slots) + 4 * sizeof(int) + 16;
     const size_t budget = 220 * 1024;
     int ns = fixed < budget ? static_cast<int>((budget - fixed) / moe::kStageBytes) : 0;
     if (ns > moe::kMaxStages) ns = moe::kMaxStages;
@@ -1051,6 +1056,13 @@ cudaError_t moe_configure_ffn_stream() {
 
 bool moe_ffn_stream_supported(int H, int I) {
     return H <= moe::kMaxK && I <= moe::kMaxK && H % 128 == 0 && I % 128 == 0;
+}
+
+// Whether a launch for this batch gets the two stages the consumer groups need.
+bool moe_ffn_stream_fits(int H, int I, int T, int max_slots, int n_ent) {
+    int ns = 0;
+    moe_ffn_stream_smem(H, I, T, max_slots, n_ent, &ns);
+    return ns >= moe::kGroups;
 }
 
 namespace {

@@ -56,3 +56,32 @@ def test_streaming_ffn_shapes_match_oracle(name):
     assert Hh.rel_l2(y.cpu().numpy(), exp) < 1e-5
     esh = oracle.expert_ffn(xn, *ox.shared())
     assert Hh.rel_l2(ysh.cpu().numpy(), esh) < 1e-5
+
+
+@pytest.mark.gpu
+def test_streaming_ffn_largest_tables_sampled():
+    """E = 1024 experts and 150 tokens through the GEMV path: the largest slot
+    and entry tables next to full fragment buffers for both consumer groups
+    (the prologue's own tables then share the stage ring).  Every slot is
+    finite and 24 sampled slots and the shared expert match the oracle."""
+    cfg = LayerConfig("big", H=2048, I=512, E=1024, k=10, tiers=((8, 256), (4, 384), (3, 384)))
+    T, seed = 150, 99
+    layer = B.build_layer(cfg, seed, DEV)
+    x = inputs.activations(T, cfg.H, seed=seed, device=DEV)
+    ids = torch.stack([torch.randperm(cfg.E, generator=torch.Generator().manual_seed(7 + t))[: cfg.k]
+                       for t in range(T)]).to(torch.int32).to(DEV)
+    off, srt, pos, act = B.bucketize(ids, cfg.E)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y, ysh = B.expert_ffn(layer, x, cfg.k, off, srt, act, mode=B.FFN_GEMV, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    y = y.cpu().numpy()
+    assert np.isfinite(y).all()
+    ox = Hh.OracleExperts(cfg, seed, DEV)
+    xn = x.float().cpu().numpy()
+    idn = ids.cpu().numpy().reshape(-1)
+    for s in np.random.default_rng(3).choice(T * cfg.k, size=24, replace=False):
+        exp = oracle.expert_ffn(xn[s // cfg.k: s // cfg.k + 1], *ox(int(idn[s])))[0]
+        assert Hh.rel_l2(y[s], exp) < 1e-5, s
+    esh = oracle.expert_ffn(xn, *ox.shared())
+    assert Hh.rel_l2(ysh.cpu().numpy(), esh) < 1e-5
