@@ -146,3 +146,42 @@ def test_route_workspace_size():
     assert L.moe_route_workspace_size(1, 2048, 512, 10) == 2048 + 256
     assert L.moe_route_workspace_size(3, 2048, 100, 10) == 1280 + 256
     assert L.moe_route_workspace_size(0, 2048, 512, 10) == 256
+
+
+def _layer_fwd(d, T=1, k=2, ws=None, wsp=0x40000, x=0x20000):
+    L = B.lib()
+    p = ctypes.c_void_p(0x30000)
+    if ws is None:
+        ws = int(L.moe_layer_workspace_size(ctypes.byref(d), T, k, 0))
+    return L.moe_layer_forward(ctypes.byref(d), p, None, ctypes.c_void_p(x), T, k, None, p, None, None,
+                               ctypes.c_void_p(wsp) if wsp else None, ws, 0, None, None)
+
+
+def test_layer_forward_rejects_bad_arguments_before_enqueueing():
+    """moe_layer_forward validates everything it can on the host first (fake
+    device pointers: nothing here reaches the GPU)."""
+    d = _fake_layer()
+    assert _layer_fwd(d, T=0) == B.MOE_OK                                # empty batch: nothing to do
+    assert _layer_fwd(d, k=0) == B.MOE_ERR_INVALID_ARG
+    assert _layer_fwd(d, k=17) == B.MOE_ERR_INVALID_ARG                  # k > E
+    assert _layer_fwd(d, ws=64) == B.MOE_ERR_WORKSPACE
+    assert _layer_fwd(d, wsp=0) == B.MOE_ERR_WORKSPACE
+    assert _layer_fwd(d, wsp=0x40008) == B.MOE_ERR_INVALID_ARG           # misaligned workspace
+    assert _layer_fwd(d, x=0x20008) == B.MOE_ERR_INVALID_ARG             # misaligned x (checked by the router)
+    bad = _fake_layer()
+    bad.tiers[1].bits = 2
+    assert _layer_fwd(bad) == B.MOE_ERR_INVALID_ARG
+    assert B.lib().moe_last_error()
+
+
+def test_layer_workspace_holds_the_route_workspace():
+    """The layer workspace covers the routing call's logits and counter, the
+    routing plan, the FFN intermediates and the slot outputs."""
+    L = B.lib()
+    d = _fake_layer(H=2048, I=512, E=512, tiers=((8, 0, 128), (4, 128, 192), (3, 320, 192)))
+    for T in (1, 16, 17, 300):
+        lay = int(L.moe_layer_workspace_size(ctypes.byref(d), T, 10, 0))
+        route = int(L.moe_route_workspace_size(T, 2048, 512, 10))
+        ffn = int(L.moe_ffn_workspace_size(ctypes.byref(d), T, 10, 0))
+        slots = T * 10 * 2048 * 4 + T * 2048 * 4
+        assert lay >= route + ffn + slots
