@@ -427,3 +427,89 @@ def test_f16_staged_ffn_equals_exact_when_staging_is_lossless():
     h = oracle.silu(x @ wgu[:I].T) * (x @ wgu[I:].T)
     assert np.allclose(y_staged, oracle.round_f16(h) @ wdn.T, rtol=0, atol=0)
     assert np.max(np.abs(y_staged - y_exact)) <= np.abs(h).max() * 2.0 ** -11 * np.abs(wdn).sum(axis=1).max()
+
+
+def test_f16_staged_ffn_rounds_x_to_f16():
+    """Activations that are not fp16 values: the staged FFN must round x to the
+    nearest fp16 (ties to even) before the products.  With W_gate = 2I, W_up = I and
+    W_down = I every product is exact, so y = fp16(silu(2X) * X) where X is the
+    fp16 rounding of x, written out here by hand from the fp16 grid (step 2^-10 in
+    [1, 2), 2^-9 in [2, 4), 2^-14 in [1/16, 1/8))."""
+    n = 8
+    x = np.array([[1 + 2.0 ** -12,       # quarter step above 1 -> 1
+                   1 + 3 * 2.0 ** -12,   # three quarters of a step -> 1 + 2^-10
+                   1 + 2.0 ** -11,       # tie between 1 and 1 + 2^-10 -> even: 1
+                   1 + 3 * 2.0 ** -11,   # tie between 1 + 2^-10 and 1 + 2^-9 -> even: 1 + 2^-9
+                   -(2 + 2.0 ** -11),    # quarter step beyond -2 -> -2
+                   0.1,                  # 1638.4 * 2^-14 -> 1638 * 2^-14
+                   3.14159,              # 1608.49 * 2^-9 -> 1608 * 2^-9
+                   -0.75]])              # an fp16 value: unchanged
+    X = np.array([[1.0, 1 + 2.0 ** -10, 1.0, 1 + 2.0 ** -9, -2.0, 1638 * 2.0 ** -14, 1608 * 2.0 ** -9, -0.75]])
+    wgu = np.concatenate([2.0 * np.eye(n), np.eye(n)])
+    y = oracle.expert_ffn_f16_staged(x, wgu, np.eye(n))
+    expect = oracle.round_f16(oracle.silu(2.0 * X) * X)
+    assert np.array_equal(y, expect)
+    # the pin has teeth: skipping the rounding of x changes six of the eight outputs
+    unrounded = oracle.round_f16(oracle.silu(2.0 * x) * x)
+    assert np.sum(unrounded != expect) == 6
+
+
+def _stack_layer_identity(n, c):
+    """One routed expert (E = 1, k = 1) whose FFN is y = silu(c x) * x elementwise,
+    and no shared expert: the layer is out = bf16(silu(c n) * n)."""
+    wgu = np.concatenate([c * np.eye(n), np.eye(n)])
+    wr = np.zeros((1, n), np.float32)
+    return (wr, None, lambda e: (wgu, np.eye(n)), None)
+
+
+def test_moe_stack_closed_form_recursion():
+    """A stack of elementwise layers has a closed form: n_l = rms_norm(x_l),
+    out_l = bf16(silu(c_l n_l) n_l), x_{l+1} = bf16(x_l + out_l).  Feeding x instead
+    of n to a layer, or adding out to n instead of x, breaks it."""
+    n = 16
+    rng = np.random.default_rng(21)
+    x0 = oracle.round_bf16(rng.standard_normal((3, n)) * 4.0)
+    cs = [0.5, 2.0, 1.0, 4.0]
+    res = oracle.moe_stack(x0, [_stack_layer_identity(n, c) for c in cs], 1, n, n)
+    x = x0.copy()
+    for l, c in enumerate(cs):
+        nl = oracle.rms_norm(x)
+        out = oracle.round_bf16(oracle.silu(c * nl) * nl)
+        assert np.array_equal(res[l]["n"], nl)
+        assert np.array_equal(res[l]["x"], x)
+        assert np.array_equal(res[l]["out"], out)
+        x = oracle.round_bf16(x + out)
+        assert np.array_equal(res[l]["x_next"], x)
+        assert np.array_equal(res[l]["n_next"], oracle.rms_norm(x))
+
+
+def test_moe_stack_zero_experts_keep_the_stream():
+    """With all-zero expert weights every layer adds 0: the stream stays x_0 exactly
+    and each layer reads rms_norm(x_0)."""
+    cfg = inputs.TINY
+    rng = np.random.default_rng(22)
+    x0 = oracle.round_bf16(rng.standard_normal((4, cfg.H)) * 3.0)
+    wr = _bf16_values((cfg.E, cfg.H), 23, 0.02)
+    zero = (np.zeros((2 * cfg.I, cfg.H)), np.zeros((cfg.H, cfg.I)))
+    layer = (wr, None, lambda e: zero, zero)
+    res = oracle.moe_stack(x0, [layer] * 3, cfg.k, cfg.H, cfg.I)
+    for r in res:
+        assert not np.any(r["out"])
+        assert np.array_equal(r["x"], x0) and np.array_equal(r["x_next"], x0)
+        assert np.array_equal(r["n"], oracle.rms_norm(x0))
+
+
+def test_moe_stack_layers_read_the_normalised_stream():
+    """The first layer's output does not change when x_0 is scaled by 2^5 (the
+    normalised stream is exactly scale invariant), while the layer evaluated on the
+    raw stream does change."""
+    cfg, x, wr, bias, shelves, shared = _tiny_layer()
+    lookup = oracle.shelves_lookup(shelves, cfg.H, cfg.I)
+    sw = shared.weights(cfg.E, cfg.H, cfg.I)
+    layer = (wr, bias, lookup, sw)
+    a = oracle.moe_stack(x, [layer], cfg.k, cfg.H, cfg.I)[0]
+    b = oracle.moe_stack(x * 32.0, [layer], cfg.k, cfg.H, cfg.I)[0]
+    assert np.array_equal(a["out"], b["out"])
+    assert np.array_equal(b["x_next"], oracle.round_bf16(32.0 * x + b["out"]))
+    raw = oracle.moe_layer(x * 32.0, wr, bias, cfg.k, lookup, sw, cfg.H, cfg.I)
+    assert not np.array_equal(raw["out"], a["out"])
