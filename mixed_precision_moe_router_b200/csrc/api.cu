@@ -1,7 +1,9 @@
 // C ABI entry points: argument validation, workspace carving and launches.
 // Every check here runs on the host before anything is enqueued; nothing here
 // allocates, frees or synchronises.
+#include <atomic>
 #include <cstdarg>
+#include <cstring>
 #include <cstdio>
 #include <mutex>
 #include <string>
@@ -31,7 +33,7 @@ cudaError_t moe_launch_bucketize(const int32_t *, int, int, int32_t *, int32_t *
 cudaError_t moe_configure_ffn_stream();
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &, cudaStream_t);
 bool moe_ffn_stream_supported(int H, int I);
-bool moe_ffn_stream_fits(int H, int I, int T, int max_slots, int n_ent);
+bool moe_ffn_stream_fits(int H, int I, int T, int k, int E, int max_slots);
 cudaError_t moe_configure_ffn_gemm();
 cudaError_t moe_launch_ffn_gemm(const moe::FfnParams &, void *ws, size_t ws_bytes, cudaStream_t, int min_count);
 bool moe_ffn_gemm_supported(int H, int I);
@@ -43,6 +45,10 @@ cudaError_t moe_launch_rmsnorm(const uint16_t *, int, int, uint16_t *, cudaStrea
 namespace {
 
 thread_local std::string g_err;
+
+// Knobs for tests of the failure paths (moe_debug_set); process-wide.
+std::atomic<long long> g_wait_limit{2000000000LL};  // ~1 s of SM clock
+std::atomic<int> g_skip_publish{-1};
 
 int fail(int code, const char *fmt, ...) {
     char buf[512];
@@ -164,18 +170,51 @@ moe::FfnParams make_params(const moe_layer_weights *w, const uint16_t *x, int T,
     p.y_slots = y_slots;
     p.y_shared = y_shared;
     p.status = status;
+    moe::PlanIn &pi = p.pi;
+    std::memset(&pi, 0, sizeof(pi));
+    pi.E = w->E;
+    pi.T = T;
+    pi.k = k;
+    pi.H = w->H;
+    pi.I = w->I;
+    pi.n_tiers = w->n_tiers;
+    pi.has_shared = p.has_shared;
+    pi.shared_bits = w->shared.bits;
+    pi.max_count = p.max_count;
+    pi.max_active = p.max_active;
+    for (int t = 0; t < w->n_tiers; ++t) {
+        pi.first[t] = w->tiers[t].first_expert;
+        pi.n[t] = w->tiers[t].n_experts;
+        pi.bits[t] = w->tiers[t].bits;
+    }
+    std::memset(&p.route, 0, sizeof(p.route));
+    p.wait_limit = g_wait_limit.load();
+    p.skip_publish = g_skip_publish.load();
     return p;
 }
 
+// The streaming path's token limit for AUTO mode also enters its schedule.
+void set_max_count(moe::FfnParams &p, int max_count) {
+    p.max_count = max_count;
+    p.pi.max_count = max_count;
+}
+
+// The streaming path's per-slot counters, followed by the two grid barrier
+// words of a batch that the FFN kernel routes itself.
 size_t ffn_ctr_bytes(const moe_layer_weights *w, int T, int k) {
     const long ma = static_cast<long>(T) * k;
-    return align_up((static_cast<size_t>(ma < w->E ? ma : w->E) + 1) * sizeof(int));
+    return align_up((static_cast<size_t>(ma < w->E ? ma : w->E) + 1 + 2) * sizeof(int));
 }
 
 // Token count from which an expert goes through the tensor-core GEMM in
 // MOE_FFN_AUTO mode (below it the streaming GEMV reads the weights once anyway
 // and wastes no tensor-core columns).
 constexpr int kGemmMinTokens = 8;
+
+// Batches the FFN kernel routes itself inside moe_layer_forward: at most as
+// many tokens as its logits pass stages, and one grouping slot per thread.
+constexpr int kFusedRouteMaxTokens = 16;
+constexpr int kFusedRouteMaxSlots = 512;
 
 bool uses_gemv(int mode) { return mode != MOE_FFN_GEMM; }
 bool uses_gemm(int mode, int T) { return mode == MOE_FFN_GEMM || (mode == MOE_FFN_AUTO && T >= kGemmMinTokens); }
@@ -314,7 +353,8 @@ int *gemv_counters(const moe_layer_weights *w, int T, int k, int mode, void *wor
 // zero already (cleared by an earlier kernel on the stream), so no memset.
 int expert_ffn(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t k, const int32_t *expert_offsets,
                const int32_t *sorted_slot, const int32_t *active, float *y_slots, float *y_shared, void *workspace,
-               size_t workspace_bytes, int32_t mode, int32_t *status, moe_stream_t stream, bool counters_clear) {
+               size_t workspace_bytes, int32_t mode, int32_t *status, moe_stream_t stream, bool counters_clear,
+               const moe::FfnParams::Route *route = nullptr) {
     int r = check_weights(w);
     if (r) return r;
     r = check_k(T, w->E, k);
@@ -338,8 +378,8 @@ int expert_ffn(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t
     if (uses_gemv(mode)) {
         const long ma = static_cast<long>(T) * k;
         const int max_slots = static_cast<int>(ma < w->E ? ma : w->E) + 1;
-        if (!moe_ffn_stream_fits(w->H, w->I, T, max_slots, T * k + T))
-            return fail(MOE_ERR_UNSUPPORTED, "GEMV path: shared memory for T = %d, k = %d leaves fewer than 2 stages",
+        if (!moe_ffn_stream_fits(w->H, w->I, T, k, w->E, max_slots))
+            return fail(MOE_ERR_UNSUPPORTED, "GEMV path: shared memory for T = %d, k = %d leaves no room for a tile",
                         T, k);
     }
     if (uses_gemm(mode, T) && !moe_ffn_gemm_supported(w->H, w->I))
@@ -354,7 +394,11 @@ int expert_ffn(const moe_layer_weights *w, const uint16_t *x, int32_t T, int32_t
     if (uses_gemv(mode)) {
         int n_ctr = 0;
         p.ctr = gemv_counters(w, T, k, mode, workspace, &n_ctr);
-        p.max_count = gemm ? split - 1 : 0x7fffffff;
+        set_max_count(p, gemm ? split - 1 : 0x7fffffff);
+        if (route) {
+            p.route = *route;
+            p.route.gbar = p.ctr + n_ctr;
+        }
         if (!counters_clear) e = cudaMemsetAsync(p.ctr, 0, ffn_ctr_bytes(w, T, k), s);
         if (e == cudaSuccess) e = moe_launch_ffn_stream(p, s);
     }
@@ -520,6 +564,31 @@ int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router, cons
     if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "layer workspace needs %zu bytes", need);
     if (!aligned16(workspace)) return fail(MOE_ERR_INVALID_ARG, "workspace not 16-byte aligned");
     LayerWs L = carve(w, T, k, mode, static_cast<char *>(workspace));
+    // A small batch on the streaming path: the FFN kernel routes it itself
+    // (no routing kernel), after one memset of its counters.
+    if (uses_gemv(mode) && T <= kFusedRouteMaxTokens && static_cast<long>(T) * k <= kFusedRouteMaxSlots &&
+        moe_ffn_stream_supported(w->H, w->I)) {
+        if (!w_router || !x) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+        if (!aligned16(x) || !aligned16(w_router)) return fail(MOE_ERR_INVALID_ARG, "x / w_router not 16-byte aligned");
+        moe::FfnParams::Route rt;
+        std::memset(&rt, 0, sizeof(rt));
+        rt.on = 1;
+        rt.wr = w_router;
+        rt.bias = bias;
+        rt.logits = static_cast<float *>(L.route_ws);
+        rt.topk_idx = L.idx;
+        rt.topk_w = L.tw;
+        rt.offsets = L.offsets;
+        rt.sorted = L.sorted;
+        rt.slot_pos = L.pos;
+        rt.active = L.active;
+        r = expert_ffn(w, x, T, k, L.offsets, L.sorted, L.active, L.y_slots,
+                       w->shared.n_experts == 1 ? L.y_shared : nullptr, L.ffn_ws, L.ffn_bytes, mode, status, stream,
+                       false, &rt);
+        if (r) return r;
+        return moe_combine(L.y_slots, w->shared.n_experts == 1 ? L.y_shared : nullptr, L.tw, T, k, w->H, residual,
+                           out, x_next, x_next_norm, stream);
+    }
     // the routing kernel also zeroes the FFN's GEMV counters on its way out
     int n_ctr = 0;
     int *ctr = gemv_counters(w, T, k, mode, L.ffn_ws, &n_ctr);

@@ -51,6 +51,14 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void *p) {
     return r;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while its predecessor on the stream still runs;
+// pdl_wait() returns once the predecessor has completed and its writes are
+// visible (immediately when there is no such predecessor), and pdl_trigger()
+// lets the successor start its own prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -100,5 +108,22 @@ __device__ __forceinline__ void u3x16_to_f32(uint32_t lo, uint32_t hi16, float *
         f[i] = __uint_as_float(0x4b000000u | c) - (kMagic + 4.0f);
     }
 }
+
+// Launch attribute list for a kernel that may overlap its predecessor
+// (programmatic dependent launch); `extra` (e.g. cooperative) is appended.
+struct PdlAttrs {
+    cudaLaunchAttribute a[2];
+    int n;
+    explicit PdlAttrs(bool cooperative = false) : n(0) {
+        a[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        a[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+        if (cooperative) {
+            a[n].id = cudaLaunchAttributeCooperative;
+            a[n].val.cooperative = 1;
+            ++n;
+        }
+    }
+};
 
 }  // namespace moe

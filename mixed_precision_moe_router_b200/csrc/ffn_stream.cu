@@ -7,38 +7,38 @@
 // shelf results add up; the decode kernel fuses gate, up and the activation.
 //
 // Design (B200):
-//  * Work is a list of tiles.  For every slot (an active expert whose token
-//    count is in (0, max_count], and the shared expert) there are gate_up
+//  * Work is a list of tiles (plan.cuh): for every slot (an active expert
+//    whose token count is in (0, max_count], and the shared expert) gate_up
 //    tiles of 8R gate rows plus the 8R matching up rows, and down tiles of
-//    16R rows, with R the largest power of two <= 8 such that a tile holds at
-//    most 32K codes.  Each CTA takes a contiguous, cost-balanced share of the
-//    gate_up tiles and then of the down tiles, so 8-, 4- and 3-bit experts
-//    spread evenly over the SMs.  The prologue turns that share into a tile
-//    range per slot, so walking the list is integer increments.
-//  * Two consumer groups of 8 warps take alternate tiles of the CTA's list,
-//    so one group's barriers, epilogue and waits overlap the other's
-//    arithmetic.  Each group stages its own tiles into a shared-memory ring
-//    with TMA tensor copies (cp.async.bulk.tensor) that complete on the
-//    stage's mbarrier.  A gate_up tile is one 5-D copy when its rows are
-//    whole 128-byte lines: [gate|up][8R rows][lines, padded to an odd count
-//    with zero-filled out-of-range lines][128 bytes]; otherwise, and for down
-//    tiles, one copy per 128-byte column chunk.  Either way the copies store
-//    the tile with the TMA swizzle, which makes the fragment reads below
-//    bank-conflict free, and one more copy brings the scales.
-//  * 8 compute warps split a tile into R row subtiles x 8/R K slices.  For
-//    each 32-weight block a warp turns its codes into exact fp16 integers
-//    (|q| <= 127), multiplies them with fp16 activation fragments on the
-//    tensor cores (mma.sync m16n8k16: exact products, fp32 accumulation) and
-//    adds d * partial into fp32 accumulators.  The only roundings besides fp32
-//    accumulation are bf16 x -> fp16 (exact for |x| in [2^-14, 65504]) and the
-//    split of the fp32 intermediate h into two fp16 columns hi + lo (relative
-//    error <= 2^-22).  Dequantisation is paid once per tile for up to 8 tokens;
-//    more tokens take further passes over the resident tile.
-//  * K slices are summed in shared memory in a fixed order.  gate_up tiles
-//    write h = silu(g) * u and count themselves done per slot; a down tile
-//    waits (bounded) for its slot's count before reading h, while its weights
-//    may already be in flight.  The grid is launched cooperatively so every
-//    CTA is resident and the waits resolve.
+//    16R rows.  Each CTA takes a contiguous, cost-balanced run of the gate_up
+//    tiles and then of the down tiles, so 8-, 4- and 3-bit experts spread
+//    evenly over the SMs.
+//  * Warp-specialised pipeline, every hand-off an mbarrier (no block-wide
+//    barrier after the prologue):
+//      - a producer warp stages tile after tile with TMA tensor copies into a
+//        byte ring (tiles of different precisions take different sizes, so
+//        the ring holds as many bytes in flight as shared memory allows);
+//      - a loader warp builds the B operand of each (slot, pass): fp16
+//        fragments of x for gate_up, of h split into hi + lo for down, after
+//        waiting (bounded) for the slot's gate_up tiles to be counted done;
+//      - 8 compute warps split every tile into R row subtiles x 8/R K
+//        slices.  For each 32-weight block a warp turns its codes into exact
+//        fp16 integers (|q| <= 127), multiplies them with the B fragments on
+//        the tensor cores (mma.sync m16n8k16: exact products, fp32
+//        accumulation) and adds d * partial into fp32 accumulators, then
+//        hands its partial sums to the epilogue through a small ring;
+//      - an epilogue warp sums the K slices in a fixed order and writes
+//        h = silu(g) * u or y, and publishes per slot how many gate_up tiles
+//        this CTA finished (fence, then an atomic add).
+//    The only roundings besides fp32 accumulation are bf16 x -> fp16 (exact
+//    for |x| in [2^-14, 65504]) and the split of the fp32 intermediate h into
+//    two fp16 columns hi + lo (relative error <= 2^-22).
+//  * A down tile's weights are in flight while its slot's h is still being
+//    produced elsewhere; the grid is launched cooperatively so every CTA is
+//    resident and the waits on other CTAs' counts resolve.  Every wait is
+//    bounded; a warp that gives up sets MOE_STATUS_TIMEOUT and a CTA-wide
+//    abort flag that releases the others, and the producer waits for its
+//    copies in flight before the CTA exits.
 #include <cuda.h>
 
 #include <cstring>
@@ -47,33 +47,31 @@
 
 #include "common.cuh"
 #include "ffn.cuh"
+#include "route_cta.cuh"
 #include "sync.cuh"
 
 namespace moe {
 
-constexpr int kWarps = 8;                          // compute warps of a group (they split a tile)
-constexpr int kThreads = kWarps * 32;              // threads of a group
-constexpr int kGroups = 2;                         // consumer groups, taking alternate tiles
-constexpr int kBlockThreads = kGroups * kThreads;
-constexpr int kBarGroup0 = 1;                      // named barrier of group g: kBarGroup0 + g
-constexpr int kStager = 32;  // the thread of a group that stages its tiles: lane 0 of its second
-                             // warp, so the staging overlaps the epilogue (low threads first)
-constexpr int kMaxStages = 6;
-constexpr int kStageBytes = 40 * 1024;
+constexpr int kWarps = 8;          // compute warps of a group: they split each tile
+constexpr int kGroups = 2;         // compute groups, taking alternate tiles
+constexpr int kComputeWarps = kGroups * kWarps;
+constexpr int kWarpProducer = kComputeWarps;      // lane 0 stages the tiles
+constexpr int kWarpLoader = kComputeWarps + 1;    // builds the B operand of each (slot, pass)
+constexpr int kWarpEpilogue0 = kComputeWarps + 2;  // one per group: sums partials, writes h / y
+constexpr int kBlockWarps = kComputeWarps + 2 + kGroups;
+constexpr int kBlockThreads = kBlockWarps * 32;
+constexpr int kND = 8;             // tiles in flight at most (full/empty barrier pairs)
+constexpr int kNR = 3;             // partial-sum buffers per group (compute warps -> epilogue)
+constexpr int kNB = 2;             // B-operand buffers (loader -> compute warps)
+constexpr int kMaxTileBytes = 40 * 1024;  // a staged tile (codes, padding, scales) at most
+constexpr int kTileAlign = 1024;   // ring allocations start on a 128-byte-swizzle atom
 constexpr int kMaxK = 2048;
-constexpr int kMaxSmemEntries = 2048;  // token-entry tables kept in shared memory up to this size
-constexpr int kTokPerPass = 8;         // gate_up token columns per pass over a resident tile
-constexpr int kRedBytes = kWarps * 32 * 4 * 4;
+constexpr int kRedBytes = kWarps * 32 * 16;  // one item's partials: a float4 per compute lane
+constexpr int kMaxSmemEntries = 2048;        // sorted slot ids kept in shared memory up to this many
 
 // ---------------------------------------------------------------------------
 // tile geometry
 // ---------------------------------------------------------------------------
-__host__ __device__ __forceinline__ int rows_pow2(int K) {
-    int R = 1;
-    while (R < 8 && 2 * R * K <= 2048) R *= 2;
-    return R;
-}
-
 // Swizzle width of a row of `bytes` bytes: the largest of 128, 64 and 32 that
 // divides it (its 16-byte chunks are permuted within that span), else 16 (no
 // swizzle).
@@ -121,7 +119,7 @@ __host__ __device__ __forceinline__ Geo geo_gu(int K, int bits) {
     if (g.W == 128) {
         const int n = g.rb / 128;
         const int nc1 = n + 1 + (n & 1);
-        if (nc1 <= 256 && g.rows * (nc1 * 128 + g.sb) <= kStageBytes) {
+        if (nc1 <= 256 && g.rows * (nc1 * 128 + g.sb) <= kMaxTileBytes) {
             g.pad = 1;
             g.nc1 = nc1;
             g.cb = g.rows * nc1 * 128;
@@ -164,150 +162,6 @@ __device__ __forceinline__ int row_x(int r, const Geo &G) {
 // x fragments in shared memory: [column][block][thread t][8 halves], with a
 // column stride that keeps the 16-byte reads of two columns in different banks.
 __host__ __device__ __forceinline__ int xf_col_stride(int K) { return (K / 32) * 64 + 64; }
-
-__host__ __device__ __forceinline__ int down_ntiles(int I) { return I <= 1024 ? 2 : 1; }
-
-// Fragment columns a pass can use with at most T tokens: gate_up one per
-// token (up to 8), down hi + lo per token in n-tiles of 8 (column 8*(n/4) +
-// 2*(n%4) + 1 is the last one written for token n).
-__host__ __device__ __forceinline__ int xf_bytes(int H, int I, int T) {
-    const int cg = T < kTokPerPass ? T : kTokPerPass;
-    const int nd = T < 4 * down_ntiles(I) ? T : 4 * down_ntiles(I);
-    const int cd = nd <= 4 ? 2 * nd : 8 + 2 * (nd - 4);
-    const int a = cg * xf_col_stride(H);
-    const int b = cd * xf_col_stride(I);
-    const int m = a > b ? a : b;
-    return (m + 127) & ~127;
-}
-
-// Thread index within its consumer group, and the group.
-__device__ __forceinline__ int gtid() { return threadIdx.x & (kThreads - 1); }
-__device__ __forceinline__ int group_of_thread() { return threadIdx.x / kThreads; }
-
-// tokens of one pass: gate_up tiles use one column per token, down tiles two
-// (h = hi + lo) in n-tiles of 8 columns
-__host__ __device__ __forceinline__ int tokens_per_pass(int phase, int I) {
-    return phase == 0 ? kTokPerPass : 4 * down_ntiles(I);
-}
-
-struct SlotTabs {  // per expert slot, in shared memory
-    int *expert, *bits, *count, *first;
-    int *tok, *row;  // entries [first, first + count) of every slot: token and h/y row
-};
-
-// Table base pointers of the shelves (index < n_tiers) and of the shared
-// expert (index n_tiers), copied from the parameters into shared memory so
-// that they can be indexed at run time.
-struct TierPtrs {
-    const uint8_t *gq, *gs, *dq, *ds;
-    int bits, first, n, pad;
-};
-
-// Balancing weight of a tile: a fixed share for the per-tile work (waits,
-// barriers, epilogue), its bytes, and a per-weight share for the
-// dequantise-and-multiply work of each pass (3-bit codes take the most).
-constexpr long long kTileFixedCost = 65536;
-__device__ __forceinline__ long long tile_cost(const FfnParams &p, int phase, int bits, int count) {
-    const int K = phase == 0 ? p.w.H : p.w.I;
-    const long long rows = 16 * rows_pow2(K);
-    const int tp = tokens_per_pass(phase, p.w.I);
-    const long long passes = (count + tp - 1) / tp;
-    return kTileFixedCost + rows * (K * bits / 8 + K / 16) + passes * (rows * K / 3) * (bits == 3 ? 3 : 2);
-}
-
-__device__ __forceinline__ int tiles_per_slot(const FfnParams &p, int phase) {
-    return phase == 0 ? p.w.I / (8 * rows_pow2(p.w.H)) : p.w.H / (16 * rows_pow2(p.w.I));
-}
-
-// Per-slot tile costs and inclusive prefix sums of the slots' total costs,
-// per phase, built once in the prologue (shared memory).
-struct Sched {
-    long long *tc0, *tc1;    // cost of one tile of each slot
-    long long *pre0, *pre1;  // inclusive prefix sums of the slots' total costs
-    int2 *rng0, *rng1;       // per slot: this CTA's tiles of it, [b0, b1)
-    int *fl;                 // per phase: first and last slot with tiles in this CTA (last < first: none)
-};
-
-// floor(x / y) for 0 <= x < 2^52, 0 < y: a double quotient corrected to the
-// exact integer result (the 64-bit integer divide is a long routine).
-__device__ __forceinline__ long long div_floor(long long x, long long y) {
-    long long q = static_cast<long long>(static_cast<double>(x) / static_cast<double>(y));
-    while (q * y > x) --q;
-    while ((q + 1) * y <= x) ++q;
-    return q;
-}
-
-// This CTA's tiles, in order: its cost-balanced contiguous share of all
-// gate_up tiles (phase 0), then of all down tiles (phase 1).  phase == 2 once
-// the list is exhausted.  The per-slot tile ranges are computed once in the
-// prologue, so stepping is a few integer operations.
-struct TileIt {
-    int phase, a, b, b1;  // current tile: slot a, tile b; b1 ends this slot's range
-};
-
-// Tiles of a slot (nt tiles of cost tb) that start before cost offset x from
-// the slot's start: ceil(x / tb) clamped to [0, nt].  A float quotient
-// corrected to the exact integer (the quotient is below nt <= 256 here).
-__device__ __forceinline__ int tiles_before(long long x, long long tb, int nt) {
-    if (x <= 0) return 0;
-    if (x >= nt * tb) return nt;
-    long long q = static_cast<long long>(__fdividef(static_cast<float>(x), static_cast<float>(tb)));
-    while (q * tb < x) ++q;
-    while (q > 0 && (q - 1) * tb >= x) --q;
-    return static_cast<int>(q);
-}
-
-__device__ __forceinline__ bool it_enter(const Sched &sc, TileIt &it, int phase) {
-    const int f = sc.fl[2 * phase], l = sc.fl[2 * phase + 1];
-    if (f > l) return false;
-    const int2 r = (phase == 0 ? sc.rng0 : sc.rng1)[f];
-    it.phase = phase;
-    it.a = f;
-    it.b = r.x;
-    it.b1 = r.y;
-    return true;
-}
-
-__device__ __forceinline__ void it_begin(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
-    (void)p;
-    it.phase = 2;
-    if (n_slots == 0) return;
-    if (!it_enter(sc, it, 0) && !it_enter(sc, it, 1)) it.phase = 2;
-}
-
-// Slots strictly between a phase's first and last slot lie wholly inside the
-// CTA's contiguous cost range, so each of them has tiles here.
-__device__ __forceinline__ void it_next(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it) {
-    (void)p;
-    (void)n_slots;
-    if (it.phase == 2) return;
-    if (++it.b < it.b1) return;
-    if (it.a < sc.fl[2 * it.phase + 1]) {
-        ++it.a;
-        const int2 r = (it.phase == 0 ? sc.rng0 : sc.rng1)[it.a];
-        it.b = r.x;
-        it.b1 = r.y;
-        return;
-    }
-    if (it.phase == 0 && it_enter(sc, it, 1)) return;
-    it.phase = 2;
-}
-
-// token and output row of the n-th entry of slot a (tables built in the prologue)
-__device__ __forceinline__ void slot_entry(const FfnParams &p, const SlotTabs &st, int a, int n, int &tok,
-                                           int &row) {
-    const int j = st.first[a] + n;
-    if (st.tok) {
-        tok = st.tok[j];
-        row = st.row[j];
-    } else if (j >= p.T * p.k) {  // shared expert
-        tok = j - p.T * p.k;
-        row = j;
-    } else {
-        row = p.sorted[j];
-        tok = row / p.k;
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Codes -> exact fp16 integers: four half2 pairs per row, block and thread.
@@ -464,25 +318,6 @@ __device__ __forceinline__ uint4 pack_frag(const uint16_t (&v)[8], int bits) {
     return r;
 }
 
-struct StreamSmem {
-    uint8_t *stages;
-    uint8_t *xf;             // [kGroups][xf_size]
-    int xf_size;
-    float4 *red;             // [kGroups][kWarps * 32]
-    uint64_t *full;          // per stage: copies landed
-    int *abort;
-    // per group: how many of its tiles (g, g + 2, ...) are staged, and the
-    // iterator at the next one to stage
-    struct Ahead { TileIt it; int n; } *ahead;
-    SlotTabs st;
-    Sched sc;
-    int *tier, *jloc;   // per slot: shelf index (n_tiers = shared) and index within the shelf
-    TierPtrs *tp;       // [MOE_MAX_TIERS + 1]
-    Geo *geo;           // [phase][8-, 4-, 3-bit]
-};
-
-__device__ __forceinline__ int bits_idx(int bits) { return bits == 8 ? 0 : (bits == 4 ? 1 : 2); }
-
 // Tensor maps of the shelf tables (index < n_tiers) and of the shared expert
 // (index n_tiers), built on the host:
 //   gq: 4-D [expert][gate|up][I][rb_H] bytes, box {W_H, 8R, 2, 1}
@@ -520,14 +355,148 @@ __device__ __forceinline__ void tma_5d(void *dst, const CUtensorMap *map, int x,
         : "memory");
 }
 
+__device__ __forceinline__ int bits_idx(int bits) { return bits == 8 ? 0 : (bits == 4 ? 1 : 2); }
+
+// Table base pointers of the shelves (index < n_tiers) and of the shared
+// expert (index n_tiers), copied from the parameters into shared memory so
+// that they can be indexed at run time.
+struct TierPtrs {
+    const uint8_t *gq, *gs, *dq, *ds;
+};
+
+// Ring bytes a staged tile takes (its start stays on a swizzle atom).
+__host__ __device__ __forceinline__ int stage_alloc_bytes(const Geo &g) {
+    return (stage_bytes(g) + kTileAlign - 1) & ~(kTileAlign - 1);
+}
+
+// Bytes of the all-token x fragments (batches of at most kTokPerPass tokens):
+// column t holds token t, once in the pair order of 8-bit codes and once in
+// that of 4- and 3-bit codes.
+__host__ __device__ __forceinline__ int xall_bytes(int H, int T) {
+    return T <= kTokPerPass ? 2 * T * xf_col_stride(H) : 0;
+}
+
+// Bytes of one B-operand buffer: the down fragments of one pass, plus the
+// gate_up fragments of one pass when gate_up does not use the all-token copy.
+__host__ __device__ __forceinline__ int bbuf_bytes(int H, int I, int T) {
+    const int nd = T < 4 * down_ntiles(I) ? T : 4 * down_ntiles(I);
+    const int cd = nd <= 4 ? 2 * nd : 8 + 2 * (nd - 4);
+    int b = cd * xf_col_stride(I);
+    if (T > kTokPerPass) {
+        const int a = kTokPerPass * xf_col_stride(H);
+        b = a > b ? a : b;
+    }
+    return (b + 127) & ~127;
+}
+
+struct StreamSmem {
+    uint8_t *ring;
+    int ring_bytes;
+    uint8_t *xall;           // all-token gate_up fragments (T <= kTokPerPass), else null
+    uint8_t *bbuf;           // [kNB][b_bytes]
+    int b_bytes;
+    float4 *red;             // [kGroups][kNR][kWarps * 32]
+    uint64_t *full, *empty;  // [kND]: a tile's copies landed / every compute warp is done with it
+    uint64_t *rfull, *rempty;  // [kGroups][kNR]: partials written / partials summed
+    uint64_t *bfull, *bempty;  // [kNB]: B operand built / every compute warp has moved past it
+    int *abort;              // set by a warp that gave up; every wait checks it
+    int *range;              // this CTA's tiles: [gs0, ge0), [gs1, ge1); then the slot count
+    int *srt;                // copy of sorted_slot when it has at most kMaxSmemEntries entries, else null
+    PlanTabs pt;
+    TierPtrs *tp;            // [MOE_MAX_TIERS + 1]
+    Geo *geo;                // [phase][8-, 4-, 3-bit]
+    int nt0, nt1;            // tiles per slot of each phase
+};
+
+__device__ __forceinline__ const Geo &tile_geo(const StreamSmem &S, int phase, int a) {
+    return S.geo[phase * 3 + bits_idx(S.pt.bits[a])];
+}
+
+__device__ __forceinline__ void abort_cta(const FfnParams &p, const StreamSmem &S) {
+    status_or(p.status, MOE_STATUS_TIMEOUT);
+    *static_cast<volatile int *>(S.abort) = 1;
+}
+
+// This CTA's tiles in order: its run of gate_up tiles (phase 0), then its run
+// of down tiles (phase 1); phase 2 once exhausted.  Tile g of a phase is tile
+// b = g % nt of slot a = g / nt.  Every warp role walks the same sequence.
+struct Walk {
+    int phase, g, ge, a, b;
+};
+
+__device__ __forceinline__ void walk_enter(const StreamSmem &S, Walk &w, int phase) {
+    const int nt = phase == 0 ? S.nt0 : S.nt1;
+    w.phase = phase;
+    w.g = S.range[2 * phase];
+    w.ge = S.range[2 * phase + 1];
+    w.a = w.g / nt;
+    w.b = w.g - w.a * nt;
+}
+
+__device__ __forceinline__ void walk_begin(const StreamSmem &S, Walk &w) {
+    if (S.range[0] < S.range[1]) walk_enter(S, w, 0);
+    else if (S.range[2] < S.range[3]) walk_enter(S, w, 1);
+    else w.phase = 2;
+}
+
+__device__ __forceinline__ void walk_next(const StreamSmem &S, Walk &w) {
+    if (++w.g < w.ge) {
+        if (++w.b == (w.phase == 0 ? S.nt0 : S.nt1)) {
+            w.b = 0;
+            ++w.a;
+        }
+        return;
+    }
+    if (w.phase == 0 && S.range[2] < S.range[3]) walk_enter(S, w, 1);
+    else w.phase = 2;
+}
+
+// Passes over a resident tile of slot a, and whether phase `phase` takes its
+// B operand from the loader (true) or from the all-token fragments.
+__device__ __forceinline__ int n_passes(const FfnParams &p, const StreamSmem &S, int phase, int a) {
+    const int tp = tokens_per_pass(phase, p.w.I);
+    return (S.pt.count[a] + tp - 1) / tp;
+}
+__device__ __forceinline__ bool loads_b(const StreamSmem &S, int phase) { return phase == 1 || S.xall == nullptr; }
+
+// Key of the B operand of (phase, slot, pass); consecutive tiles of one slot
+// with a single pass share it.
+__device__ __forceinline__ long long b_key(int phase, int a, int pass) {
+    return (static_cast<long long>(2 * a + phase) << 32) | static_cast<unsigned>(pass);
+}
+
+// The ring offset of each tile, in order: every role that needs it takes the
+// same allocations (wrapping to 0 when a tile does not fit before the end).
+__device__ __forceinline__ int ring_take(int &head, int sz, int ring_bytes) {
+    if (head + sz > ring_bytes) head = 0;
+    const int s = head;
+    head += sz;
+    return s;
+}
+
+// h / y row of entry n of slot a: the slot's sorted slot ids, or for the
+// shared expert (entries from T*k on) the row T*k + t of token t.
+__device__ __forceinline__ int entry_row(const FfnParams &p, const StreamSmem &S, int a, int n) {
+    const int j = S.pt.first[a] + n;
+    const int Sk = p.T * p.k;
+    if (j >= Sk) return j;
+    const int r = S.srt ? S.srt[j] : __ldg(p.sorted + j);
+    return (r >= 0 && r < Sk) ? r : 0;
+}
+
+__device__ __forceinline__ int row_token(const FfnParams &p, int row) {
+    const int Sk = p.T * p.k;
+    return row >= Sk ? row - Sk : row / p.k;
+}
+
 // Stage the codes and scales of tile (phase, a, tile) into `dst`, completing
 // on `bar`: a gate_up tile is its 8R gate rows and the matching 8R up rows, a
 // down tile 16R consecutive rows; codes as column chunks of W bytes.
 __device__ __forceinline__ void issue_tile(const FfnParams &p, const StreamMaps &M, const StreamSmem &S, int phase,
                                            int a, int tile, uint8_t *dst, uint64_t *bar) {
     const int I = p.w.I;
-    const Geo &G = S.geo[phase * 3 + bits_idx(S.st.bits[a])];
-    const int ti = S.tier[a], j = S.jloc[a];
+    const Geo &G = tile_geo(S, phase, a);
+    const int ti = S.pt.tier[a], j = S.pt.jloc[a];
     const TierPtrs &T = S.tp[ti];
     uint8_t *dsc = dst + G.cb;
     const int chunk = G.rows << G.lw;  // bytes of one column chunk of the tile
@@ -557,337 +526,506 @@ __device__ __forceinline__ void issue_tile(const FfnParams &p, const StreamMaps 
     }
 }
 
-// Barrier of one consumer group that also ANDs a flag over it.
-__device__ __forceinline__ bool bar_and(bool ok) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(ok ? 1u : 0u), "r"(kBarGroup0 + group_of_thread()), "n"(kThreads)
-        : "memory");
-    return r != 0;
+// ---------------------------------------------------------------------------
+// B operands
+// ---------------------------------------------------------------------------
+
+// 8 consecutive bf16 values -> fp16 fragment words in both pair orders.
+__device__ __forceinline__ void x_frags(const uint4 q, bool &bad, uint4 &f8, uint4 &f43) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint16_t v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        v[2 * j] = to_f16(bf16lo(w[j]), bad);
+        v[2 * j + 1] = to_f16(bf16hi(w[j]), bad);
+    }
+    f8 = pack_frag(v, 8);
+    f43 = pack_frag(v, 4);
 }
 
-__device__ __forceinline__ void bar_compute() { named_bar_sync(kBarGroup0 + group_of_thread(), kThreads); }
-
-
-// gate_up fragments of one pass: column n holds the token of entry pass*8 + n.
-__device__ __forceinline__ bool build_xf_gu(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
-                                         int bits, uint8_t *xf) {
+// All-token gate_up fragments (T <= kTokPerPass) from the bf16 rows of x
+// staged in shared memory: column t of copy 0 (8-bit order) and of copy 1
+// (4- and 3-bit order) is token t.  Every thread of the CTA takes a share.
+__device__ __forceinline__ bool build_xall(const FfnParams &p, const uint8_t *x_s, uint8_t *xall) {
     bool bad = false;
-    const int H = p.w.H, nb = H / 32, cs = xf_col_stride(H);
-    const int n_chunks = ntok * nb * 4;
-    for (int i = gtid(); i < n_chunks; i += kThreads) {
-        const int n = i / (nb * 4), rem = i % (nb * 4);  // rem = 4 * block + t
-        int tok, row;
-        slot_entry(p, st, a, pass * kTokPerPass + n, tok, row);
-        const uint4 q = *reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(tok) * H + 8 * rem);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-        uint16_t v[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[2 * j] = to_f16(bf16lo(w[j]), bad);
-            v[2 * j + 1] = to_f16(bf16hi(w[j]), bad);
-        }
-        *reinterpret_cast<uint4 *>(xf + n * cs + rem * 16) = pack_frag(v, bits);
+    const int H = p.w.H, nchunk = H / 8, cs = xf_col_stride(H);
+    const int n = p.T * nchunk;
+    uint8_t *x43 = xall + p.T * cs;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int t = i / nchunk, rem = i - t * nchunk;
+        const uint4 q = reinterpret_cast<const uint4 *>(x_s)[i];
+        uint4 f8, f43;
+        x_frags(q, bad, f8, f43);
+        *reinterpret_cast<uint4 *>(xall + t * cs + rem * 16) = f8;
+        *reinterpret_cast<uint4 *>(x43 + t * cs + rem * 16) = f43;
     }
     return bad;
 }
 
-// down fragments of one pass: in n-tile nt, column 2m holds hi and column
-// 2m + 1 lo of h for the token of entry pass*tp + 4nt + m.
-__device__ __forceinline__ bool build_xf_dn(const FfnParams &p, const SlotTabs &st, int a, int pass, int ntok,
-                                         int bits, uint8_t *xf) {
+// gate_up fragments of one pass (loader warp): column n holds the token of
+// entry pass * 8 + n of slot a, in the pair order of the slot's codes.
+__device__ __forceinline__ bool load_b_gu(const FfnParams &p, const StreamSmem &S, int a, int pass, int ntok,
+                                          uint8_t *xf) {
     bool bad = false;
-    const int I = p.w.I, nb = I / 32, cs = xf_col_stride(I);
+    const int lane = threadIdx.x & 31;
+    const int H = p.w.H, nchunk = H / 8, cs = xf_col_stride(H), bits = S.pt.bits[a];
+    const int my_row = lane < ntok ? entry_row(p, S, a, pass * kTokPerPass + lane) : 0;
+    for (int n = 0; n < ntok; ++n) {
+        const int tok = row_token(p, __shfl_sync(0xffffffffu, my_row, n));
+        const uint16_t *xr = p.x + static_cast<size_t>(tok) * H;
+#pragma unroll 4
+        for (int rem = lane; rem < nchunk; rem += 32) {
+            const uint4 q = *reinterpret_cast<const uint4 *>(xr + 8 * rem);
+            uint4 f8, f43;
+            x_frags(q, bad, f8, f43);
+            *reinterpret_cast<uint4 *>(xf + n * cs + rem * 16) = bits == 8 ? f8 : f43;
+        }
+    }
+    return bad;
+}
+
+// down fragments of one pass (loader warp): in n-tile nt, column 2m holds hi
+// and column 2m + 1 lo of h for the entry pass * tp + 4nt + m of slot a.
+__device__ __forceinline__ bool load_b_dn(const FfnParams &p, const StreamSmem &S, int a, int pass, int ntok,
+                                          uint8_t *xf) {
+    bool bad = false;
+    const int lane = threadIdx.x & 31;
+    const int I = p.w.I, nchunk = I / 8, cs = xf_col_stride(I), bits = S.pt.bits[a];
     const int tp = tokens_per_pass(1, I);
-    const int n_chunks = ntok * nb * 4;
-    for (int i = gtid(); i < n_chunks; i += kThreads) {
-        const int n = i / (nb * 4), rem = i % (nb * 4);
-        int tok, row;
-        slot_entry(p, st, a, pass * tp + n, tok, row);
-        const float *src = p.h + static_cast<size_t>(row) * I + 8 * rem;
-        const float4 f0 = __ldcg(reinterpret_cast<const float4 *>(src));
-        const float4 f1 = __ldcg(reinterpret_cast<const float4 *>(src + 4));
-        const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-        uint16_t hi[8], lo[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            hi[j] = to_f16(f[j], bad);
-            lo[j] = __half_as_ushort(__float2half_rn(f[j] - __half2float(__ushort_as_half(hi[j]))));
-        }
+    const int my_row = lane < ntok ? entry_row(p, S, a, pass * tp + lane) : 0;
+    for (int n = 0; n < ntok; ++n) {
+        const int row = __shfl_sync(0xffffffffu, my_row, n);
+        const float *hr = p.h + static_cast<size_t>(row) * I;
         const int col = (n >> 2) * 8 + 2 * (n & 3);
-        *reinterpret_cast<uint4 *>(xf + col * cs + rem * 16) = pack_frag(hi, bits);
-        *reinterpret_cast<uint4 *>(xf + (col + 1) * cs + rem * 16) = pack_frag(lo, bits);
+#pragma unroll 2
+        for (int rem = lane; rem < nchunk; rem += 32) {
+            const float4 f0 = __ldcg(reinterpret_cast<const float4 *>(hr + 8 * rem));
+            const float4 f1 = __ldcg(reinterpret_cast<const float4 *>(hr + 8 * rem + 4));
+            const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+            uint16_t hi[8], lo[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                hi[j] = to_f16(f[j], bad);
+                lo[j] = __half_as_ushort(__float2half_rn(f[j] - __half2float(__ushort_as_half(hi[j]))));
+            }
+            *reinterpret_cast<uint4 *>(xf + col * cs + rem * 16) = pack_frag(hi, bits);
+            *reinterpret_cast<uint4 *>(xf + (col + 1) * cs + rem * 16) = pack_frag(lo, bits);
+        }
     }
     return bad;
 }
 
-// This warp's partial sums of the resident tile, to red[warp][lane].
+// ---------------------------------------------------------------------------
+// warp roles
+// ---------------------------------------------------------------------------
+
+// One compute warp's partial sums of a resident tile for one pass.
 template <int BITS>
-__device__ __forceinline__ void compute_tile(const FfnParams &p, const Geo &G, int phase, const uint8_t *stage,
-                                             const uint8_t *xf, int ntok, float4 *red) {
-    const int warp = gtid() >> 5, lane = threadIdx.x & 31;
-    const int r = warp % G.R, s = warp / G.R;
+__device__ __forceinline__ float4 compute_part(const Geo &G, int phase, const uint8_t *stage, const uint8_t *xf,
+                                               int ncol, int warp) {
+    const int r = warp & (G.R - 1), s = warp / G.R;
     const int b0 = min(G.nb, s * G.bps), b1 = min(G.nb, (s + 1) * G.bps);
     const int cs = xf_col_stride(G.K);
-    const int g = lane >> 2;
+    const int g = (threadIdx.x & 31) >> 2;
     if (phase == 0) {
-        const TileAcc t = G.pad ? warp_tile<BITS, 1, true>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs, ntok, 0)
-                                : warp_tile<BITS, 1, false>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs, ntok, 0);
-        const float(&acc)[2][4] = t.acc;
-        red[warp * 32 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-    } else {
-        const int nc0 = 2 * max(0, min(4, ntok)), nc1 = 2 * max(0, min(4, ntok - 4));
-        const TileAcc t = down_ntiles(p.w.I) == 2
-                              ? warp_tile<BITS, 2, false>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1)
-                              : warp_tile<BITS, 1, false>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs, nc0, nc1);
-        const float(&acc)[2][4] = t.acc;
-        // hi + lo columns of each token
-        red[warp * 32 + lane] =
-            make_float4(acc[0][0] + acc[0][1], acc[0][2] + acc[0][3], acc[1][0] + acc[1][1], acc[1][2] + acc[1][3]);
+        const TileAcc t = G.pad ? warp_tile<BITS, 1, true>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs,
+                                                           ncol, 0)
+                                : warp_tile<BITS, 1, false>(stage, G, 8 * r + g, 8 * G.R + 8 * r + g, b0, b1, xf, cs,
+                                                            ncol, 0);
+        return make_float4(t.acc[0][0], t.acc[0][1], t.acc[0][2], t.acc[0][3]);
     }
+    const int nc0 = 2 * max(0, min(4, ncol)), nc1 = 2 * max(0, min(4, ncol - 4));
+    const TileAcc t = nc1 > 0 ? warp_tile<BITS, 2, false>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs,
+                                                          nc0, nc1)
+                              : warp_tile<BITS, 1, false>(stage, G, 16 * r + g, 16 * r + g + 8, b0, b1, xf, cs,
+                                                          nc0, 0);
+    // hi + lo columns of each token
+    return make_float4(t.acc[0][0] + t.acc[0][1], t.acc[0][2] + t.acc[0][3], t.acc[1][0] + t.acc[1][1],
+                       t.acc[1][2] + t.acc[1][3]);
 }
 
-// K slices summed in a fixed order; gate_up -> h = silu(g) * u, down -> y.
-__device__ __forceinline__ void epilogue(const FfnParams &p, const SlotTabs &st, int phase, int a, int tile,
-                                         int pass, int ntok, const float4 *red) {
-    const int K = phase == 0 ? p.w.H : p.w.I;
-    const int R = rows_pow2(K), S = kWarps / R;
-    const float *rf = reinterpret_cast<const float *>(red);
-    if (phase == 0) {
-        const int I = p.w.I;
-        const int n_out = R * 8 * ntok;
-        for (int o = gtid(); o < n_out; o += kThreads) {
-            const int n = o % ntok, rg = o / ntok, g = rg % 8, r = rg / 8;
-            const int lane = 4 * g + (n >> 1), sub = n & 1;
-            float gate = 0.f, up = 0.f;
-            for (int s = 0; s < S; ++s) {
-                const float *v = rf + ((r + R * s) * 32 + lane) * 4;
-                gate += v[sub];
-                up += v[2 + sub];
+// Producer (lane 0 of its warp): allocate each tile in the byte ring, wait
+// until no tile still being read overlaps it (tiles are released oldest
+// first), and stage it.  Before returning it waits for every copy it issued.
+__device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMaps &M, StreamSmem &S) {
+    if ((threadIdx.x & 31) != 0) return;
+    int head = 0, rel = 0, i = 0;
+    int st[kND], en[kND];
+    bool ok = true;
+    Walk w;
+    walk_begin(S, w);
+    for (; w.phase < 2; walk_next(S, w), ++i) {
+        const int sz = stage_alloc_bytes(tile_geo(S, w.phase, w.a));
+        const int s0 = ring_take(head, sz, S.ring_bytes);
+        while (rel < i) {
+            bool clash = i - rel >= kND;
+            for (int j = rel; j < i && !clash; ++j) clash = st[j % kND] < s0 + sz && s0 < en[j % kND];
+            if (!clash) break;
+            if (!mbar_wait_abortable(&S.empty[rel % kND], (rel / kND) & 1, S.abort, p.wait_limit)) {
+                ok = false;
+                break;
             }
-            int tok, row;
-            slot_entry(p, st, a, pass * kTokPerPass + n, tok, row);
-            p.h[static_cast<size_t>(row) * I + tile * 8 * R + 8 * r + g] = gate / (1.0f + expf(-gate)) * up;
+            ++rel;
         }
-    } else {
-        const int H = p.w.H, tp = tokens_per_pass(1, p.w.I);
-        const int n_out = R * 16 * ntok;
-        for (int o = gtid(); o < n_out; o += kThreads) {
-            const int rr = o % (R * 16), n = o / (R * 16);
-            const int r = rr / 16, row16 = rr % 16;
-            const int lane = 4 * (row16 % 8) + (n & 3), idx = 2 * (n >> 2) + row16 / 8;
-            float v = 0.f;
-            for (int s = 0; s < S; ++s) v += rf[((r + R * s) * 32 + lane) * 4 + idx];
-            int tok, row;
-            slot_entry(p, st, a, pass * tp + n, tok, row);
-            float *dst = row >= p.T * p.k ? p.y_shared + static_cast<size_t>(row - p.T * p.k) * H
-                                          : p.y_slots + static_cast<size_t>(row) * H;
-            dst[tile * 16 * R + rr] = v;
-        }
+        if (!ok) break;
+        st[i % kND] = s0;
+        en[i % kND] = s0 + sz;
+        issue_tile(p, M, S, w.phase, w.a, w.b, S.ring + s0, &S.full[i % kND]);
     }
+    if (!ok) abort_cta(p, S);
+    // tiles [0, i) were issued and those before rel consumed: the rest must land
+    for (int j = max(rel, i - kND); j < i; ++j)
+        if (!mbar_wait_limit(&S.full[j % kND], (j / kND) & 1, p.wait_limit)) status_or(p.status, MOE_STATUS_TIMEOUT);
 }
 
-// Advance an iterator by `n` tiles.
-__device__ __forceinline__ void it_skip(const FfnParams &p, const Sched &sc, int n_slots, TileIt &it, int n) {
-    for (int k = 0; k < n; ++k) it_next(p, sc, n_slots, it);
-}
-
-// The persistent FFN kernel body; `n_slots` slots are described in S.
-//
-// Two consumer groups of 8 warps take alternate tiles of the CTA's list
-// (group g: tiles g, g + 2, ...), so one group's barriers, epilogue and
-// dependency waits overlap the other's dequantise-and-multiply.  Tile i lives
-// in stage i % nstages; nstages is even, so a stage always serves the same
-// group.  The first nstages tiles are staged in the prologue; afterwards a
-// group stages its tile i + nstages as soon as its barrier after the last
-// pass over tile i shows the stage drained.  A group therefore never waits
-// on copies the other group issues, and a group waiting on another slot's
-// gate_up count cannot hold back the tiles that produce that count.
-__device__ __forceinline__ void ffn_stream_body(const FfnParams &p, const StreamMaps &M, StreamSmem &S, int n_slots,
-                                                int nstages) {
-    const int grp = group_of_thread(), gt = gtid(), lane = threadIdx.x & 31;
-    const int I = p.w.I;
-    uint8_t *xf = S.xf + grp * S.xf_size;
-    float4 *red = S.red + grp * kWarps * 32;
-    const int gu_tiles = tiles_per_slot(p, 0);
-    TileIt it;
-    it_begin(p, S.sc, n_slots, it);
-    it_skip(p, S.sc, n_slots, it, grp);
-    if (gt == kStager) {
-        // the group's stager stages its first nstages / 2 tiles
-        StreamSmem::Ahead &ah = S.ahead[grp];
-        ah.it = it;
-        ah.n = 0;
-        while (ah.n < nstages / kGroups && ah.it.phase < 2) {
-            const int k = grp + kGroups * ah.n;
-            issue_tile(p, M, S, ah.it.phase, ah.it.a, ah.it.b, S.stages + static_cast<size_t>(k) * kStageBytes,
-                       &S.full[k]);
-            it_skip(p, S.sc, n_slots, ah.it, kGroups);
-            ++ah.n;
-        }
-    }
-    int xf_key = -1;      // (slot, phase, pass) whose fragments xf holds
-    int ready_slot = -1;  // a slot whose h is known to be complete
-    int pend_tiles = 0;   // gate_up tiles of the current slot not yet counted
-    int consumed = 0;     // this group's tiles whose copies have landed
-    bool bad = false;
-    int i = grp;
-    for (; it.phase < 2; i += kGroups) {
-        const int phase = it.phase, a = it.a, tile = it.b;
-        const int s = i % nstages;
-        if (phase == 0) {
-            // gate_up fragments of the first pass do not depend on the tile:
-            // build them while its copies are in flight (every reader of the
-            // old fragments is past the previous tile's barriers, and the
-            // barrier below orders these writes before the reads)
-            const int key0 = (a * 2) * 65536;
-            if (key0 != xf_key) {
-                bad |= build_xf_gu(p, S.st, a, 0, min(kTokPerPass, S.st.count[a]), S.st.bits[a], xf);
-                xf_key = key0;
-            }
-        }
-        bool ok = mbar_wait(&S.full[s], (i / nstages) & 1);
-        // one thread polls the slot's gate_up count (with backoff, so that
-        // pollers do not crowd the counters' L2 slice); the barrier passes
-        // the result on and orders every thread's reads of h after it
-        if (phase == 1 && a != ready_slot && gt == 0) ok = ok && wait_geq_backoff(p.ctr + a, gu_tiles);
-        if (!bar_and(ok && !*static_cast<volatile int *>(S.abort))) {
-            if (gt == 0) {
-                status_or(p.status, MOE_STATUS_TIMEOUT);
-                *static_cast<volatile int *>(S.abort) = 1;
-            }
+// Compute warp `cw` (0..kComputeWarps-1): group cw / kWarps computes the
+// tiles i with i % kGroups == group, its K slice cw % kWarps of each.  Every
+// compute warp follows the whole tile sequence so that it keeps the ring
+// offsets and, for the B operands, releases every buffer in order: on each
+// change of operand it waits until the next one is built (even when its group
+// has no tile that uses it) and releases the previous one, so no release can
+// run ahead of the loader.
+__device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, int cw) {
+    const int lane = threadIdx.x & 31, grp = cw / kWarps, warp = cw % kWarps;
+    int head = 0, i = 0, m = 0, kb = -1;
+    long long key = -1;
+    bool ok = true;
+    float4 *red = S.red + grp * kNR * (kWarps * 32);
+    uint64_t *rfull = S.rfull + grp * kNR, *rempty = S.rempty + grp * kNR;
+    Walk w;
+    walk_begin(S, w);
+    for (; ok && w.phase < 2; walk_next(S, w), ++i) {
+        const int phase = w.phase, a = w.a;
+        const int bits = S.pt.bits[a], cnt = S.pt.count[a];
+        const Geo &G = tile_geo(S, phase, a);
+        const int s0 = ring_take(head, stage_alloc_bytes(G), S.ring_bytes);
+        const bool mine = i % kGroups == grp;
+        if (mine && !mbar_wait_warp(&S.full[i % kND], (i / kND) & 1, S.abort, p.wait_limit)) {
+            ok = false;
             break;
         }
-        ++consumed;
-        if (phase == 1) ready_slot = a;
-        const uint8_t *stage = S.stages + static_cast<size_t>(s) * kStageBytes;
-        const int bits = S.st.bits[a], cnt = S.st.count[a];
-        const Geo &G = S.geo[phase * 3 + bits_idx(bits)];
-        const int tp = tokens_per_pass(phase, I);
-        const int np = (cnt + tp - 1) / tp;
+        const uint8_t *stage = S.ring + s0;
+        const int tp = tokens_per_pass(phase, p.w.I), np = n_passes(p, S, phase, a);
         for (int pass = 0; pass < np; ++pass) {
-            const int ntok = min(tp, cnt - pass * tp);
-            const int key = (a * 2 + phase) * 65536 + pass;
-            if (key != xf_key) {  // the last readers of xf passed a barrier since
-                bad |= phase == 0 ? build_xf_gu(p, S.st, a, pass, ntok, bits, xf)
-                                  : build_xf_dn(p, S.st, a, pass, ntok, bits, xf);
-                xf_key = key;
-                bar_compute();
-            }
-            if (bits == 8)
-                compute_tile<8>(p, G, phase, stage, xf, ntok, red);
-            else if (bits == 4)
-                compute_tile<4>(p, G, phase, stage, xf, ntok, red);
-            else
-                compute_tile<3>(p, G, phase, stage, xf, ntok, red);
-            bar_compute();
-            if (pass == np - 1 && gt == kStager) {
-                // every warp of the group is past its reads of the stage:
-                // stage this group's tile i + nstages into it
-                StreamSmem::Ahead &ah = S.ahead[grp];
-                if (ah.it.phase < 2) {
-                    const int k = grp + kGroups * ah.n;  // == i + nstages
-                    issue_tile(p, M, S, ah.it.phase, ah.it.a, ah.it.b,
-                               S.stages + static_cast<size_t>(k % nstages) * kStageBytes, &S.full[k % nstages]);
-                    it_skip(p, S.sc, n_slots, ah.it, kGroups);
-                    ++ah.n;
+            const uint8_t *xf;
+            int ncol;
+            if (loads_b(S, phase)) {
+                const long long nk = b_key(phase, a, pass);
+                if (nk != key) {
+                    ++kb;
+                    key = nk;
+                    if (!mbar_wait_warp(&S.bfull[kb % kNB], (kb / kNB) & 1, S.abort, p.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    if (kb > 0) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.bempty[(kb - 1) % kNB]);
+                    }
                 }
+                xf = S.bbuf + static_cast<size_t>(kb % kNB) * S.b_bytes;
+                ncol = min(tp, cnt - pass * tp);
+            } else {  // every token is a column; the epilogue keeps the slot's
+                xf = S.xall + (bits == 8 ? 0 : p.T * xf_col_stride(p.w.H));
+                ncol = p.T;
             }
-            epilogue(p, S.st, phase, a, tile, pass, ntok, red);
-            if (pass + 1 < np) bar_compute();  // red is written again by the next pass
+            if (!mine) continue;
+            const float4 part = bits == 8 ? compute_part<8>(G, phase, stage, xf, ncol, warp)
+                                          : (bits == 4 ? compute_part<4>(G, phase, stage, xf, ncol, warp)
+                                                       : compute_part<3>(G, phase, stage, xf, ncol, warp));
+            if (pass == np - 1) {  // every read of the stage is done
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.empty[i % kND]);
+            }
+            const int r = m % kNR;
+            if (!mbar_wait_warp(&rempty[r], ((m / kNR) & 1) ^ 1, S.abort, p.wait_limit)) {
+                ok = false;
+                break;
+            }
+            red[r * (kWarps * 32) + warp * 32 + lane] = part;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rfull[r]);
+            ++m;
         }
-        it_skip(p, S.sc, n_slots, it, kGroups);
-        if (phase == 0) {
-            // when this group leaves the slot, count its gate_up tiles of it:
-            // after every thread's h writes (barrier) and a fence, and before
-            // this group waits on any other slot's count
-            ++pend_tiles;
-            if (it.phase != 0 || it.a != a) {
-                bar_compute();
-                if (gt == 0) {
-                    __threadfence();
-                    atomicAdd(p.ctr + a, pend_tiles);
-                }
-                pend_tiles = 0;
+    }
+    if (!ok && lane == 0) abort_cta(p, S);
+}
+
+// Loader warp: the B operand of every (phase, slot, pass) that takes one, in
+// the order the compute warps use them; before a slot's first down operand it
+// waits (bounded) until every gate_up tile of the slot has been counted done.
+__device__ __forceinline__ void run_loader(const FfnParams &p, StreamSmem &S) {
+    const int lane = threadIdx.x & 31;
+    int kb = -1, ready = -1;
+    long long key = -1;
+    bool ok = true, bad = false;
+    Walk w;
+    walk_begin(S, w);
+    for (; ok && w.phase < 2; walk_next(S, w)) {
+        const int phase = w.phase, a = w.a;
+        if (!loads_b(S, phase)) continue;
+        const int tp = tokens_per_pass(phase, p.w.I), np = n_passes(p, S, phase, a), cnt = S.pt.count[a];
+        for (int pass = 0; pass < np; ++pass) {
+            const long long nk = b_key(phase, a, pass);
+            if (nk == key) continue;
+            key = nk;
+            ++kb;
+            if (!mbar_wait_warp(&S.bempty[kb % kNB], ((kb / kNB) & 1) ^ 1, S.abort, p.wait_limit)) {
+                ok = false;
+                break;
             }
+            if (phase == 1 && a != ready) {
+                bool got = true;
+                if (lane == 0) got = wait_geq_abortable(p.ctr + a, S.nt0, S.abort, p.wait_limit);
+                got = __shfl_sync(0xffffffffu, got, 0);
+                __syncwarp();
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                ready = a;
+            }
+            uint8_t *xf = S.bbuf + static_cast<size_t>(kb % kNB) * S.b_bytes;
+            const int ntok = min(tp, cnt - pass * tp);
+            bad |= phase == 0 ? load_b_gu(p, S, a, pass, ntok, xf) : load_b_dn(p, S, a, pass, ntok, xf);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.bfull[kb % kNB]);
         }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(p.status, MOE_STATUS_FP16_RANGE);
-    // after an abort, copies this group staged but never consumed must land
-    // before the CTA exits (on a normal exit there are none)
-    if (gt == kStager) {
-        for (int m = consumed; m < S.ahead[grp].n; ++m) {
-            const int k = grp + kGroups * m;
-            if (!mbar_wait(&S.full[k % nstages], (k / nstages) & 1)) status_or(p.status, MOE_STATUS_TIMEOUT);
+    if (!ok && lane == 0) abort_cta(p, S);
+}
+
+// Epilogue of one (tile, pass): the K slices of every output summed in a
+// fixed order; gate_up -> h = silu(g) * u, down -> y.
+__device__ __forceinline__ void epilogue_item(const FfnParams &p, const StreamSmem &S, int phase, int a, int tile,
+                                              int pass, const float4 *red) {
+    const int lane = threadIdx.x & 31;
+    const float *rf = reinterpret_cast<const float *>(red);
+    const int cnt = S.pt.count[a];
+    if (phase == 0) {
+        const int I = p.w.I, R = S.geo[0].R, S_ = kWarps / R, lr = __ffs(8 * R) - 1;
+        // with the all-token fragments the column of entry n is its token;
+        // otherwise entry pass*8 + n sits in column n
+        const int ntok = S.xall ? cnt : min(kTokPerPass, cnt - pass * kTokPerPass);
+        const int base = S.xall ? 0 : pass * kTokPerPass;
+        const int my_row = lane < ntok ? entry_row(p, S, a, base + lane) : 0;
+        const int n_out = ntok << lr;
+        for (int o0 = 0; o0 < n_out; o0 += 32) {
+            const int o = o0 + lane;
+            const int n = min(o >> lr, ntok - 1);
+            const int row = __shfl_sync(0xffffffffu, my_row, n);
+            if (o < n_out) {
+                const int rg = o & (8 * R - 1), g = rg & 7, r = rg >> 3;
+                const int col = S.xall ? row_token(p, row) : n;
+                const int ln = 4 * g + (col >> 1), sub = col & 1;
+                float gate = 0.f, up = 0.f;
+                for (int s = 0; s < S_; ++s) {
+                    const float *v = rf + ((r + R * s) * 32 + ln) * 4;
+                    gate += v[sub];
+                    up += v[2 + sub];
+                }
+                p.h[static_cast<size_t>(row) * I + tile * 8 * R + 8 * r + g] = gate / (1.0f + expf(-gate)) * up;
+            }
+        }
+    } else {
+        const int H = p.w.H, R = S.geo[3].R, S_ = kWarps / R, tp = tokens_per_pass(1, p.w.I);
+        const int lr = __ffs(16 * R) - 1;
+        const int ntok = min(tp, cnt - pass * tp);
+        const int my_row = lane < ntok ? entry_row(p, S, a, pass * tp + lane) : 0;
+        const int n_out = ntok << lr;
+        const int Sk = p.T * p.k;
+        for (int o0 = 0; o0 < n_out; o0 += 32) {
+            const int o = o0 + lane;
+            const int n = min(o >> lr, ntok - 1);
+            const int row = __shfl_sync(0xffffffffu, my_row, n);
+            if (o < n_out) {
+                const int rr = o & (16 * R - 1), r = rr >> 4, row16 = rr & 15;
+                const int ln = 4 * (row16 & 7) + (n & 3), idx = 2 * (n >> 2) + (row16 >> 3);
+                float v = 0.f;
+                for (int s = 0; s < S_; ++s) v += rf[((r + R * s) * 32 + ln) * 4 + idx];
+                float *dst = row >= Sk ? p.y_shared + static_cast<size_t>(row - Sk) * H
+                                       : p.y_slots + static_cast<size_t>(row) * H;
+                dst[tile * 16 * R + rr] = v;
+            }
         }
     }
 }
 
-__global__ void __launch_bounds__(kBlockThreads, 1)
-ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ StreamMaps M, int nstages) {
-    extern __shared__ __align__(1024) uint8_t smem[];
-    StreamSmem S;
-    S.stages = smem;
-    S.xf_size = xf_bytes(p.w.H, p.w.I, p.T);
-    S.xf = smem + static_cast<size_t>(nstages) * kStageBytes;
-    S.red = reinterpret_cast<float4 *>(S.xf + kGroups * S.xf_size);
-    S.full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(S.red) + kGroups * kRedBytes);
-    S.ahead = reinterpret_cast<StreamSmem::Ahead *>(S.full + kMaxStages);
-    S.tp = reinterpret_cast<TierPtrs *>(S.ahead + kGroups);
-    S.geo = reinterpret_cast<Geo *>(S.tp + MOE_MAX_TIERS + 1);
-    S.abort = reinterpret_cast<int *>(S.geo + 6);
-    int *tabs = S.abort + 2;
-    const int max_slots = p.max_active + 1;
-    S.st.expert = tabs;
-    S.st.bits = tabs + max_slots;
-    S.st.count = tabs + 2 * max_slots;
-    S.st.first = tabs + 3 * max_slots;
-    S.tier = tabs + 4 * max_slots;
-    S.jloc = tabs + 5 * max_slots;
-    // entry tables in shared memory when they fit, else read from global
-    const int n_ent = p.T * p.k + p.T;
-    const bool ent_smem = n_ent <= kMaxSmemEntries;
-    S.st.tok = ent_smem ? tabs + 6 * max_slots : nullptr;
-    S.st.row = ent_smem ? S.st.tok + n_ent : nullptr;
-    // 8-byte aligned: every table before it has an even number of ints
-    S.sc.rng0 = reinterpret_cast<int2 *>(tabs + 6 * max_slots + (ent_smem ? 2 * n_ent : 0));
-    S.sc.rng1 = S.sc.rng0 + max_slots;
-    S.sc.fl = reinterpret_cast<int *>(S.sc.rng1 + max_slots);
-    // Tables the prologue alone uses live in the stage ring, which no copy
-    // touches before the prologue's last barrier (the ring holds at least two
-    // 40 KB stages; these take at most 36 * 1025 + 4 * 1025 bytes): the tile
-    // costs and prefix sums, and copies of the active list and the expert
-    // offsets.
-    long long *sched = reinterpret_cast<long long *>(S.stages);
-    S.sc.tc0 = sched;
-    S.sc.tc1 = sched + max_slots;
-    S.sc.pre0 = sched + 2 * max_slots;
-    S.sc.pre1 = sched + 3 * max_slots;
-    int *act_s = reinterpret_cast<int *>(sched + 4 * max_slots);
-    int *off_s = act_s + max_slots;
-    // one round of independent global loads fills every table below
-    const int S_ = p.T * p.k;
-    for (int i = threadIdx.x; i < max_slots; i += blockDim.x) act_s[i] = p.active[i];
-    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) off_s[e] = p.offsets[e];
-    if (ent_smem) {
-        for (int j = threadIdx.x; j < S_; j += blockDim.x) {
-            const int sl = p.sorted[j];
-            const bool okj = sl >= 0 && sl < S_;
-            S.st.tok[j] = okj ? sl / p.k : 0;
-            S.st.row[j] = okj ? sl : 0;
+// Epilogue warp of group `grp`: the group's items in order; when the tile
+// sequence leaves a slot's gate_up tiles it publishes how many of them the
+// group finished (after a fence, so that another CTA that sees the count also
+// sees the h values).
+__device__ __forceinline__ void run_epilogue(const FfnParams &p, StreamSmem &S, int grp) {
+    const int lane = threadIdx.x & 31;
+    int m = 0, pend = 0, i = 0;
+    bool ok = true;
+    float4 *red = S.red + grp * kNR * (kWarps * 32);
+    uint64_t *rfull = S.rfull + grp * kNR, *rempty = S.rempty + grp * kNR;
+    Walk w;
+    walk_begin(S, w);
+    for (; ok && w.phase < 2; ++i) {
+        const int phase = w.phase, a = w.a, tile = w.b;
+        if (i % kGroups == grp) {
+            const int np = n_passes(p, S, phase, a);
+            for (int pass = 0; pass < np; ++pass) {
+                const int r = m % kNR;
+                if (!mbar_wait_warp(&rfull[r], (m / kNR) & 1, S.abort, p.wait_limit)) {
+                    ok = false;
+                    break;
+                }
+                epilogue_item(p, S, phase, a, tile, pass, red + r * (kWarps * 32));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&rempty[r]);
+                ++m;
+            }
+            if (!ok) break;
+            if (phase == 0) ++pend;
         }
-        for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
-            S.st.tok[S_ + t] = t;
-            S.st.row[S_ + t] = S_ + t;
+        walk_next(S, w);
+        if (phase == 0 && pend > 0 && (w.phase != 0 || w.a != a)) {
+            __syncwarp();
+            if (lane == 0 && a != p.skip_publish) {
+                __threadfence();
+                atomicAdd(p.ctr + a, pend);
+            }
+            pend = 0;
         }
     }
-    // shelf table pointers (constant-index reads of the parameters), tile
-    // geometry of each phase and precision, and the stage barriers
+    if (!ok && lane == 0) abort_cta(p, S);
+}
+
+// Layout of the prologue's scratch inside the ring (byte offsets): the
+// routing lists, the bf16 rows of x, and for a
+// batch routed in the kernel the top-k candidates, choices, weights, slot
+// positions and a few ints of scan space.
+struct PrologueScratch {
+    size_t lists, x, cand, idx, w, pos, tmp, end;
+};
+
+__host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
+
+__host__ __device__ __forceinline__ PrologueScratch prologue_scratch(int H, int T, int k, int E, int max_slots,
+                                                                     bool fused) {
+    PrologueScratch ps;
+    const size_t lists = static_cast<size_t>(max_slots) + E + 1;
+    const size_t S_ = static_cast<size_t>(T) * k;
+    ps.lists = 0;
+    ps.x = align16(lists * sizeof(int));
+    const bool need_x = fused || T <= kTokPerPass;
+    ps.cand = align16(ps.x + (need_x ? static_cast<size_t>(T) * H * 2 : 0));
+    ps.idx = align16(ps.cand + (fused ? cta_topk_smem(T, E, k) : 0));
+    ps.w = align16(ps.idx + (fused ? S_ * sizeof(int) : 0));
+    ps.pos = align16(ps.w + (fused ? S_ * sizeof(float) : 0));
+    ps.tmp = align16(ps.pos + (fused ? S_ * sizeof(int) : 0));
+    ps.end = ps.tmp + (fused ? 32 * sizeof(int) : 0);
+    return ps;
+}
+
+// The batch routed by the FFN kernel itself (every thread of every CTA): the
+// logits of this CTA's share of the experts, a grid barrier, then the top-k
+// of every token and the stable grouping of the T*k slots, into the same
+// shared-memory lists the prologue otherwise copies from global memory.  CTA 0
+// also writes the routing outputs.  False when the grid barrier gave up.
+__device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, const uint16_t *x_s, int *act_s,
+                                          int *off_s, const PrologueScratch &ps) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int T = p.T, E = p.E, k = p.k, H = p.w.H, S_ = T * k;
+    const PlanIn &pi = p.pi;
+    (void)pi;
+    // logits of experts [E * c / G, E * (c + 1) / G): one warp per expert
+    const int e0 = static_cast<int>(static_cast<long long>(E) * blockIdx.x / gridDim.x);
+    const int e1 = static_cast<int>(static_cast<long long>(E) * (blockIdx.x + 1) / gridDim.x);
+    for (int e = e0 + warp; e < e1; e += nwarps) {
+        float acc[kRouterTokTile];
+        expert_dots(x_s, p.route.wr + static_cast<size_t>(e) * H, T, H / 8, acc);
+        const float b = p.route.bias ? p.route.bias[e] : 0.f;
+#pragma unroll
+        for (int t = 0; t < kRouterTokTile; ++t) {
+            if (t < T) {
+                const float v = warp_sum(acc[t]);
+                if (lane == 0) p.route.logits[static_cast<size_t>(t) * E + e] = v + b;
+            }
+        }
+    }
+    __syncthreads();
+    int *barrier_ok = S.range + 5;
+    if (threadIdx.x == 0) {
+        const bool ok = grid_barrier(p.route.gbar, S.abort, p.wait_limit);
+        if (!ok) {
+            status_or(p.status, MOE_STATUS_TIMEOUT);
+            *static_cast<volatile int *>(S.abort) = 1;
+        }
+        *barrier_ok = ok;
+    }
+    __syncthreads();
+    if (!*barrier_ok) return false;
+    int *idx_s = reinterpret_cast<int *>(S.ring + ps.idx);
+    float *w_s = reinterpret_cast<float *>(S.ring + ps.w);
+    int *pos_s = reinterpret_cast<int *>(S.ring + ps.pos);
+    cta_topk(p.route.logits, T, E, k, S.ring + ps.cand, idx_s, w_s);
+    cta_group(idx_s, S_, E, S.srt, pos_s, act_s, off_s, reinterpret_cast<int *>(S.ring + ps.tmp));
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < S_; i += blockDim.x) {
+            p.route.topk_idx[i] = idx_s[i];
+            p.route.topk_w[i] = w_s[i];
+            p.route.sorted[i] = S.srt[i];
+            p.route.slot_pos[i] = pos_s[i];
+        }
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) p.route.offsets[e] = off_s[e];
+        for (int a = threadIdx.x; a <= act_s[0]; a += blockDim.x) p.route.active[a] = act_s[a];
+    }
+    (void)lane;
+    return true;
+}
+
+__global__ void __launch_bounds__(kBlockThreads, 1)
+ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ StreamMaps M, int ring_bytes) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int max_slots = p.max_active + 1;
+    StreamSmem S;
+    uint8_t *q = smem;
+    S.ring = q;
+    S.ring_bytes = ring_bytes;
+    q += ring_bytes;
+    const int xb = xall_bytes(p.w.H, p.T);
+    S.xall = xb ? q : nullptr;
+    q += xb;
+    S.b_bytes = bbuf_bytes(p.w.H, p.w.I, p.T);
+    S.bbuf = q;
+    q += kNB * S.b_bytes;
+    S.red = reinterpret_cast<float4 *>(q);
+    q += kGroups * kNR * kRedBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(q);
+    S.full = bars;
+    S.empty = bars + kND;
+    S.rfull = bars + 2 * kND;
+    S.rempty = S.rfull + kGroups * kNR;
+    S.bfull = S.rempty + kGroups * kNR;
+    S.bempty = S.bfull + kNB;
+    q = reinterpret_cast<uint8_t *>(S.bempty + kNB);
+    S.abort = reinterpret_cast<int *>(q);
+    S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots (16-byte aligned)
+    q += 12 * sizeof(int);
+    S.tp = reinterpret_cast<TierPtrs *>(q);
+    q += (MOE_MAX_TIERS + 1) * sizeof(TierPtrs);
+    S.geo = reinterpret_cast<Geo *>(q);
+    q += 6 * sizeof(Geo);
+    q = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q) + 15) & ~static_cast<uintptr_t>(15));
+    S.pt = plan_tabs(q, max_slots);
+    q += plan_tab_bytes(max_slots);
+    const int n_srt = p.T * p.k;
+    S.srt = n_srt <= kMaxSmemEntries ? reinterpret_cast<int *>(q) : nullptr;
+    S.nt0 = tiles_per_slot(p.w.H, p.w.I, 0);
+    S.nt1 = tiles_per_slot(p.w.H, p.w.I, 1);
+
+    // Prologue.  One round of asynchronous copies brings into shared memory
+    // either the plan the routing kernel wrote (the slot rows and this CTA's
+    // tile runs) or the active list and the expert offsets to build it from,
+    // and the sorted slot ids and (T <= kTokPerPass) the bf16 rows of x.  The
+    // scratch copies sit in the ring, which no TMA copy touches before the
+    // prologue's last barrier.
     if (threadIdx.x == 0) {
 #pragma unroll
         for (int t = 0; t < MOE_MAX_TIERS; ++t) {
@@ -896,9 +1034,6 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
                 S.tp[t].gs = reinterpret_cast<const uint8_t *>(p.w.tiers[t].gu_scale);
                 S.tp[t].dq = p.w.tiers[t].dn_qs;
                 S.tp[t].ds = reinterpret_cast<const uint8_t *>(p.w.tiers[t].dn_scale);
-                S.tp[t].bits = p.w.tiers[t].bits;
-                S.tp[t].first = p.w.tiers[t].first_expert;
-                S.tp[t].n = p.w.tiers[t].n_experts;
             }
         }
         const int t = p.w.n_tiers;
@@ -906,163 +1041,127 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
         S.tp[t].gs = reinterpret_cast<const uint8_t *>(p.w.shared.gu_scale);
         S.tp[t].dq = p.w.shared.dn_qs;
         S.tp[t].ds = reinterpret_cast<const uint8_t *>(p.w.shared.dn_scale);
-        S.tp[t].bits = p.w.shared.bits;
-        S.tp[t].first = p.E;
-        S.tp[t].n = 1;
-        for (int st = 0; st < nstages; ++st) mbar_init(&S.full[st], 1);  // the stager's expect_tx arrival
+        for (int i = 0; i < kND; ++i) {
+            mbar_init(&S.full[i], 1);  // the producer's expect_tx arrival
+            mbar_init(&S.empty[i], kWarps);
+        }
+        for (int i = 0; i < kGroups * kNR; ++i) {
+            mbar_init(&S.rfull[i], kWarps);
+            mbar_init(&S.rempty[i], 1);
+        }
+        for (int i = 0; i < kNB; ++i) {
+            mbar_init(&S.bfull[i], 1);
+            mbar_init(&S.bempty[i], kComputeWarps);
+        }
         *S.abort = 0;
         mbar_fence_init();
+        // the tensor maps of the shelves in use
+        for (int t = 0; t <= p.w.n_tiers; ++t) {
+            if (t == p.w.n_tiers && !p.has_shared) break;
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&M.gq[t])) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&M.dq[t])) : "memory");
+        }
     }
     if (threadIdx.x < 6) {
         const int phase = threadIdx.x / 3, bi = threadIdx.x % 3;
         const int bits = bi == 0 ? 8 : (bi == 1 ? 4 : 3);
         S.geo[threadIdx.x] = phase == 0 ? geo_gu(p.w.H, bits) : geo(p.w.I, bits);
     }
-    __syncthreads();
-    // slot table: active routed experts with work for this path, compacted in
-    // order by warp 0 (no block-wide barrier per step), then the shared
-    // expert; then the schedule (unit costs and their prefix sums)
-    __shared__ int n_keep;
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        const int n_active_all = min(act_s[0], p.max_active);
-        int run = 0;
-        for (int a0 = 0; a0 < n_active_all; a0 += 32) {
-            const int a = a0 + lane;
-            int e = -1, f = 0, cnt = 0;
-            if (a < n_active_all) {
-                e = act_s[1 + a];
-                if (e >= 0 && e < p.E) {
-                    f = off_s[e];
-                    cnt = off_s[e + 1] - f;
-                }
-            }
-            const bool keep = a < n_active_all && e >= 0 && e < p.E && cnt > 0 && cnt <= p.max_count;
-            const unsigned m = __ballot_sync(0xffffffffu, keep);
-            if (keep) {
-                const int pos = run + __popc(m & ((1u << lane) - 1u));
-                int ti = 0;  // the shelf holding e (shelves cover [0, E) without overlap)
-                for (int t = 0; t < p.w.n_tiers; ++t)
-                    if (e >= S.tp[t].first && e - S.tp[t].first < S.tp[t].n) ti = t;
-                S.st.expert[pos] = e;
-                S.st.bits[pos] = S.tp[ti].bits;
-                S.st.first[pos] = f;
-                S.st.count[pos] = cnt;
-                S.tier[pos] = ti;
-                S.jloc[pos] = e - S.tp[ti].first;
-            }
-            run += __popc(m);
-        }
-        const bool shared_here = p.has_shared && p.T <= p.max_count;
-        if (lane == 0 && shared_here) {
-            S.st.expert[run] = p.E;
-            S.st.bits[run] = p.w.shared.bits;
-            S.st.first[run] = S_;
-            S.st.count[run] = p.T;
-            S.tier[run] = p.w.n_tiers;
-            S.jloc[run] = 0;
-        }
-        const int ns = run + (shared_here ? 1 : 0);
-        if (lane == 0) n_keep = ns;
+    // everything above reads only the parameters; what follows reads the
+    // routing kernel's outputs
+    pdl_wait();
+    pdl_trigger();
+    const bool fused = p.route.on != 0;
+    const PrologueScratch ps = prologue_scratch(p.w.H, p.T, p.k, p.E, max_slots, fused);
+    int *act_s = reinterpret_cast<int *>(S.ring + ps.lists);  // active list + offsets
+    int *off_s = act_s + max_slots;
+    const uint8_t *x_s = S.ring + ps.x;
+    if (!fused) {
+        for (int i = threadIdx.x; i <= p.max_active; i += blockDim.x) cp_async_4b(act_s + i, p.active + i);
+        for (int e = threadIdx.x; e <= p.E; e += blockDim.x) cp_async_4b(off_s + e, p.offsets + e);
     }
+    if (S.srt && !fused)
+        for (int j = threadIdx.x; j < n_srt; j += blockDim.x) cp_async_4b(S.srt + j, p.sorted + j);
+    if (S.xall || fused)
+        for (int c = threadIdx.x; c < p.T * p.w.H / 8; c += blockDim.x)
+            cp_async_16b(const_cast<uint8_t *>(x_s) + 16 * c, p.x + 8 * static_cast<size_t>(c));
+    cp_async_wait_all();
     __syncthreads();
-    // the schedule: warp 0 for the gate_up tiles, warp 1 for the down tiles
-    if (threadIdx.x < 64) {
-        const int lane = threadIdx.x & 31, phase = threadIdx.x >> 5;
-        const int ns = n_keep;
-        {
-            const long long nt = tiles_per_slot(p, phase);
-            long long *tc = phase == 0 ? S.sc.tc0 : S.sc.tc1;
-            long long *pre = phase == 0 ? S.sc.pre0 : S.sc.pre1;
-            long long base = 0;
-            for (int a0 = 0; a0 < ns; a0 += 32) {
-                const int a = a0 + lane;
-                long long v = 0;
-                if (a < ns) {
-                    const long long c = tile_cost(p, phase, S.st.bits[a], S.st.count[a]);
-                    tc[a] = c;
-                    v = nt * c;
-                }
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const long long u = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += u;
-                }
-                if (a < ns) pre[a] = base + v;
-                base += __shfl_sync(0xffffffffu, v, 31);
-            }
-            // this CTA's contiguous share [lo, hi) of the phase's total cost,
-            // and each slot's tiles whose start falls in it
-            const long long lo = div_floor(base * blockIdx.x, gridDim.x);
-            const long long hi = div_floor(base * (blockIdx.x + 1), gridDim.x);
-            int2 *rng = phase == 0 ? S.sc.rng0 : S.sc.rng1;
-            int first = 0x7fffffff, last = -1;
-            for (int a0 = 0; a0 < ns; a0 += 32) {
-                const int a = a0 + lane;
-                bool has = false;
-                if (a < ns) {
-                    const long long tb = tc[a], off = pre[a] - nt * tb;
-                    const int b0 = tiles_before(lo - off, tb, static_cast<int>(nt));
-                    const int b1 = tiles_before(hi - off, tb, static_cast<int>(nt));
-                    rng[a] = make_int2(b0, b1);
-                    has = b0 < b1;
-                }
-                const unsigned m = __ballot_sync(0xffffffffu, has);
-                if (m) {
-                    first = min(first, a0 + __ffs(m) - 1);
-                    last = max(last, a0 + 31 - __clz(m));
-                }
-            }
+    if (S.xall) {
+        const bool xbad = build_xall(p, x_s, S.xall);
+        if (__any_sync(0xffffffffu, xbad) && lane == 0) status_or(p.status, MOE_STATUS_FP16_RANGE);
+    }
+    bool routed = true;
+    if (fused) routed = route_in_cta(p, S, reinterpret_cast<const uint16_t *>(x_s), act_s, off_s, ps);
+    if (!routed) {  // the grid barrier gave up: stream nothing
+        if (threadIdx.x < 5) S.range[threadIdx.x] = 0;
+    } else {
+        if (warp == 0) {
+            const int ns = plan_compact(p.pi, act_s, off_s, S.pt);
+            if (lane == 0) S.range[4] = ns;
+        }
+        __syncthreads();
+        if (warp < 2) {
+            const int ns = S.range[4];
+            const long long total = plan_costs(p.pi, ns, warp, S.pt);
             if (lane == 0) {
-                S.sc.fl[2 * phase] = first;
-                S.sc.fl[2 * phase + 1] = last;
+                const int2 r = plan_cta_range(S.pt, ns, warp == 0 ? S.nt0 : S.nt1, warp, total, blockIdx.x,
+                                              gridDim.x);
+                S.range[2 * warp] = r.x;
+                S.range[2 * warp + 1] = r.y;
             }
         }
     }
-    // the prologue's tables in the stage ring are overwritten by TMA copies
-    // from here on: order this thread's generic accesses before them
+    // the ring's scratch is overwritten by TMA copies from here on: order
+    // this thread's generic accesses before them
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
-    const int n_slots = n_keep;
-    ffn_stream_body(p, M, S, n_slots, nstages);
+
+    if (warp == kWarpProducer) {
+        run_producer(p, M, S);
+        return;
+    }
+    if (warp < kComputeWarps) run_compute(p, S, warp);
+    else if (warp == kWarpLoader) run_loader(p, S);
+    else if (warp >= kWarpEpilogue0) run_epilogue(p, S, warp - kWarpEpilogue0);
 }
 
 }  // namespace moe
 
-// Shared memory of one CTA: the stage ring, each group's x fragments and
-// K-slice partials, shelf and geometry tables, and the slot/entry/schedule
-// tables.  Returns the byte count and the number of stages that fit in the
-// budget (even: each stage serves one group).
-size_t moe_ffn_stream_smem(int H, int I, int T, int max_slots, int n_ent, int *nstages) {
-    const size_t ent = n_ent <= moe::kMaxSmemEntries ? 2 * sizeof(int) * static_cast<size_t>(n_ent) : 0;
-    const size_t fixed = moe::kGroups * (static_cast<size_t>(moe::xf_bytes(H, I, T)) + moe::kRedBytes) +
-                         moe::kMaxStages * sizeof(uint64_t) + moe::kGroups * sizeof(moe::StreamSmem::Ahead) +
-                         (MOE_MAX_TIERS + 1) * sizeof(moe::TierPtrs) +
-                         6 * sizeof(moe::Geo) + 8 + 6 * sizeof(int) * static_cast<size_t>(max_slots) + ent +
-                         2 * sizeof(int2) * static_cast<size_t>(max_slots) + 4 * sizeof(int) + 16;
-    const size_t budget = 220 * 1024;
-    int ns = fixed < budget ? static_cast<int>((budget - fixed) / moe::kStageBytes) : 0;
-    if (ns > moe::kMaxStages) ns = moe::kMaxStages;
-    ns &= ~(moe::kGroups - 1);
-    *nstages = ns;
-    return static_cast<size_t>(ns) * moe::kStageBytes + fixed;
+// Shared memory of one CTA: the byte ring for staged tiles, the all-token x
+// fragments, the B-operand and partial-sum buffers, barriers, and the slot
+// tables.  Returns the byte count and the ring size in *ring_bytes (0 when
+// the ring cannot hold the largest tile and the prologue's scratch).
+size_t moe_ffn_stream_smem(int H, int I, int T, int k, int E, int max_slots, bool fused, int *ring_bytes) {
+    const size_t n_srt = static_cast<size_t>(T) * k;
+    const size_t fixed = static_cast<size_t>(moe::xall_bytes(H, T)) + moe::kNB * static_cast<size_t>(moe::bbuf_bytes(H, I, T)) +
+                         moe::kGroups * moe::kNR * static_cast<size_t>(moe::kRedBytes) +
+                         (2 * moe::kND + 2 * moe::kGroups * moe::kNR + 2 * moe::kNB) * sizeof(uint64_t) +
+                         12 * sizeof(int) +
+                         (MOE_MAX_TIERS + 1) * sizeof(moe::TierPtrs) + 6 * sizeof(moe::Geo) + 16 +
+                         moe::plan_tab_bytes(max_slots) + (n_srt <= moe::kMaxSmemEntries ? n_srt * sizeof(int) : 0);
+    const size_t budget = 227 * 1024;
+    size_t ring = fixed < budget ? ((budget - fixed) & ~static_cast<size_t>(moe::kTileAlign - 1)) : 0;
+    const size_t scratch = moe::prologue_scratch(H, T, k, E, max_slots, fused).end;
+    if (ring < static_cast<size_t>(moe::kMaxTileBytes) || ring < scratch) ring = 0;
+    *ring_bytes = static_cast<int>(ring);
+    return ring + fixed;
 }
 
 cudaError_t moe_configure_ffn_stream() {
-    // the opt-in limit is 227 KB per CTA including static shared memory
-    return cudaFuncSetAttribute(moe::ffn_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                227 * 1024 - 1024);
+    return cudaFuncSetAttribute(moe::ffn_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
 }
 
 bool moe_ffn_stream_supported(int H, int I) {
     return H <= moe::kMaxK && I <= moe::kMaxK && H % 128 == 0 && I % 128 == 0;
 }
 
-// Whether a launch for this batch gets the two stages the consumer groups need.
-bool moe_ffn_stream_fits(int H, int I, int T, int max_slots, int n_ent) {
-    int ns = 0;
-    moe_ffn_stream_smem(H, I, T, max_slots, n_ent, &ns);
-    return ns >= moe::kGroups;
+// Whether a launch for this batch gets a ring that holds the largest tile.
+bool moe_ffn_stream_fits(int H, int I, int T, int k, int E, int max_slots) {
+    int ring = 0, ring2 = 0;
+    moe_ffn_stream_smem(H, I, T, k, E, max_slots, false, &ring);
+    moe_ffn_stream_smem(H, I, T, k, E, max_slots, T <= moe::kRouterTokTile, &ring2);
+    return ring > 0 && ring2 > 0;
 }
 
 namespace {
@@ -1173,11 +1272,12 @@ bool shelf_maps(moe::StreamMaps &M, int t, const moe_tier &tier, int H, int I) {
 
 }  // namespace
 
+
 // counters (int[max_active + 1]) must be zero on entry; the caller clears them.
 cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
-    int nstages = 0;
-    const size_t smem = moe_ffn_stream_smem(p.w.H, p.w.I, p.T, p.max_active + 1, p.T * p.k + p.T, &nstages);
-    if (nstages < moe::kGroups) return cudaErrorInvalidConfiguration;
+    int ring = 0;
+    const size_t smem = moe_ffn_stream_smem(p.w.H, p.w.I, p.T, p.k, p.E, p.max_active + 1, p.route.on != 0, &ring);
+    if (ring == 0) return cudaErrorInvalidConfiguration;
     int dev = 0;
     cudaGetDevice(&dev);
     int sms = 0;
@@ -1187,15 +1287,20 @@ cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     cfg.blockDim = dim3(moe::kBlockThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    moe::PdlAttrs at(true);
+    cfg.attrs = at.a;
+    cfg.numAttrs = at.n;
     moe::StreamMaps M;
     std::memset(&M, 0, sizeof(M));
     for (int t = 0; t < p.w.n_tiers; ++t)
         if (!shelf_maps(M, t, p.w.tiers[t], p.w.H, p.w.I)) return cudaErrorInvalidValue;
     if (p.has_shared && !shelf_maps(M, p.w.n_tiers, p.w.shared, p.w.H, p.w.I)) return cudaErrorInvalidValue;
-    return cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, M, nstages);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, M, ring);
+    if (e != cudaSuccess) {  // without overlapping the predecessor
+        cudaGetLastError();
+        cfg.attrs = at.a + 1;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, M, ring);
+    }
+    return e;
 }

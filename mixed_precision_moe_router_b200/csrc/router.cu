@@ -7,45 +7,9 @@
 #include <float.h>
 
 #include "common.cuh"
+#include "route_cta.cuh"
 
 namespace moe {
-
-constexpr int kRouterTokTile = 16;   // tokens staged in shared memory per CTA
-constexpr int kRouterWarps = 4;      // one expert per warp
-
-// Dot products of one expert row with the nt (<= kRouterTokTile) tokens staged
-// in xs, by one warp: lane-strided 8-element chunks and an fma chain per token
-// (per-lane partial sums; the caller adds them with warp_sum).  Every routing
-// kernel below uses this one function, so a logit has the same bits whichever
-// kernel computed it.
-__device__ __forceinline__ void expert_dots(const uint16_t *xs, const uint16_t *wrow, int nt, int vec_per_row,
-                                            float (&acc)[kRouterTokTile]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
-#pragma unroll 4
-    for (int c = lane; c < vec_per_row; c += 32) {
-        const uint4 wv = ld_stream_v4(wrow + c * 8);
-        const float w[8] = {bf16lo(wv.x), bf16hi(wv.x), bf16lo(wv.y), bf16hi(wv.y),
-                            bf16lo(wv.z), bf16hi(wv.z), bf16lo(wv.w), bf16hi(wv.w)};
-#pragma unroll
-        for (int t = 0; t < kRouterTokTile; ++t) {
-            if (t < nt) {
-                const uint4 xv = reinterpret_cast<const uint4 *>(xs)[t * vec_per_row + c];
-                float a = acc[t];
-                a = fmaf(w[0], bf16lo(xv.x), a);
-                a = fmaf(w[1], bf16hi(xv.x), a);
-                a = fmaf(w[2], bf16lo(xv.y), a);
-                a = fmaf(w[3], bf16hi(xv.y), a);
-                a = fmaf(w[4], bf16lo(xv.z), a);
-                a = fmaf(w[5], bf16hi(xv.z), a);
-                a = fmaf(w[6], bf16lo(xv.w), a);
-                a = fmaf(w[7], bf16hi(xv.w), a);
-                acc[t] = a;
-            }
-        }
-    }
-}
 
 // Stage nt tokens of x (bf16 rows of H) into shared memory, 16 bytes a thread.
 __device__ __forceinline__ void stage_tokens(const uint16_t *x, int nt, int vec_per_row, uint16_t *xs) {
@@ -80,11 +44,6 @@ router_logits_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
             if (lane == 0) logits[static_cast<size_t>(t0 + t) * E + e] = v + b;
         }
     }
-}
-
-// Is (va, ia) ranked before (vb, ib)?  Larger logit first, then lower id.
-__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
-    return va > vb || (va == vb && ia < ib);
 }
 
 // Top-k of one logit row by one warp: k rounds of a warp-wide arg-max over
@@ -203,6 +162,8 @@ route_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
     __shared__ int total_slots, total_active, is_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int vec_per_row = H / 8;
+    pdl_wait();  // x is the previous kernel's output
+    pdl_trigger();
     stage_tokens(x, T, vec_per_row, xs);
     __syncthreads();
     const int e = blockIdx.x * kRouteWarps + warp;
@@ -343,11 +304,20 @@ cudaError_t moe_launch_route_small(const uint16_t *x, const uint16_t *wr, const 
     const int grid = (E + moe::kRouteWarps - 1) / moe::kRouteWarps;
     const int threads = moe::kRouteWarps * 32;
     const int nj = (E + 31) / 32;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    moe::PdlAttrs at;
+    cfg.attrs = at.a;
+    cfg.numAttrs = at.n;
 #define MOE_ROUTE_ARGS x, wr, bias, T, H, E, k, logits, idx, w, offsets, sorted, pos, active, status, ticket, clear, n_clear
-    if (nj <= 4) moe::route_small_kernel<4><<<grid, threads, smem, s>>>(MOE_ROUTE_ARGS);
-    else if (nj <= 8) moe::route_small_kernel<8><<<grid, threads, smem, s>>>(MOE_ROUTE_ARGS);
-    else if (nj <= 16) moe::route_small_kernel<16><<<grid, threads, smem, s>>>(MOE_ROUTE_ARGS);
-    else moe::route_small_kernel<32><<<grid, threads, smem, s>>>(MOE_ROUTE_ARGS);
+    cudaError_t e;
+    if (nj <= 4) e = cudaLaunchKernelEx(&cfg, moe::route_small_kernel<4>, MOE_ROUTE_ARGS);
+    else if (nj <= 8) e = cudaLaunchKernelEx(&cfg, moe::route_small_kernel<8>, MOE_ROUTE_ARGS);
+    else if (nj <= 16) e = cudaLaunchKernelEx(&cfg, moe::route_small_kernel<16>, MOE_ROUTE_ARGS);
+    else e = cudaLaunchKernelEx(&cfg, moe::route_small_kernel<32>, MOE_ROUTE_ARGS);
 #undef MOE_ROUTE_ARGS
-    return cudaGetLastError();
+    return e;
 }

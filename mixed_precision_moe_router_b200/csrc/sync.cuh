@@ -46,6 +46,55 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a caller-chosen suspend-time hint in nanoseconds.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity; false once *abort is set (by
+// another warp of the CTA giving up) or after `limit` SM clock cycles.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t parity, const volatile int *abort,
+                                                    long long limit) {
+    if (mbar_try_wait_ns(bar, parity, 20000u)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_ns(bar, parity, 20000u)) {
+        if (*abort || clock64() - t0 > limit) return false;
+    }
+    return true;
+}
+
+// Warp-wide wait for the phase with the given parity: lane 0 polls (with the
+// abort flag and the cycle limit of mbar_wait_abortable), then every lane
+// confirms with one try_wait of its own (which acquires the phase; it cannot
+// have moved on, since advancing it takes an action of this warp).  Returns the
+// same result in every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, const volatile int *abort,
+                                               long long limit) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_abortable(bar, parity, abort, limit);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) mbar_try_wait_ns(bar, parity, 0u);
+    return ok;
+}
+
+// Wait for the phase with the given parity; false after `limit` cycles.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit) return false;
+    }
+    return true;
+}
+
 // Wait until the phase with the given parity has completed; false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -66,6 +115,18 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Asynchronous global -> shared copies of 4 and 16 bytes (cp.async), waited
+// for with cp_async_wait_all.
+__device__ __forceinline__ void cp_async_4b(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_16b(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ int ld_acquire(const int *p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -82,6 +143,45 @@ __device__ __forceinline__ bool wait_geq_backoff(const int *ctr, int target) {
         if (clock64() - t0 > kWaitLimitCycles) return false;
         __nanosleep(ns);
         if (ns < 1024) ns *= 2;
+    }
+    return true;
+}
+
+// Spin until *ctr >= target (acquire), with backoff; false once *abort is
+// set or after `limit` cycles.
+__device__ __forceinline__ bool wait_geq_abortable(const int *ctr, int target, const volatile int *abort,
+                                                   long long limit) {
+    if (ld_acquire(ctr) >= target) return true;
+    const long long t0 = clock64();
+    unsigned ns = 32;
+    while (ld_acquire(ctr) < target) {
+        if (*abort || clock64() - t0 > limit) return false;
+        __nanosleep(ns);
+        if (ns < 512) ns *= 2;
+    }
+    return true;
+}
+
+// Grid-wide barrier of a cooperative launch.  bar[0] counts arrivals (zero on
+// entry; the last arriver resets it), bar[1] is a generation number.  Thread 0
+// of each CTA arrives after a fence and waits (bounded, abortable) for the
+// generation to move; the caller follows with __syncthreads.  Returns false
+// when the wait gave up.
+__device__ __forceinline__ bool grid_barrier(int *bar, const volatile int *abort, long long limit) {
+    const int gen = ld_acquire(bar + 1);
+    __threadfence();
+    if (atomicAdd(bar, 1) == static_cast<int>(gridDim.x * gridDim.y * gridDim.z) - 1) {
+        bar[0] = 0;
+        __threadfence();
+        atomicAdd(bar + 1, 1);
+        return true;
+    }
+    const long long t0 = clock64();
+    unsigned ns = 32;
+    while (ld_acquire(bar + 1) == gen) {
+        if (*abort || clock64() - t0 > limit) return false;
+        __nanosleep(ns);
+        if (ns < 256) ns *= 2;
     }
     return true;
 }
