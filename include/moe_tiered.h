@@ -315,6 +315,47 @@ int moe_layer_forward(const moe_layer_weights *w, const uint16_t *w_router,
                       uint16_t *x_next_norm, void *workspace, size_t workspace_bytes, int32_t mode,
                       int32_t *status, moe_stream_t stream);
 
+/*
+ * A stack of decode layers in one persistent launch ([P5] "What the model
+ * actually is": 48 layers with a residual design; [P1] "step 3: split every
+ * layer into hot and cold": the per-token time goes to thousands of launches
+ * and syncs rather than to expert bytes, so the whole stack runs as one).
+ * For each layer l, with x_0 = x_in:
+ *   n_l     = bf16_rne(x_l / sqrt(mean_h(x_l^2) + MOE_NORM_EPS))
+ *   out_l   = the layer on n_l: router top-k, the tiered expert FFN (every
+ *             expert on the streaming path, MOE_FFN_GEMV numerics) and combine
+ *   x_{l+1} = bf16_rne(x_l + out_l)
+ * x_out = x_L; x_out_norm = n_L when given.  x_layers, when given, receives
+ * x_0 .. x_L ([n_layers + 1][T][H]) for inspection.
+ *
+ * moe_stack_prepare writes a device descriptor of the layers (their weights
+ * descriptors, routers and the tensor maps of their shelves):
+ *   layers    host array [n_layers]; all share H, I and E
+ *   w_router  host array [n_layers] of device pointers, bf16 [E][H]
+ *   bias      host array [n_layers] of device pointers fp32 [E] (entries may
+ *             be NULL), or NULL for no bias at all
+ *   desc      device buffer of moe_stack_desc_bytes(n_layers) bytes, 64-byte
+ *             aligned, owned by the caller
+ * Unlike every other call it copies synchronously (a set-up step, run once
+ * per set of weights; run it again whenever a weight pointer changes).
+ *
+ * moe_stack_forward enqueues one memset and one cooperative launch:
+ *   x_in, x_out bf16 [T][H]; x_out_norm bf16 [T][H] or NULL; x_layers or NULL
+ *   workspace  moe_stack_workspace_size() bytes, 16-byte aligned
+ *   status     as for the other calls (MOE_STATUS_TIMEOUT if a grid-wide or
+ *              pipeline wait gave up; outputs are then undefined)
+ * Limits: 1 <= T <= 8; k, E, H and I as for moe_layer_forward on the
+ * streaming path.  Calls sharing a workspace must not overlap on the GPU.
+ */
+size_t moe_stack_desc_bytes(int32_t n_layers);
+int moe_stack_prepare(const moe_layer_weights *layers, const uint16_t *const *w_router,
+                      const float *const *bias, int32_t n_layers, void *desc, size_t desc_bytes);
+size_t moe_stack_workspace_size(int32_t H, int32_t I, int32_t E, int32_t T, int32_t k);
+int moe_stack_forward(const void *desc, int32_t n_layers, int32_t H, int32_t I, int32_t E,
+                      int32_t T, int32_t k, const uint16_t *x_in, uint16_t *x_out,
+                      uint16_t *x_out_norm, uint16_t *x_layers, void *workspace,
+                      size_t workspace_bytes, int32_t *status, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

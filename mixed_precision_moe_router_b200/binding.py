@@ -65,6 +65,12 @@ SIGNATURES = [
     ("moe_layer_workspace_size", c_size, [ctypes.POINTER(LayerWeights), c_i32, c_i32, c_i32]),
     ("moe_layer_forward", c_i32, [ctypes.POINTER(LayerWeights), c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp,
                                   c_vp, c_vp, c_vp, c_size, c_i32, c_vp, c_vp]),
+    ("moe_stack_desc_bytes", c_size, [c_i32]),
+    ("moe_stack_prepare", c_i32, [ctypes.POINTER(LayerWeights), ctypes.POINTER(c_vp), ctypes.POINTER(c_vp), c_i32,
+                                  c_vp, c_size]),
+    ("moe_stack_workspace_size", c_size, [c_i32, c_i32, c_i32, c_i32, c_i32]),
+    ("moe_stack_forward", c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                  c_size, c_vp, c_vp]),
 ]
 
 _lib = None
@@ -378,3 +384,46 @@ def layer_forward(layer, w_router, bias, x, k, residual=None, mode=FFN_AUTO, wor
                                    _ptr(out), _ptr(x_next), _ptr(x_next_norm), _ptr(workspace), workspace.numel(),
                                    mode, _ptr(status), _stream()))
     return out if residual is None else (out, x_next, x_next_norm)
+
+
+# ---------------------------------------------------------------------------
+# a stack of decode layers in one persistent launch
+# ---------------------------------------------------------------------------
+
+class Stack:
+    """Device descriptor of a stack of layers for :func:`stack_forward`
+    (moe_stack_prepare; the layers and routers must outlive it)."""
+
+    def __init__(self, layers, routers):
+        n = len(layers)
+        self.layers, self.routers = layers, routers
+        self.H, self.I, self.E = layers[0].H, layers[0].I, layers[0].E
+        self.n = n
+        descs = (LayerWeights * n)(*[l.descriptor() for l in layers])
+        wr = (c_vp * n)(*[r[0].data_ptr() for r in routers])
+        bias = (c_vp * n)(*[(r[1].data_ptr() if r[1] is not None else None) for r in routers])
+        nbytes = int(lib().moe_stack_desc_bytes(n))
+        dev = routers[0][0].device
+        self._buf = torch.empty(nbytes + 64, dtype=torch.uint8, device=dev)
+        off = (-self._buf.data_ptr()) % 64
+        self.desc = self._buf[off:off + nbytes]
+        _check(lib().moe_stack_prepare(descs, wr, bias, n, _ptr(self.desc), nbytes))
+
+    def workspace_size(self, T, k):
+        return int(lib().moe_stack_workspace_size(self.H, self.I, self.E, T, k))
+
+
+def stack_forward(stack, x_in, k, out=None, out_norm=None, x_layers=None, workspace=None, status=None):
+    """x_in (bf16 [T, H], the residual stream) through every layer of `stack`
+    in one launch; returns x_out (and fills out_norm / x_layers when given)."""
+    _need(x_in, torch.bfloat16, name="x_in")
+    T, H = x_in.shape
+    if out is None:
+        out = torch.empty_like(x_in)
+    nws = stack.workspace_size(T, k)
+    if workspace is None:
+        workspace = torch.empty(max(nws, 1), dtype=torch.uint8, device=x_in.device)
+    _check(lib().moe_stack_forward(_ptr(stack.desc), stack.n, stack.H, stack.I, stack.E, T, k, _ptr(x_in), _ptr(out),
+                                   _ptr(out_norm), _ptr(x_layers), _ptr(workspace), workspace.numel(), _ptr(status),
+                                   _stream()))
+    return out

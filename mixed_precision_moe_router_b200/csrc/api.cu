@@ -41,6 +41,13 @@ size_t moe_ffn_gemm_workspace(const moe_layer_weights *, int T, int k);
 cudaError_t moe_launch_combine(const float *, const float *, const float *, int, int, int, const uint16_t *,
                                uint16_t *, uint16_t *, uint16_t *, cudaStream_t);
 cudaError_t moe_launch_rmsnorm(const uint16_t *, int, int, uint16_t *, cudaStream_t);
+size_t moe_stack_layer_bytes();
+cudaError_t moe_stack_encode_layer(const moe_layer_weights *, const uint16_t *, const float *, void *);
+size_t moe_stack_smem(int H, int I, int T, int k, int E, int *ring_bytes);
+cudaError_t moe_configure_stack();
+cudaError_t moe_launch_stack(const void *, int, int, int, int, int, int, const uint16_t *, uint16_t *, uint16_t *,
+                             uint16_t *, uint16_t *, float *, float *, float *, float *, int *, int *, int32_t *,
+                             long long, cudaStream_t);
 
 namespace {
 
@@ -87,6 +94,7 @@ int ensure_configured() {
         if (r == cudaSuccess) r = moe_configure_bucketize();
         if (r == cudaSuccess) r = moe_configure_ffn_stream();
         if (r == cudaSuccess) r = moe_configure_ffn_gemm();
+        if (r == cudaSuccess) r = moe_configure_stack();
         g_dev_err[dev] = r;
     });
     if (g_dev_err[dev] != cudaSuccess) return cuda_fail(g_dev_err[dev], "kernel configuration");
@@ -683,3 +691,114 @@ extern "C" int moe_expert_ffn_tiered_static(const moe_layer_weights *w, const ui
     if (e == cudaSuccess) e = moe_launch_ffn_stream(p, s);
     return e == cudaSuccess ? ok() : cuda_fail(e, "ffn launch");
 }
+
+// ---------------------------------------------------------------------------
+// A stack of decode layers in one persistent launch
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kStackMaxTokens = 8;
+
+struct StackWs {
+    float *logits, *h, *y_slots, *y_shared;
+    uint16_t *xbuf;
+    int *ctr;  // per-slot counts, then the two grid barrier words
+    size_t ctr_bytes;
+    size_t total;
+};
+
+StackWs carve_stack(int H, int I, int E, int T, int k, char *base) {
+    StackWs L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *p = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return p;
+    };
+    const size_t S = static_cast<size_t>(T) * k;
+    const long ma = static_cast<long>(S) < E ? static_cast<long>(S) : E;
+    L.logits = reinterpret_cast<float *>(take(static_cast<size_t>(T) * E * sizeof(float)));
+    L.h = reinterpret_cast<float *>(take((S + T) * I * sizeof(float)));
+    L.y_slots = reinterpret_cast<float *>(take(S * H * sizeof(float)));
+    L.y_shared = reinterpret_cast<float *>(take(static_cast<size_t>(T) * H * sizeof(float)));
+    L.xbuf = reinterpret_cast<uint16_t *>(take(2 * static_cast<size_t>(T) * H * sizeof(uint16_t)));
+    L.ctr_bytes = align_up((static_cast<size_t>(ma) + 1 + 2) * sizeof(int));
+    L.ctr = reinterpret_cast<int *>(take(L.ctr_bytes));
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_stack_desc_bytes(int32_t n_layers) {
+    if (n_layers < 1) return 0;
+    return static_cast<size_t>(n_layers) * moe_stack_layer_bytes();
+}
+
+int moe_stack_prepare(const moe_layer_weights *layers, const uint16_t *const *w_router, const float *const *bias,
+                      int32_t n_layers, void *desc, size_t desc_bytes) {
+    if (n_layers < 1) return fail(MOE_ERR_INVALID_ARG, "n_layers = %d", n_layers);
+    if (!layers || !w_router) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    const size_t need = moe_stack_desc_bytes(n_layers);
+    if (!desc || desc_bytes < need) return fail(MOE_ERR_WORKSPACE, "stack descriptor needs %zu bytes", need);
+    if ((reinterpret_cast<uintptr_t>(desc) & 63u) != 0) return fail(MOE_ERR_INVALID_ARG, "descriptor not 64-byte aligned");
+    for (int l = 0; l < n_layers; ++l) {
+        int r = check_weights(&layers[l]);
+        if (r) return fail(r, "layer %d: %s", l, g_err.c_str());
+        if (layers[l].H != layers[0].H || layers[l].I != layers[0].I || layers[l].E != layers[0].E)
+            return fail(MOE_ERR_INVALID_ARG, "layer %d: H, I and E must match layer 0", l);
+        if (!w_router[l] || !aligned16(w_router[l])) return fail(MOE_ERR_INVALID_ARG, "layer %d: router NULL or misaligned", l);
+    }
+    if (!moe_ffn_stream_supported(layers[0].H, layers[0].I))
+        return fail(MOE_ERR_UNSUPPORTED, "the streaming path supports H, I <= 2048");
+    int r = ensure_configured();
+    if (r) return r;
+    const size_t lb = moe_stack_layer_bytes();
+    std::string host(need, '\0');
+    for (int l = 0; l < n_layers; ++l) {
+        cudaError_t e = moe_stack_encode_layer(&layers[l], w_router[l], bias ? bias[l] : nullptr, &host[l * lb]);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor map encoding");
+    }
+    cudaError_t e = cudaMemcpy(desc, host.data(), need, cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "descriptor copy");
+}
+
+size_t moe_stack_workspace_size(int32_t H, int32_t I, int32_t E, int32_t T, int32_t k) {
+    if (H <= 0 || I <= 0 || E <= 0 || T <= 0 || k <= 0) return 0;
+    return carve_stack(H, I, E, T, k, nullptr).total;
+}
+
+int moe_stack_forward(const void *desc, int32_t n_layers, int32_t H, int32_t I, int32_t E, int32_t T, int32_t k,
+                      const uint16_t *x_in, uint16_t *x_out, uint16_t *x_out_norm, uint16_t *x_layers,
+                      void *workspace, size_t workspace_bytes, int32_t *status, moe_stream_t stream) {
+    if (n_layers < 1) return fail(MOE_ERR_INVALID_ARG, "n_layers = %d", n_layers);
+    int r = check_k(T, E, k);
+    if (r) return r;
+    if (T < 1 || T > kStackMaxTokens) return fail(MOE_ERR_UNSUPPORTED, "T = %d (the stack kernel takes 1..%d tokens)", T, kStackMaxTokens);
+    if (H <= 0 || H % 128 != 0 || I <= 0 || I % 128 != 0) return fail(MOE_ERR_INVALID_ARG, "H = %d, I = %d", H, I);
+    if (!moe_ffn_stream_supported(H, I)) return fail(MOE_ERR_UNSUPPORTED, "the streaming path supports H, I <= 2048");
+    if (!desc || !x_in || !x_out) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(x_in) || !aligned16(x_out) || (x_out_norm && !aligned16(x_out_norm)) || (x_layers && !aligned16(x_layers)))
+        return fail(MOE_ERR_INVALID_ARG, "stream pointers not 16-byte aligned");
+    const size_t need = moe_stack_workspace_size(H, I, E, T, k);
+    if (!workspace || workspace_bytes < need) return fail(MOE_ERR_WORKSPACE, "stack workspace needs %zu bytes", need);
+    if (!aligned16(workspace)) return fail(MOE_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    int ring = 0;
+    moe_stack_smem(H, I, T, k, E, &ring);
+    if (ring == 0) return fail(MOE_ERR_UNSUPPORTED, "shared memory for T = %d, k = %d leaves no room for a tile", T, k);
+    r = ensure_configured();
+    if (r) return r;
+    StackWs L = carve_stack(H, I, E, T, k, static_cast<char *>(workspace));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(L.ctr, 0, L.ctr_bytes, s);
+    const long ma = static_cast<long>(T) * k < E ? static_cast<long>(T) * k : E;
+    if (e == cudaSuccess)
+        e = moe_launch_stack(desc, n_layers, T, k, H, I, E, x_in, x_out, x_out_norm, x_layers, L.xbuf, L.logits, L.h,
+                             L.y_slots, L.y_shared, L.ctr, L.ctr + ma + 1, status, g_wait_limit.load(), s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "stack launch");
+}
+
+}  // extern "C"

@@ -68,6 +68,7 @@ constexpr int kTileAlign = 1024;   // ring allocations start on a 128-byte-swizz
 constexpr int kMaxK = 2048;
 constexpr int kRedBytes = kWarps * 32 * 16;  // one item's partials: a float4 per compute lane
 constexpr int kMaxSmemEntries = 2048;        // sorted slot ids kept in shared memory up to this many
+constexpr int kMaxExpertShare = 16;          // router rows a CTA computes when it routes the batch itself
 
 // ---------------------------------------------------------------------------
 // tile geometry
@@ -647,10 +648,30 @@ __device__ __forceinline__ float4 compute_part(const Geo &G, int phase, const ui
 // Producer (lane 0 of its warp): allocate each tile in the byte ring, wait
 // until no tile still being read overlaps it (tiles are released oldest
 // first), and stage it.  Before returning it waits for every copy it issued.
-__device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMaps &M, StreamSmem &S) {
-    if ((threadIdx.x & 31) != 0) return;
-    int head = 0, rel = 0, i = 0;
+// State a role keeps from one layer to the next in a persistent launch (tile
+// and item counts fix the barrier phases and ring offsets).
+struct ProducerState {
+    int head, rel, i;
     int st[kND], en[kND];
+};
+struct ComputeState {
+    int head, i, m, kb;
+};
+struct LoaderState {
+    int kb;
+};
+struct EpilogueState {
+    int m, i;
+};
+
+// Producer for the current tile list; `drain`: wait for every copy in
+// flight before returning (the last list of a launch).
+__device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMaps &M, StreamSmem &S,
+                                             ProducerState &ps, bool drain) {
+    if ((threadIdx.x & 31) != 0) return;
+    int head = ps.head, rel = ps.rel, i = ps.i;
+    int(&st)[kND] = ps.st;
+    int(&en)[kND] = ps.en;
     bool ok = true;
     Walk w;
     walk_begin(S, w);
@@ -673,9 +694,14 @@ __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMap
         issue_tile(p, M, S, w.phase, w.a, w.b, S.ring + s0, &S.full[i % kND]);
     }
     if (!ok) abort_cta(p, S);
-    // tiles [0, i) were issued and those before rel consumed: the rest must land
-    for (int j = max(rel, i - kND); j < i; ++j)
-        if (!mbar_wait_limit(&S.full[j % kND], (j / kND) & 1, p.wait_limit)) status_or(p.status, MOE_STATUS_TIMEOUT);
+    ps.head = head;
+    ps.rel = rel;
+    ps.i = i;
+    // tiles before i were issued and those before rel consumed: the rest must land
+    if (drain || !ok)
+        for (int j = max(rel, i - kND); j < i; ++j)
+            if (!mbar_wait_limit(&S.full[j % kND], (j / kND) & 1, p.wait_limit))
+                status_or(p.status, MOE_STATUS_TIMEOUT);
 }
 
 // Compute warp `cw` (0..kComputeWarps-1): group cw / kWarps computes the
@@ -685,9 +711,9 @@ __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMap
 // change of operand it waits until the next one is built (even when its group
 // has no tile that uses it) and releases the previous one, so no release can
 // run ahead of the loader.
-__device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, int cw) {
+__device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, int cw, ComputeState &cs) {
     const int lane = threadIdx.x & 31, grp = cw / kWarps, warp = cw % kWarps;
-    int head = 0, i = 0, m = 0, kb = -1;
+    int head = cs.head, i = cs.i, m = cs.m, kb = cs.kb;
     long long key = -1;
     bool ok = true;
     float4 *red = S.red + grp * kNR * (kWarps * 32);
@@ -748,15 +774,19 @@ __device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, i
             ++m;
         }
     }
+    cs.head = head;
+    cs.i = i;
+    cs.m = m;
+    cs.kb = kb;
     if (!ok && lane == 0) abort_cta(p, S);
 }
 
 // Loader warp: the B operand of every (phase, slot, pass) that takes one, in
 // the order the compute warps use them; before a slot's first down operand it
 // waits (bounded) until every gate_up tile of the slot has been counted done.
-__device__ __forceinline__ void run_loader(const FfnParams &p, StreamSmem &S) {
+__device__ __forceinline__ void run_loader(const FfnParams &p, StreamSmem &S, LoaderState &ls) {
     const int lane = threadIdx.x & 31;
-    int kb = -1, ready = -1;
+    int kb = ls.kb, ready = -1;
     long long key = -1;
     bool ok = true, bad = false;
     Walk w;
@@ -792,6 +822,7 @@ __device__ __forceinline__ void run_loader(const FfnParams &p, StreamSmem &S) {
             if (lane == 0) mbar_arrive(&S.bfull[kb % kNB]);
         }
     }
+    ls.kb = kb;
     if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(p.status, MOE_STATUS_FP16_RANGE);
     if (!ok && lane == 0) abort_cta(p, S);
 }
@@ -856,9 +887,9 @@ __device__ __forceinline__ void epilogue_item(const FfnParams &p, const StreamSm
 // sequence leaves a slot's gate_up tiles it publishes how many of them the
 // group finished (after a fence, so that another CTA that sees the count also
 // sees the h values).
-__device__ __forceinline__ void run_epilogue(const FfnParams &p, StreamSmem &S, int grp) {
+__device__ __forceinline__ void run_epilogue(const FfnParams &p, StreamSmem &S, int grp, EpilogueState &es) {
     const int lane = threadIdx.x & 31;
-    int m = 0, pend = 0, i = 0;
+    int m = es.m, pend = 0, i = es.i;
     bool ok = true;
     float4 *red = S.red + grp * kNR * (kWarps * 32);
     uint64_t *rfull = S.rfull + grp * kNR, *rempty = S.rempty + grp * kNR;
@@ -892,6 +923,8 @@ __device__ __forceinline__ void run_epilogue(const FfnParams &p, StreamSmem &S, 
             pend = 0;
         }
     }
+    es.m = m;
+    es.i = i;
     if (!ok && lane == 0) abort_cta(p, S);
 }
 
@@ -914,7 +947,8 @@ __host__ __device__ __forceinline__ PrologueScratch prologue_scratch(int H, int 
     ps.x = align16(lists * sizeof(int));
     const bool need_x = fused || T <= kTokPerPass;
     ps.cand = align16(ps.x + (need_x ? static_cast<size_t>(T) * H * 2 : 0));
-    ps.idx = align16(ps.cand + (fused ? cta_topk_smem(T, E, k) : 0));
+    // the logits partials: 4 quarters x kMaxExpertShare experts x 16 tokens
+    ps.idx = align16(ps.cand + (fused ? 4 * static_cast<size_t>(kMaxExpertShare) * 16 * sizeof(float) : 0));
     ps.w = align16(ps.idx + (fused ? S_ * sizeof(int) : 0));
     ps.pos = align16(ps.w + (fused ? S_ * sizeof(float) : 0));
     ps.tmp = align16(ps.pos + (fused ? S_ * sizeof(int) : 0));
@@ -929,26 +963,12 @@ __host__ __device__ __forceinline__ PrologueScratch prologue_scratch(int H, int 
 // also writes the routing outputs.  False when the grid barrier gave up.
 __device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, const uint16_t *x_s, int *act_s,
                                           int *off_s, const PrologueScratch &ps) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int T = p.T, E = p.E, k = p.k, H = p.w.H, S_ = T * k;
-    const PlanIn &pi = p.pi;
-    (void)pi;
-    // logits of experts [E * c / G, E * (c + 1) / G): one warp per expert
+    // logits of experts [E * c / G, E * (c + 1) / G), all warps
     const int e0 = static_cast<int>(static_cast<long long>(E) * blockIdx.x / gridDim.x);
     const int e1 = static_cast<int>(static_cast<long long>(E) * (blockIdx.x + 1) / gridDim.x);
-    for (int e = e0 + warp; e < e1; e += nwarps) {
-        float acc[kRouterTokTile];
-        expert_dots(x_s, p.route.wr + static_cast<size_t>(e) * H, T, H / 8, acc);
-        const float b = p.route.bias ? p.route.bias[e] : 0.f;
-#pragma unroll
-        for (int t = 0; t < kRouterTokTile; ++t) {
-            if (t < T) {
-                const float v = warp_sum(acc[t]);
-                if (lane == 0) p.route.logits[static_cast<size_t>(t) * E + e] = v + b;
-            }
-        }
-    }
-    __syncthreads();
+    cta_logits(x_s, T, H, E, p.route.wr, p.route.bias, e0, e1,
+               reinterpret_cast<float *>(S.ring + ps.cand), p.route.logits);
     int *barrier_ok = S.range + 5;
     if (threadIdx.x == 0) {
         const bool ok = grid_barrier(p.route.gbar, S.abort, p.wait_limit);
@@ -963,9 +983,9 @@ __device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, 
     int *idx_s = reinterpret_cast<int *>(S.ring + ps.idx);
     float *w_s = reinterpret_cast<float *>(S.ring + ps.w);
     int *pos_s = reinterpret_cast<int *>(S.ring + ps.pos);
-    cta_topk(p.route.logits, T, E, k, S.ring + ps.cand, idx_s, w_s);
+    cta_topk_rows(p.route.logits, T, E, k, idx_s, w_s);
     cta_group(idx_s, S_, E, S.srt, pos_s, act_s, off_s, reinterpret_cast<int *>(S.ring + ps.tmp));
-    if (blockIdx.x == 0) {
+    if (blockIdx.x == 0 && p.route.topk_idx) {
         for (int i = threadIdx.x; i < S_; i += blockDim.x) {
             p.route.topk_idx[i] = idx_s[i];
             p.route.topk_w[i] = w_s[i];
@@ -975,24 +995,23 @@ __device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, 
         for (int e = threadIdx.x; e <= E; e += blockDim.x) p.route.offsets[e] = off_s[e];
         for (int a = threadIdx.x; a <= act_s[0]; a += blockDim.x) p.route.active[a] = act_s[a];
     }
-    (void)lane;
     return true;
 }
 
-__global__ void __launch_bounds__(kBlockThreads, 1)
-ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ StreamMaps M, int ring_bytes) {
-    extern __shared__ __align__(1024) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int max_slots = p.max_active + 1;
-    StreamSmem S;
+// Shared memory of a CTA (same layout for every launch shape): the ring,
+// the all-token x fragments, B-operand and partial-sum buffers, barriers,
+// flags, shelf pointers, geometry, slot tables and the sorted slot ids.
+// Returns the first byte past it.
+__device__ __forceinline__ uint8_t *carve_stream_smem(uint8_t *smem, int ring_bytes, int H, int I, int T, int k,
+                                                      int max_slots, StreamSmem &S) {
     uint8_t *q = smem;
     S.ring = q;
     S.ring_bytes = ring_bytes;
     q += ring_bytes;
-    const int xb = xall_bytes(p.w.H, p.T);
+    const int xb = xall_bytes(H, T);
     S.xall = xb ? q : nullptr;
     q += xb;
-    S.b_bytes = bbuf_bytes(p.w.H, p.w.I, p.T);
+    S.b_bytes = bbuf_bytes(H, I, T);
     S.bbuf = q;
     q += kNB * S.b_bytes;
     S.red = reinterpret_cast<float4 *>(q);
@@ -1006,7 +1025,7 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     S.bempty = S.bfull + kNB;
     q = reinterpret_cast<uint8_t *>(S.bempty + kNB);
     S.abort = reinterpret_cast<int *>(q);
-    S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots (16-byte aligned)
+    S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots, flag (16-byte aligned)
     q += 12 * sizeof(int);
     S.tp = reinterpret_cast<TierPtrs *>(q);
     q += (MOE_MAX_TIERS + 1) * sizeof(TierPtrs);
@@ -1015,32 +1034,28 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     q = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q) + 15) & ~static_cast<uintptr_t>(15));
     S.pt = plan_tabs(q, max_slots);
     q += plan_tab_bytes(max_slots);
-    const int n_srt = p.T * p.k;
+    const int n_srt = T * k;
     S.srt = n_srt <= kMaxSmemEntries ? reinterpret_cast<int *>(q) : nullptr;
-    S.nt0 = tiles_per_slot(p.w.H, p.w.I, 0);
-    S.nt1 = tiles_per_slot(p.w.H, p.w.I, 1);
+    if (S.srt) q += ((n_srt * sizeof(int) + 15) / 16) * 16;
+    S.nt0 = tiles_per_slot(H, I, 0);
+    S.nt1 = tiles_per_slot(H, I, 1);
+    return q;
+}
 
-    // Prologue.  One round of asynchronous copies brings into shared memory
-    // either the plan the routing kernel wrote (the slot rows and this CTA's
-    // tile runs) or the active list and the expert offsets to build it from,
-    // and the sorted slot ids and (T <= kTokPerPass) the bf16 rows of x.  The
-    // scratch copies sit in the ring, which no TMA copy touches before the
-    // prologue's last barrier.
+// Host mirror of carve_stream_smem: bytes past the ring.
+__host__ __forceinline__ size_t stream_smem_fixed(int H, int I, int T, int k, int max_slots) {
+    const size_t n_srt = static_cast<size_t>(T) * k;
+    return static_cast<size_t>(xall_bytes(H, T)) + kNB * static_cast<size_t>(bbuf_bytes(H, I, T)) +
+           kGroups * kNR * static_cast<size_t>(kRedBytes) +
+           (2 * kND + 2 * kGroups * kNR + 2 * kNB) * sizeof(uint64_t) + 12 * sizeof(int) +
+           (MOE_MAX_TIERS + 1) * sizeof(TierPtrs) + 6 * sizeof(Geo) + 16 + plan_tab_bytes(max_slots) +
+           (n_srt <= static_cast<size_t>(kMaxSmemEntries) ? (n_srt * sizeof(int) + 15) / 16 * 16 : 0);
+}
+
+// The pipeline's barriers, the abort flag and the tile geometry (thread 0
+// and threads < 6; the caller synchronises).
+__device__ __forceinline__ void init_stream_smem(StreamSmem &S, int H, int I) {
     if (threadIdx.x == 0) {
-#pragma unroll
-        for (int t = 0; t < MOE_MAX_TIERS; ++t) {
-            if (t < p.w.n_tiers) {
-                S.tp[t].gq = p.w.tiers[t].gu_qs;
-                S.tp[t].gs = reinterpret_cast<const uint8_t *>(p.w.tiers[t].gu_scale);
-                S.tp[t].dq = p.w.tiers[t].dn_qs;
-                S.tp[t].ds = reinterpret_cast<const uint8_t *>(p.w.tiers[t].dn_scale);
-            }
-        }
-        const int t = p.w.n_tiers;
-        S.tp[t].gq = p.w.shared.gu_qs;
-        S.tp[t].gs = reinterpret_cast<const uint8_t *>(p.w.shared.gu_scale);
-        S.tp[t].dq = p.w.shared.dn_qs;
-        S.tp[t].ds = reinterpret_cast<const uint8_t *>(p.w.shared.dn_scale);
         for (int i = 0; i < kND; ++i) {
             mbar_init(&S.full[i], 1);  // the producer's expect_tx arrival
             mbar_init(&S.empty[i], kWarps);
@@ -1055,17 +1070,77 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
         }
         *S.abort = 0;
         mbar_fence_init();
+    }
+    if (threadIdx.x < 6) {
+        const int phase = threadIdx.x / 3, bi = threadIdx.x % 3;
+        const int bits = bi == 0 ? 8 : (bi == 1 ? 4 : 3);
+        S.geo[threadIdx.x] = phase == 0 ? geo_gu(H, bits) : geo(I, bits);
+    }
+}
+
+// Table pointers of the layer's shelves and shared expert (thread 0).
+__device__ __forceinline__ void fill_tier_ptrs(const moe_layer_weights &w, StreamSmem &S) {
+    if (threadIdx.x != 0) return;
+#pragma unroll
+    for (int t = 0; t < MOE_MAX_TIERS; ++t) {
+        if (t < w.n_tiers) {
+            S.tp[t].gq = w.tiers[t].gu_qs;
+            S.tp[t].gs = reinterpret_cast<const uint8_t *>(w.tiers[t].gu_scale);
+            S.tp[t].dq = w.tiers[t].dn_qs;
+            S.tp[t].ds = reinterpret_cast<const uint8_t *>(w.tiers[t].dn_scale);
+        }
+    }
+    const int t = w.n_tiers;
+    S.tp[t].gq = w.shared.gu_qs;
+    S.tp[t].gs = reinterpret_cast<const uint8_t *>(w.shared.gu_scale);
+    S.tp[t].dq = w.shared.dn_qs;
+    S.tp[t].ds = reinterpret_cast<const uint8_t *>(w.shared.dn_scale);
+}
+
+// The slot table and this CTA's tile runs from the active list and the expert
+// offsets in shared memory (every thread; ends before a barrier).
+__device__ __forceinline__ void plan_in_cta(const FfnParams &p, StreamSmem &S, const int *act_s, const int *off_s) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0) {
+        const int ns = plan_compact(p.pi, act_s, off_s, S.pt);
+        if (lane == 0) S.range[4] = ns;
+    }
+    __syncthreads();
+    if (warp < 2) {
+        const int ns = S.range[4];
+        const long long total = plan_costs(p.pi, ns, warp, S.pt);
+        if (lane == 0) {
+            const int2 r = plan_cta_range(S.pt, ns, warp == 0 ? S.nt0 : S.nt1, warp, total, blockIdx.x, gridDim.x);
+            S.range[2 * warp] = r.x;
+            S.range[2 * warp + 1] = r.y;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kBlockThreads, 1)
+ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ StreamMaps M, int ring_bytes) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int max_slots = p.max_active + 1;
+    StreamSmem S;
+    carve_stream_smem(smem, ring_bytes, p.w.H, p.w.I, p.T, p.k, max_slots, S);
+    const int n_srt = p.T * p.k;
+
+    // Prologue.  One round of asynchronous copies brings into shared memory
+    // either the plan the routing kernel wrote (the slot rows and this CTA's
+    // tile runs) or the active list and the expert offsets to build it from,
+    // and the sorted slot ids and (T <= kTokPerPass) the bf16 rows of x.  The
+    // scratch copies sit in the ring, which no TMA copy touches before the
+    // prologue's last barrier.
+    init_stream_smem(S, p.w.H, p.w.I);
+    fill_tier_ptrs(p.w, S);
+    if (threadIdx.x == 0) {
         // the tensor maps of the shelves in use
         for (int t = 0; t <= p.w.n_tiers; ++t) {
             if (t == p.w.n_tiers && !p.has_shared) break;
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&M.gq[t])) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&M.dq[t])) : "memory");
         }
-    }
-    if (threadIdx.x < 6) {
-        const int phase = threadIdx.x / 3, bi = threadIdx.x % 3;
-        const int bits = bi == 0 ? 8 : (bi == 1 ? 4 : 3);
-        S.geo[threadIdx.x] = phase == 0 ? geo_gu(p.w.H, bits) : geo(p.w.I, bits);
     }
     // everything above reads only the parameters; what follows reads the
     // routing kernel's outputs
@@ -1096,21 +1171,7 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     if (!routed) {  // the grid barrier gave up: stream nothing
         if (threadIdx.x < 5) S.range[threadIdx.x] = 0;
     } else {
-        if (warp == 0) {
-            const int ns = plan_compact(p.pi, act_s, off_s, S.pt);
-            if (lane == 0) S.range[4] = ns;
-        }
-        __syncthreads();
-        if (warp < 2) {
-            const int ns = S.range[4];
-            const long long total = plan_costs(p.pi, ns, warp, S.pt);
-            if (lane == 0) {
-                const int2 r = plan_cta_range(S.pt, ns, warp == 0 ? S.nt0 : S.nt1, warp, total, blockIdx.x,
-                                              gridDim.x);
-                S.range[2 * warp] = r.x;
-                S.range[2 * warp + 1] = r.y;
-            }
-        }
+        plan_in_cta(p, S, act_s, off_s);
     }
     // the ring's scratch is overwritten by TMA copies from here on: order
     // this thread's generic accesses before them
@@ -1118,12 +1179,20 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     __syncthreads();
 
     if (warp == kWarpProducer) {
-        run_producer(p, M, S);
+        ProducerState ps0 = {};
+        run_producer(p, M, S, ps0, true);
         return;
     }
-    if (warp < kComputeWarps) run_compute(p, S, warp);
-    else if (warp == kWarpLoader) run_loader(p, S);
-    else if (warp >= kWarpEpilogue0) run_epilogue(p, S, warp - kWarpEpilogue0);
+    if (warp < kComputeWarps) {
+        ComputeState cs = {0, 0, 0, -1};
+        run_compute(p, S, warp, cs);
+    } else if (warp == kWarpLoader) {
+        LoaderState ls = {-1};
+        run_loader(p, S, ls);
+    } else if (warp >= kWarpEpilogue0) {
+        EpilogueState es = {0, 0};
+        run_epilogue(p, S, warp - kWarpEpilogue0, es);
+    }
 }
 
 }  // namespace moe
@@ -1133,13 +1202,7 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
 // tables.  Returns the byte count and the ring size in *ring_bytes (0 when
 // the ring cannot hold the largest tile and the prologue's scratch).
 size_t moe_ffn_stream_smem(int H, int I, int T, int k, int E, int max_slots, bool fused, int *ring_bytes) {
-    const size_t n_srt = static_cast<size_t>(T) * k;
-    const size_t fixed = static_cast<size_t>(moe::xall_bytes(H, T)) + moe::kNB * static_cast<size_t>(moe::bbuf_bytes(H, I, T)) +
-                         moe::kGroups * moe::kNR * static_cast<size_t>(moe::kRedBytes) +
-                         (2 * moe::kND + 2 * moe::kGroups * moe::kNR + 2 * moe::kNB) * sizeof(uint64_t) +
-                         12 * sizeof(int) +
-                         (MOE_MAX_TIERS + 1) * sizeof(moe::TierPtrs) + 6 * sizeof(moe::Geo) + 16 +
-                         moe::plan_tab_bytes(max_slots) + (n_srt <= moe::kMaxSmemEntries ? n_srt * sizeof(int) : 0);
+    const size_t fixed = moe::stream_smem_fixed(H, I, T, k, max_slots);
     const size_t budget = 227 * 1024;
     size_t ring = fixed < budget ? ((budget - fixed) & ~static_cast<size_t>(moe::kTileAlign - 1)) : 0;
     const size_t scratch = moe::prologue_scratch(H, T, k, E, max_slots, fused).end;
@@ -1282,6 +1345,7 @@ cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
     cudaGetDevice(&dev);
     int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (p.route.on && (p.E + sms - 1) / sms > moe::kMaxExpertShare) return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(moe::kBlockThreads);
@@ -1301,6 +1365,380 @@ cudaError_t moe_launch_ffn_stream(const moe::FfnParams &p, cudaStream_t s) {
         cfg.attrs = at.a + 1;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, moe::ffn_stream_kernel, p, M, ring);
+    }
+    return e;
+}
+
+// ---------------------------------------------------------------------------
+// A stack of decode layers in one persistent launch ([P5] "What the model
+// actually is": 48 layers, a residual design; [P1] "step 3": the per-token
+// profile is dominated by launches and syncs, not by expert bytes).
+//
+// Every CTA loops over the layers.  Per layer: the RMS norm of the residual
+// stream (each CTA recomputes it, in one fixed order), the router logits of
+// its share of the experts, a grid barrier, then every CTA ranks and groups
+// the tokens and plans its tiles; the warp-role pipeline streams the layer's
+// experts; a grid barrier; each CTA adds its slice of the combined output
+// into the next residual buffer; a grid barrier.  The pipeline's barriers,
+// ring offsets and operand buffers carry over from layer to layer, and the
+// code stays resident in the instruction caches.
+// ---------------------------------------------------------------------------
+namespace moe {
+
+struct __align__(64) StackLayer {
+    StreamMaps maps;
+    moe_layer_weights w;
+    const uint16_t *wr;
+    const float *bias;
+};
+
+struct StackParams {
+    const StackLayer *layers;
+    int n_layers, T, k, H, I, E;
+    const uint16_t *x_in;  // bf16 [T][H] residual stream entering the first layer
+    uint16_t *x_out;       // bf16 [T][H] residual stream leaving the last layer
+    uint16_t *x_out_norm;  // its RMS-normalised copy, or null
+    uint16_t *x_layers;    // [n_layers + 1][T][H] the stream at every layer boundary, or null
+    uint16_t *xbuf;        // [2][T][H] residual stream between layers
+    float *logits, *h, *y_slots, *y_shared;
+    int *ctr;              // [min(T*k, E) + 1] per-slot gate_up counts (zero on entry)
+    int *gbar;             // [2] grid barrier words (zero on entry)
+    int32_t *status;
+    long long wait_limit;
+    int ring_bytes;
+};
+
+// Bytes past the shared stream layout: this layer's parameters, its top-k
+// weights and the norm's scratch.
+__host__ __device__ __forceinline__ size_t stack_smem_extra(int T, int k) {
+    return (sizeof(FfnParams) + 15) / 16 * 16 + (static_cast<size_t>(T) * k * sizeof(float) + 15) / 16 * 16 +
+           (static_cast<size_t>(T) + 32) * sizeof(float);
+}
+
+// n = bf16(x / sqrt(mean(x^2) + eps)) of every row of the bf16 tile x_s
+// [T][H], in place (whole CTA; red: 32 + T floats of scratch).
+__device__ __forceinline__ void cta_rms_norm_rows(uint16_t *x_s, int T, int H, float *red) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    float *rinv = red + 32;
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *xr = x_s + static_cast<size_t>(t) * H;
+        float ss = 0.f;
+        for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(xr + 4 * c);
+            const float f0 = bf16lo(v.x), f1 = bf16hi(v.x), f2 = bf16lo(v.y), f3 = bf16hi(v.y);
+            ss = fmaf(f0, f0, fmaf(f1, f1, fmaf(f2, f2, fmaf(f3, f3, ss))));
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        if (warp == 0) {
+            float tot = lane < nwarps ? red[lane] : 0.f;
+            tot = warp_sum(tot);
+            if (lane == 0) rinv[t] = 1.0f / sqrtf(tot / static_cast<float>(H) + MOE_NORM_EPS);
+        }
+        __syncthreads();
+    }
+    for (int i = threadIdx.x; i < T * H / 2; i += blockDim.x) {
+        const int t = (2 * i) / H;
+        uint32_t v = reinterpret_cast<uint32_t *>(x_s)[i];
+        const float r = rinv[t];
+        v = static_cast<uint32_t>(f32_to_bf16_rne(bf16lo(v) * r)) |
+            (static_cast<uint32_t>(f32_to_bf16_rne(bf16hi(v) * r)) << 16);
+        reinterpret_cast<uint32_t *>(x_s)[i] = v;
+    }
+    __syncthreads();
+}
+
+// thread 0 of every CTA at a grid barrier; the result in every thread
+__device__ __forceinline__ bool stack_barrier(const StackParams &P, StreamSmem &S) {
+    if (threadIdx.x == 0) {
+        const bool ok = !*static_cast<volatile int *>(S.abort) && grid_barrier(P.gbar, S.abort, P.wait_limit);
+        if (!ok) {
+            status_or(P.status, MOE_STATUS_TIMEOUT);
+            *static_cast<volatile int *>(S.abort) = 1;
+        }
+        S.range[6] = ok;
+    }
+    __syncthreads();
+    return S.range[6] != 0;
+}
+
+__global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_constant__ StackParams P) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const int T = P.T, k = P.k, H = P.H, E = P.E, S_ = T * k;
+    const int max_active = min(S_, E), max_slots = max_active + 1;
+    StreamSmem S;
+    uint8_t *q = carve_stream_smem(smem, P.ring_bytes, H, P.I, T, k, max_slots, S);
+    FfnParams &p = *reinterpret_cast<FfnParams *>(q);
+    q += (sizeof(FfnParams) + 15) / 16 * 16;
+    float *wkeep = reinterpret_cast<float *>(q);
+    q += (static_cast<size_t>(S_) * sizeof(float) + 15) / 16 * 16;
+    float *red = reinterpret_cast<float *>(q);
+    init_stream_smem(S, H, P.I);
+    ProducerState prs = {};
+    ComputeState cst = {0, 0, 0, -1};
+    LoaderState lds = {-1};
+    EpilogueState eps = {0, 0};
+    const PrologueScratch ps = prologue_scratch(H, T, k, E, max_slots, true);
+    int *act_s = reinterpret_cast<int *>(S.ring + ps.lists);
+    int *off_s = act_s + max_slots;
+    uint16_t *x_s = reinterpret_cast<uint16_t *>(S.ring + ps.x);
+    pdl_wait();
+    pdl_trigger();
+    if (P.x_layers && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < T * H / 8; i += blockDim.x)
+            reinterpret_cast<uint4 *>(P.x_layers)[i] = reinterpret_cast<const uint4 *>(P.x_in)[i];
+    if (threadIdx.x == 0) {
+        p.E = E;
+        p.T = T;
+        p.k = k;
+        p.max_active = max_active;
+        p.x = nullptr;
+        p.offsets = p.sorted = p.active = nullptr;
+        p.h = P.h;
+        p.ctr = P.ctr;
+        p.max_count = 0x7fffffff;
+        p.y_slots = P.y_slots;
+        p.y_shared = P.y_shared;
+        p.status = P.status;
+        PlanIn &pi = p.pi;
+        pi.E = E;
+        pi.T = T;
+        pi.k = k;
+        pi.H = H;
+        pi.I = P.I;
+        pi.max_count = 0x7fffffff;
+        pi.max_active = max_active;
+        p.route.on = 1;
+        p.route.logits = P.logits;
+        p.route.topk_idx = nullptr;
+        p.route.topk_w = nullptr;
+        p.route.offsets = p.route.sorted = p.route.slot_pos = p.route.active = nullptr;
+        p.route.gbar = P.gbar;
+        p.wait_limit = P.wait_limit;
+        p.skip_publish = -1;
+    }
+    bool alive = true;
+    for (int l = 0; l < P.n_layers && alive; ++l) {
+        const StackLayer &Ld = P.layers[l];
+        const uint16_t *xl = l == 0 ? P.x_in : P.xbuf + static_cast<size_t>((l - 1) & 1) * T * H;
+        uint16_t *xn = l + 1 == P.n_layers ? P.x_out : P.xbuf + static_cast<size_t>(l & 1) * T * H;
+        // this layer's weights descriptor into shared memory (every thread a word)
+        {
+            const int *src = reinterpret_cast<const int *>(&Ld.w);
+            int *dst = reinterpret_cast<int *>(&p.w);
+            for (int w = threadIdx.x; w < static_cast<int>(sizeof(moe_layer_weights) / sizeof(int)); w += blockDim.x)
+                dst[w] = __ldg(src + w);
+            if (threadIdx.x == 0) {
+                p.route.wr = Ld.wr;
+                p.route.bias = Ld.bias;
+                for (int t = 0; t <= MOE_MAX_TIERS; ++t) {
+                    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&Ld.maps.gq[t])) : "memory");
+                    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&Ld.maps.dq[t])) : "memory");
+                }
+            }
+        }
+        // the residual stream entering the layer
+        for (int c = threadIdx.x; c < T * H / 8; c += blockDim.x)
+            cp_async_16b(x_s + 8 * c, xl + 8 * static_cast<size_t>(c));
+        cp_async_wait_all();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            p.has_shared = p.w.shared.n_experts == 1;
+            PlanIn &pi = p.pi;
+            pi.n_tiers = p.w.n_tiers;
+            pi.has_shared = p.has_shared;
+            pi.shared_bits = p.w.shared.bits;
+            for (int t = 0; t < MOE_MAX_TIERS; ++t) {
+                pi.first[t] = t < p.w.n_tiers ? p.w.tiers[t].first_expert : 0;
+                pi.n[t] = t < p.w.n_tiers ? p.w.tiers[t].n_experts : 0;
+                pi.bits[t] = t < p.w.n_tiers ? p.w.tiers[t].bits : 8;
+            }
+        }
+        fill_tier_ptrs(p.w, S);
+        // normalised in place (its barriers also publish the parameters above)
+        cta_rms_norm_rows(x_s, T, H, red);
+        {
+            const bool xbad = build_xall(p, reinterpret_cast<const uint8_t *>(x_s), S.xall);
+            if (__any_sync(0xffffffffu, xbad) && (threadIdx.x & 31) == 0) status_or(P.status, MOE_STATUS_FP16_RANGE);
+        }
+        if (!route_in_cta(p, S, x_s, act_s, off_s, ps)) {
+            alive = false;
+            break;
+        }
+        for (int i = threadIdx.x; i < S_; i += blockDim.x) wkeep[i] = reinterpret_cast<const float *>(S.ring + ps.w)[i];
+        plan_in_cta(p, S, act_s, off_s);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        const bool last = l + 1 == P.n_layers;
+        if (!last && threadIdx.x == 32 * kWarpLoader) {
+            // the next layer's router rows of this CTA and a slice of its shared
+            // expert (needed whatever the routing) into L2 while this layer streams
+            const StackLayer &Nx = P.layers[l + 1];
+            const int e0 = static_cast<int>(static_cast<long long>(E) * blockIdx.x / gridDim.x);
+            const int e1 = static_cast<int>(static_cast<long long>(E) * (blockIdx.x + 1) / gridDim.x);
+            prefetch_l2(Nx.wr + static_cast<size_t>(e0) * H, static_cast<uint32_t>((e1 - e0) * H * 2));
+            if (Nx.w.shared.n_experts == 1) {
+                const moe_tier &sh = Nx.w.shared;
+                const size_t gq = static_cast<size_t>(2) * P.I * H * sh.bits / 8, gs = static_cast<size_t>(2) * P.I * (H / 32) * 2;
+                const size_t dq = static_cast<size_t>(H) * P.I * sh.bits / 8, ds = static_cast<size_t>(H) * (P.I / 32) * 2;
+                const void *base[4] = {sh.gu_qs, sh.gu_scale, sh.dn_qs, sh.dn_scale};
+                const size_t len[4] = {gq, gs, dq, ds};
+                for (int a = 0; a < 4; ++a) {
+                    const size_t c0 = (len[a] * blockIdx.x / gridDim.x) & ~static_cast<size_t>(15);
+                    const size_t c1 = blockIdx.x + 1 == gridDim.x ? len[a] : ((len[a] * (blockIdx.x + 1) / gridDim.x) & ~static_cast<size_t>(15));
+                    prefetch_l2(static_cast<const uint8_t *>(base[a]) + c0, static_cast<uint32_t>(c1 - c0));
+                }
+            }
+        }
+        if (warp == kWarpProducer) run_producer(p, Ld.maps, S, prs, last);
+        else if (warp < kComputeWarps) run_compute(p, S, warp, cst);
+        else if (warp == kWarpLoader) run_loader(p, S, lds);
+        else if (warp >= kWarpEpilogue0) run_epilogue(p, S, warp - kWarpEpilogue0, eps);
+        __syncthreads();
+        if (!stack_barrier(P, S)) {
+            alive = false;
+            break;
+        }
+        // this CTA's slice of out = bf16(sum_j w_j y_j + y_shared), x' = bf16(x + out)
+        const int nch = T * H / 4;
+        const int c0 = static_cast<int>(static_cast<long long>(nch) * blockIdx.x / gridDim.x);
+        const int c1 = static_cast<int>(static_cast<long long>(nch) * (blockIdx.x + 1) / gridDim.x);
+        for (int c = c0 + static_cast<int>(threadIdx.x); c < c1; c += blockDim.x) {
+            const int t = c / (H / 4), col = c - t * (H / 4);
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < k; ++j) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(P.y_slots + (static_cast<size_t>(t) * k + j) * H) + col);
+                const float wj = wkeep[t * k + j];
+                a.x = fmaf(wj, v.x, a.x);
+                a.y = fmaf(wj, v.y, a.y);
+                a.z = fmaf(wj, v.z, a.z);
+                a.w = fmaf(wj, v.w, a.w);
+            }
+            if (p.has_shared) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(P.y_shared + static_cast<size_t>(t) * H) + col);
+                a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+            }
+            const uint2 r = __ldcg(reinterpret_cast<const uint2 *>(xl + static_cast<size_t>(t) * H) + col);
+            const uint16_t n0 = f32_to_bf16_rne(bf16lo(r.x) + bf16_to_f32(f32_to_bf16_rne(a.x)));
+            const uint16_t n1 = f32_to_bf16_rne(bf16hi(r.x) + bf16_to_f32(f32_to_bf16_rne(a.y)));
+            const uint16_t n2 = f32_to_bf16_rne(bf16lo(r.y) + bf16_to_f32(f32_to_bf16_rne(a.z)));
+            const uint16_t n3 = f32_to_bf16_rne(bf16hi(r.y) + bf16_to_f32(f32_to_bf16_rne(a.w)));
+            const uint2 o = make_uint2(static_cast<uint32_t>(n0) | (static_cast<uint32_t>(n1) << 16),
+                                       static_cast<uint32_t>(n2) | (static_cast<uint32_t>(n3) << 16));
+            reinterpret_cast<uint2 *>(xn + static_cast<size_t>(t) * H)[col] = o;
+            if (P.x_layers)
+                reinterpret_cast<uint2 *>(P.x_layers + (static_cast<size_t>(l + 1) * T + t) * H)[col] = o;
+        }
+        // the per-slot counts start from zero in the next layer (nobody reads them now)
+        if (blockIdx.x == 0)
+            for (int i = threadIdx.x; i < max_slots; i += blockDim.x) P.ctr[i] = 0;
+        if (!stack_barrier(P, S)) {
+            alive = false;
+            break;
+        }
+    }
+    // after a failed barrier: wait for any copy this CTA still has in flight
+    if (!alive && warp == kWarpProducer && (threadIdx.x & 31) == 0)
+        for (int j = max(prs.rel, prs.i - kND); j < prs.i; ++j)
+            if (!mbar_wait_limit(&S.full[j % kND], (j / kND) & 1, P.wait_limit)) status_or(P.status, MOE_STATUS_TIMEOUT);
+    if (alive && P.x_out_norm && blockIdx.x == 0) {
+        for (int c = threadIdx.x; c < T * H / 8; c += blockDim.x)
+            reinterpret_cast<uint4 *>(x_s)[c] = __ldcg(reinterpret_cast<const uint4 *>(P.x_out) + c);
+        __syncthreads();
+        cta_rms_norm_rows(x_s, T, H, red);
+        for (int c = threadIdx.x; c < T * H / 8; c += blockDim.x)
+            reinterpret_cast<uint4 *>(P.x_out_norm)[c] = reinterpret_cast<const uint4 *>(x_s)[c];
+    }
+}
+
+}  // namespace moe
+
+size_t moe_stack_layer_bytes() { return sizeof(moe::StackLayer); }
+
+// One layer of a stack descriptor, encoded on the host into `dst`
+// (sizeof(StackLayer) bytes): the tensor maps of its shelves, the weights
+// descriptor and the router.
+cudaError_t moe_stack_encode_layer(const moe_layer_weights *w, const uint16_t *wr, const float *bias, void *dst) {
+    moe::StackLayer L;
+    std::memset(&L, 0, sizeof(L));
+    for (int t = 0; t < w->n_tiers; ++t)
+        if (!shelf_maps(L.maps, t, w->tiers[t], w->H, w->I)) return cudaErrorInvalidValue;
+    if (w->shared.n_experts == 1 && !shelf_maps(L.maps, w->n_tiers, w->shared, w->H, w->I)) return cudaErrorInvalidValue;
+    L.w = *w;
+    L.wr = wr;
+    L.bias = bias;
+    std::memcpy(dst, &L, sizeof(L));
+    return cudaSuccess;
+}
+
+// Shared memory of the stack kernel; *ring_bytes = 0 when the ring cannot
+// hold the largest tile and the per-layer scratch.
+size_t moe_stack_smem(int H, int I, int T, int k, int E, int *ring_bytes) {
+    const int max_slots = (T * k < E ? T * k : E) + 1;
+    const size_t fixed = moe::stream_smem_fixed(H, I, T, k, max_slots) + moe::stack_smem_extra(T, k);
+    const size_t budget = 227 * 1024;
+    size_t ring = fixed < budget ? ((budget - fixed) & ~static_cast<size_t>(moe::kTileAlign - 1)) : 0;
+    const size_t scratch = moe::prologue_scratch(H, T, k, E, max_slots, true).end;
+    if (ring < static_cast<size_t>(moe::kMaxTileBytes) || ring < scratch) ring = 0;
+    *ring_bytes = static_cast<int>(ring);
+    return ring + fixed;
+}
+
+cudaError_t moe_configure_stack() {
+    return cudaFuncSetAttribute(moe::stack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+}
+
+// ctr and gbar must be zero on entry; the caller clears them.
+cudaError_t moe_launch_stack(const void *layers, int n_layers, int T, int k, int H, int I, int E, const uint16_t *x_in,
+                             uint16_t *x_out, uint16_t *x_out_norm, uint16_t *x_layers, uint16_t *xbuf, float *logits,
+                             float *h, float *y_slots, float *y_shared, int *ctr, int *gbar, int32_t *status,
+                             long long wait_limit, cudaStream_t s) {
+    moe::StackParams P;
+    std::memset(&P, 0, sizeof(P));
+    P.layers = static_cast<const moe::StackLayer *>(layers);
+    P.n_layers = n_layers;
+    P.T = T;
+    P.k = k;
+    P.H = H;
+    P.I = I;
+    P.E = E;
+    P.x_in = x_in;
+    P.x_out = x_out;
+    P.x_out_norm = x_out_norm;
+    P.x_layers = x_layers;
+    P.xbuf = xbuf;
+    P.logits = logits;
+    P.h = h;
+    P.y_slots = y_slots;
+    P.y_shared = y_shared;
+    P.ctr = ctr;
+    P.gbar = gbar;
+    P.status = status;
+    P.wait_limit = wait_limit;
+    int ring = 0;
+    const size_t smem = moe_stack_smem(H, I, T, k, E, &ring);
+    if (ring == 0) return cudaErrorInvalidConfiguration;
+    P.ring_bytes = ring;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if ((E + sms - 1) / sms > moe::kMaxExpertShare) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(moe::kBlockThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    moe::PdlAttrs at(true);
+    cfg.attrs = at.a;
+    cfg.numAttrs = at.n;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, moe::stack_kernel, P);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        cfg.attrs = at.a + 1;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, moe::stack_kernel, P);
     }
     return e;
 }

@@ -181,24 +181,18 @@ __device__ __forceinline__ int plan_first_tile(const PlanTabs &t, int ns, int nt
     if (lo == ns) return ns * nt;
     const long long tc = t.tc(phase)[lo];
     const long long off = pre[lo] - nt * tc;  // start cost of the slot's first tile
-    // ceil((x - off) / tc) clamped to [0, nt]: a double quotient corrected to
-    // the exact integer (the quotient is at most nt)
+    // ceil((x - off) / tc) clamped to [0, nt], as a double quotient: every CTA
+    // evaluates the same monotone function of x, so neighbouring CTAs agree on
+    // the tile where one run ends and the next begins
     if (x <= off) return lo * nt;
-    long long b = static_cast<long long>(static_cast<double>(x - off) / static_cast<double>(tc));
-    while (b * tc < x - off) ++b;
-    while (b > 0 && (b - 1) * tc >= x - off) --b;
+    long long b = static_cast<long long>(ceil(static_cast<double>(x - off) / static_cast<double>(tc)));
     if (b > nt) b = nt;
     return lo * nt + static_cast<int>(b);
 }
 
-// floor(a * c / g) for 0 <= a < 2^50, 0 <= c <= g: a double quotient corrected
-// to the exact integer (a 64-bit integer division is a long routine).
+// floor(a * c / g) as a double quotient (deterministic and monotone in c).
 __device__ __forceinline__ long long share_floor(long long a, int c, int g) {
-    const long long num = a * c;
-    long long q = static_cast<long long>(static_cast<double>(num) / static_cast<double>(g));
-    while (q * g > num) --q;
-    while ((q + 1) * g <= num) ++q;
-    return q;
+    return static_cast<long long>(static_cast<double>(a) * c / static_cast<double>(g));
 }
 
 // CTA c's run of phase-`phase` tiles: [gs, ge) in global tile indices.

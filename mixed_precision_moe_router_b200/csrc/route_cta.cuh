@@ -55,109 +55,153 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
 }
 
 // ---------------------------------------------------------------------------
-// Top-k of T logit rows by a whole CTA.  Each row is cut into quarters of
-// 128 logits (4 per lane); a warp finds a quarter's top-k by k rounds of a
-// warp arg-max, then one warp per row merges the quarters' candidates the
-// same way.  Ties go to the lower id at every stage, so the result is the
-// top-k of the whole row in (logit desc, id asc) order.
+// Top-k of one logit row by one warp with warp-wide reductions: lane l holds
+// logits l, l+32, ... (16 for E <= 512, 32 for E <= 1024); each of the k
+// rounds takes every lane's best untaken value, the warp maximum of an
+// order-preserving 32-bit key of the logit (redux.sync) and, among the lanes
+// holding that maximum, the lowest id.  Lane r < k returns choice r and its
+// renormalised softmax weight, with the same arithmetic as topk_row.
 // ---------------------------------------------------------------------------
-constexpr int kTopkQuarter = 128;
-
-// Shared memory for cta_topk: candidates [T][quarters][k] as (value, id).
-__host__ __device__ __forceinline__ size_t cta_topk_smem(int T, int E, int k) {
-    const int nq = (E + kTopkQuarter - 1) / kTopkQuarter;
-    return static_cast<size_t>(T) * nq * k * (sizeof(float) + sizeof(int));
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// k rounds of a warp arg-max over NJ values per lane (v, id), skipping the
-// ones already taken; lane r < k returns choice r.
 template <int NJ>
-__device__ __forceinline__ void warp_topk(const float (&v)[NJ], const int (&id)[NJ], int k, float &out_v,
-                                          int &out_i) {
+__device__ __forceinline__ void warp_topk_redux(const float *row, int E, int k, int &out_i, float &out_w) {
     const int lane = threadIdx.x & 31;
+    uint32_t key[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const int e = lane + 32 * j;
+        key[j] = e < E ? order_key(__ldcg(row + e) + 0.0f) : 0u;  // -0 keys as +0
+    }
     uint32_t taken = 0;
-    out_v = -FLT_MAX;
-    out_i = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j)
+        if (lane + 32 * j >= E) taken |= 1u << j;
+    float my_v = 0.f;
+    int my_i = 0;
     for (int r = 0; r < k; ++r) {
-        float bv = -FLT_MAX;
-        int bi = 0x7fffffff, bj = -1;
+        // this lane's best untaken entry: the largest key, then the lowest id
+        // (ids grow with j, so the first j with the largest key)
+        uint32_t bk = 0;
+        int bj = -1;
 #pragma unroll
         for (int j = 0; j < NJ; ++j)
-            if (!((taken >> j) & 1u) && id[j] != 0x7fffffff && ranks_before(v[j], id[j], bv, bi)) {
-                bv = v[j];
-                bi = id[j];
+            if (!((taken >> j) & 1u) && (bj < 0 || key[j] > bk)) {
+                bk = key[j];
                 bj = j;
             }
-        float wv = bv;
-        int wi = bi;
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t id = (bj >= 0 && bk == wk) ? static_cast<uint32_t>(lane + 32 * bj) : 0xffffffffu;
+        const uint32_t wi = __reduce_min_sync(0xffffffffu, id);
+        if (static_cast<int>(wi & 31u) == lane) taken |= 1u << (wi >> 5);
+        if (lane == r) {
+            my_i = static_cast<int>(wi);
+            my_v = __ldcg(row + wi);
+        }
+    }
+    const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
+    const float z = lane < k ? expf(my_v - l0) : 0.f;
+    const float sum = warp_sum(z);
+    out_i = my_i;
+    out_w = z / sum;
+}
+
+// Top-k of T rows by a whole CTA: one warp per row (E <= 1024, k <= 32).
+// idx_s / w_s [T][k]; ends with a barrier.
+__device__ __forceinline__ void cta_topk_rows(const float *logits, int T, int E, int k, int *idx_s, float *w_s) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    for (int t = warp; t < T; t += nwarps) {
+        int i;
+        float w;
+        if (E <= 512) warp_topk_redux<16>(logits + static_cast<size_t>(t) * E, E, k, i, w);
+        else warp_topk_redux<32>(logits + static_cast<size_t>(t) * E, E, k, i, w);
+        if (lane < k) {
+            idx_s[t * k + lane] = i;
+            w_s[t * k + lane] = w;
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// Router logits of experts [e0, e1) for T <= NT tokens by a whole CTA: each
+// warp takes (expert, quarter of the row) tasks, so one round of row loads
+// covers the CTA's share; the quarters are added in order afterwards.
+//   x_s bf16 [T][H] in shared memory; part: 4 * (e1 - e0) * NT floats of
+//   shared scratch; logits fp32 [T][E] (global).  Ends with a barrier.
+// ---------------------------------------------------------------------------
+template <int NT>
+__device__ __forceinline__ void cta_logits_nt(const uint16_t *x_s, int T, int H, int E, const uint16_t *wr,
+                                              const float *bias, int e0, int e1, float *part, float *logits) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int vec = H / 8, qv = vec / 4;  // 16-byte chunks per row and per quarter
+    const int ntask = 4 * (e1 - e0);
+    for (int task = warp; task < ntask; task += nwarps) {
+        const int el = task >> 2, q = task & 3;
+        const uint16_t *row = wr + static_cast<size_t>(e0 + el) * H;
+        float acc[NT];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, wi, o);
-            if (ranks_before(ov, oi, wv, wi)) {
-                wv = ov;
-                wi = oi;
+        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+        for (int c0 = q * qv; c0 < (q + 1) * qv; c0 += 32 * 4) {
+            uint4 wv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = c0 + lane + 32 * u;
+                wv[u] = c < (q + 1) * qv ? ld_stream_v4(row + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = c0 + lane + 32 * u;
+                if (c >= (q + 1) * qv) continue;
+                const float w[8] = {bf16lo(wv[u].x), bf16hi(wv[u].x), bf16lo(wv[u].y), bf16hi(wv[u].y),
+                                    bf16lo(wv[u].z), bf16hi(wv[u].z), bf16lo(wv[u].w), bf16hi(wv[u].w)};
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (t < T) {
+                        const uint4 xv = reinterpret_cast<const uint4 *>(x_s)[t * vec + c];
+                        float a = acc[t];
+                        a = fmaf(w[0], bf16lo(xv.x), a);
+                        a = fmaf(w[1], bf16hi(xv.x), a);
+                        a = fmaf(w[2], bf16lo(xv.y), a);
+                        a = fmaf(w[3], bf16hi(xv.y), a);
+                        a = fmaf(w[4], bf16lo(xv.z), a);
+                        a = fmaf(w[5], bf16hi(xv.z), a);
+                        a = fmaf(w[6], bf16lo(xv.w), a);
+                        a = fmaf(w[7], bf16hi(xv.w), a);
+                        acc[t] = a;
+                    }
+                }
             }
         }
-        if (bj >= 0 && bi == wi) taken |= 1u << bj;  // ids are unique: only the owner matches
-        if (lane == r) {
-            out_v = wv;
-            out_i = wi;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const float v = warp_sum(acc[t]);
+            if (lane == 0) part[(el * 4 + q) * NT + t] = v;
         }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < (e1 - e0) * T; i += blockDim.x) {
+        const int el = i / T, t = i - el * T;
+        const float *pp = part + el * 4 * NT + t;
+        const float v = ((pp[0] + pp[NT]) + pp[2 * NT]) + pp[3 * NT];
+        logits[static_cast<size_t>(t) * E + e0 + el] = v + (bias ? bias[e0 + el] : 0.f);
     }
 }
 
-// Every thread of the CTA calls it.  logits fp32 [T][E] (read through L2);
-// on return (after a barrier) idx_s / w_s [T][k] hold each row's choices and
-// their renormalised softmax weights, bit-identical to the top-k kernels.
-__device__ __forceinline__ void cta_topk(const float *logits, int T, int E, int k, void *scratch, int *idx_s,
-                                         float *w_s) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    const int nq = (E + kTopkQuarter - 1) / kTopkQuarter;
-    float *cv = static_cast<float *>(scratch);
-    int *ci = reinterpret_cast<int *>(cv + T * nq * k);
-    for (int task = warp; task < T * nq; task += nwarps) {
-        const int t = task / nq, q = task - t * nq;
-        float v[4];
-        int id[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = q * kTopkQuarter + lane + 32 * j;
-            v[j] = e < E ? __ldcg(logits + static_cast<size_t>(t) * E + e) : -FLT_MAX;
-            id[j] = e < E ? e : 0x7fffffff;
-        }
-        float ov;
-        int oi;
-        warp_topk<4>(v, id, k, ov, oi);
-        if (lane < k) {
-            cv[(t * nq + q) * k + lane] = ov;
-            ci[(t * nq + q) * k + lane] = oi;
-        }
+__host__ __device__ __forceinline__ int cta_logits_nt_for(int T) { return T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : (T <= 8 ? 8 : 16))); }
+
+__device__ __forceinline__ void cta_logits(const uint16_t *x_s, int T, int H, int E, const uint16_t *wr,
+                                           const float *bias, int e0, int e1, float *part, float *logits) {
+    switch (cta_logits_nt_for(T)) {
+        case 1: cta_logits_nt<1>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
+        case 2: cta_logits_nt<2>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
+        case 4: cta_logits_nt<4>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
+        case 8: cta_logits_nt<8>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
+        default: cta_logits_nt<16>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
     }
-    __syncthreads();
-    for (int t = warp; t < T; t += nwarps) {
-        // at most 8 quarters (E <= 1024) x k <= 32 candidates: 8 per lane
-        float v[8];
-        int id[8];
-        const int nc = nq * k;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c = lane + 32 * j;
-            v[j] = c < nc ? cv[t * nc + c] : -FLT_MAX;
-            id[j] = c < nc ? ci[t * nc + c] : 0x7fffffff;
-        }
-        float my_v;
-        int my_i;
-        warp_topk<8>(v, id, k, my_v, my_i);
-        const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
-        const float z = lane < k ? expf(my_v - l0) : 0.f;
-        const float sum = warp_sum(z);
-        if (lane < k) {
-            idx_s[t * k + lane] = my_i;
-            w_s[t * k + lane] = z / sum;
-        }
-    }
-    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
