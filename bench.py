@@ -6,8 +6,9 @@ layers of the decode configuration (hidden 2048, 512 experts of intermediate
 3 bits, blocks of 32 with fp16 scales -- plus one 8-bit shared expert, top-10
 Zipf-skewed routing, bf16 residual stream).  The 48 layers have independent
 seeded weights (~49.5 GB resident), so no layer's weights are in L2 when it
-runs.  One step = one token through all 48 layers; the metric counts
-layer-tokens (tokens x layers) per second.
+runs.  One step = one token through all 48 layers, which is one launch of the
+persistent stack kernel (routing, expert FFN and combine of every layer); the
+metric counts layer-tokens (tokens x layers) per second.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -35,13 +36,25 @@ from mixed_precision_moe_router_b200 import inputs  # noqa: E402
 METRIC = "MoE-layer tokens/s; decode expert-weight GB/s vs HBM peak; prefill TFLOP/s"
 UNIT = "layer-tokens/s"
 N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
-KERNELS_PER_LAYER = 3  # fused routing, streaming FFN, combine (+1 rmsnorm per step)
 
-# DRAM bytes (read + write) per launch measured by ncu for the kernel versions
-# in this tree (profiles/ffn_stream_decode_T1.md, profiles/ffn_gemm_prefill_T4096.md);
-# to be re-measured whenever those kernels change.
-DECODE_FFN_TRAFFIC = 28.80e6  # streaming FFN kernel, one decode token: mean DRAM bytes of 2 captured launches
-PREFILL_FFN_TRAFFIC = 1.519e9  # the gate_up and down GEMM launches of one 4096-token call
+# Sources the persistent decode kernel is compiled from.  The DRAM traffic
+# below was captured (ncu dram__bytes_read.sum + dram__bytes_write.sum, cold
+# L2, one launch of a 4-layer stack, one token) for the sources with this
+# digest; when they change, the bench reports traffic as null until the
+# capture is taken again.
+STACK_SOURCES = ("csrc/ffn_stream.cu", "csrc/ffn.cuh", "csrc/plan.cuh", "csrc/route_cta.cuh", "csrc/sync.cuh",
+                 "csrc/common.cuh")
+STACK_TRAFFIC = {"digest": None, "dram_bytes": None, "algorithmic_bytes": None, "layers": 4}
+PREFILL_FFN_TRAFFIC = None  # the GEMM kernels changed since their last capture
+
+
+def source_digest(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "mixed_precision_moe_router_b200", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def peaks():
@@ -251,7 +264,8 @@ def run_prefill(args, rank, world):
     return {
         "metric": METRIC, "value": round(world * T / (pf["layer_ms"] / 1e3), 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pf["layer_ms"], 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 tensor-core MMA on dequantised codes and fp16 activations, fp32 accumulation",
         "data": "synthetic",
         "config": {"workload": f"prefill: one MoE layer (H=2048, I=512, E=512, top-10 + 1 shared, 3 shelves, "
                                f"Zipf routing), {T} tokens per step per GPU", "global_batch": world * T,
@@ -266,6 +280,66 @@ def run_prefill(args, rank, world):
     }
 
 
+class StackStep:
+    """One decode step: T tokens through every layer of the stack in one launch
+    of the persistent kernel (moe_stack_forward)."""
+
+    def __init__(self, layers, routers, x0):
+        from mixed_precision_moe_router_b200 import binding as B
+        self.B, self.k = B, inputs.DECODE.k
+        self.st = B.Stack(layers, routers)
+        self.x_in = x0.clone()
+        self.out = torch.empty_like(x0)
+        self.ws = torch.empty(max(self.st.workspace_size(x0.shape[0], self.k), 1), dtype=torch.uint8,
+                              device=x0.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=x0.device)
+
+    def step(self, x_layers=None):
+        return self.B.stack_forward(self.st, self.x_in, self.k, out=self.out, x_layers=x_layers, workspace=self.ws,
+                                    status=self.status)
+
+    def check(self):
+        st = int(self.status.item())
+        if st:
+            raise RuntimeError(f"stack kernel status {st:#x}")
+
+    def time(self, stream, steps, warmup):
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                self.step()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                self.step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        self.check()
+        return a.elapsed_time(b) / steps
+
+
+def stack_touched_bytes(run, layers, routers, stream):
+    """Per layer: bytes of the expert blocks the step reads (the distinct routed
+    experts of the step's tokens plus the shared expert) and of the router
+    (bf16 [E][H] weights and fp32 bias).  Routing is redone from each layer's
+    input as the kernel saw it (x_layers of one extra step)."""
+    B, cfg = run.B, inputs.DECODE
+    T = run.x_in.shape[0]
+    xl = torch.empty(len(layers) + 1, T, cfg.H, dtype=torch.bfloat16, device=run.x_in.device)
+    with torch.cuda.stream(stream):
+        run.step(x_layers=xl)
+        ex, rt = [], []
+        for l, layer in enumerate(layers):
+            wr, bias = routers[l]
+            idx, _, _ = B.router_topk(B.rmsnorm(xl[l]), wr, bias, cfg.k)
+            touched = set(idx.cpu().numpy().reshape(-1).tolist())
+            ex.append(sum(layer.nbytes_expert(e) for e in touched) + layer.nbytes_expert(cfg.E))
+            rt.append(wr.numel() * 2 + (bias.numel() * 4 if bias is not None else 0))
+    torch.cuda.synchronize()
+    run.check()
+    return ex, rt
+
+
 def run_native(args, rank, world):
     from mixed_precision_moe_router_b200 import binding as B
     device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -273,28 +347,34 @@ def run_native(args, rank, world):
     cfg = inputs.DECODE
     T = 1
     layers, routers = build_stack(cfg, N_LAYERS, device)
-    k = cfg.k
     stream = torch.cuda.Stream(device)
     x0 = inputs.activations(T, cfg.H, seed=inputs.X_SEED + 1000 * rank, device=device)
-    run = StackRunner(layers, routers, x0, stream)
-    graph = run.graph
-    for _ in range(args.warmup):
-        graph.replay()
+    run = StackStep(layers, routers, x0)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            run.step()
     torch.cuda.synchronize()
+    run.check()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the timed region: K launches of the persistent kernel on `stream`, one
+    # event before each launch and one after the last
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with ClockSampler(device.index) as clk:
         time.sleep(0.3)
-        cur = torch.cuda.current_stream(device)
-        ev0.record(cur)
-        for _ in range(args.steps):
-            graph.replay()
-        ev1.record(cur)
+        with torch.cuda.stream(stream):
+            torch.cuda.nvtx.range_push("timed")
+            for i in range(args.steps):
+                evs[i].record(stream)
+                run.step()
+            evs[-1].record(stream)
+            torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         time.sleep(0.2)
-    ms = ev0.elapsed_time(ev1)
+    run.check()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    ms = evs[0].elapsed_time(evs[-1])
     if world > 1:
         t = torch.tensor([ms], device=device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -303,12 +383,19 @@ def run_native(args, rank, world):
     ms_per_step = ms / args.steps
     value = world * T * N_LAYERS * args.steps / (ms / 1e3)
 
-    # the dominant kernel: the expert FFN call of each layer, on the inputs the
-    # timed steps gave each layer, device-timed with the host kept ahead
+    # the roofline of the one kernel of the step: the bytes it must read (every
+    # layer's touched expert blocks and router) over its launch time
     hbm, tf, peak_kind = peaks()
-    fp = ffn_profile(layers, routers, run.ns[:N_LAYERS], stream)
+    ex, rt = stack_touched_bytes(run, layers, routers, stream)
+    launch_s = float(np.mean(per)) / 1e3
+    alg = float(sum(ex) + sum(rt))
+    achieved = alg / launch_s / 1e9
+    traffic = None
+    if STACK_TRAFFIC["digest"] == source_digest(STACK_SOURCES) and STACK_TRAFFIC["dram_bytes"]:
+        traffic = round(STACK_TRAFFIC["dram_bytes"] / STACK_TRAFFIC["algorithmic_bytes"] * alg)
 
-    # end to end through the public API: pinned host input, eager calls, host output
+    # end to end through the public API: the token copied in from pinned host
+    # memory, one stack_forward, the result copied back, every step
     h_in = x0.cpu().pin_memory()
     h_out = torch.empty(T, cfg.H, dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
@@ -318,19 +405,20 @@ def run_native(args, rank, world):
                 torch.cuda.synchronize()
                 e0 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            run.xs[0].copy_(h_in, non_blocking=True)
+            run.x_in.copy_(h_in, non_blocking=True)
             run.step()
-            h_out.copy_(run.xs[N_LAYERS], non_blocking=True)
+            h_out.copy_(run.out, non_blocking=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e1.record(stream)
-        torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    run.check()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if world > 1:
         t = torch.tensor([e2e_ms], device=device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_val = world * T * N_LAYERS / (e2e_ms / 1e3)
-    del graph, run
+    del run
 
     # the other workloads of the layer, reported beside the headline
     extra = {}
@@ -340,19 +428,25 @@ def run_native(args, rank, world):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "int codes x fp16 activations, fp32 accumulation; bf16 residual stream",
+        "data": "synthetic",
         "config": {"workload": f"decode: {N_LAYERS} stacked MoE layers (H=2048, I=512, E=512, top-10 + 1 shared, "
                                "shelves 128x8-bit/192x4-bit/192x3-bit, Zipf routing), 1 token per step per GPU",
                    "global_batch": world * T, "layers": N_LAYERS, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2: ~1.37 GB of distinct expert weights touched per step",
-                   "graph": f"one CUDA graph per step (rmsnorm + {N_LAYERS} x layer_forward)"},
-        "roofline": {"bound": "hbm", "kernel": "expert FFN call of one layer (counter clear + streaming GEMV)",
-                     "achieved": round(fp["gbs"], 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(fp["gbs"] / hbm, 4), "traffic": DECODE_FFN_TRAFFIC, "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": round(fp["bytes"]), "avg_launch_us": round(fp["ms"] * 1e3, 2)},
+                   "l2": f"inputs larger than L2: {sum(ex) / 1e9:.2f} GB of expert blocks touched per step",
+                   "launch": f"one launch of the persistent stack kernel per step (all {N_LAYERS} layers)"},
+        "roofline": {"bound": "hbm", "kernel": f"stack kernel: one decode step through {N_LAYERS} layers",
+                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": traffic, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": round(alg),
+                     "expert_bytes_per_launch": round(sum(ex)), "router_bytes_per_launch": round(sum(rt)),
+                     "expert_only_frac": round(sum(ex) / launch_s / 1e9 / hbm, 4),
+                     "avg_launch_us": round(launch_s * 1e6, 2),
+                     "avg_layer_us": round(launch_s * 1e6 / N_LAYERS, 2)},
         "e2e": {"value": round(e2e_val, 1), "unit": UNIT,
                 "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2},
-        "gpu_launches": args.steps * (N_LAYERS * KERNELS_PER_LAYER + 1),
+        "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }
     if extra:
@@ -370,11 +464,19 @@ def other_workloads(args, layers, routers, stream, rank):
     for name, x0 in (("decode_T8", inputs.activations(8, cfg.H, seed=inputs.X_SEED + 1000 * rank + 8, device=dev)),
                      ("verify_T5", inputs.correlated_activations(inputs.VERIFY_T, cfg.H,
                                                                  seed=inputs.X_SEED + 1000 * rank, device=dev))):
-        run = StackRunner(layers, routers, x0, stream)
-        ms = run.time(args.steps, args.warmup)
+        run = StackStep(layers, routers, x0)
+        ms = run.time(stream, args.steps, args.warmup)
         res[name] = {"layer_tokens_per_s": round(x0.shape[0] * n / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
-                     "layers": n, "tokens": x0.shape[0]}
+                     "layers": n, "tokens": x0.shape[0], "path": "stack kernel"}
         del run
+    # the same one-token step through the per-layer entry points (routing,
+    # FFN and combine kernels per layer, one CUDA graph per step)
+    x0 = inputs.activations(1, cfg.H, seed=inputs.X_SEED + 1000 * rank, device=dev)
+    run = StackRunner(layers, routers, x0, stream)
+    ms = run.time(args.steps, args.warmup)
+    res["decode_T1_layer_path"] = {"layer_tokens_per_s": round(n / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+                                   "layers": n, "tokens": 1, "path": "rmsnorm + per-layer routing/FFN/combine graph"}
+    del run
     hbm, tf, _ = peaks()
     pf = prefill_profile(layers[0], routers[0], stream)
     res["prefill_T4096"] = {"layer_tokens_per_s": round(pf["T"] / (pf["layer_ms"] / 1e3), 1),

@@ -402,6 +402,7 @@ struct StreamSmem {
     uint64_t *bfull, *bempty;  // [kNB]: B operand built / every compute warp has moved past it
     int *abort;              // set by a warp that gave up; every wait checks it
     int *range;              // this CTA's tiles: [gs0, ge0), [gs1, ge1); then the slot count
+    int *pst;                // producer: ring byte range [pst[d], pst[kND + d]) of the tile in descriptor d
     int *srt;                // copy of sorted_slot when it has at most kMaxSmemEntries entries, else null
     PlanTabs pt;
     TierPtrs *tp;            // [MOE_MAX_TIERS + 1]
@@ -652,7 +653,6 @@ __device__ __forceinline__ float4 compute_part(const Geo &G, int phase, const ui
 // and item counts fix the barrier phases and ring offsets).
 struct ProducerState {
     int head, rel, i;
-    int st[kND], en[kND];
 };
 struct ComputeState {
     int head, i, m, kb;
@@ -670,8 +670,10 @@ __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMap
                                              ProducerState &ps, bool drain) {
     if ((threadIdx.x & 31) != 0) return;
     int head = ps.head, rel = ps.rel, i = ps.i;
-    int(&st)[kND] = ps.st;
-    int(&en)[kND] = ps.en;
+    // the ring ranges of the tiles in flight sit in shared memory: a thread's
+    // dynamically indexed array would live in local memory, which has almost
+    // no L1 behind a full shared-memory carve-out
+    int *st = S.pst, *en = S.pst + kND;
     bool ok = true;
     Walk w;
     walk_begin(S, w);
@@ -1026,7 +1028,8 @@ __device__ __forceinline__ uint8_t *carve_stream_smem(uint8_t *smem, int ring_by
     q = reinterpret_cast<uint8_t *>(S.bempty + kNB);
     S.abort = reinterpret_cast<int *>(q);
     S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots, flag (16-byte aligned)
-    q += 12 * sizeof(int);
+    S.pst = S.abort + 12;
+    q += (12 + 2 * kND) * sizeof(int);
     S.tp = reinterpret_cast<TierPtrs *>(q);
     q += (MOE_MAX_TIERS + 1) * sizeof(TierPtrs);
     S.geo = reinterpret_cast<Geo *>(q);
@@ -1047,7 +1050,7 @@ __host__ __forceinline__ size_t stream_smem_fixed(int H, int I, int T, int k, in
     const size_t n_srt = static_cast<size_t>(T) * k;
     return static_cast<size_t>(xall_bytes(H, T)) + kNB * static_cast<size_t>(bbuf_bytes(H, I, T)) +
            kGroups * kNR * static_cast<size_t>(kRedBytes) +
-           (2 * kND + 2 * kGroups * kNR + 2 * kNB) * sizeof(uint64_t) + 12 * sizeof(int) +
+           (2 * kND + 2 * kGroups * kNR + 2 * kNB) * sizeof(uint64_t) + (12 + 2 * kND) * sizeof(int) +
            (MOE_MAX_TIERS + 1) * sizeof(TierPtrs) + 6 * sizeof(Geo) + 16 + plan_tab_bytes(max_slots) +
            (n_srt <= static_cast<size_t>(kMaxSmemEntries) ? (n_srt * sizeof(int) + 15) / 16 * 16 : 0);
 }

@@ -67,6 +67,11 @@ __device__ __forceinline__ uint32_t order_key(float v) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float whose order_key is `key`.
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 template <int NJ>
 __device__ __forceinline__ void warp_topk_redux(const float *row, int E, int k, int &out_i, float &out_w) {
     const int lane = threadIdx.x & 31;
@@ -97,9 +102,9 @@ __device__ __forceinline__ void warp_topk_redux(const float *row, int E, int k, 
         const uint32_t id = (bj >= 0 && bk == wk) ? static_cast<uint32_t>(lane + 32 * bj) : 0xffffffffu;
         const uint32_t wi = __reduce_min_sync(0xffffffffu, id);
         if (static_cast<int>(wi & 31u) == lane) taken |= 1u << (wi >> 5);
-        if (lane == r) {
+        if (lane == r) {  // the value from its key: no load in the loop
             my_i = static_cast<int>(wi);
-            my_v = __ldcg(row + wi);
+            my_v = key_value(wk);
         }
     }
     const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
