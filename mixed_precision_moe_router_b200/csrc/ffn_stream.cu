@@ -400,7 +400,7 @@ struct StreamSmem {
     uint64_t *full, *empty;  // [kND]: a tile's copies landed / every compute warp is done with it
     uint64_t *rfull, *rempty;  // [kGroups][kNR]: partials written / partials summed
     uint64_t *bfull, *bempty;  // [kNB]: B operand built / every compute warp has moved past it
-    int *abort;              // set by a warp that gave up; every wait checks it
+    int *abort;              // [0] set by a warp that gave up (every wait checks it); [1] grid barriers passed
     int *range;              // this CTA's tiles: [gs0, ge0), [gs1, ge1); then the slot count
     int *pst;                // producer: ring byte range [pst[d], pst[kND + d]) of the tile in descriptor d
     int *srt;                // copy of sorted_slot when it has at most kMaxSmemEntries entries, else null
@@ -958,12 +958,129 @@ __host__ __device__ __forceinline__ PrologueScratch prologue_scratch(int H, int 
     return ps;
 }
 
+// First tile (global index) of a phase whose start cost is >= x, with the
+// slots' inclusive cost prefix `pre` and tile cost `tc` held by lanes < ns
+// (warp-uniform result): the warp form of plan_first_tile.
+__device__ __forceinline__ int lanes_first_tile(long long pre, long long tc, int nt, int ns, long long x) {
+    const int lane = threadIdx.x & 31;
+    const unsigned m = __ballot_sync(0xffffffffu, lane < ns && pre > x);
+    if (!m) return ns * nt;
+    const int L = __ffs(m) - 1;
+    int r = 0;
+    if (lane == L) {
+        const long long off = pre - nt * tc;  // start cost of the slot's first tile
+        if (x <= off) {
+            r = L * nt;
+        } else {
+            long long b = static_cast<long long>(ceil(static_cast<double>(x - off) / static_cast<double>(tc)));
+            if (b > nt) b = nt;
+            r = L * nt + static_cast<int>(b);
+        }
+    }
+    return __shfl_sync(0xffffffffu, r, L);
+}
+
+// One token (T == 1, k <= 31): warp 0 alone ends the routing from the grid's
+// logits and builds this CTA's schedule.  It writes what cta_topk_rows,
+// cta_group and plan_in_cta write (the choices and weights, the sorted slots,
+// their positions, the active list, the slot tables and the tile runs), with
+// the chosen experts held one per lane: the k choices of one token are
+// distinct, so each is one slot and its sorted position is its rank.  The
+// offsets are written only when fill_offsets.  The caller synchronises.
+__device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S, int *act_s, int *off_s, int *idx_s,
+                                               float *w_s, int *pos_s, bool fill_offsets) {
+    const int lane = threadIdx.x & 31;
+    const int E = p.E, k = p.k;
+    int e_r;
+    float w_r;
+    if (E <= 512) warp_topk_redux<16>(p.route.logits, E, k, e_r, w_r);
+    else warp_topk_redux<32>(p.route.logits, E, k, e_r, w_r);
+    int rank = 0;
+    for (int j = 0; j < k; ++j) rank += __shfl_sync(0xffffffffu, e_r, j) < e_r;
+    if (lane < k) {
+        idx_s[lane] = e_r;
+        w_s[lane] = w_r;
+        pos_s[lane] = rank;
+        S.srt[rank] = lane;
+        act_s[1 + rank] = e_r;
+    }
+    if (lane == 0) act_s[0] = k;
+    __syncwarp();
+    // slot a = lane: the a-th chosen expert in id order, then the shared expert
+    const PlanIn &pi = p.pi;
+    const bool shared = pi.has_shared && pi.T <= pi.max_count;
+    const int ns = k + (shared ? 1 : 0);
+    int e = -1, bits = 0, ti = 0, jl = 0, first = 0;
+    if (lane < k) {
+        e = act_s[1 + lane];
+        for (int t = 0; t < pi.n_tiers; ++t)
+            if (e >= pi.first[t] && e - pi.first[t] < pi.n[t]) ti = t;
+        bits = pi.bits[ti];
+        jl = e - pi.first[ti];
+        first = lane;
+    } else if (lane == k && shared) {
+        e = pi.E;
+        bits = pi.shared_bits;
+        ti = pi.n_tiers;
+        first = k;
+    }
+    if (fill_offsets)  // offsets[x] = chosen experts below x
+        for (int x0 = 0; x0 <= E; x0 += 32) {
+            int c = 0;
+            for (int a = 0; a < k; ++a) c += __shfl_sync(0xffffffffu, e, a) < x0 + lane;
+            if (x0 + lane <= E) off_s[x0 + lane] = c;
+        }
+    const int nt0 = S.nt0, nt1 = S.nt1;
+    long long tc0 = 0, tc1 = 0, v0 = 0, v1 = 0;
+    if (lane < ns) {
+        tc0 = tile_cost(pi.H, pi.I, 0, bits, 1);
+        tc1 = tile_cost(pi.H, pi.I, 1, bits, 1);
+        v0 = nt0 * tc0;
+        v1 = nt1 * tc1;
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long u0 = __shfl_up_sync(0xffffffffu, v0, o), u1 = __shfl_up_sync(0xffffffffu, v1, o);
+        if (lane >= o) {
+            v0 += u0;
+            v1 += u1;
+        }
+    }
+    if (lane < ns) {
+        const PlanTabs &t = S.pt;
+        t.expert[lane] = e;
+        t.bits[lane] = bits;
+        t.tier[lane] = ti;
+        t.jloc[lane] = jl;
+        t.first[lane] = first;
+        t.count[lane] = 1;
+        t.tc0[lane] = tc0;
+        t.tc1[lane] = tc1;
+        t.pre0[lane] = v0;
+        t.pre1[lane] = v1;
+    }
+    const int c = blockIdx.x, G = gridDim.x;
+    const long long tot0 = __shfl_sync(0xffffffffu, v0, 31), tot1 = __shfl_sync(0xffffffffu, v1, 31);
+    const int gs0 = lanes_first_tile(v0, tc0, nt0, ns, share_floor(tot0, c, G));
+    const int ge0 = c + 1 == G ? ns * nt0 : lanes_first_tile(v0, tc0, nt0, ns, share_floor(tot0, c + 1, G));
+    const int gs1 = lanes_first_tile(v1, tc1, nt1, ns, share_floor(tot1, c, G));
+    const int ge1 = c + 1 == G ? ns * nt1 : lanes_first_tile(v1, tc1, nt1, ns, share_floor(tot1, c + 1, G));
+    if (lane == 0) {
+        S.range[0] = gs0;
+        S.range[1] = ge0;
+        S.range[2] = gs1;
+        S.range[3] = ge1;
+        S.range[4] = ns;
+    }
+}
+
 // The batch routed by the FFN kernel itself (every thread of every CTA): the
 // logits of this CTA's share of the experts, a grid barrier, then the top-k
 // of every token and the stable grouping of the T*k slots, into the same
 // shared-memory lists the prologue otherwise copies from global memory.  CTA 0
-// also writes the routing outputs.  False when the grid barrier gave up.
-__device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, const uint16_t *x_s, int *act_s,
+// also writes the routing outputs.  Returns 0 when the grid barrier gave up,
+// 2 when the schedule is built too (one token), else 1.
+__device__ __forceinline__ int route_in_cta(const FfnParams &p, StreamSmem &S, const uint16_t *x_s, int *act_s,
                                           int *off_s, const PrologueScratch &ps) {
     const int T = p.T, E = p.E, k = p.k, H = p.w.H, S_ = T * k;
     // logits of experts [E * c / G, E * (c + 1) / G), all warps
@@ -972,8 +1089,9 @@ __device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, 
     cta_logits(x_s, T, H, E, p.route.wr, p.route.bias, e0, e1,
                reinterpret_cast<float *>(S.ring + ps.cand), p.route.logits);
     int *barrier_ok = S.range + 5;
+    __syncthreads();  // every thread's logits are written before thread 0 arrives
     if (threadIdx.x == 0) {
-        const bool ok = grid_barrier(p.route.gbar, S.abort, p.wait_limit);
+        const bool ok = grid_barrier(p.route.gbar, S.abort[1]++, S.abort, p.wait_limit);
         if (!ok) {
             status_or(p.status, MOE_STATUS_TIMEOUT);
             *static_cast<volatile int *>(S.abort) = 1;
@@ -981,12 +1099,19 @@ __device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, 
         *barrier_ok = ok;
     }
     __syncthreads();
-    if (!*barrier_ok) return false;
+    if (!*barrier_ok) return 0;
     int *idx_s = reinterpret_cast<int *>(S.ring + ps.idx);
     float *w_s = reinterpret_cast<float *>(S.ring + ps.w);
     int *pos_s = reinterpret_cast<int *>(S.ring + ps.pos);
-    cta_topk_rows(p.route.logits, T, E, k, idx_s, w_s);
-    cta_group(idx_s, S_, E, S.srt, pos_s, act_s, off_s, reinterpret_cast<int *>(S.ring + ps.tmp));
+    const bool one = T == 1 && k <= 31 && E <= 1024 && p.pi.max_count >= 1 && S.srt != nullptr;
+    if (one) {
+        if (threadIdx.x < 32)
+            route_plan_one(p, S, act_s, off_s, idx_s, w_s, pos_s, blockIdx.x == 0 && p.route.topk_idx != nullptr);
+        __syncthreads();
+    } else {
+        cta_topk_rows(p.route.logits, T, E, k, idx_s, w_s);
+        cta_group(idx_s, S_, E, S.srt, pos_s, act_s, off_s, reinterpret_cast<int *>(S.ring + ps.tmp));
+    }
     if (blockIdx.x == 0 && p.route.topk_idx) {
         for (int i = threadIdx.x; i < S_; i += blockDim.x) {
             p.route.topk_idx[i] = idx_s[i];
@@ -997,7 +1122,7 @@ __device__ __forceinline__ bool route_in_cta(const FfnParams &p, StreamSmem &S, 
         for (int e = threadIdx.x; e <= E; e += blockDim.x) p.route.offsets[e] = off_s[e];
         for (int a = threadIdx.x; a <= act_s[0]; a += blockDim.x) p.route.active[a] = act_s[a];
     }
-    return true;
+    return one ? 2 : 1;
 }
 
 // Shared memory of a CTA (same layout for every launch shape): the ring,
@@ -1071,7 +1196,8 @@ __device__ __forceinline__ void init_stream_smem(StreamSmem &S, int H, int I) {
             mbar_init(&S.bfull[i], 1);
             mbar_init(&S.bempty[i], kComputeWarps);
         }
-        *S.abort = 0;
+        S.abort[0] = 0;
+        S.abort[1] = 0;  // grid barriers this CTA has passed
         mbar_fence_init();
     }
     if (threadIdx.x < 6) {
@@ -1169,11 +1295,11 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
         const bool xbad = build_xall(p, x_s, S.xall);
         if (__any_sync(0xffffffffu, xbad) && lane == 0) status_or(p.status, MOE_STATUS_FP16_RANGE);
     }
-    bool routed = true;
+    int routed = 1;
     if (fused) routed = route_in_cta(p, S, reinterpret_cast<const uint16_t *>(x_s), act_s, off_s, ps);
     if (!routed) {  // the grid barrier gave up: stream nothing
         if (threadIdx.x < 5) S.range[threadIdx.x] = 0;
-    } else {
+    } else if (routed == 1) {
         plan_in_cta(p, S, act_s, off_s);
     }
     // the ring's scratch is overwritten by TMA copies from here on: order
@@ -1454,8 +1580,10 @@ __device__ __forceinline__ void cta_rms_norm_rows(uint16_t *x_s, int T, int H, f
 
 // thread 0 of every CTA at a grid barrier; the result in every thread
 __device__ __forceinline__ bool stack_barrier(const StackParams &P, StreamSmem &S) {
+    __syncthreads();  // the CTA's writes before the barrier precede thread 0's arrival
     if (threadIdx.x == 0) {
-        const bool ok = !*static_cast<volatile int *>(S.abort) && grid_barrier(P.gbar, S.abort, P.wait_limit);
+        const bool ok =
+            !*static_cast<volatile int *>(S.abort) && grid_barrier(P.gbar, S.abort[1]++, S.abort, P.wait_limit);
         if (!ok) {
             status_or(P.status, MOE_STATUS_TIMEOUT);
             *static_cast<volatile int *>(S.abort) = 1;
@@ -1566,12 +1694,13 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
             const bool xbad = build_xall(p, reinterpret_cast<const uint8_t *>(x_s), S.xall);
             if (__any_sync(0xffffffffu, xbad) && (threadIdx.x & 31) == 0) status_or(P.status, MOE_STATUS_FP16_RANGE);
         }
-        if (!route_in_cta(p, S, x_s, act_s, off_s, ps)) {
+        const int routed = route_in_cta(p, S, x_s, act_s, off_s, ps);
+        if (!routed) {
             alive = false;
             break;
         }
         for (int i = threadIdx.x; i < S_; i += blockDim.x) wkeep[i] = reinterpret_cast<const float *>(S.ring + ps.w)[i];
-        plan_in_cta(p, S, act_s, off_s);
+        if (routed == 1) plan_in_cta(p, S, act_s, off_s);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
         const bool last = l + 1 == P.n_layers;

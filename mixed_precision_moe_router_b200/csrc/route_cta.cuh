@@ -75,33 +75,56 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 template <int NJ>
 __device__ __forceinline__ void warp_topk_redux(const float *row, int E, int k, int &out_i, float &out_w) {
     const int lane = threadIdx.x & 31;
+    // key 0 marks an entry out of range or already taken (no float maps to 0
+    // but a NaN with every bit set)
     uint32_t key[NJ];
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
         const int e = lane + 32 * j;
         key[j] = e < E ? order_key(__ldcg(row + e) + 0.0f) : 0u;  // -0 keys as +0
     }
-    uint32_t taken = 0;
-#pragma unroll
-    for (int j = 0; j < NJ; ++j)
-        if (lane + 32 * j >= E) taken |= 1u << j;
     float my_v = 0.f;
     int my_i = 0;
     for (int r = 0; r < k; ++r) {
-        // this lane's best untaken entry: the largest key, then the lowest id
-        // (ids grow with j, so the first j with the largest key)
-        uint32_t bk = 0;
-        int bj = -1;
+        // this lane's best untaken entry, the largest key then the lowest id:
+        // up to 16 keys by a tree over adjacent pairs (a left subtree holds
+        // the lower ids), more by one pass (fewer registers)
+        uint32_t bk = 0u;
+        int bj = 0;
+        if constexpr (NJ <= 16) {
+            uint32_t kk[NJ];
+            int jj[NJ];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j)
-            if (!((taken >> j) & 1u) && (bj < 0 || key[j] > bk)) {
-                bk = key[j];
-                bj = j;
+            for (int j = 0; j < NJ; ++j) {
+                kk[j] = key[j];
+                jj[j] = j;
             }
+#pragma unroll
+            for (int s = 1; s < NJ; s *= 2)
+#pragma unroll
+                for (int m = 0; m + s < NJ; m += 2 * s)
+                    if (kk[m + s] > kk[m]) {
+                        kk[m] = kk[m + s];
+                        jj[m] = jj[m + s];
+                    }
+            bk = kk[0];
+            bj = jj[0];
+        } else {
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+                if (key[j] > bk) {
+                    bk = key[j];
+                    bj = j;
+                }
+        }
         const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-        const uint32_t id = (bj >= 0 && bk == wk) ? static_cast<uint32_t>(lane + 32 * bj) : 0xffffffffu;
+        const uint32_t id = (bk != 0u && bk == wk) ? static_cast<uint32_t>(lane + 32 * bj) : 0xffffffffu;
         const uint32_t wi = __reduce_min_sync(0xffffffffu, id);
-        if (static_cast<int>(wi & 31u) == lane) taken |= 1u << (wi >> 5);
+        // the winner's lane marks it taken (a select per key: a conditional
+        // store would send the array to local memory)
+        const int wj = static_cast<int>(wi & 31u) == lane ? static_cast<int>(wi >> 5) : -1;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) key[j] = j == wj ? 0u : key[j];
         if (lane == r) {  // the value from its key: no load in the loop
             my_i = static_cast<int>(wi);
             my_v = key_value(wk);

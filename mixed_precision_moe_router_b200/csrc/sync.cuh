@@ -167,27 +167,19 @@ __device__ __forceinline__ bool wait_geq_abortable(const int *ctr, int target, c
     return true;
 }
 
-// Grid-wide barrier of a cooperative launch.  bar[0] counts arrivals (zero on
-// entry; the last arriver resets it), bar[1] is a generation number.  Thread 0
-// of each CTA arrives after a fence and waits (bounded, abortable) for the
-// generation to move; the caller follows with __syncthreads.  Returns false
-// when the wait gave up.
-__device__ __forceinline__ bool grid_barrier(int *bar, const volatile int *abort, long long limit) {
-    const int gen = ld_acquire(bar + 1);
-    __threadfence();
-    if (atomicAdd(bar, 1) == static_cast<int>(gridDim.x * gridDim.y * gridDim.z) - 1) {
-        bar[0] = 0;
-        __threadfence();
-        atomicAdd(bar + 1, 1);
-        return true;
-    }
+// Grid-wide barrier, called by thread 0 of every CTA with the CTA synchronised
+// before and after.  `bar` counts arrivals over the launch (zero at launch,
+// never reset), so barrier number n (0, 1, ...) is passed once it reaches
+// (n + 1) * grid.  The arrival is a release add, which orders the writes the
+// CTA made before the barrier; the wait polls with acquire loads, bounded and
+// abortable.  Returns false when the wait gave up.
+__device__ __forceinline__ bool grid_barrier(int *bar, int n, const volatile int *abort, long long limit) {
+    const int target = (n + 1) * static_cast<int>(gridDim.x * gridDim.y * gridDim.z);
+    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(bar) : "memory");
+    if (ld_acquire(bar) >= target) return true;
     const long long t0 = clock64();
-    unsigned ns = 32;
-    while (ld_acquire(bar + 1) == gen) {
+    while (ld_acquire(bar) < target)
         if (*abort || clock64() - t0 > limit) return false;
-        __nanosleep(ns);
-        if (ns < 256) ns *= 2;
-    }
     return true;
 }
 
