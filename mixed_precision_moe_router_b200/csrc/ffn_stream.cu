@@ -652,10 +652,10 @@ __device__ __forceinline__ float4 compute_part(const Geo &G, int phase, const ui
 // State a role keeps from one layer to the next in a persistent launch (tile
 // and item counts fix the barrier phases and ring offsets).
 struct ProducerState {
-    int head, rel, i;
+    int i;  // tiles issued so far
 };
 struct ComputeState {
-    int head, i, m, kb;
+    int i, m, kb;
 };
 struct LoaderState {
     int kb;
@@ -664,46 +664,89 @@ struct EpilogueState {
     int m, i;
 };
 
-// Producer for the current tile list; `drain`: wait for every copy in
-// flight before returning (the last list of a launch).
+// Producer warp for the current tile list; `drain`: wait for every copy in
+// flight before returning (the last list of a launch).  Every tile issued
+// before the call has been consumed (the previous list's roles have ended),
+// so the ring starts empty: the first tiles that fit it, up to kND, take
+// consecutive ranges from offset 0 (a warp prefix sum of their sizes) and are
+// issued at once, one per lane.  Lane 0 then issues the rest in order, each
+// once the ranges it overlaps have been released.  The ring range of the tile
+// in descriptor d is [pst[d], pst[kND + d]) (in shared memory: a dynamically
+// indexed array of a thread lives in local memory, which has almost no L1
+// behind a full shared-memory carve-out); the compute warps read the stage
+// offset from there.
 __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMaps &M, StreamSmem &S,
                                              ProducerState &ps, bool drain) {
-    if ((threadIdx.x & 31) != 0) return;
-    int head = ps.head, rel = ps.rel, i = ps.i;
-    // the ring ranges of the tiles in flight sit in shared memory: a thread's
-    // dynamically indexed array would live in local memory, which has almost
-    // no L1 behind a full shared-memory carve-out
+    const int lane = threadIdx.x & 31;
     int *st = S.pst, *en = S.pst + kND;
-    bool ok = true;
-    Walk w;
-    walk_begin(S, w);
-    for (; w.phase < 2; walk_next(S, w), ++i) {
-        const int sz = stage_alloc_bytes(tile_geo(S, w.phase, w.a));
-        const int s0 = ring_take(head, sz, S.ring_bytes);
-        while (rel < i) {
-            bool clash = i - rel >= kND;
-            for (int j = rel; j < i && !clash; ++j) clash = st[j % kND] < s0 + sz && s0 < en[j % kND];
-            if (!clash) break;
-            if (!mbar_wait_abortable(&S.empty[rel % kND], (rel / kND) & 1, S.abort, p.wait_limit)) {
-                ok = false;
-                break;
-            }
-            ++rel;
+    const int i0 = ps.i;
+    const int gs0 = S.range[0], n0 = max(S.range[1] - gs0, 0);
+    const int gs1 = S.range[2], n1 = max(S.range[3] - gs1, 0);
+    int nfit, head;
+    {
+        const int j = lane;
+        const bool real = j < n0 + n1 && j < kND;
+        int phase = 0, a = 0, b = 0, sz = 0;
+        if (real) {
+            phase = j < n0 ? 0 : 1;
+            const int g = phase == 0 ? gs0 + j : gs1 + (j - n0);
+            const int nt = phase == 0 ? S.nt0 : S.nt1;
+            a = g / nt;
+            b = g - a * nt;
+            sz = stage_alloc_bytes(tile_geo(S, phase, a));
         }
-        if (!ok) break;
-        st[i % kND] = s0;
-        en[i % kND] = s0 + sz;
-        issue_tile(p, M, S, w.phase, w.a, w.b, S.ring + s0, &S.full[i % kND]);
+        int end = sz;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, end, o);
+            if (lane >= o) end += v;
+        }
+        const bool fits = real && end <= S.ring_bytes;  // a prefix of the lanes
+        nfit = __popc(__ballot_sync(0xffffffffu, fits));
+        head = nfit > 0 ? __shfl_sync(0xffffffffu, end, nfit - 1) : 0;
+        if (fits) {
+            const int d = (i0 + j) % kND;
+            st[d] = end - sz;
+            en[d] = end;
+            issue_tile(p, M, S, phase, a, b, S.ring + (end - sz), &S.full[d]);
+        }
     }
-    if (!ok) abort_cta(p, S);
-    ps.head = head;
-    ps.rel = rel;
-    ps.i = i;
-    // tiles before i were issued and those before rel consumed: the rest must land
-    if (drain || !ok)
-        for (int j = max(rel, i - kND); j < i; ++j)
-            if (!mbar_wait_limit(&S.full[j % kND], (j / kND) & 1, p.wait_limit))
-                status_or(p.status, MOE_STATUS_TIMEOUT);
+    __syncwarp();  // lane 0 reads the other lanes' ring ranges below
+    // every lane keeps the count: the next list's descriptors follow from it
+    ps.i = i0 + n0 + n1;
+    if (lane == 0) {
+        int rel = i0, i = i0 + nfit;
+        bool ok = true;
+        Walk w;
+        walk_begin(S, w);
+        for (int n = 0; n < nfit; ++n) walk_next(S, w);
+        for (; w.phase < 2; walk_next(S, w), ++i) {
+            const int sz = stage_alloc_bytes(tile_geo(S, w.phase, w.a));
+            const int s0 = ring_take(head, sz, S.ring_bytes);
+            while (rel < i) {
+                bool clash = i - rel >= kND;
+                for (int j = rel; j < i && !clash; ++j) clash = st[j % kND] < s0 + sz && s0 < en[j % kND];
+                if (!clash) break;
+                if (!mbar_wait_abortable(&S.empty[rel % kND], (rel / kND) & 1, S.abort, p.wait_limit)) {
+                    ok = false;
+                    break;
+                }
+                ++rel;
+            }
+            if (!ok) break;
+            st[i % kND] = s0;
+            en[i % kND] = s0 + sz;
+            issue_tile(p, M, S, w.phase, w.a, w.b, S.ring + s0, &S.full[i % kND]);
+        }
+        if (!ok) abort_cta(p, S);
+        ps.i = i;  // short of i0 + n0 + n1 only after giving up
+        // tiles before i were issued and those before rel consumed: the rest must land
+        if (drain || !ok)
+            for (int j = max(rel, i - kND); j < i; ++j)
+                if (!mbar_wait_limit(&S.full[j % kND], (j / kND) & 1, p.wait_limit))
+                    status_or(p.status, MOE_STATUS_TIMEOUT);
+    }
+    __syncwarp();
 }
 
 // Compute warp `cw` (0..kComputeWarps-1): group cw / kWarps computes the
@@ -715,7 +758,7 @@ __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMap
 // run ahead of the loader.
 __device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, int cw, ComputeState &cs) {
     const int lane = threadIdx.x & 31, grp = cw / kWarps, warp = cw % kWarps;
-    int head = cs.head, i = cs.i, m = cs.m, kb = cs.kb;
+    int i = cs.i, m = cs.m, kb = cs.kb;
     long long key = -1;
     bool ok = true;
     float4 *red = S.red + grp * kNR * (kWarps * 32);
@@ -726,13 +769,13 @@ __device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, i
         const int phase = w.phase, a = w.a;
         const int bits = S.pt.bits[a], cnt = S.pt.count[a];
         const Geo &G = tile_geo(S, phase, a);
-        const int s0 = ring_take(head, stage_alloc_bytes(G), S.ring_bytes);
         const bool mine = i % kGroups == grp;
         if (mine && !mbar_wait_warp(&S.full[i % kND], (i / kND) & 1, S.abort, p.wait_limit)) {
             ok = false;
             break;
         }
-        const uint8_t *stage = S.ring + s0;
+        // the stage's offset, written by the producer before the copy it waited for
+        const uint8_t *stage = S.ring + (mine ? S.pst[i % kND] : 0);
         const int tp = tokens_per_pass(phase, p.w.I), np = n_passes(p, S, phase, a);
         for (int pass = 0; pass < np; ++pass) {
             const uint8_t *xf;
@@ -776,7 +819,6 @@ __device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, i
             ++m;
         }
     }
-    cs.head = head;
     cs.i = i;
     cs.m = m;
     cs.kb = kb;
@@ -1313,7 +1355,7 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
         return;
     }
     if (warp < kComputeWarps) {
-        ComputeState cs = {0, 0, 0, -1};
+        ComputeState cs = {0, 0, -1};
         run_compute(p, S, warp, cs);
     } else if (warp == kWarpLoader) {
         LoaderState ls = {-1};
@@ -1608,7 +1650,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
     float *red = reinterpret_cast<float *>(q);
     init_stream_smem(S, H, P.I);
     ProducerState prs = {};
-    ComputeState cst = {0, 0, 0, -1};
+    ComputeState cst = {0, 0, -1};
     LoaderState lds = {-1};
     EpilogueState eps = {0, 0};
     const PrologueScratch ps = prologue_scratch(H, T, k, E, max_slots, true);
@@ -1772,8 +1814,9 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
         }
     }
     // after a failed barrier: wait for any copy this CTA still has in flight
+    // (the last kND tiles issued: each was the last use of its descriptor)
     if (!alive && warp == kWarpProducer && (threadIdx.x & 31) == 0)
-        for (int j = max(prs.rel, prs.i - kND); j < prs.i; ++j)
+        for (int j = max(0, prs.i - kND); j < prs.i; ++j)
             if (!mbar_wait_limit(&S.full[j % kND], (j / kND) & 1, P.wait_limit)) status_or(P.status, MOE_STATUS_TIMEOUT);
     if (alive && P.x_out_norm && blockIdx.x == 0) {
         for (int c = threadIdx.x; c < T * H / 8; c += blockDim.x)
