@@ -356,6 +356,23 @@ int moe_stack_forward(const void *desc, int32_t n_layers, int32_t H, int32_t I, 
                       uint16_t *x_out_norm, uint16_t *x_layers, void *workspace,
                       size_t workspace_bytes, int32_t *status, moe_stream_t stream);
 
+/* ------------------------------------------------------------------------ *
+ * Test hook for the failure-detection paths (not for production use).
+ *
+ * Every device-side wait (mbarrier phases, the per-slot gate_up counters, the
+ * grid barriers) gives up after a number of SM clock cycles, about 1 s by
+ * default, and the call then reports MOE_STATUS_TIMEOUT in its status word.
+ * moe_debug_set_waits sets that limit for the calls enqueued after it
+ * (wait_limit_cycles <= 0 restores the default), and with skip_publish_slot
+ * >= 0 makes the streaming FFN kernels never publish the gate_up completions
+ * of that slot (the slot's position in the kernel's plan order; -1: none), so
+ * that a wait on them runs out without any fault.  The setting is
+ * process-wide and applies to moe_expert_ffn_tiered, moe_layer_forward and
+ * moe_stack_forward; calls already enqueued keep the values they were
+ * launched with.  Always returns MOE_OK.
+ * ------------------------------------------------------------------------ */
+int moe_debug_set_waits(int64_t wait_limit_cycles, int32_t skip_publish_slot);
+
 #ifdef __cplusplus
 }
 #endif

@@ -71,6 +71,7 @@ SIGNATURES = [
     ("moe_stack_workspace_size", c_size, [c_i32, c_i32, c_i32, c_i32, c_i32]),
     ("moe_stack_forward", c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
                                   c_size, c_vp, c_vp]),
+    ("moe_debug_set_waits", c_i32, [ctypes.c_int64, c_i32]),
 ]
 
 _lib = None
@@ -427,3 +428,10 @@ def stack_forward(stack, x_in, k, out=None, out_norm=None, x_layers=None, worksp
                                    _ptr(out_norm), _ptr(x_layers), _ptr(workspace), workspace.numel(), _ptr(status),
                                    _stream()))
     return out
+
+
+def debug_set_waits(wait_limit_cycles=0, skip_publish_slot=-1):
+    """Test hook (moe_debug_set_waits): the device-side wait limit in SM clock
+    cycles (<= 0: the default, about 1 s) and a slot whose gate_up completions
+    the streaming FFN kernels never publish (-1: none)."""
+    _check(lib().moe_debug_set_waits(int(wait_limit_cycles), int(skip_publish_slot)))

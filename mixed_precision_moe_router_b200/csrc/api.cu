@@ -47,14 +47,15 @@ size_t moe_stack_smem(int H, int I, int T, int k, int E, int *ring_bytes);
 cudaError_t moe_configure_stack();
 cudaError_t moe_launch_stack(const void *, int, int, int, int, int, int, const uint16_t *, uint16_t *, uint16_t *,
                              uint16_t *, uint16_t *, float *, float *, float *, float *, int *, int *, int32_t *,
-                             long long, cudaStream_t);
+                             long long, int, cudaStream_t);
 
 namespace {
 
 thread_local std::string g_err;
 
 // Knobs for tests of the failure paths (moe_debug_set); process-wide.
-std::atomic<long long> g_wait_limit{2000000000LL};  // ~1 s of SM clock
+constexpr long long kDefaultWaitLimit = 2000000000LL;  // ~1 s of SM clock
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 std::atomic<int> g_skip_publish{-1};
 
 int fail(int code, const char *fmt, ...) {
@@ -797,8 +798,15 @@ int moe_stack_forward(const void *desc, int32_t n_layers, int32_t H, int32_t I, 
     const long ma = static_cast<long>(T) * k < E ? static_cast<long>(T) * k : E;
     if (e == cudaSuccess)
         e = moe_launch_stack(desc, n_layers, T, k, H, I, E, x_in, x_out, x_out_norm, x_layers, L.xbuf, L.logits, L.h,
-                             L.y_slots, L.y_shared, L.ctr, L.ctr + ma + 1, status, g_wait_limit.load(), s);
+                             L.y_slots, L.y_shared, L.ctr, L.ctr + ma + 1, status, g_wait_limit.load(),
+                             g_skip_publish.load(), s);
     return e == cudaSuccess ? ok() : cuda_fail(e, "stack launch");
+}
+
+int moe_debug_set_waits(int64_t wait_limit_cycles, int32_t skip_publish_slot) {
+    g_wait_limit.store(wait_limit_cycles > 0 ? wait_limit_cycles : kDefaultWaitLimit);
+    g_skip_publish.store(skip_publish_slot < 0 ? -1 : skip_publish_slot);
+    return ok();
 }
 
 }  // extern "C"

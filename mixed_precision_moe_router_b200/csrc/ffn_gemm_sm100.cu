@@ -448,7 +448,7 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
                 pend = -1;
             }
             const int s = L % STAGES;
-            if (!__all_sync(0xffffffffu, mbar_wait(&S.empty[s], ((L / STAGES) & 1) ^ 1))) { fail(P, S); break; }
+            if (!__all_sync(0xffffffffu, mbar_wait_limit(&S.empty[s], ((L / STAGES) & 1) ^ 1, P.f.wait_limit))) { fail(P, S); break; }
             tc_fence_after();
             tmem_st32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + ACC_COLS + s * A_COLS + 32 * half, o);
             pend = s;
@@ -524,7 +524,7 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
             pend = -1;
         }
         const int s = L % STAGES;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&S.empty[s], ((L / STAGES) & 1) ^ 1));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_limit(&S.empty[s], ((L / STAGES) & 1) ^ 1, P.f.wait_limit));
         if (!ok) { fail(P, S); break; }
         tc_fence_after();
         // lanes 32*(warp%4).. of the stage's A columns; this thread's row and half
@@ -580,7 +580,7 @@ __device__ __forceinline__ void role_tokens(const Params &P, const Shared &S, in
 #pragma unroll 1
         for (int kc = 0; kc < NK; ++kc, ++q) {
             const int s = q % STAGES;
-            if (!mbar_wait(&S.empty[s], ((q / STAGES) & 1) ^ 1)) { fail(P, S); break; }
+            if (!mbar_wait_limit(&S.empty[s], ((q / STAGES) & 1) ^ 1, P.f.wait_limit)) { fail(P, S); break; }
             const uint32_t B = smem_u32(S.stages + s * STAGE_BYTES);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -614,7 +614,7 @@ __device__ __forceinline__ void role_mma(const Params &P, const Shared &S, int t
         const int Nt = (nvalid + 15) & ~15;
         const uint32_t idesc = idesc_f16(Nt, P.phase == 2);
         const int buf = acc & 1;
-        if (!mbar_wait(&S.acc_empty[buf], ((acc >> 1) & 1) ^ 1)) { fail(P, S); break; }
+        if (!mbar_wait_limit(&S.acc_empty[buf], ((acc >> 1) & 1) ^ 1, P.f.wait_limit)) { fail(P, S); break; }
         tc_fence_after();
         const uint32_t d = tmem + buf * MAXN;
         bool ok = true;
@@ -622,7 +622,7 @@ __device__ __forceinline__ void role_mma(const Params &P, const Shared &S, int t
         for (int kc = 0; kc < NK; ++kc, ++q) {
             const int s = q % STAGES;
             const uint32_t par = (q / STAGES) & 1;
-            if (!mbar_wait(&S.full_a[s], par) || !mbar_wait(&S.full_b[s], par)) { ok = false; break; }
+            if (!mbar_wait_limit(&S.full_a[s], par, P.f.wait_limit) || !mbar_wait_limit(&S.full_b[s], par, P.f.wait_limit)) { ok = false; break; }
             tc_fence_after();
             const uint32_t b0 = smem_u32(S.stages + s * STAGE_BYTES);
             const uint32_t a = tmem + ACC_COLS + s * A_COLS;
@@ -638,7 +638,7 @@ __device__ __forceinline__ void role_mma(const Params &P, const Shared &S, int t
     }
     // all MMAs issued by this thread are complete before the CTA tears down
     mma_commit(S.fin);
-    if (!mbar_wait(S.fin, 0)) status_or(P.f.status, MOE_STATUS_TIMEOUT);
+    if (!mbar_wait_limit(S.fin, 0, P.f.wait_limit)) status_or(P.f.status, MOE_STATUS_TIMEOUT);
 }
 
 // Epilogue: warp q of the epilogue group owns accumulator lanes 32q..32q+31.
@@ -656,7 +656,7 @@ __device__ __forceinline__ void role_epilogue(const Params &P, const Shared &S, 
         const int first = S.slots.first[tl.slot];
         const int nvalid = min(MAXN, S.slots.count[tl.slot] - tl.nc * MAXN);
         const int buf = acc & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&S.acc_full[buf], (acc >> 1) & 1))) { fail(P, S); break; }
+        if (!__all_sync(0xffffffffu, mbar_wait_limit(&S.acc_full[buf], (acc >> 1) & 1, P.f.wait_limit))) { fail(P, S); break; }
         tc_fence_after();
         const int row = 32 * q + lane;  // accumulator lane = tile row
 #pragma unroll 1
@@ -894,6 +894,7 @@ bool moe_router_gemm_supported(int T, int H, int E) {
 cudaError_t moe_launch_router_gemm(const uint16_t *x, const uint16_t *wr, const float *bias, int T, int H, int E,
                                    float *logits, cudaStream_t s) {
     moe::gemm::Params P{};
+    P.f.wait_limit = moe::kWaitLimitCycles;
     P.f.w.H = H;
     P.f.w.I = 128;
     P.f.E = E;

@@ -1576,6 +1576,7 @@ struct StackParams {
     int *gbar;             // [2] grid barrier words (zero on entry)
     int32_t *status;
     long long wait_limit;
+    int skip_publish;  // test hook, as in FfnParams (-1: none)
     int ring_bytes;
 };
 
@@ -1690,7 +1691,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
         p.route.offsets = p.route.sorted = p.route.slot_pos = p.route.active = nullptr;
         p.route.gbar = P.gbar;
         p.wait_limit = P.wait_limit;
-        p.skip_publish = -1;
+        p.skip_publish = P.skip_publish;
     }
     bool alive = true;
     for (int l = 0; l < P.n_layers && alive; ++l) {
@@ -1869,7 +1870,7 @@ cudaError_t moe_configure_stack() {
 cudaError_t moe_launch_stack(const void *layers, int n_layers, int T, int k, int H, int I, int E, const uint16_t *x_in,
                              uint16_t *x_out, uint16_t *x_out_norm, uint16_t *x_layers, uint16_t *xbuf, float *logits,
                              float *h, float *y_slots, float *y_shared, int *ctr, int *gbar, int32_t *status,
-                             long long wait_limit, cudaStream_t s) {
+                             long long wait_limit, int skip_publish, cudaStream_t s) {
     moe::StackParams P;
     std::memset(&P, 0, sizeof(P));
     P.layers = static_cast<const moe::StackLayer *>(layers);
@@ -1892,6 +1893,7 @@ cudaError_t moe_launch_stack(const void *layers, int n_layers, int T, int k, int
     P.gbar = gbar;
     P.status = status;
     P.wait_limit = wait_limit;
+    P.skip_publish = skip_publish;
     int ring = 0;
     const size_t smem = moe_stack_smem(H, I, T, k, E, &ring);
     if (ring == 0) return cudaErrorInvalidConfiguration;
