@@ -255,9 +255,12 @@ int moe_expert_ffn_tiered(const moe_layer_weights *w, const uint16_t *x, int32_t
  * counters) is one array of MOE_STATIC_SCRATCH_BYTES bytes compiled into the
  * library: every GPU that loads the library holds it until the process
  * exits.  The call needs
- *   align256((T*k + T) * I * 4) + align256((min(T*k, E) + 1) * 4)
- * bytes of it (at I = 512, k = 10: up to 46 tokens) and returns
- * MOE_ERR_UNSUPPORTED, enqueueing nothing, when that exceeds the array.
+ *   align256((T*k + T) * I * 4) + align256((min(T*k, E) + 1 + 2) * 4)
+ * bytes of it (the intermediates, then the per-slot counters and two words a
+ * grid barrier may use; at I = 512, k = 10: up to 46 tokens) and returns
+ * MOE_ERR_UNSUPPORTED, enqueueing nothing, when that exceeds the array or
+ * when the batch's shared-memory layout leaves the streaming kernel no room
+ * for a tile (the same check as moe_expert_ffn_tiered in MOE_FFN_GEMV mode).
  * Arguments, outputs and results are those of moe_expert_ffn_tiered in
  * MOE_FFN_GEMV mode.  It allocates nothing: it clears the counters with an
  * asynchronous memset on `stream` and launches the streaming kernel.

@@ -625,29 +625,31 @@ static __device__ __align__(256) unsigned char moe_static_scratch[MOE_STATIC_SCR
 
 namespace {
 
-std::once_flag g_scratch_once[kMaxDevices];
-void *g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::atomic<void *> g_scratch_ptr[kMaxDevices];
+std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device, looked up on the
-// first call per device (which therefore must not run under stream capture).
+// Device address of the scratch array on the current device.  Only a
+// successful lookup is kept: a failed one (say under stream capture, or with
+// an error pending) is reported and tried again by the next call.
 int static_scratch(char **ptr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d", dev);
-    std::call_once(g_scratch_once[dev], [dev]() {
-        void *p = nullptr;
-        cudaError_t r = cudaGetSymbolAddress(&p, moe_static_scratch);
-        if (r != cudaSuccess) {
-            cudaGetLastError();
-            p = nullptr;
+    void *p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            const cudaError_t r = cudaGetSymbolAddress(&p, moe_static_scratch);
+            if (r != cudaSuccess || !p) {
+                cudaGetLastError();
+                return cuda_fail(r != cudaSuccess ? r : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
+            }
+            g_scratch_ptr[dev].store(p, std::memory_order_release);
         }
-        g_scratch_err[dev] = r;
-        g_scratch_ptr[dev] = p;
-    });
-    if (g_scratch_err[dev] != cudaSuccess) return cuda_fail(g_scratch_err[dev], "cudaGetSymbolAddress(scratch)");
-    *ptr = static_cast<char *>(g_scratch_ptr[dev]);
+    }
+    *ptr = static_cast<char *>(p);
     return MOE_OK;
 }
 
@@ -678,6 +680,13 @@ extern "C" int moe_expert_ffn_tiered_static(const moe_layer_weights *w, const ui
     r = ensure_configured();
     if (r) return r;
     if (!moe_ffn_stream_supported(w->H, w->I)) return fail(MOE_ERR_UNSUPPORTED, "GEMV path supports H, I <= 2048");
+    {
+        const long ma = static_cast<long>(T) * k;
+        const int max_slots = static_cast<int>(ma < w->E ? ma : w->E) + 1;
+        if (!moe_ffn_stream_fits(w->H, w->I, T, k, w->E, max_slots))
+            return fail(MOE_ERR_UNSUPPORTED, "GEMV path: shared memory for T = %d, k = %d leaves no room for a tile",
+                        T, k);
+    }
     char *ws = nullptr;
     r = static_scratch(&ws);
     if (r) return r;

@@ -99,17 +99,20 @@ def test_decode_stack_teacher_forced_and_free_running(decode_stack):
 
 
 def test_decode_stack_eight_tokens_batch_invariant(decode_stack):
-    """The 8-token decode batch: each token's result equals its 1-token run
+    """The 8-token decode batch: every token's result equals its 1-token run
     (GEMV path), so the 1-token oracle comparison above covers it."""
     cfg, layers = decode_stack
     xs = inputs.activations(8, cfg.H, seed=inputs.X_SEED + 1, device=DEV)
     g_x, g_n = xs.clone(), B.rmsnorm(xs)
-    one_x, one_n = xs[3:4].clone(), B.rmsnorm(xs[3:4].contiguous())
-    for l in range(min(STACK_LAYERS, 8)):
+    ones = [(xs[t:t + 1].clone(), B.rmsnorm(xs[t:t + 1].contiguous())) for t in range(8)]
+    for l in range(min(STACK_LAYERS, 6)):
         wr, bias = inputs.router(cfg, inputs.layer_seed(cfg, l), DEV)
         _, g_x, g_n = B.layer_forward(layers[l], wr, bias, g_n, cfg.k, residual=g_x, mode=B.FFN_GEMV)
-        _, one_x, one_n = B.layer_forward(layers[l], wr, bias, one_n, cfg.k, residual=one_x, mode=B.FFN_GEMV)
-        assert torch.equal(g_x[3:4], one_x)
+        for t in range(8):
+            one_x, one_n = ones[t]
+            _, one_x, one_n = B.layer_forward(layers[l], wr, bias, one_n, cfg.k, residual=one_x, mode=B.FFN_GEMV)
+            ones[t] = (one_x, one_n)
+            assert torch.equal(g_x[t:t + 1], one_x), (l, t)
 
 
 @pytest.mark.parametrize("T", [1, 2, 5, 16, 64, 256])
@@ -129,29 +132,26 @@ def test_token_sweep_one_layer(decode_stack, T):
 
 
 def test_verify_batch_correlated_drafts(decode_stack):
-    """1 base token + 4 correlated drafts through the stack: the base token is
-    compared with the oracle at every layer (drafts only share experts)."""
+    """1 base token + 4 correlated drafts through the stack, every token on the
+    oracle's own layer inputs: all five tokens' outputs and routing match the
+    oracle at every layer, and the drafts share most of the base token's
+    experts."""
     cfg, layers = decode_stack
-    xs = inputs.correlated_activations(5, cfg.H, device=DEV)
-    x = xs[0:1].float().cpu().numpy()
+    xs = inputs.correlated_activations(inputs.VERIFY_T, cfg.H, device=DEV)
+    x = xs.float().cpu().numpy()
     n = oracle.rms_norm(x).astype(np.float32)
-    g_x = xs.clone()
-    g_n = B.rmsnorm(xs)
     overlaps = []
-    for l in range(min(STACK_LAYERS, 12)):
+    for l in range(min(STACK_LAYERS, 6)):
         seed = inputs.layer_seed(cfg, l)
         ox = Hh.OracleExperts(cfg, seed, DEV)
         res, wrn, bn = _oracle_layer(cfg, seed, n, x, ox)
         wr, bias = inputs.router(cfg, seed, DEV)
-        # drafts run on their own GPU chain, the base token on the oracle's input
-        g_n[0:1] = _bf16(n)
-        g_x[0:1] = _bf16(x)
-        out, g_x, g_n = B.layer_forward(layers[l], wr, bias, g_n, cfg.k, residual=g_x)
-        _check_layer_outputs(out[0:1], res, wrn, bn, n)
+        out, _, _ = B.layer_forward(layers[l], wr, bias, _bf16(n), cfg.k, residual=_bf16(x))
+        idx, w, _ = B.router_topk(_bf16(n), wr, bias, cfg.k)
+        d = idx.cpu().numpy()
+        _check_layer_outputs(out, res, wrn, bn, n, got_idx=d, got_w=w.cpu().numpy())
+        overlaps += [len(set(d[0]) & set(d[t])) / cfg.k for t in range(1, inputs.VERIFY_T)]
         x, n = res["x_next"].astype(np.float32), res["n_next"].astype(np.float32)
-        d_idx, _, _ = B.router_topk(g_n, wr, bias, cfg.k)
-        d = d_idx.cpu().numpy()
-        overlaps += [len(set(d[0]) & set(d[t])) / cfg.k for t in range(1, 5)]
     assert 0.3 < np.mean(overlaps) < 0.9
 
 
@@ -172,8 +172,9 @@ def test_prefill_layer_4096_tokens():
     assert status.item() == 0
     wrn, bn = wr.float().cpu().numpy(), bias.cpu().numpy()
     L = oracle.router_logits(nn, wrn, bn)
-    cert, near = Hh.check_routing(idx.cpu().numpy(), w.cpu().numpy(), L, cfg.k, Hh.logit_error_bound(nn, wrn, bn))
-    assert cert > 0.5 * T
+    bound = Hh.logit_error_bound(nn, wrn, bn, Hh.TENSOR_CORE_ROUTER_FACTOR)
+    cert, near = Hh.check_routing(idx.cpu().numpy(), w.cpu().numpy(), L, cfg.k, bound)
+    Hh.assert_few_near_ties(near, T, 0.15, "prefill router")
     # token -> expert lists: every slot once, counts sum to T*k, some experts carry hundreds of tokens
     off, srt, pos, act = B.bucketize(idx, cfg.E)
     off = off.cpu().numpy()

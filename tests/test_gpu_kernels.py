@@ -84,10 +84,12 @@ def test_router_topk_matches_oracle(cfg, T):
     xn, wn = x.float().cpu().numpy(), wr.float().cpu().numpy()
     bn = None if bias is None else bias.cpu().numpy()
     L = oracle.router_logits(xn, wn, bn)
-    bound = Hh.logit_error_bound(xn, wn, bn)
+    tensor = T >= 64  # logits on the tensor cores
+    bound = Hh.logit_error_bound(xn, wn, bn, Hh.TENSOR_CORE_ROUTER_FACTOR if tensor else 1.0)
     assert np.all(np.abs(logits.cpu().numpy() - L) <= bound)
     cert, near = Hh.check_routing(idx.cpu().numpy(), w.cpu().numpy(), L, cfg.k, bound)
-    assert cert + near == T and cert >= 0.5 * T
+    assert cert + near == T
+    Hh.assert_few_near_ties(near, T, 0.15 if tensor else 0.1, f"router T={T}")
     # the ids come from the GPU's own logits by the exact top-k rule
     oi, _ = oracle.select_topk(logits.cpu().numpy().astype(np.float64), cfg.k)
     assert np.array_equal(idx.cpu().numpy(), oi)
@@ -247,10 +249,10 @@ def test_layer_tiny_tier_split_is_bit_identical():
     three = B.build_layer(cfg, seed, DEV, tier_ranges=[(8, 0, 5), (8, 5, 2), (8, 7, 9)])
     x = inputs.activations(8, cfg.H, seed=seed, device=DEV)
     wr, bias = inputs.router(cfg, seed, DEV)
-    for mode in (B.FFN_GEMV,):
+    for mode in (B.FFN_GEMV, B.FFN_GEMM, B.FFN_AUTO):
         a = B.layer_forward(one, wr, bias, x, cfg.k, mode=mode)
         b = B.layer_forward(three, wr, bias, x, cfg.k, mode=mode)
-        assert torch.equal(a, b)
+        assert torch.equal(a, b), mode
 
 
 def test_layer_tiny_edge_token_counts():

@@ -66,7 +66,8 @@ def test_route_against_oracle(T):
     L = oracle.router_logits(xn, wn, bn)
     bound = Hh.logit_error_bound(xn, wn, bn)
     cert, near = Hh.check_routing(idx.cpu().numpy(), w.cpu().numpy(), L, cfg.k, bound)
-    assert cert + near == T and cert >= 0.5 * T
+    assert cert + near == T
+    Hh.assert_few_near_ties(near, T, 0.1, f"fused route T={T}")
     o_off, o_srt, o_pos = oracle.bucketize(idx.cpu().numpy(), cfg.E)
     assert np.array_equal(off.cpu().numpy(), o_off)
     assert np.array_equal(srt.cpu().numpy(), o_srt)

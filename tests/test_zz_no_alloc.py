@@ -7,7 +7,8 @@ front): its scratch is one array inside the library, shared by every call on a
 device, so each call finds the previous call's intermediates and counters
 there and must clear what has to start at zero.  The GPU test makes two calls
 in a row with different tokens and routing on one stream and checks both
-against moe_expert_ffn_tiered in GEMV mode.
+against moe_expert_ffn_tiered in GEMV mode, bit for bit, up to the largest
+decode batch the array holds (46 tokens at I = 512, k = 10).
 
 The file name sorts last, so pytest collects it after the other tests; it
 passes alone in a fresh process (where its first call does the per-device
@@ -20,7 +21,6 @@ import torch
 
 from mixed_precision_moe_router_b200 import binding as B
 from mixed_precision_moe_router_b200 import inputs
-from tests import helpers as Hh
 
 DEV = "cuda"
 
@@ -32,7 +32,7 @@ def _routing(cfg, T, seed):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name,T", [("tiny", 8), ("decode", 1), ("decode", 8)])
+@pytest.mark.parametrize("name,T", [("tiny", 8), ("decode", 1), ("decode", 8), ("decode", 46)])
 def test_static_call_matches_workspace_call_twice_in_a_row(name, T):
     cfg = {"tiny": inputs.TINY, "decode": inputs.DECODE}[name]
     seed = inputs.layer_seed(cfg)
@@ -50,12 +50,12 @@ def test_static_call_matches_workspace_call_twice_in_a_row(name, T):
             for x, (off, srt, pos, act) in batches]
     torch.cuda.synchronize()
     assert status.item() == 0
+    # the same kernel on the same inputs sums in the same order: any stale
+    # intermediate or counter left by the first call would show as a difference
     for (ys, yshs), (yw, yshw) in zip(got, want):
         assert torch.isfinite(ys).all()
-        assert Hh.rel_l2(ys.cpu().numpy(), yw.cpu().numpy()) < Hh.REL_L2
-        assert Hh.max_abs(ys.cpu().numpy(), yw.cpu().numpy()) < Hh.MAX_ABS
-        assert Hh.rel_l2(yshs.cpu().numpy(), yshw.cpu().numpy()) < Hh.REL_L2
-        assert Hh.max_abs(yshs.cpu().numpy(), yshw.cpu().numpy()) < Hh.MAX_ABS
+        assert torch.equal(ys, yw)
+        assert torch.equal(yshs, yshw)
 
 
 def test_static_call_rejects_batches_beyond_its_scratch():
