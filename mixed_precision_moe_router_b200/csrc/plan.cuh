@@ -17,7 +17,7 @@
 namespace moe {
 
 constexpr int kTokPerPass = 8;               // gate_up token columns per pass over a resident tile
-constexpr long long kTileFixedCost = 65536;  // per-tile share of waits, hand-offs and epilogue
+constexpr long long kTileFixedCost = 4000;  // per-tile waits and hand-offs (tenths of a ns, as tile_cost)
 
 // Rows per tile are 16R: the largest power of two R <= 8 with 2RK <= 2048, so
 // a tile holds at most 32K weights.
@@ -38,14 +38,24 @@ __host__ __device__ __forceinline__ int tiles_per_slot(int H, int I, int phase) 
     return phase == 0 ? I / (8 * rows_pow2(H)) : H / (16 * rows_pow2(I));
 }
 
-// Balancing weight of one tile: the fixed per-tile work, its bytes, and the
-// dequantise-and-multiply work of each pass (3-bit codes take the most).
+// Balancing weight of one tile, in tenths of a nanosecond of its CTA's time:
+// a fixed share for waits and hand-offs, then the larger of the time to copy
+// its bytes at an even share of HBM (about 44 GB/s per SM) and its dequantise-
+// and-multiply time for every pass.  The two compute groups work side by
+// side, so a tile occupies the CTA for half of one group's time, which was
+// measured on B200 per 32K-weight tile and pass as 1.42 / 1.50 / 2.30 us for
+// gate_up and 1.36 / 1.38 / 1.72 us for down with 8- / 4- / 3-bit codes.
 __host__ __device__ __forceinline__ long long tile_cost(int H, int I, int phase, int bits, int count) {
     const int K = phase == 0 ? H : I;
     const long long rows = 16 * rows_pow2(K);
     const int tp = tokens_per_pass(phase, I);
     const long long passes = (count + tp - 1) / tp;
-    return kTileFixedCost + rows * (K * bits / 8 + K / 16) + passes * (rows * K / 3) * (bits == 3 ? 3 : 2);
+    const long long bytes = rows * (K * bits / 8 + K / 16);
+    const long long copy = bytes * 227 / 1000;
+    const long long per_tile = phase == 0 ? (bits == 8 ? 14200 : (bits == 4 ? 15000 : 23000))
+                                          : (bits == 8 ? 13600 : (bits == 4 ? 13800 : 17200));
+    const long long compute = passes * per_tile * rows * K / (2 * 32768);
+    return kTileFixedCost + (copy > compute ? copy : compute);
 }
 
 // What the schedule needs to know about a layer and a call (no device pointers).
