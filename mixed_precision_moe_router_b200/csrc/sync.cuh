@@ -152,17 +152,17 @@ __device__ __forceinline__ bool wait_geq_backoff(const int *ctr, int target) {
     return true;
 }
 
-// Spin until *ctr >= target (acquire), with backoff; false once *abort is
-// set or after `limit` cycles.
+// Spin until *ctr >= target (acquire); false once *abort is set or after
+// `limit` cycles.  The polling thread has nothing else to do, so it polls at
+// the L2 round-trip rate with a short pause: a longer backoff would add its
+// own length to the dependency it waits for.
 __device__ __forceinline__ bool wait_geq_abortable(const int *ctr, int target, const volatile int *abort,
                                                    long long limit) {
     if (ld_acquire(ctr) >= target) return true;
     const long long t0 = clock64();
-    unsigned ns = 32;
     while (ld_acquire(ctr) < target) {
         if (*abort || clock64() - t0 > limit) return false;
-        __nanosleep(ns);
-        if (ns < 512) ns *= 2;
+        __nanosleep(32);
     }
     return true;
 }
