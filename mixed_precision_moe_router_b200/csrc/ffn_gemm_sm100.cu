@@ -7,7 +7,7 @@
 //
 // Orientation: the expert's weight rows are the MMA M side (128 rows per
 // tile) and the expert's tokens the N side (padded to a multiple of 16, at most
-// 256 per accumulator), so an expert with few tokens wastes at most 15 columns.
+// 128 per accumulator), so an expert with few tokens wastes at most 15 columns.
 //   gate_up:  D[row, tok] = W_gu[row] . x[tok],  rows interleaved gate/up so a
 //             thread and its neighbour lane hold g and u of the same pair;
 //             epilogue h = silu(g) * u written as fp16 in expert-grouped order.
@@ -17,16 +17,18 @@
 //
 // Warp roles (480 threads, one CTA per SM, persistent over tiles):
 //   warps 0-7  dequant: thread (warp w, lane l) owns tile row 32*(w%4)+l, which
-//              is the tensor-memory lane its warp may access, and half of each
-//              64-wide K chunk; its packed codes and scales stream through a
-//              4-deep cp.async ring in shared memory, are converted with packed
-//              half2 arithmetic and stored straight into tensor memory
-//              (tcgen05.st), where the MMA reads its A operand.
+//              is the tensor-memory lane its warp may access, and one 64-wide
+//              half (w/4) of each 128-wide K chunk (BK); its packed codes and
+//              scales stream through a RAW-deep (4) cp.async ring in shared
+//              memory, are converted with packed half2 arithmetic and stored
+//              straight into tensor memory (tcgen05.st), where the MMA reads
+//              its A operand (STAGES = 4 stages of BK/2 columns).
 //   warps 8-11 epilogue: tcgen05.ld of their 32 accumulator lanes.
 //   warps 12-13 token rows: cp.async gather of fp16 rows into 128B-swizzled
-//              K-major shared memory (zero-filled past the expert's last token).
-//   warp  14   allocates 512 TMEM columns (two 128-column accumulators, then the
-//              A stages); lane 0 issues tcgen05.mma and tcgen05.commit.
+//              K-major shared memory, BK wide per stage (zero-filled past the
+//              expert's last token).
+//   warp  14   allocates 512 TMEM columns (two MAXN = 128-column accumulators,
+//              then the A stages); lane 0 issues tcgen05.mma and tcgen05.commit.
 #include "common.cuh"
 #include "ffn.cuh"
 #include "sync.cuh"
@@ -392,8 +394,9 @@ __device__ __forceinline__ void fail(const Params &P, const Shared &S) {
 // ---------------------------------------------------------------------------
 // roles
 // ---------------------------------------------------------------------------
-// Dequant producer: threads 2r and 2r+1 stream the two 32-weight halves of
-// row r of every tile's 64-wide K chunk.
+// Dequant producer: lane l of warps w and w + 4 (w < 4) owns tile row
+// 32*w + l, each streaming one 64-weight half (two 32-weight blocks) of every
+// tile's 128-wide K chunk.
 __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, int total_tiles, uint32_t tmem) {
     const int tid = threadIdx.x;  // 0..255
     const int warp = tid >> 5, lane = tid & 31;
