@@ -1561,7 +1561,15 @@ struct __align__(64) StackLayer {
     moe_layer_weights w;
     const uint16_t *wr;
     const float *bias;
+    PlanShelves shelves;                // the schedule's view of w, prepared on the host
+    TierPtrs tp[MOE_MAX_TIERS + 1];     // the shelves' table pointers, shared expert last
 };
+
+// Copy n 4-byte words from global to shared memory, one word per thread.
+__device__ __forceinline__ void copy_words(void *dst, const void *src, int n) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        static_cast<int *>(dst)[i] = __ldg(static_cast<const int *>(src) + i);
+}
 
 struct StackParams {
     const StackLayer *layers;
@@ -1698,13 +1706,18 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
         const StackLayer &Ld = P.layers[l];
         const uint16_t *xl = l == 0 ? P.x_in : P.xbuf + static_cast<size_t>((l - 1) & 1) * T * H;
         uint16_t *xn = l + 1 == P.n_layers ? P.x_out : P.xbuf + static_cast<size_t>(l & 1) * T * H;
-        // this layer's weights descriptor into shared memory (every thread a word)
+        // the residual stream entering the layer (in flight while the
+        // descriptor below is read)
+        for (int c = threadIdx.x; c < T * H / 8; c += blockDim.x)
+            cp_async_16b(x_s + 8 * c, xl + 8 * static_cast<size_t>(c));
+        // this layer's weights descriptor, the schedule's view of its shelves and
+        // their table pointers into shared memory (a word per thread, one round)
         {
-            const int *src = reinterpret_cast<const int *>(&Ld.w);
-            int *dst = reinterpret_cast<int *>(&p.w);
-            for (int w = threadIdx.x; w < static_cast<int>(sizeof(moe_layer_weights) / sizeof(int)); w += blockDim.x)
-                dst[w] = __ldg(src + w);
+            copy_words(&p.w, &Ld.w, sizeof(moe_layer_weights) / sizeof(int));
+            copy_words(p.pi.shelves(), &Ld.shelves, sizeof(PlanShelves) / sizeof(int));
+            copy_words(S.tp, Ld.tp, sizeof(Ld.tp) / sizeof(int));
             if (threadIdx.x == 0) {
+                p.has_shared = __ldg(&Ld.shelves.has_shared);
                 p.route.wr = Ld.wr;
                 p.route.bias = Ld.bias;
                 for (int t = 0; t <= MOE_MAX_TIERS; ++t) {
@@ -1713,24 +1726,8 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
                 }
             }
         }
-        // the residual stream entering the layer
-        for (int c = threadIdx.x; c < T * H / 8; c += blockDim.x)
-            cp_async_16b(x_s + 8 * c, xl + 8 * static_cast<size_t>(c));
         cp_async_wait_all();
         __syncthreads();
-        if (threadIdx.x == 0) {
-            p.has_shared = p.w.shared.n_experts == 1;
-            PlanIn &pi = p.pi;
-            pi.n_tiers = p.w.n_tiers;
-            pi.has_shared = p.has_shared;
-            pi.shared_bits = p.w.shared.bits;
-            for (int t = 0; t < MOE_MAX_TIERS; ++t) {
-                pi.first[t] = t < p.w.n_tiers ? p.w.tiers[t].first_expert : 0;
-                pi.n[t] = t < p.w.n_tiers ? p.w.tiers[t].n_experts : 0;
-                pi.bits[t] = t < p.w.n_tiers ? p.w.tiers[t].bits : 8;
-            }
-        }
-        fill_tier_ptrs(p.w, S);
         // normalised in place (its barriers also publish the parameters above)
         cta_rms_norm_rows(x_s, T, H, red);
         {
@@ -1845,6 +1842,20 @@ cudaError_t moe_stack_encode_layer(const moe_layer_weights *w, const uint16_t *w
     L.w = *w;
     L.wr = wr;
     L.bias = bias;
+    L.shelves.n_tiers = w->n_tiers;
+    L.shelves.has_shared = w->shared.n_experts == 1;
+    L.shelves.shared_bits = w->shared.bits;
+    for (int t = 0; t < MOE_MAX_TIERS; ++t) {
+        const bool on = t < w->n_tiers;
+        L.shelves.first[t] = on ? w->tiers[t].first_expert : 0;
+        L.shelves.n[t] = on ? w->tiers[t].n_experts : 0;
+        L.shelves.bits[t] = on ? w->tiers[t].bits : 8;
+        if (on)
+            L.tp[t] = {w->tiers[t].gu_qs, reinterpret_cast<const uint8_t *>(w->tiers[t].gu_scale), w->tiers[t].dn_qs,
+                       reinterpret_cast<const uint8_t *>(w->tiers[t].dn_scale)};
+    }
+    L.tp[w->n_tiers] = {w->shared.gu_qs, reinterpret_cast<const uint8_t *>(w->shared.gu_scale), w->shared.dn_qs,
+                        reinterpret_cast<const uint8_t *>(w->shared.dn_scale)};
     std::memcpy(dst, &L, sizeof(L));
     return cudaSuccess;
 }

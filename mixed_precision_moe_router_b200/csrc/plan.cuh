@@ -59,13 +59,20 @@ __host__ __device__ __forceinline__ long long tile_cost(int H, int I, int phase,
 }
 
 // What the schedule needs to know about a layer and a call (no device pointers).
-struct PlanIn {
-    int E, T, k, H, I;
+struct PlanShelves {  // the shelves of a layer
     int n_tiers, has_shared, shared_bits;
-    int max_count;   // slots with more tokens are left to the tensor-core path
-    int max_active;  // routed slots at most: min(E, T*k)
     int first[MOE_MAX_TIERS], n[MOE_MAX_TIERS], bits[MOE_MAX_TIERS];
 };
+struct PlanIn {
+    int E, T, k, H, I;
+    int max_count;   // slots with more tokens are left to the tensor-core path
+    int max_active;  // routed slots at most: min(E, T*k)
+    int n_tiers, has_shared, shared_bits;
+    int first[MOE_MAX_TIERS], n[MOE_MAX_TIERS], bits[MOE_MAX_TIERS];
+    // the fields from n_tiers on, as one block
+    __host__ __device__ __forceinline__ PlanShelves *shelves() { return reinterpret_cast<PlanShelves *>(&n_tiers); }
+};
+static_assert(sizeof(PlanIn) == 7 * sizeof(int) + sizeof(PlanShelves), "PlanIn ends with its shelves block");
 
 // Per-slot tables in shared memory.  tc/pre: per phase, the cost of one tile
 // of the slot and the inclusive prefix sum of the slots' total costs.
