@@ -44,7 +44,7 @@ N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
 # capture is taken again.
 STACK_SOURCES = ("csrc/ffn_stream.cu", "csrc/ffn.cuh", "csrc/plan.cuh", "csrc/route_cta.cuh", "csrc/sync.cuh",
                  "csrc/common.cuh")
-STACK_TRAFFIC = {"digest": None, "dram_bytes": None, "algorithmic_bytes": None, "layers": 4}
+STACK_TRAFFIC = {"digest": "f8b4c7810afb4e16", "dram_bytes": 119538944 + 4555776, "algorithmic_bytes": 118497280, "layers": 4}
 PREFILL_FFN_TRAFFIC = None  # the GEMM kernels changed since their last capture
 
 
