@@ -45,7 +45,10 @@ N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
 STACK_SOURCES = ("csrc/ffn_stream.cu", "csrc/ffn.cuh", "csrc/plan.cuh", "csrc/route_cta.cuh", "csrc/sync.cuh",
                  "csrc/common.cuh")
 STACK_TRAFFIC = {"digest": "f8b4c7810afb4e16", "dram_bytes": 119538944 + 4555776, "algorithmic_bytes": 118497280, "layers": 4}
-PREFILL_FFN_TRAFFIC = None  # the GEMM kernels changed since their last capture
+# The same for the prefill FFN call's two GEMM launches (gate_up and down; ncu
+# DRAM read + write of one call of the 4096-token workload).
+PREFILL_SOURCES = ("csrc/ffn_gemm_sm100.cu", "csrc/ffn.cuh", "csrc/plan.cuh", "csrc/sync.cuh", "csrc/common.cuh")
+PREFILL_TRAFFIC = {"digest": "0be2e99b13526a72", "dram_bytes": 765743104 + 39737856 + 391481600 + 315155712}
 
 
 def source_digest(files):
@@ -273,7 +276,9 @@ def run_prefill(args, rank, world):
                    "l2": "inputs larger than L2: every expert of the layer (~0.6 GB) is read each step"},
         "roofline": {"bound": "tensor", "kernel": "expert FFN call (f16 staging + gate_up GEMM + down GEMM)",
                      "achieved": round(pf["tflops"], 1), "peak": tf, "unit": "TFLOP/s",
-                     "frac": round(pf["tflops"] / tf, 4), "traffic": PREFILL_FFN_TRAFFIC, "peak_kind": peak_kind + " burst",
+                     "frac": round(pf["tflops"] / tf, 4),
+                     "traffic": PREFILL_TRAFFIC["dram_bytes"]
+                     if PREFILL_TRAFFIC["digest"] == source_digest(PREFILL_SOURCES) else None, "peak_kind": peak_kind + " burst",
                      "algorithmic_flops_per_launch": pf["flops"], "avg_launch_us": round(pf["ffn_ms"] * 1e3, 1)},
         "gpu_launches": max(args.steps, 3) * 8,
         "clocks": clk.summary(),
