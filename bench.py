@@ -495,7 +495,66 @@ def other_workloads(args, layers, routers, stream, rank):
                       "frac_hbm": round(fp["gbs"] / hbm, 4), "tflops": round(fp["tflops"], 2),
                       "frac_bf16": round(fp["tflops"] / tf, 4), "touched_mb": round(fp["bytes"] / 1e6, 2)})
     res["sweep_one_layer_ffn"] = sweep
+    res["tier_planner"] = tier_planner_curve(layers[0], routers[0], stream)
     return res
+
+
+def tier_planner_curve(layer0, router, stream, fractions=(0.75, 1.0, 1.3, 1.6)):
+    """The tier planner's speed/size curve on the decode configuration: expert
+    use from routing 4096 synthetic tokens through layer 0's router, the
+    expected error per precision from the library's own quantiser on one
+    expert (the synthetic experts share one weight distribution), a plan at
+    each byte budget (a fraction of the configured 128/192/192 shelves), and
+    that plan's layer built (experts renumbered so that each shelf is one
+    contiguous id range) and its one-token FFN call timed, next to the
+    configured shelves' own."""
+    from mixed_precision_moe_router_b200 import binding as B
+    from mixed_precision_moe_router_b200 import ep, planner
+    cfg = inputs.DECODE
+    dev = torch.device("cuda", torch.cuda.current_device())
+    seed = inputs.layer_seed(cfg, 0)
+    wr, bias = router
+    xs = inputs.activations(4096, cfg.H, seed=inputs.X_SEED + 77, device=dev)
+    idx, _, _ = B.router_topk(B.rmsnorm(xs), wr, bias, cfg.k)
+    freq = torch.bincount(idx.reshape(-1).long(), minlength=cfg.E).double().cpu().numpy()
+    freq = list(freq / freq.sum())
+    wgu, wdn = inputs.expert_source(cfg, seed, 0, dev)
+    sq = {}
+    for b in planner.BITS:
+        tot = 0.0
+        for w in (wgu.contiguous(), wdn.contiguous()):
+            qs, sc = B.quantize(w, b)
+            back, _ = B.dequantize(qs, sc, w.shape[1], b)
+            tot += float(((back - w).double() ** 2).sum())
+        sq[b] = tot
+    err = [dict(sq) for _ in range(cfg.E)]
+    nb = {b: ep.expert_bytes(cfg.H, cfg.I, b) for b in planner.BITS}
+    configured = [b for b, f, n in cfg.tier_ranges() for _ in range(n)]
+    ref_bytes, ref_err = planner.plan_bytes(configured, nb), planner.expected_error(configured, freq, err)
+    tokens = [inputs.activations(1, cfg.H, seed=inputs.X_SEED + 500 + i, device=dev) for i in range(8)]
+    out = []
+    for frac in fractions:
+        plan = planner.plan_tiers(freq, err, nb, frac * ref_bytes)
+        order, shelves = planner.shelves_from_bits(plan)
+        row = {"budget_gb": round(frac * ref_bytes / 1e9, 3), "layer_gb": round(planner.plan_bytes(plan, nb) / 1e9, 3),
+               "shelves": {f"{b}-bit": n for b, _, n in shelves},
+               "expected_error_vs_configured": round(planner.expected_error(plan, freq, err) / ref_err, 4)}
+        # shelves are contiguous id ranges: expert e of the planned layer is
+        # expert order[e] of the original one (its router row and bias move
+        # with it), so the planned layer computes what the original does
+        perm = torch.tensor(order, device=dev)
+        src = (lambda c, sd, e, d: inputs.expert_source(c, sd, order[e] if e < c.E else e, d))
+        layer = B.build_layer(cfg, seed, dev, source=src, tier_ranges=shelves)
+        prouter = (wr[perm].contiguous(), None if bias is None else bias[perm].contiguous())
+        fp = ffn_profile([layer] * len(tokens), [prouter] * len(tokens), tokens, stream)
+        row.update({"ffn_us_T1": round(fp["ms"] * 1e3, 2), "touched_mb_T1": round(fp["bytes"] / 1e6, 2),
+                    "permuted_ids": order != list(range(cfg.E))})
+        del layer
+        out.append(row)
+    fp = ffn_profile([layer0] * len(tokens), [router] * len(tokens), tokens, stream)
+    return {"configured": {"layer_gb": round(ref_bytes / 1e9, 3), "shelves": {f"{b}-bit": n for b, _, n in cfg.tier_ranges()},
+                           "ffn_us_T1": round(fp["ms"] * 1e3, 2), "touched_mb_T1": round(fp["bytes"] / 1e6, 2)},
+            "plans": out}
 
 
 class OracleStack:

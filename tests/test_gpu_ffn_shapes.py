@@ -85,3 +85,32 @@ def test_streaming_ffn_largest_tables_sampled():
         assert Hh.rel_l2(y[s], exp) < 1e-5, s
     esh = oracle.expert_ffn(xn, *ox.shared())
     assert Hh.rel_l2(ysh.cpu().numpy(), esh) < 1e-5
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", [B.FFN_GEMV, B.FFN_GEMM])
+def test_down_width_640_matches_oracle(mode):
+    """I = 640, the down width the pages' model has ([P1] "step 4": rows 640
+    wide): 20 scale blocks per down row (3-bit rows of 240 bytes, staged in
+    16-byte columns; scale rows of 40 bytes, staged as bulk copies) through the
+    streaming and the tensor-core paths, against the oracle."""
+    cfg = LayerConfig("i640", H=2048, I=640, E=16, k=2, tiers=((8, 4), (4, 6), (3, 6)))
+    T, seed = 8, 640
+    layer = B.build_layer(cfg, seed, DEV)
+    x = inputs.activations(T, cfg.H, seed=seed, device=DEV)
+    ids = torch.stack([torch.randperm(cfg.E, generator=torch.Generator().manual_seed(31 + t))[: cfg.k]
+                       for t in range(T)]).to(torch.int32).to(DEV)
+    off, srt, pos, act = B.bucketize(ids, cfg.E)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y, ysh = B.expert_ffn(layer, x, cfg.k, off, srt, act, mode=mode, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ox = Hh.OracleExperts(cfg, seed, DEV)
+    xn = x.float().cpu().numpy()
+    idn = ids.cpu().numpy().reshape(-1)
+    exp = np.stack([oracle.expert_ffn(xn[s // cfg.k: s // cfg.k + 1], *ox(int(idn[s])))[0]
+                    for s in range(T * cfg.k)])
+    esh = oracle.expert_ffn(xn, *ox.shared())
+    tol = 1e-5 if mode == B.FFN_GEMV else Hh.REL_L2  # exact products vs fp16-staged tensor-core operands
+    assert Hh.rel_l2(y.cpu().numpy(), exp) < tol
+    assert Hh.rel_l2(ysh.cpu().numpy(), esh) < tol
