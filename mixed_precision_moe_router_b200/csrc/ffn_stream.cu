@@ -252,7 +252,9 @@ __device__ __forceinline__ TileAcc warp_tile(const uint8_t *stage, const Geo G, 
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-#pragma unroll 2
+    // one pair of blocks per iteration: a larger unroll measured slower, its
+    // extra code competing with the other roles' for the instruction cache
+#pragma unroll 1
     for (int b = b0; b < b1; b += 2) {
         const float2 da = half2_to_float2(*reinterpret_cast<const uint32_t *>(scl + rA * G.sb + ((2 * b) ^ sxa)));
         const float2 db = half2_to_float2(*reinterpret_cast<const uint32_t *>(scl + rB * G.sb + ((2 * b) ^ sxb)));
