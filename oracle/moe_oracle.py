@@ -155,6 +155,82 @@ def quantize_pack(w, bits: int):
 
 
 # ---------------------------------------------------------------------------
+# FP4 (E2M1) shelf.  [P1] "step 4" stores the rarest down projections as
+# MXFP4: a 4-bit floating-point code per weight and a power-of-two scale per
+# block of 32 weights.
+# READING (the pages name the format only): the OCP MX conversion.  The block's
+# shared scale is X = 2^(floor(log2 amax) - 2) (2 = the largest exponent of
+# E2M1, so amax / X lies in [4, 8)); each weight becomes w / X rounded to the
+# nearest E2M1 value (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the even
+# code, saturating at 6; a weight that rounds to 0 keeps code 0.  In the shelf
+# format the nibbles are packed as the 4-bit codes are (code = sign * 8 +
+# magnitude index) and the fp16 scale array holds d = X / 2, so that
+# w = d * q with the integer q = 2 * value(code) in {0, +-1, +-2, +-3, +-4, +-6,
+# +-8, +-12}; d is a power of two kept within fp16's exact range [2^-24, 2^15]
+# (the block exponent is raised or lowered to it), and d = 0 for a zero block.
+# ---------------------------------------------------------------------------
+
+FP4_VALUES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)  # E2M1 magnitude of index 0..7
+
+
+def quantize_rows_fp4(w):
+    """fp32 rows -> (codes uint8 [R,K] in 0..15, scales d fp16 [R,K/32])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    R, K = w.shape
+    assert K % BLOCK == 0
+    blocks = w.reshape(R, K // BLOCK, BLOCK).astype(np.float64)
+    amax = np.abs(blocks).max(axis=2)
+    _, e = np.frexp(amax)                    # amax = f * 2^e, f in [0.5, 1): floor(log2 amax) = e - 1
+    shared = np.clip(e - 1 - 2, -23, 16)     # d = 2^(shared - 1) within [2^-24, 2^15]
+    X = np.ldexp(1.0, shared)[..., None]
+    v = blocks / X                           # exact: a power-of-two divisor
+    a = np.abs(v)
+    vals = np.asarray(FP4_VALUES)
+    dist = np.abs(a[..., None] - vals)       # exact differences of short binary fractions
+    m = np.argmin(dist, axis=-1)             # the first (lower) index on a tie ...
+    nxt = np.minimum(m + 1, 7)
+    tie = (np.take_along_axis(dist, nxt[..., None], -1)[..., 0] == np.take_along_axis(dist, m[..., None], -1)[..., 0]) & (nxt != m)
+    m = np.where(tie & (m % 2 == 1), nxt, m)  # ... moved to the even index
+    code = m + np.where((v < 0) & (m > 0), 8, 0)
+    code = np.where(amax[..., None] == 0, 0, code)
+    d = np.where(amax == 0, 0.0, np.ldexp(1.0, shared - 1)).astype(np.float16)
+    return code.reshape(R, K).astype(np.uint8), d
+
+
+def fp4_integers(codes):
+    """Codes 0..15 -> the integers q = 2 * value (sign from bit 3)."""
+    c = np.asarray(codes, np.int64)
+    mag = (2 * np.asarray(FP4_VALUES))[c & 7]
+    return np.where(c & 8, -mag, mag).astype(np.int64)
+
+
+def pack_rows_fp4(codes):
+    """Nibbles as in the 4-bit shelf: weight 2m low, 2m+1 high in byte m."""
+    c = np.asarray(codes, np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_rows_fp4(packed, K: int):
+    p = np.asarray(packed, np.uint8)
+    c = np.empty((p.shape[0], K), np.uint8)
+    c[:, 0::2] = p & 0xF
+    c[:, 1::2] = p >> 4
+    return c
+
+
+def dequantize_fp4_f32(packed, scale, K: int):
+    """w = float(d) * float(q); exact in fp32 (a power of two times |q| <= 12)."""
+    q = fp4_integers(unpack_rows_fp4(packed, K)).astype(np.float32)
+    d = np.repeat(np.asarray(scale, np.float16).astype(np.float32), BLOCK, axis=1)
+    return d * q
+
+
+def quantize_pack_fp4(w):
+    c, d = quantize_rows_fp4(w)
+    return pack_rows_fp4(c), d
+
+
+# ---------------------------------------------------------------------------
 # Router: logits, top-k, weights
 # [P1] "a small dictionary before we start": each layer has 512 experts and a
 # router picks the best 10 for each word.  [P5] "What the model actually is":

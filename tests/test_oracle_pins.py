@@ -513,3 +513,61 @@ def test_moe_stack_layers_read_the_normalised_stream():
     assert np.array_equal(b["x_next"], oracle.round_bf16(32.0 * x + b["out"]))
     raw = oracle.moe_layer(x * 32.0, wr, bias, cfg.k, lookup, sw, cfg.H, cfg.I)
     assert not np.array_equal(raw["out"], a["out"])
+
+
+# ---------------------------------------------------------------------------
+# FP4 (E2M1) shelf: codes and scales derived by hand from the format (OCP MX:
+# shared scale X = 2^(floor(log2 amax) - 2), nearest E2M1 value, ties to the
+# even code, saturation at 6; stored as d = X / 2 and q = 2 * value)
+# ---------------------------------------------------------------------------
+
+def test_fp4_hand_derived_block():
+    # amax = 3.0: floor(log2 3) = 1, X = 2^-1, v = 2w, d = 0.25
+    w = np.zeros((1, 32), np.float32)
+    w[0, :10] = [3.0, 0.125, 0.375, -1.25, 2.5, 0.7, -0.1, 1.6, 2.9, -3.0]
+    # v:          6    0.25   0.75   -2.5   5    1.4   -0.2  3.2  5.8  -6
+    # nearest:    6    0|0.5  0.5|1  2|3    4|6  1.5   0     3    6    -6
+    #                  tie->0 tie->1 tie->2 tie->4
+    codes, d = oracle.quantize_rows_fp4(w)
+    assert d.tolist() == [[0.25]]
+    assert codes[0, :10].tolist() == [7, 0, 2, 12, 6, 3, 0, 5, 7, 15]
+    assert codes[0, 10:].tolist() == [0] * 22
+    assert oracle.fp4_integers(codes[0, :10]).tolist() == [12, 0, 2, -4, 8, 3, 0, 6, 12, -12]
+    back = oracle.dequantize_fp4_f32(oracle.pack_rows_fp4(codes), d, 32)[0, :10]
+    assert back.tolist() == [3.0, 0.0, 0.5, -1.0, 2.0, 0.75, 0.0, 1.5, 3.0, -3.0]
+    # the nibble order of the 4-bit shelf: weight 2m low, 2m+1 high
+    assert oracle.pack_rows_fp4(codes)[0, :2].tolist() == [7 | (0 << 4), 2 | (12 << 4)]
+
+
+def test_fp4_edge_blocks():
+    w = np.zeros((4, 32), np.float32)
+    w[0, 5] = 4.0            # amax a power of two: X = 1, d = 0.5, code 6
+    w[1, 3] = 2.0 ** -30     # below fp16's range: d = 2^-24, X = 2^-23, v = 2^-7 -> 0
+    w[3, :] = -7.9           # every weight saturates: amax/X = 7.9 / 1 -> 6
+    codes, d = oracle.quantize_rows_fp4(w)
+    assert float(d[0, 0]) == 0.5 and codes[0, 5] == 6 and codes[0].sum() == 6
+    assert float(d[1, 0]) == 2.0 ** -24 and codes[1].sum() == 0
+    assert float(d[2, 0]) == 0.0 and codes[2].sum() == 0          # a zero block
+    assert float(d[3, 0]) == 0.5 and set(codes[3].tolist()) == {15}
+    assert oracle.dequantize_fp4_f32(oracle.pack_rows_fp4(codes), d, 32)[3].tolist() == [-6.0] * 32
+
+
+def test_fp4_codes_are_the_nearest_of_all_sixteen():
+    """Brute force: at the block's scale, every weight's code gives the value
+    nearest to it among all 16 codes (ties: the even magnitude index, and 0
+    rather than -0), and the round trip is within half a grid step."""
+    rng = np.random.default_rng(11)
+    w = (rng.standard_normal((16, 64)) * rng.choice([1e-3, 0.02, 1.0, 50.0], size=(16, 1))).astype(np.float32)
+    w[0, :4] = [0.0, -0.0, 1e-9, -1e-9]
+    codes, d = oracle.quantize_rows_fp4(w)
+    grid = np.array([(1 if c < 8 else -1) * oracle.FP4_VALUES[c & 7] for c in range(16)])
+    for r in range(w.shape[0]):
+        for i in range(w.shape[1]):
+            X = 2.0 * float(d[r, i // 32])
+            v = float(w[r, i]) / X
+            dist = np.abs(grid - v)
+            best = [c for c in range(16) if dist[c] == dist.min()]
+            best = [c for c in best if c != 8] or best           # 0 rather than -0
+            even = [c for c in best if (c & 7) % 2 == 0]
+            assert codes[r, i] == (even or best)[0], (r, i, v, best)
+            assert abs(v - grid[codes[r, i]]) <= (1.0 if abs(v) <= 6 else 2.0)
