@@ -64,6 +64,7 @@ typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
 #define MOE_MAX_TOPK 32
 #define MOE_MAX_EXPERTS 1024
 #define MOE_NORM_EPS 1e-6f /* epsilon of the residual-stream RMS norm */
+#define MOE_FP4 5 /* `bits` of an FP4 (E2M1) shelf: 4-bit storage, see below */
 
 /*
  * Packed shelf format ([P1] "step 4: three shelves, all on the GPU": each
@@ -82,22 +83,39 @@ typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
  *   bits 3: c = q + 4; a low plane of K/4 bytes (bits 0-1 of weight i at bit
  *           2*(i%4) of byte i/4) followed by a high plane of K/8 bytes (bit 2
  *           of weight i at bit i%8 of byte K/4 + i/8).
+ *
+ * FP4 shelf (bits = MOE_FP4; [P1] "step 4": MXFP4 for the rarest experts'
+ * weights).  The OCP MX conversion with E2M1 elements and a power-of-two
+ * block scale, stored in the layout above with 4-bit storage (K/2 code bytes
+ * per row):
+ *   X = 2^(floor(log2 amax) - 2), clamped to [2^-23, 2^16]; amax == 0 -> d = 0,
+ *       every code 0;
+ *   v = the E2M1 value (0, 0.5, 1, 1.5, 2, 3, 4, 6, signed) nearest to w / X,
+ *       a tie to the one of even magnitude index, saturating at 6;
+ *   c = 8 * sign + m, m the magnitude index 0..7 (a zero is stored as +0);
+ *       weight 2m in the low nibble of byte m, 2m+1 in the high;
+ *   d = X / 2 (exact in fp16), q = 2 * v in {0, +-1, +-2, +-3, +-4, +-6, +-8,
+ *       +-12}, so that w = d * q as for the integer shelves.
  */
-size_t moe_packed_row_bytes(int32_t K, int32_t bits);
+size_t moe_packed_row_bytes(int32_t K, int32_t bits); /* K*bits/8, K/2 for MOE_FP4;
+                                                         0 for an invalid K or bits */
 
 /*
- * One shelf: experts [first_expert, first_expert + n_experts) at `bits`.
- * Per expert (expert j of the shelf at index j), hidden H, intermediate I:
- *   gu_qs    [n_experts][2*I][H*bits/8]   gate rows 0..I-1, up rows I..2I-1
+ * One shelf: experts [first_expert, first_expert + n_experts), gate_up at
+ * `bits` and down at `dn_bits` ([P1] "step 4": the down projections take a
+ * ladder of their own, MXFP4 on the rarest shelf).  Per expert (expert j of
+ * the shelf at index j), hidden H, intermediate I, b = bits, c = dn_bits:
+ *   gu_qs    [n_experts][2*I][H*b/8]   gate rows 0..I-1, up rows I..2I-1
  *   gu_scale [n_experts][2*I][H/32]
- *   dn_qs    [n_experts][H][I*bits/8]
+ *   dn_qs    [n_experts][H][I*c/8]
  *   dn_scale [n_experts][H][I/32]
+ * (in these sizes and in moe_quantize's, MOE_FP4 counts as 4 bits).
  */
 typedef struct moe_tier {
-    int32_t bits;          /* 8, 4 or 3 */
+    int32_t bits;          /* gate_up format: 8, 4, 3 or MOE_FP4 */
     int32_t first_expert;  /* first id of this shelf's contiguous id range */
     int32_t n_experts;     /* experts on the shelf (0 for an unused shared slot) */
-    int32_t reserved;      /* must be 0 */
+    int32_t dn_bits;       /* down format: 8, 4, 3 or MOE_FP4; 0 = same as bits */
     const uint8_t *gu_qs;
     const uint16_t *gu_scale;
     const uint8_t *dn_qs;

@@ -31,7 +31,7 @@ c_i32, c_i64, c_size, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ct
 
 
 class Tier(ctypes.Structure):
-    _fields_ = [("bits", c_i32), ("first_expert", c_i32), ("n_experts", c_i32), ("reserved", c_i32),
+    _fields_ = [("bits", c_i32), ("first_expert", c_i32), ("n_experts", c_i32), ("dn_bits", c_i32),
                 ("gu_qs", c_vp), ("gu_scale", c_vp), ("dn_qs", c_vp), ("dn_scale", c_vp)]
 
 
@@ -121,6 +121,20 @@ def _need(t, dtype, shape=None, name="tensor"):
         raise ValueError(f"{name}: shape {tuple(t.shape)}, want {tuple(shape)}")
 
 
+# `bits` of an FP4 (E2M1, power-of-two block scale) shelf; stored as 4-bit codes
+FP4 = 5
+
+
+def storage_bits(bits):
+    """Code bits per weight in memory (4 for an FP4 shelf)."""
+    return 4 if bits == FP4 else bits
+
+
+def formats(bits):
+    """(gate_up format, down format) of a shelf given as one format or a pair."""
+    return (bits, bits) if isinstance(bits, int) else (int(bits[0]), int(bits[1]))
+
+
 def packed_row_bytes(K, bits):
     return int(lib().moe_packed_row_bytes(K, bits))
 
@@ -130,10 +144,12 @@ def packed_row_bytes(K, bits):
 # ---------------------------------------------------------------------------
 
 def quantize(src, bits, out_qs=None, out_scale=None):
-    """fp32 [rows, K] -> (codes uint8 [rows, K*bits/8], fp16 scale bits int16 [rows, K/32])."""
+    """fp32 [rows, K] -> (codes uint8 [rows, K*bits/8], fp16 scale bits int16 [rows, K/32]);
+    bits 8, 4, 3 or FP4."""
     _need(src, torch.float32, name="src")
     rows, K = src.shape
-    qs = out_qs if out_qs is not None else torch.empty(rows, K * bits // 8, dtype=torch.uint8, device=src.device)
+    qs = out_qs if out_qs is not None else torch.empty(rows, K * storage_bits(bits) // 8, dtype=torch.uint8,
+                                                       device=src.device)
     sc = out_scale if out_scale is not None else torch.empty(rows, K // 32, dtype=torch.int16, device=src.device)
     _check(lib().moe_quantize(_ptr(src), rows, K, bits, _ptr(qs), _ptr(sc), _stream()))
     return qs, sc
@@ -167,10 +183,11 @@ class TieredLayer:
     @staticmethod
     def allocate(H, I, E, tier_ranges, shared_bits, device):
         def shelf(bits, first, n):
-            return dict(bits=bits, first=first, n=n,
-                        gu_qs=torch.empty(n, 2 * I, H * bits // 8, dtype=torch.uint8, device=device),
+            gu, dn = formats(bits)
+            return dict(bits=gu, dn_bits=dn, first=first, n=n,
+                        gu_qs=torch.empty(n, 2 * I, H * storage_bits(gu) // 8, dtype=torch.uint8, device=device),
                         gu_scale=torch.empty(n, 2 * I, H // 32, dtype=torch.int16, device=device),
-                        dn_qs=torch.empty(n, H, I * bits // 8, dtype=torch.uint8, device=device),
+                        dn_qs=torch.empty(n, H, I * storage_bits(dn) // 8, dtype=torch.uint8, device=device),
                         dn_scale=torch.empty(n, H, I // 32, dtype=torch.int16, device=device))
         tiers = [shelf(b, f, n) for b, f, n in tier_ranges]
         shared = shelf(shared_bits, E, 1) if shared_bits else None
@@ -188,14 +205,14 @@ class TieredLayer:
         """Quantise one expert's fp32 source weights into its shelf (on the GPU)."""
         t, j = self.shelf_of(e)
         quantize(w_gate_up.contiguous(), t["bits"], t["gu_qs"][j], t["gu_scale"][j])
-        quantize(w_down.contiguous(), t["bits"], t["dn_qs"][j], t["dn_scale"][j])
+        quantize(w_down.contiguous(), t["dn_bits"], t["dn_qs"][j], t["dn_scale"][j])
         self._desc = None
 
     def nbytes_expert(self, e):
         t, _ = self.shelf_of(e)
-        b = t["bits"]
+        gu, dn = storage_bits(t["bits"]), storage_bits(t["dn_bits"])
         rows_k = 2 * self.I * self.H + self.H * self.I
-        return rows_k * b // 8 + rows_k // 32 * 2
+        return (2 * self.I * self.H * gu + self.H * self.I * dn) // 8 + rows_k // 32 * 2
 
     def descriptor(self):
         if self._desc is None:
@@ -203,7 +220,8 @@ class TieredLayer:
             d.H, d.I, d.E, d.n_tiers = self.H, self.I, self.E, len(self.tiers)
 
             def fill(dst, t):
-                dst.bits, dst.first_expert, dst.n_experts, dst.reserved = t["bits"], t["first"], t["n"], 0
+                dst.bits, dst.first_expert, dst.n_experts = t["bits"], t["first"], t["n"]
+                dst.dn_bits = 0 if t["dn_bits"] == t["bits"] else t["dn_bits"]
                 dst.gu_qs, dst.gu_scale = t["gu_qs"].data_ptr(), t["gu_scale"].data_ptr()
                 dst.dn_qs, dst.dn_scale = t["dn_qs"].data_ptr(), t["dn_scale"].data_ptr()
             for i, t in enumerate(self.tiers):

@@ -102,13 +102,14 @@ int ensure_configured() {
     return MOE_OK;
 }
 
-bool valid_bits(int b) { return b == 8 || b == 4 || b == 3; }
+bool valid_bits(int b) { return b == 8 || b == 4 || b == 3 || b == MOE_FP4; }
 
 size_t align_up(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 int check_tier(const moe_tier &t, const char *name, int idx) {
-    if (!valid_bits(t.bits)) return fail(MOE_ERR_INVALID_ARG, "%s[%d].bits = %d (want 8, 4 or 3)", name, idx, t.bits);
-    if (t.reserved != 0) return fail(MOE_ERR_INVALID_ARG, "%s[%d].reserved must be 0", name, idx);
+    if (!valid_bits(t.bits)) return fail(MOE_ERR_INVALID_ARG, "%s[%d].bits = %d (want 8, 4, 3 or MOE_FP4)", name, idx, t.bits);
+    if (t.dn_bits != 0 && !valid_bits(t.dn_bits))
+        return fail(MOE_ERR_INVALID_ARG, "%s[%d].dn_bits = %d (want 0, 8, 4, 3 or MOE_FP4)", name, idx, t.dn_bits);
     if (!t.gu_qs || !t.gu_scale || !t.dn_qs || !t.dn_scale)
         return fail(MOE_ERR_INVALID_ARG, "%s[%d] has a NULL table pointer", name, idx);
     if (!aligned16(t.gu_qs) || !aligned16(t.gu_scale) || !aligned16(t.dn_qs) || !aligned16(t.dn_scale))
@@ -188,13 +189,13 @@ moe::FfnParams make_params(const moe_layer_weights *w, const uint16_t *x, int T,
     pi.I = w->I;
     pi.n_tiers = w->n_tiers;
     pi.has_shared = p.has_shared;
-    pi.shared_bits = w->shared.bits;
+    pi.shared_bits = moe::tier_formats(w->shared);
     pi.max_count = p.max_count;
     pi.max_active = p.max_active;
     for (int t = 0; t < w->n_tiers; ++t) {
         pi.first[t] = w->tiers[t].first_expert;
         pi.n[t] = w->tiers[t].n_experts;
-        pi.bits[t] = w->tiers[t].bits;
+        pi.bits[t] = moe::tier_formats(w->tiers[t]);
     }
     std::memset(&p.route, 0, sizeof(p.route));
     p.wait_limit = g_wait_limit.load();
@@ -249,12 +250,12 @@ const char *moe_version(void) { return "moe_tiered 0.1 (sm_100a)"; }
 
 size_t moe_packed_row_bytes(int32_t K, int32_t bits) {
     if (K <= 0 || K % 64 != 0 || !valid_bits(bits)) return 0;
-    return static_cast<size_t>(K) * bits / 8;
+    return static_cast<size_t>(K) * moe::storage_bits(bits) / 8;
 }
 
 int moe_quantize(const float *src, int64_t rows, int32_t K, int32_t bits, uint8_t *qs, uint16_t *scale,
                  moe_stream_t stream) {
-    if (!valid_bits(bits)) return fail(MOE_ERR_INVALID_ARG, "bits = %d (want 8, 4 or 3)", bits);
+    if (!valid_bits(bits)) return fail(MOE_ERR_INVALID_ARG, "bits = %d (want 8, 4, 3 or MOE_FP4)", bits);
     if (K <= 0 || K % 64 != 0) return fail(MOE_ERR_INVALID_ARG, "K = %d must be a positive multiple of 64", K);
     if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "rows = %lld", (long long)rows);
     if (rows == 0) return ok();
@@ -268,7 +269,7 @@ int moe_quantize(const float *src, int64_t rows, int32_t K, int32_t bits, uint8_
 
 int moe_dequantize(const uint8_t *qs, const uint16_t *scale, int64_t rows, int32_t K, int32_t bits, float *out_f32,
                    uint16_t *out_f16, moe_stream_t stream) {
-    if (!valid_bits(bits)) return fail(MOE_ERR_INVALID_ARG, "bits = %d (want 8, 4 or 3)", bits);
+    if (!valid_bits(bits)) return fail(MOE_ERR_INVALID_ARG, "bits = %d (want 8, 4, 3 or MOE_FP4)", bits);
     if (K <= 0 || K % 64 != 0) return fail(MOE_ERR_INVALID_ARG, "K = %d must be a positive multiple of 64", K);
     if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "rows = %lld", (long long)rows);
     if (!out_f32 && !out_f16) return fail(MOE_ERR_INVALID_ARG, "both outputs are NULL");

@@ -109,6 +109,47 @@ __device__ __forceinline__ void u3x16_to_f32(uint32_t lo, uint32_t hi16, float *
     }
 }
 
+// ---------------------------------------------------------------------------
+// FP4 (E2M1) codes of an FP4 shelf ([P1] "step 4": MXFP4 for the rarest
+// down projections).  A code is sign * 8 + m, the magnitude index m of
+// 0, 0.5, 1, 1.5, 2, 3, 4, 6; the shelf stores d = X / 2 for the block scale X,
+// so a weight is d * q with the integer q = 2 * value in {0, +-1, +-2, +-3,
+// +-4, +-6, +-8, +-12}, exact in fp16 like the integer shelves' codes.
+// Plans and kernels carry an FP4 shelf as bits = kBitsFp4 (4-bit storage).
+// ---------------------------------------------------------------------------
+constexpr int kBitsFp4 = MOE_FP4;
+__host__ __device__ __forceinline__ int storage_bits(int bits) { return bits == kBitsFp4 ? 4 : bits; }
+
+// A shelf's two formats as one int (plans and per-slot tables): the gate_up
+// format in the low byte, the down format in the next.
+__host__ __device__ __forceinline__ int tier_dn_bits(const moe_tier &t) { return t.dn_bits ? t.dn_bits : t.bits; }
+__host__ __device__ __forceinline__ int tier_formats(const moe_tier &t) { return t.bits | (tier_dn_bits(t) << 8); }
+__host__ __device__ __forceinline__ int phase_bits(int formats, int phase) {
+    return phase == 0 ? (formats & 0xff) : (formats >> 8);
+}
+
+// The 8 codes of one 32-bit word (nibble i = weight i) as four half2 of the
+// integers q: P[j] = (q_j, q_{j+4}), the pairing the 4-bit decoders use.  The
+// magnitudes 2|value| come from a byte table (prmt selects table bytes by the
+// 3-bit index of each nibble), the sign bit flips the half's sign.
+__device__ __forceinline__ void fp4_pairs(uint32_t v, uint32_t (&P)[4]) {
+    constexpr uint32_t kLo = 0x03020100u, kHi = 0x0C080604u;  // 0 1 2 3 | 4 6 8 12
+    uint32_t m0, m1;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m0) : "r"(kLo), "r"(kHi), "r"(v & 0x7777u));          // |q0..q3|
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m1) : "r"(kLo), "r"(kHi), "r"((v >> 16) & 0x7777u));  // |q4..q7|
+    // byte pairs (|q_j|, 0, |q_{j+4}|, 0): a selector nibble with bit 3 set
+    // copies the sign of a table byte, which is 0
+    const uint32_t sel[4] = {0xC480u, 0xD591u, 0xE6A2u, 0xF7B3u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t y, h;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(y) : "r"(m0), "r"(m1), "r"(sel[j]));
+        // fp16(1024 + |q|) - 1024 = |q| exactly, then the sign bits 4j+3 and 4j+19
+        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(y | 0x64006400u), "r"(0x64006400u));
+        P[j] = h ^ ((v << (12 - 4 * j)) & 0x80008000u);
+    }
+}
+
 // Launch attribute list for a kernel that may overlap its predecessor
 // (programmatic dependent launch); `extra` (e.g. cooperative) is appended.
 struct PdlAttrs {

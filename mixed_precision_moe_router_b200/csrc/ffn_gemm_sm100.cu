@@ -200,70 +200,6 @@ __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
 // w = fp16_rne(d * q): q is built exactly as fp16 from the code bits with the
 // 1024-offset exponent trick, then one fp16 multiply rounds the exact product.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void dequant8(const uint8_t *raw, uint32_t d2a, uint32_t d2b, uint32_t (&o)[32]) {
-    const uint4 *q = reinterpret_cast<const uint4 *>(raw);
-    const uint32_t bias = 0x64806480u;  // (1152, 1152) = 1024 + 128
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-        const uint4 w = q[v];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const uint32_t u = ws[m] ^ 0x80808080u;
-            const uint32_t d2 = (v < 2) ? d2a : d2b;
-            o[v * 8 + 2 * m] = hmul2_u(hsub2_u(__byte_perm(u, 0x64646464u, 0x4140), bias), d2);
-            o[v * 8 + 2 * m + 1] = hmul2_u(hsub2_u(__byte_perm(u, 0x64646464u, 0x4342), bias), d2);
-        }
-    }
-}
-
-__device__ __forceinline__ void dequant4(const uint8_t *raw, uint32_t d2a, uint32_t d2b, uint32_t (&o)[32]) {
-    const uint4 *q = reinterpret_cast<const uint4 *>(raw);
-    const uint32_t bias = 0x64086408u;  // (1032, 1032) = 1024 + 8
-#pragma unroll
-    for (int v = 0; v < 2; ++v) {
-        const uint4 w = q[v];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {  // word m holds weights 8m..8m+7 of this 32-weight block
-            const uint32_t d2 = v == 0 ? d2a : d2b;
-            uint32_t P[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)  // P[j] = (w_j, w_{j+4})
-                P[j] = hsub2_u(((ws[m] >> (4 * j)) & 0x000f000fu) | 0x64006400u, bias);
-            uint32_t *dst = o + v * 16 + m * 4;
-            dst[0] = hmul2_u(__byte_perm(P[0], P[1], 0x5410), d2);
-            dst[1] = hmul2_u(__byte_perm(P[2], P[3], 0x5410), d2);
-            dst[2] = hmul2_u(__byte_perm(P[0], P[1], 0x7632), d2);
-            dst[3] = hmul2_u(__byte_perm(P[2], P[3], 0x7632), d2);
-        }
-    }
-}
-
-__device__ __forceinline__ void dequant3(const uint8_t *raw, uint32_t d2a, uint32_t d2b, uint32_t (&o)[32]) {
-    const uint4 lo = *reinterpret_cast<const uint4 *>(raw);
-    const uint2 hi = *reinterpret_cast<const uint2 *>(raw + 16);
-    const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w};
-    const uint32_t bias = 0x64046404u;  // (1028, 1028) = 1024 + 4
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {  // 16 weights: lo word p, high bits 16(p%2).. of hi word p/2
-        const uint32_t hw = (p < 2 ? hi.x : hi.y) >> (16 * (p & 1));
-        // spread: bit j (weight j) -> bit j+2, bit 8+j (weight 8+j) -> bit 18+j
-        const uint32_t Y = ((hw & 0xffu) | ((hw & 0xff00u) << 8)) << 2;
-        const uint32_t d2 = p < 2 ? d2a : d2b;
-        uint32_t P[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)  // P[j] = (c_j, c_{j+8})
-            P[j] = hsub2_u(((lw[p] >> (2 * j)) & 0x00030003u) | ((Y >> j) & 0x00040004u) | 0x64006400u, bias);
-        uint32_t *dst = o + p * 8;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            dst[j] = hmul2_u(__byte_perm(P[2 * j], P[2 * j + 1], 0x5410), d2);      // (c_2j, c_2j+1)
-            dst[4 + j] = hmul2_u(__byte_perm(P[2 * j], P[2 * j + 1], 0x7632), d2);  // (c_8+2j, c_9+2j)
-        }
-    }
-}
-
 // 32-weight variants (one quantisation block, one scale pair d2)
 __device__ __forceinline__ void dequant8_32(const uint8_t *raw, uint32_t d2, uint32_t (&o)[16]) {
     const uint4 *q = reinterpret_cast<const uint4 *>(raw);
@@ -290,6 +226,22 @@ __device__ __forceinline__ void dequant4_32(const uint8_t *raw, uint32_t d2, uin
         uint32_t P[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) P[j] = hsub2_u(((ws[m] >> (4 * j)) & 0x000f000fu) | 0x64006400u, bias);
+        o[4 * m] = hmul2_u(__byte_perm(P[0], P[1], 0x5410), d2);
+        o[4 * m + 1] = hmul2_u(__byte_perm(P[2], P[3], 0x5410), d2);
+        o[4 * m + 2] = hmul2_u(__byte_perm(P[0], P[1], 0x7632), d2);
+        o[4 * m + 3] = hmul2_u(__byte_perm(P[2], P[3], 0x7632), d2);
+    }
+}
+
+// FP4 codes: the nibble layout of 4-bit codes, the integers q = 2 * value
+// from the E2M1 table (exact fp16), so d * q is exact as well.
+__device__ __forceinline__ void dequant_fp4_32(const uint8_t *raw, uint32_t d2, uint32_t (&o)[16]) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(raw);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        uint32_t P[4];
+        fp4_pairs(ws[m], P);
         o[4 * m] = hmul2_u(__byte_perm(P[0], P[1], 0x5410), d2);
         o[4 * m + 1] = hmul2_u(__byte_perm(P[2], P[3], 0x5410), d2);
         o[4 * m + 2] = hmul2_u(__byte_perm(P[0], P[1], 0x7632), d2);
@@ -352,7 +304,7 @@ __device__ __forceinline__ void expert_rows(const Params &P, int e, int &bits, c
                                             const uint16_t *&sc) {
     const int H = P.f.w.H, I = P.f.w.I;
     if (e == P.f.E) {
-        bits = P.f.w.shared.bits;
+        bits = P.phase == 0 ? P.f.w.shared.bits : tier_dn_bits(P.f.w.shared);
         qs = P.phase == 0 ? P.f.w.shared.gu_qs : P.f.w.shared.dn_qs;
         sc = P.phase == 0 ? P.f.w.shared.gu_scale : P.f.w.shared.dn_scale;
         return;
@@ -362,13 +314,13 @@ __device__ __forceinline__ void expert_rows(const Params &P, int e, int &bits, c
         if (i < P.f.w.n_tiers && e >= P.f.w.tiers[i].first_expert &&
             e < P.f.w.tiers[i].first_expert + P.f.w.tiers[i].n_experts) {
             const size_t j = static_cast<size_t>(e - P.f.w.tiers[i].first_expert);
-            const int b = P.f.w.tiers[i].bits;
+            const int b = P.phase == 0 ? P.f.w.tiers[i].bits : tier_dn_bits(P.f.w.tiers[i]);
             bits = b;
             if (P.phase == 0) {
-                qs = P.f.w.tiers[i].gu_qs + j * 2 * I * (H * b / 8);
+                qs = P.f.w.tiers[i].gu_qs + j * 2 * I * (H * storage_bits(b) / 8);
                 sc = P.f.w.tiers[i].gu_scale + j * 2 * I * (H / 32);
             } else {
-                qs = P.f.w.tiers[i].dn_qs + j * H * (I * b / 8);
+                qs = P.f.w.tiers[i].dn_qs + j * H * (I * storage_bits(b) / 8);
                 sc = P.f.w.tiers[i].dn_scale + j * H * (I / 32);
             }
         }
@@ -427,7 +379,7 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
         const uint16_t *sc;
         expert_rows(P, S.slots.expert[tl.slot], c.bits, qs, sc);
         const int row = P.phase == 0 ? ((r & 1) ? P.f.w.I : 0) + tl.mt * (BM / 2) + (r >> 1) : tl.mt * BM + r;
-        c.qrow = qs + static_cast<size_t>(row) * (K * c.bits / 8);
+        c.qrow = qs + static_cast<size_t>(row) * (K * storage_bits(c.bits) / 8);
         c.srow = sc + static_cast<size_t>(row) * (K / 32);
     };
     if (P.phase == 2) {  // router: bf16 weight rows go to tensor memory unchanged
@@ -475,7 +427,7 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
             if (ci.bits == 8) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) cp_async16(dst + 16 * c, qrow + 32 * blk + 16 * c, 16);
-            } else if (ci.bits == 4) {
+            } else if (ci.bits == 4 || ci.bits == kBitsFp4) {
                 cp_async16(dst, qrow + 16 * blk, 16);
                 cp_async16(dst + 16, qrow + 16 * blk + 16, 16);
             } else {
@@ -509,6 +461,9 @@ __device__ __forceinline__ void role_dequant(const Params &P, const Shared &S, i
         } else if (bits == 4) {
             dequant4_32(raw, d2a, o0);
             dequant4_32(raw + 16, d2b, o1);
+        } else if (bits == kBitsFp4) {
+            dequant_fp4_32(raw, d2a, o0);
+            dequant_fp4_32(raw + 16, d2b, o1);
         } else {
             // lo plane: 8 bytes per block; hi plane: 4 bytes per block
             uint8_t tmp[16];

@@ -95,7 +95,7 @@ __host__ __device__ __forceinline__ Geo geo(int K, int bits) {
     g.K = K;
     g.R = rows_pow2(K);
     g.rows = 16 * g.R;
-    g.rb = K * bits / 8;
+    g.rb = K * storage_bits(bits) / 8;
     g.sb = K / 16;
     g.W = swizzle_width(g.rb);
     g.lw = g.W == 128 ? 7 : (g.W == 64 ? 6 : (g.W == 32 ? 5 : 4));
@@ -169,7 +169,8 @@ __host__ __device__ __forceinline__ int xf_col_stride(int K) { return (K / 32) *
 // A code c placed at mantissa bit s under the exponent of 2^(10-s) reads as
 // the half 2^(10-s) + c; subtracting 2^(10-s) + offset leaves q exactly.
 // Thread t owns weights 8t .. 8t+7 of each 32-weight block, paired as
-// (2p, 2p+1) for 8-bit codes and (p, p+4) for 4- and 3-bit codes, p = 0..3.
+// (2p, 2p+1) for 8-bit codes and (p, p+4) for 4-bit, FP4 and 3-bit codes,
+// p = 0..3.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
@@ -202,6 +203,10 @@ __device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int 
         P[1] = hsub2((v & 0x00F000F0u) | 0x54005400u, 0x54805480u);   // 64 + c - 72
         P[2] = hsub2((v8 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
         P[3] = hsub2((v8 & 0x00F000F0u) | 0x54005400u, 0x54805480u);
+    } else if constexpr (BITS == kBitsFp4) {
+        // FP4 codes in the 4-bit layout: nibble i of the word at byte 16b + 4t
+        // is weight 8t + i
+        fp4_pairs(*reinterpret_cast<const uint32_t *>(tile + tile_off<PAD>(16 * b + 4 * t, r, G, xr)), P);
     } else {
         // low plane: bits 0-1 of weight 8t+i at bit 2i of the u16 at byte 8b+2t;
         // high plane: bit 2 at bit i of byte K/4 + 4b + t (c = q + 4)
@@ -358,7 +363,8 @@ __device__ __forceinline__ void tma_5d(void *dst, const CUtensorMap *map, int x,
         : "memory");
 }
 
-__device__ __forceinline__ int bits_idx(int bits) { return bits == 8 ? 0 : (bits == 4 ? 1 : 2); }
+// geometry index of a shelf: 8-bit, 4-bit storage (integer or FP4), 3-bit
+__device__ __forceinline__ int bits_idx(int bits) { return bits == 8 ? 0 : (bits == 3 ? 2 : 1); }
 
 // Table base pointers of the shelves (index < n_tiers) and of the shared
 // expert (index n_tiers), copied from the parameters into shared memory so
@@ -413,7 +419,7 @@ struct StreamSmem {
 };
 
 __device__ __forceinline__ const Geo &tile_geo(const StreamSmem &S, int phase, int a) {
-    return S.geo[phase * 3 + bits_idx(S.pt.bits[a])];
+    return S.geo[phase * 3 + bits_idx(phase_bits(S.pt.bits[a], phase))];
 }
 
 __device__ __forceinline__ void abort_cta(const FfnParams &p, const StreamSmem &S) {
@@ -572,7 +578,7 @@ __device__ __forceinline__ bool load_b_gu(const FfnParams &p, const StreamSmem &
                                           uint8_t *xf) {
     bool bad = false;
     const int lane = threadIdx.x & 31;
-    const int H = p.w.H, nchunk = H / 8, cs = xf_col_stride(H), bits = S.pt.bits[a];
+    const int H = p.w.H, nchunk = H / 8, cs = xf_col_stride(H), bits = phase_bits(S.pt.bits[a], 0);
     const int my_row = lane < ntok ? entry_row(p, S, a, pass * kTokPerPass + lane) : 0;
     for (int n = 0; n < ntok; ++n) {
         const int tok = row_token(p, __shfl_sync(0xffffffffu, my_row, n));
@@ -594,7 +600,7 @@ __device__ __forceinline__ bool load_b_dn(const FfnParams &p, const StreamSmem &
                                           uint8_t *xf) {
     bool bad = false;
     const int lane = threadIdx.x & 31;
-    const int I = p.w.I, nchunk = I / 8, cs = xf_col_stride(I), bits = S.pt.bits[a];
+    const int I = p.w.I, nchunk = I / 8, cs = xf_col_stride(I), bits = phase_bits(S.pt.bits[a], 1);
     const int tp = tokens_per_pass(1, I);
     const int my_row = lane < ntok ? entry_row(p, S, a, pass * tp + lane) : 0;
     for (int n = 0; n < ntok; ++n) {
@@ -769,7 +775,7 @@ __device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, i
     walk_begin(S, w);
     for (; ok && w.phase < 2; walk_next(S, w), ++i) {
         const int phase = w.phase, a = w.a;
-        const int bits = S.pt.bits[a], cnt = S.pt.count[a];
+        const int bits = phase_bits(S.pt.bits[a], phase), cnt = S.pt.count[a];
         const Geo &G = tile_geo(S, phase, a);
         const bool mine = i % kGroups == grp;
         if (mine && !mbar_wait_warp(&S.full[i % kND], (i / kND) & 1, S.abort, p.wait_limit)) {
@@ -803,9 +809,11 @@ __device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, i
                 ncol = p.T;
             }
             if (!mine) continue;
-            const float4 part = bits == 8 ? compute_part<8>(G, phase, stage, xf, ncol, warp)
-                                          : (bits == 4 ? compute_part<4>(G, phase, stage, xf, ncol, warp)
-                                                       : compute_part<3>(G, phase, stage, xf, ncol, warp));
+            float4 part;
+            if (bits == 8) part = compute_part<8>(G, phase, stage, xf, ncol, warp);
+            else if (bits == 4) part = compute_part<4>(G, phase, stage, xf, ncol, warp);
+            else if (bits == 3) part = compute_part<3>(G, phase, stage, xf, ncol, warp);
+            else part = compute_part<kBitsFp4>(G, phase, stage, xf, ncol, warp);
             if (pass == np - 1) {  // every read of the stage is done
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.empty[i % kND]);
@@ -1077,8 +1085,8 @@ __device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S
     const int nt0 = S.nt0, nt1 = S.nt1;
     long long tc0 = 0, tc1 = 0, v0 = 0, v1 = 0;
     if (lane < ns) {
-        tc0 = tile_cost(pi.H, pi.I, 0, bits, 1);
-        tc1 = tile_cost(pi.H, pi.I, 1, bits, 1);
+        tc0 = tile_cost(pi.H, pi.I, 0, phase_bits(bits, 0), 1);
+        tc1 = tile_cost(pi.H, pi.I, 1, phase_bits(bits, 1), 1);
         v0 = nt0 * tc0;
         v1 = nt1 * tc1;
     }
@@ -1469,7 +1477,7 @@ bool byte_map(CUtensorMap *out, const void *ptr, int rank, const uint64_t *dims,
 // Maps of one shelf (or of the shared expert) at table index t.
 bool shelf_maps(moe::StreamMaps &M, int t, const moe_tier &tier, int H, int I) {
     const uint64_t n = static_cast<uint64_t>(tier.n_experts);
-    const moe::Geo g0 = moe::geo_gu(H, tier.bits), g1 = moe::geo(I, tier.bits);
+    const moe::Geo g0 = moe::geo_gu(H, tier.bits), g1 = moe::geo(I, moe::tier_dn_bits(tier));
     if (g0.pad) {
         // [expert][gate|up][row][line][128 bytes], box {128, nc1, 8R, 2, 1}
         const uint64_t dims[5] = {128, static_cast<uint64_t>(g0.rb / 128), static_cast<uint64_t>(I), 2, n};
@@ -1755,8 +1763,9 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
             prefetch_l2(Nx.wr + static_cast<size_t>(e0) * H, static_cast<uint32_t>((e1 - e0) * H * 2));
             if (Nx.w.shared.n_experts == 1) {
                 const moe_tier &sh = Nx.w.shared;
-                const size_t gq = static_cast<size_t>(2) * P.I * H * sh.bits / 8, gs = static_cast<size_t>(2) * P.I * (H / 32) * 2;
-                const size_t dq = static_cast<size_t>(H) * P.I * sh.bits / 8, ds = static_cast<size_t>(H) * (P.I / 32) * 2;
+                const int gbits = storage_bits(sh.bits), dbits = storage_bits(tier_dn_bits(sh));
+                const size_t gq = static_cast<size_t>(2) * P.I * H * gbits / 8, gs = static_cast<size_t>(2) * P.I * (H / 32) * 2;
+                const size_t dq = static_cast<size_t>(H) * P.I * dbits / 8, ds = static_cast<size_t>(H) * (P.I / 32) * 2;
                 const void *base[4] = {sh.gu_qs, sh.gu_scale, sh.dn_qs, sh.dn_scale};
                 const size_t len[4] = {gq, gs, dq, ds};
                 for (int a = 0; a < 4; ++a) {
@@ -1846,12 +1855,12 @@ cudaError_t moe_stack_encode_layer(const moe_layer_weights *w, const uint16_t *w
     L.bias = bias;
     L.shelves.n_tiers = w->n_tiers;
     L.shelves.has_shared = w->shared.n_experts == 1;
-    L.shelves.shared_bits = w->shared.bits;
+    L.shelves.shared_bits = moe::tier_formats(w->shared);
     for (int t = 0; t < MOE_MAX_TIERS; ++t) {
         const bool on = t < w->n_tiers;
         L.shelves.first[t] = on ? w->tiers[t].first_expert : 0;
         L.shelves.n[t] = on ? w->tiers[t].n_experts : 0;
-        L.shelves.bits[t] = on ? w->tiers[t].bits : 8;
+        L.shelves.bits[t] = on ? moe::tier_formats(w->tiers[t]) : 8 | (8 << 8);
         if (on)
             L.tp[t] = {w->tiers[t].gu_qs, reinterpret_cast<const uint8_t *>(w->tiers[t].gu_scale), w->tiers[t].dn_qs,
                        reinterpret_cast<const uint8_t *>(w->tiers[t].dn_scale)};

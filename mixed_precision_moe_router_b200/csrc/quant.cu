@@ -3,13 +3,35 @@
 // [P1] "step 4: three shelves, all on the GPU": popular experts keep more bits,
 // rare ones are squeezed harder.  [P3] "Why the model fits at all": a code per
 // weight plus one 16-bit scale per 32 weights (4.5 bits/weight at 4 bits).
-// The exact rules (absmax, fp16 scale, fp32 division, half-away rounding) and
-// the byte layout are stated in moe_tiered.h.
+// The exact rules (absmax, fp16 scale, fp32 division, half-away rounding; for
+// an FP4 shelf the MX power-of-two scale and E2M1 rounding) and the byte
+// layout are stated in moe_tiered.h.  Internally an FP4 shelf is bits = 5.
 #include "common.cuh"
 
 namespace moe {
 
 __device__ __forceinline__ int qmax_of(int bits) { return bits == 8 ? 127 : (bits == 4 ? 7 : 3); }
+
+// FP4 (E2M1) code of w in a block whose largest magnitude is amax, the
+// OCP MX conversion: X = 2^(floor(log2 amax) - 2), the E2M1 value nearest to
+// w / X (a tie goes to the even magnitude index; beyond 6 it saturates);
+// *d receives X / 2 as fp16 bits (0 for an all-zero block).
+__device__ __forceinline__ uint32_t fp4_code(float w, float amax, uint16_t *d) {
+    if (amax == 0.0f) {
+        *d = 0;
+        return 0;
+    }
+    int e = 0;
+    frexpf(amax, &e);  // amax = f * 2^e, f in [0.5, 1): floor(log2 amax) = e - 1
+    const int shared = min(max(e - 3, -23), 16);
+    *d = __half_as_ushort(__float2half_rn(ldexpf(1.0f, shared - 1)));
+    const float a = fabsf(ldexpf(w, -shared));  // |w| / X, exact
+    // magnitude index: midpoints between 0, 0.5, 1, 1.5, 2, 3, 4, 6; a value
+    // on a midpoint after an odd index moves up to the even one
+    int m = (a > 0.25f) + (a > 0.75f) + (a > 1.25f) + (a > 1.75f) + (a > 2.5f) + (a > 3.5f) + (a > 5.0f);
+    m += (a == 0.75f) + (a == 1.75f) + (a == 3.5f);
+    return static_cast<uint32_t>(m | ((w < 0.0f && m > 0) ? 8 : 0));
+}
 
 // One warp per block of 32 weights; lane i owns weight i of the block.
 __global__ void quantize_kernel(const float *__restrict__ src, int64_t rows, int K, int bits,
@@ -19,7 +41,7 @@ __global__ void quantize_kernel(const float *__restrict__ src, int64_t rows, int
     const int64_t total = rows * nblk_row;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    const size_t row_bytes = static_cast<size_t>(K) * bits / 8;
+    const size_t row_bytes = static_cast<size_t>(K) * storage_bits(bits) / 8;
     const float qmax = static_cast<float>(qmax_of(bits));
     for (int64_t b = warp0; b < total; b += nwarps) {
         const int64_t row = b / nblk_row;
@@ -28,6 +50,15 @@ __global__ void quantize_kernel(const float *__restrict__ src, int64_t rows, int
         float amax = fabsf(w);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        uint8_t *rowp = qs + row * row_bytes;
+        if (bits == kBitsFp4) {
+            uint16_t d4;
+            const uint32_t c = fp4_code(w, amax, &d4);
+            if (lane == 0) scale[row * nblk_row + blk] = d4;
+            const uint32_t nb = __shfl_down_sync(0xffffffffu, c, 1);
+            if ((lane & 1) == 0) rowp[blk * 16 + (lane >> 1)] = static_cast<uint8_t>(c | (nb << 4));
+            continue;
+        }
         const __half d = __float2half_rn(__fdiv_rn(amax, qmax));
         const float df = __half2float(d);
         int q = 0;
@@ -37,7 +68,6 @@ __global__ void quantize_kernel(const float *__restrict__ src, int64_t rows, int
             q = static_cast<int>(r);
         }
         if (lane == 0) scale[row * nblk_row + blk] = __half_as_ushort(d);
-        uint8_t *rowp = qs + row * row_bytes;
         if (bits == 8) {
             rowp[blk * 32 + lane] = static_cast<uint8_t>(static_cast<int8_t>(q));
         } else if (bits == 4) {
@@ -68,14 +98,18 @@ __global__ void dequantize_kernel(const uint8_t *__restrict__ qs, const uint16_t
                                   int64_t rows, int K, int bits, float *__restrict__ out_f32,
                                   uint16_t *__restrict__ out_f16) {
     const int64_t n = rows * K;
-    const size_t row_bytes = static_cast<size_t>(K) * bits / 8;
+    const size_t row_bytes = static_cast<size_t>(K) * storage_bits(bits) / 8;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t row = i / K;
         const int k = static_cast<int>(i - row * K);
         const uint8_t *rowp = qs + row * row_bytes;
         int q;
-        if (bits == 8) {
+        if (bits == kBitsFp4) {
+            const int c = (rowp[k >> 1] >> (4 * (k & 1))) & 0xf;
+            const int mag = static_cast<int>((0x0C08060403020100ull >> (8 * (c & 7))) & 0xff);  // 2|value|
+            q = (c & 8) ? -mag : mag;
+        } else if (bits == 8) {
             q = static_cast<int8_t>(rowp[k]);
         } else if (bits == 4) {
             q = static_cast<int>((rowp[k >> 1] >> (4 * (k & 1))) & 0xf) - 8;

@@ -28,9 +28,12 @@ def token_range(T, world, rank):
 
 def expert_bytes(H, I, bits, block=32):
     """Bytes of one expert's codes and fp16 block scales (gate_up [2I, H] and
-    down [H, I], blocks of `block` weights along each row)."""
+    down [H, I], blocks of `block` weights along each row).  `bits` is one
+    format for both or a (gate_up, down) pair; FP4 (5) stores 4-bit codes."""
+    gu, dn = (bits, bits) if isinstance(bits, int) else bits
+    code = {5: 4}
     weights = 2 * I * H + H * I
-    return weights * bits // 8 + (weights // block) * 2
+    return (2 * I * H * code.get(gu, gu) + H * I * code.get(dn, dn)) // 8 + (weights // block) * 2
 
 
 def layer_expert_bytes(H, I, tiers):

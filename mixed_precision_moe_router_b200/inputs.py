@@ -39,7 +39,7 @@ class LayerConfig:
     tiers: tuple  # ((bits, n_experts), ...) in id order, hottest first
     shared: bool = True
     zipf_alpha: float = ZIPF_ALPHA
-    shared_bits: int = 8
+    shared_bits: object = 8  # a format, or a (gate_up, down) pair
 
     def tier_ranges(self):
         out, first = [], 0
@@ -55,6 +55,17 @@ TINY = LayerConfig("tiny", H=256, I=128, E=16, k=2, tiers=((8, 4), (4, 6), (3, 6
                    zipf_alpha=0.0)
 DECODE = LayerConfig("decode", H=2048, I=512, E=512, k=10,
                      tiers=((8, 128), (4, 192), (3, 192)))
+# FP4 (E2M1) shelves: the library numbers that format 5.  A shelf's format is
+# one number, or a (gate_up, down) pair.  TINY_FP4 has every kind of FP4 shelf
+# (gate_up and down, down only, a shared expert with an FP4 down); the
+# ladder layer follows the pages' repacking recipe, whose down projections
+# drop to MXFP4 on the rarest shelf while gate_up drops to 3 bits.
+FP4 = 5
+TINY_FP4 = LayerConfig("tiny_fp4", H=256, I=128, E=16, k=2,
+                       tiers=((8, 4), (FP4, 4), ((3, FP4), 4), ((4, FP4), 4)),
+                       zipf_alpha=0.0, shared_bits=(8, FP4))
+DECODE_LADDER = LayerConfig("decode_fp4_down", H=2048, I=512, E=512, k=10,
+                            tiers=((8, 128), (4, 192), ((3, FP4), 192)))
 CONFIGS = {"tiny": TINY, "decode": DECODE}
 
 TINY_SEED = 0

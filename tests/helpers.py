@@ -34,13 +34,30 @@ def to_np(t):
     return t.detach().cpu().numpy()
 
 
+FP4 = 5  # the library's format number of an FP4 (E2M1) shelf
+
+
+def formats(bits):
+    """(gate_up, down) formats of a shelf given as one format or a pair."""
+    return (bits, bits) if isinstance(bits, int) else (int(bits[0]), int(bits[1]))
+
+
+def oracle_quantize_pack(w, fmt):
+    return oracle.quantize_pack_fp4(w) if fmt == FP4 else oracle.quantize_pack(w, fmt)
+
+
+def oracle_dequantize(q, s, fmt, K):
+    return oracle.dequantize_fp4_f32(q, s, K) if fmt == FP4 else oracle.dequantize_f32(q, s, fmt, K)
+
+
 def _prepare_expert(args):
     """Worker: oracle quantisation + dequantisation of one expert (runs in a
     spawned process; pure numpy, no GPU)."""
     wgu, wdn, bits, H, I = args
-    gq, gs = oracle.quantize_pack(wgu, bits)
-    dq, ds = oracle.quantize_pack(wdn, bits)
-    return oracle.dequantize_f32(gq, gs, bits, H), oracle.dequantize_f32(dq, ds, bits, I)
+    gf, df = formats(bits)
+    gq, gs = oracle_quantize_pack(wgu, gf)
+    dq, ds = oracle_quantize_pack(wdn, df)
+    return oracle_dequantize(gq, gs, gf, H), oracle_dequantize(dq, ds, df, I)
 
 
 _POOL = None
@@ -90,16 +107,15 @@ class OracleExperts:
     def packed(self, e):
         if e not in self._packed:
             wgu, wdn = inputs.expert_source(self.cfg, self.seed, e, self.device)
-            b = self.bits(e)
-            self._packed[e] = (oracle.quantize_pack(wgu.cpu().numpy(), b), oracle.quantize_pack(wdn.cpu().numpy(), b))
+            gf, df = formats(self.bits(e))
+            self._packed[e] = (oracle_quantize_pack(wgu.cpu().numpy(), gf), oracle_quantize_pack(wdn.cpu().numpy(), df))
         return self._packed[e]
 
     def __call__(self, e):
         if e not in self._cache:
             (gq, gs), (dq, ds) = self.packed(e)
-            b = self.bits(e)
-            self._cache[e] = (oracle.dequantize_f32(gq, gs, b, self.cfg.H),
-                              oracle.dequantize_f32(dq, ds, b, self.cfg.I))
+            gf, df = formats(self.bits(e))
+            self._cache[e] = (oracle_dequantize(gq, gs, gf, self.cfg.H), oracle_dequantize(dq, ds, df, self.cfg.I))
         return self._cache[e]
 
     def shared(self):

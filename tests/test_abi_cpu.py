@@ -36,7 +36,16 @@ def test_packed_row_bytes():
     assert B.packed_row_bytes(2048, 4) == 1024
     assert B.packed_row_bytes(2048, 3) == 768
     assert B.packed_row_bytes(100, 4) == 0
-    assert B.packed_row_bytes(128, 5) == 0
+    assert B.packed_row_bytes(128, B.FP4) == 64  # FP4: 4-bit storage
+    assert B.packed_row_bytes(128, 6) == 0
+    assert B.packed_row_bytes(128, 2) == 0
+
+
+def test_fp4_format_number_agrees_with_the_header():
+    from mixed_precision_moe_router_b200 import inputs
+    from tests import helpers
+    src = open(os.path.join(ROOT, "include", "moe_tiered.h")).read()
+    assert int(re.search(r"#define MOE_FP4 (\d+)", src).group(1)) == B.FP4 == inputs.FP4 == helpers.FP4
 
 
 def _fake_layer(tiers=((8, 0, 4), (4, 4, 6), (3, 10, 6)), H=256, I=128, E=16, shared=True, ptr=0x10000):
@@ -65,6 +74,9 @@ def _ffn(d, T=8, k=2, ws=1 << 30, mode=0):
     (lambda d: setattr(d, "E", 0), B.MOE_ERR_INVALID_ARG),
     (lambda d: setattr(d, "n_tiers", 5), B.MOE_ERR_INVALID_ARG),
     (lambda d: setattr(d.tiers[1], "bits", 2), B.MOE_ERR_INVALID_ARG),
+    (lambda d: setattr(d.tiers[1], "bits", 6), B.MOE_ERR_INVALID_ARG),
+    (lambda d: setattr(d.tiers[2], "dn_bits", 2), B.MOE_ERR_INVALID_ARG),     # down format
+    (lambda d: setattr(d.shared, "dn_bits", 7), B.MOE_ERR_INVALID_ARG),
     (lambda d: setattr(d.tiers[1], "first_expert", 3), B.MOE_ERR_INVALID_ARG),  # overlap
     (lambda d: setattr(d.tiers[2], "n_experts", 5), B.MOE_ERR_INVALID_ARG),     # gap
     (lambda d: setattr(d.tiers[2], "first_expert", -1), B.MOE_ERR_INVALID_ARG),  # negative id
@@ -94,7 +106,7 @@ def test_ffn_rejects_bad_sizes_and_workspace():
 def test_router_and_quantize_reject_bad_args():
     L = B.lib()
     p = ctypes.c_void_p(0x20000)
-    assert L.moe_quantize(p, 4, 128, 5, p, p, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize(p, 4, 128, 6, p, p, None) == B.MOE_ERR_INVALID_ARG  # no such format
     assert L.moe_quantize(p, 4, 100, 8, p, p, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_quantize(ctypes.c_void_p(0x20004), 4, 128, 8, p, p, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_router_topk(p, p, None, 4, 256, 16, 17, None, p, p, None, 0, None) == B.MOE_ERR_INVALID_ARG

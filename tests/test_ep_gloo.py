@@ -135,6 +135,10 @@ def test_expert_bytes_match_the_shelf_format():
     assert ep.expert_bytes(H, I, 8) == w + w // 16
     assert ep.expert_bytes(H, I, 4) == w // 2 + w // 16
     assert ep.expert_bytes(H, I, 3) == 3 * w // 8 + w // 16
+    # FP4 stores 4-bit codes; a (gate_up, down) pair counts each table at its own width
+    assert ep.expert_bytes(H, I, 5) == ep.expert_bytes(H, I, 4)
+    assert ep.expert_bytes(H, I, (3, 5)) == (2 * H * I * 3 + H * I * 4) // 8 + w // 16
+    assert ep.expert_bytes(H, I, (8, 8)) == ep.expert_bytes(H, I, 8)
 
 
 @pytest.mark.parametrize("T,world", [(1, 1), (8, 2), (5, 4), (3, 8), (4096, 8)])
