@@ -160,6 +160,7 @@ class StackRunner:
         self.xs = [x0.clone()] + [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev) for _ in range(n)]
         self.ns = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev) for _ in range(n + 1)]
         self.outs = [torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev) for _ in range(n)]
+        torch.cuda.synchronize()  # x0's copy is on the default stream
         with torch.cuda.stream(stream):
             self.step()  # first run outside capture
         torch.cuda.synchronize()
@@ -200,6 +201,7 @@ def ffn_calls(layers, routers, xs, mode, stream):
     from mixed_precision_moe_router_b200 import binding as B
     cfg = inputs.DECODE
     calls, nbytes, pairs = [], [], []
+    torch.cuda.synchronize()  # inputs made on other streams (a permuted router, a new layer) are complete
     for l, layer in enumerate(layers):
         wr, bias = routers[l]
         x = xs[l]
@@ -298,6 +300,7 @@ class StackStep:
         self.ws = torch.empty(max(self.st.workspace_size(x0.shape[0], self.k), 1), dtype=torch.uint8,
                               device=x0.device)
         self.status = torch.zeros(1, dtype=torch.int32, device=x0.device)
+        torch.cuda.synchronize()  # the launches may go to another stream
 
     def step(self, x_layers=None):
         return self.B.stack_forward(self.st, self.x_in, self.k, out=self.out, x_layers=x_layers, workspace=self.ws,
@@ -496,7 +499,38 @@ def other_workloads(args, layers, routers, stream, rank):
                       "frac_bf16": round(fp["tflops"] / tf, 4), "touched_mb": round(fp["bytes"] / 1e6, 2)})
     res["sweep_one_layer_ffn"] = sweep
     res["tier_planner"] = tier_planner_curve(layers[0], routers[0], stream)
+    res["fp4_down_ladder"] = fp4_down_ladder(args, layers[:8], routers[:8], stream, rank)
     return res
+
+
+def fp4_down_ladder(args, int_layers, int_routers, stream, rank):
+    """The pages' down-projection ladder at decode size: shelves 8/8, 4/4 and
+    3-bit gate_up with FP4 (E2M1) down, against the 8/4/3-bit shelves, both as
+    stacks of the same depth through the stack kernel (microseconds per layer
+    at 1 and 8 tokens), and the relative squared quantisation error of one
+    down matrix at 3 bits, FP4 and 4 bits (the library's own quantiser)."""
+    from mixed_precision_moe_router_b200 import binding as B
+    cfg = inputs.DECODE_LADDER
+    dev = torch.device("cuda", torch.cuda.current_device())
+    n = len(int_layers)
+    layers, routers = build_stack(cfg, n, dev)
+    out = {"layers": n, "shelves": "8/8, 4/4, 3/FP4 (gate_up/down)"}
+    for T in (1, 8):
+        x0 = inputs.activations(T, cfg.H, seed=inputs.X_SEED + 1000 * rank + 50 + T, device=dev)
+        for name, (ls, rs) in (("fp4_ladder", (layers, routers)), ("int_8_4_3", (int_layers, int_routers))):
+            run = StackStep(ls, rs, x0)
+            ms = run.time(stream, args.steps, args.warmup)
+            out[f"{name}_T{T}_us_per_layer"] = round(ms * 1e3 / n, 2)
+            del run
+    _, wdn = inputs.expert_source(cfg, inputs.layer_seed(cfg, 0), 0, dev)
+    w = wdn.contiguous()
+    for fmt, label in ((3, "3bit"), (B.FP4, "fp4"), (4, "4bit")):
+        qs, sc = B.quantize(w, fmt)
+        back, _ = B.dequantize(qs, sc, w.shape[1], fmt)
+        out[f"down_rel_sq_err_{label}"] = round(float(((back - w).double() ** 2).sum() / (w.double() ** 2).sum()), 5)
+    del layers, routers
+    torch.cuda.empty_cache()
+    return out
 
 
 def tier_planner_curve(layer0, router, stream, fractions=(0.75, 1.0, 1.3, 1.6)):

@@ -130,23 +130,22 @@ __host__ __device__ __forceinline__ int phase_bits(int formats, int phase) {
 
 // The 8 codes of one 32-bit word (nibble i = weight i) as four half2 of the
 // integers q: P[j] = (q_j, q_{j+4}), the pairing the 4-bit decoders use.  The
-// magnitudes 2|value| come from a byte table (prmt selects table bytes by the
-// 3-bit index of each nibble), the sign bit flips the half's sign.
+// fp16 encodings of 0, 1, 2, 3, 4, 6, 8 and 12 all have a zero low byte, so a
+// byte table of their high bytes, indexed by each nibble's magnitude bits
+// through prmt, builds the halves directly; the sign bit is then or-ed in.
 __device__ __forceinline__ void fp4_pairs(uint32_t v, uint32_t (&P)[4]) {
-    constexpr uint32_t kLo = 0x03020100u, kHi = 0x0C080604u;  // 0 1 2 3 | 4 6 8 12
+    constexpr uint32_t kLo = 0x42403C00u, kHi = 0x4A484644u;  // 0 1 2 3 | 4 6 8 12 (high bytes)
     uint32_t m0, m1;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m0) : "r"(kLo), "r"(kHi), "r"(v & 0x7777u));          // |q0..q3|
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m1) : "r"(kLo), "r"(kHi), "r"((v >> 16) & 0x7777u));  // |q4..q7|
-    // byte pairs (|q_j|, 0, |q_{j+4}|, 0): a selector nibble with bit 3 set
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m0) : "r"(kLo), "r"(kHi), "r"(v & 0x7777u));          // q0..q3
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m1) : "r"(kLo), "r"(kHi), "r"((v >> 16) & 0x7777u));  // q4..q7
+    // bytes (0, hb(q_j), 0, hb(q_{j+4})): a selector nibble with bit 3 set
     // copies the sign of a table byte, which is 0
-    const uint32_t sel[4] = {0xC480u, 0xD591u, 0xE6A2u, 0xF7B3u};
+    const uint32_t sel[4] = {0x4808u, 0x5818u, 0x6828u, 0x7838u};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        uint32_t y, h;
+        uint32_t y;
         asm("prmt.b32 %0, %1, %2, %3;" : "=r"(y) : "r"(m0), "r"(m1), "r"(sel[j]));
-        // fp16(1024 + |q|) - 1024 = |q| exactly, then the sign bits 4j+3 and 4j+19
-        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(y | 0x64006400u), "r"(0x64006400u));
-        P[j] = h ^ ((v << (12 - 4 * j)) & 0x80008000u);
+        P[j] = y | ((v << (12 - 4 * j)) & 0x80008000u);  // sign bits 4j+3 and 4j+19
     }
 }
 

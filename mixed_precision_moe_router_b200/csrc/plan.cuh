@@ -44,8 +44,8 @@ __host__ __device__ __forceinline__ int tiles_per_slot(int H, int I, int phase) 
 // and-multiply time for every pass.  The two compute groups work side by
 // side, so a tile occupies the CTA for half of one group's time, which was
 // measured on B200 per 32K-weight tile and pass as 1.42 / 1.50 / 2.30 us for
-// gate_up and 1.36 / 1.38 / 1.72 us for down with 8- / 4- / 3-bit codes
-// (FP4 codes: 4-bit storage, a longer decode).
+// gate_up and 1.36 / 1.38 / 1.72 us for down with 8- / 4- / 3-bit codes;
+// FP4 codes (4-bit storage, a longer decode) measured 5 % above 4-bit ones.
 __host__ __device__ __forceinline__ long long tile_cost(int H, int I, int phase, int bits, int count) {
     const int K = phase == 0 ? H : I;
     const long long rows = 16 * rows_pow2(K);
@@ -53,8 +53,8 @@ __host__ __device__ __forceinline__ long long tile_cost(int H, int I, int phase,
     const long long passes = (count + tp - 1) / tp;
     const long long bytes = rows * (K * storage_bits(bits) / 8 + K / 16);
     const long long copy = bytes * 227 / 1000;
-    const long long per_tile = phase == 0 ? (bits == 8 ? 14200 : (bits == 4 ? 15000 : (bits == 3 ? 23000 : 16500)))
-                                          : (bits == 8 ? 13600 : (bits == 4 ? 13800 : (bits == 3 ? 17200 : 15000)));
+    const long long per_tile = phase == 0 ? (bits == 8 ? 14200 : (bits == 4 ? 15000 : (bits == 3 ? 23000 : 15750)))
+                                          : (bits == 8 ? 13600 : (bits == 4 ? 13800 : (bits == 3 ? 17200 : 14500)));
     const long long compute = passes * per_tile * rows * K / (2 * 32768);
     return kTileFixedCost + (copy > compute ? copy : compute);
 }
