@@ -69,6 +69,7 @@ constexpr int kMaxK = 2048;
 constexpr int kRedBytes = kWarps * 32 * 16;  // one item's partials: a float4 per compute lane
 constexpr int kMaxSmemEntries = 2048;        // sorted slot ids kept in shared memory up to this many
 constexpr int kMaxExpertShare = 16;          // router rows a CTA computes when it routes the batch itself
+constexpr int kDealtMaxTokens = 2;          // tiles dealt out in turn up to this many tokens (plan_in_cta)
 
 // ---------------------------------------------------------------------------
 // tile geometry
@@ -430,6 +431,9 @@ __device__ __forceinline__ void abort_cta(const FfnParams &p, const StreamSmem &
 // This CTA's tiles in order: its run of gate_up tiles (phase 0), then its run
 // of down tiles (phase 1); phase 2 once exhausted.  Tile g of a phase is tile
 // b = g % nt of slot a = g / nt.  Every warp role walks the same sequence.
+// A CTA's tiles of a phase are the global indices g = range[2 phase] +
+// n * range[5] below range[2 phase + 1]: a contiguous run (stride 1) or every
+// grid-th tile (stride = grid).
 struct Walk {
     int phase, g, ge, a, b;
 };
@@ -443,6 +447,12 @@ __device__ __forceinline__ void walk_enter(const StreamSmem &S, Walk &w, int pha
     w.b = w.g - w.a * nt;
 }
 
+// tiles of `phase` in this CTA's list
+__device__ __forceinline__ int phase_tiles(const StreamSmem &S, int phase) {
+    const int g = S.range[2 * phase], ge = S.range[2 * phase + 1], s = S.range[5];
+    return g < ge ? (ge - g + s - 1) / s : 0;
+}
+
 __device__ __forceinline__ void walk_begin(const StreamSmem &S, Walk &w) {
     if (S.range[0] < S.range[1]) walk_enter(S, w, 0);
     else if (S.range[2] < S.range[3]) walk_enter(S, w, 1);
@@ -450,10 +460,18 @@ __device__ __forceinline__ void walk_begin(const StreamSmem &S, Walk &w) {
 }
 
 __device__ __forceinline__ void walk_next(const StreamSmem &S, Walk &w) {
-    if (++w.g < w.ge) {
-        if (++w.b == (w.phase == 0 ? S.nt0 : S.nt1)) {
-            w.b = 0;
-            ++w.a;
+    const int stride = S.range[5];
+    w.g += stride;
+    if (w.g < w.ge) {
+        const int nt = w.phase == 0 ? S.nt0 : S.nt1;
+        if (stride == 1) {
+            if (++w.b == nt) {
+                w.b = 0;
+                ++w.a;
+            }
+        } else {
+            w.a = w.g / nt;
+            w.b = w.g - w.a * nt;
         }
         return;
     }
@@ -688,8 +706,8 @@ __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMap
     const int lane = threadIdx.x & 31;
     int *st = S.pst, *en = S.pst + kND;
     const int i0 = ps.i;
-    const int gs0 = S.range[0], n0 = max(S.range[1] - gs0, 0);
-    const int gs1 = S.range[2], n1 = max(S.range[3] - gs1, 0);
+    const int gs0 = S.range[0], n0 = phase_tiles(S, 0);
+    const int gs1 = S.range[2], n1 = phase_tiles(S, 1), stride = S.range[5];
     int nfit, head;
     {
         const int j = lane;
@@ -697,7 +715,7 @@ __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMap
         int phase = 0, a = 0, b = 0, sz = 0;
         if (real) {
             phase = j < n0 ? 0 : 1;
-            const int g = phase == 0 ? gs0 + j : gs1 + (j - n0);
+            const int g = phase == 0 ? gs0 + j * stride : gs1 + (j - n0) * stride;
             const int nt = phase == 0 ? S.nt0 : S.nt1;
             a = g / nt;
             b = g - a * nt;
@@ -1010,28 +1028,6 @@ __host__ __device__ __forceinline__ PrologueScratch prologue_scratch(int H, int 
     return ps;
 }
 
-// First tile (global index) of a phase whose start cost is >= x, with the
-// slots' inclusive cost prefix `pre` and tile cost `tc` held by lanes < ns
-// (warp-uniform result): the warp form of plan_first_tile.
-__device__ __forceinline__ int lanes_first_tile(long long pre, long long tc, int nt, int ns, long long x) {
-    const int lane = threadIdx.x & 31;
-    const unsigned m = __ballot_sync(0xffffffffu, lane < ns && pre > x);
-    if (!m) return ns * nt;
-    const int L = __ffs(m) - 1;
-    int r = 0;
-    if (lane == L) {
-        const long long off = pre - nt * tc;  // start cost of the slot's first tile
-        if (x <= off) {
-            r = L * nt;
-        } else {
-            long long b = static_cast<long long>(ceil(static_cast<double>(x - off) / static_cast<double>(tc)));
-            if (b > nt) b = nt;
-            r = L * nt + static_cast<int>(b);
-        }
-    }
-    return __shfl_sync(0xffffffffu, r, L);
-}
-
 // One token (T == 1, k <= 31): warp 0 alone ends the routing from the grid's
 // logits and builds this CTA's schedule.  It writes what cta_topk_rows,
 // cta_group and plan_in_cta write (the choices and weights, the sorted slots,
@@ -1111,18 +1107,15 @@ __device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S
         t.pre0[lane] = v0;
         t.pre1[lane] = v1;
     }
-    const int c = blockIdx.x, G = gridDim.x;
-    const long long tot0 = __shfl_sync(0xffffffffu, v0, 31), tot1 = __shfl_sync(0xffffffffu, v1, 31);
-    const int gs0 = lanes_first_tile(v0, tc0, nt0, ns, share_floor(tot0, c, G));
-    const int ge0 = c + 1 == G ? ns * nt0 : lanes_first_tile(v0, tc0, nt0, ns, share_floor(tot0, c + 1, G));
-    const int gs1 = lanes_first_tile(v1, tc1, nt1, ns, share_floor(tot1, c, G));
-    const int ge1 = c + 1 == G ? ns * nt1 : lanes_first_tile(v1, tc1, nt1, ns, share_floor(tot1, c + 1, G));
+    // one token: every tile is a single pass, so the tiles are dealt out in
+    // turn (tile g to CTA g mod grid; see plan_in_cta)
     if (lane == 0) {
-        S.range[0] = gs0;
-        S.range[1] = ge0;
-        S.range[2] = gs1;
-        S.range[3] = ge1;
+        S.range[0] = blockIdx.x;
+        S.range[1] = ns * nt0;
+        S.range[2] = blockIdx.x;
+        S.range[3] = ns * nt1;
         S.range[4] = ns;
+        S.range[5] = gridDim.x;
     }
 }
 
@@ -1204,7 +1197,7 @@ __device__ __forceinline__ uint8_t *carve_stream_smem(uint8_t *smem, int ring_by
     S.bempty = S.bfull + kNB;
     q = reinterpret_cast<uint8_t *>(S.bempty + kNB);
     S.abort = reinterpret_cast<int *>(q);
-    S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots, flag (16-byte aligned)
+    S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots, stride, flag (16-byte aligned)
     S.pst = S.abort + 12;
     q += (12 + 2 * kND) * sizeof(int);
     S.tp = reinterpret_cast<TierPtrs *>(q);
@@ -1287,13 +1280,27 @@ __device__ __forceinline__ void plan_in_cta(const FfnParams &p, StreamSmem &S, c
         if (lane == 0) S.range[4] = ns;
     }
     __syncthreads();
+    // With one or two tokens (every tile a single pass), the tiles of a
+    // phase are dealt out in turn: CTA c takes the global tiles c, c + grid,
+    // ...  Each CTA then works through the slots in order, so the slots'
+    // gate_up results complete one after another and the down tiles of early
+    // slots find their operand ready, where contiguous runs finish every slot
+    // only near the end of the phase (decode layer at one token: 44.9 ->
+    // 42.6 us).  Dealt tiles change slot at every tile, so the loader builds
+    // a down operand per tile; from about five tokens on that costs more than
+    // it saves, and each CTA takes the contiguous run of an equal share of
+    // the phase's cost instead.
+    const bool dealt = p.T <= kDealtMaxTokens && p.T <= tokens_per_pass(1, p.w.I);
     if (warp < 2) {
         const int ns = S.range[4];
         const long long total = plan_costs(p.pi, ns, warp, S.pt);
         if (lane == 0) {
-            const int2 r = plan_cta_range(S.pt, ns, warp == 0 ? S.nt0 : S.nt1, warp, total, blockIdx.x, gridDim.x);
+            const int nt = warp == 0 ? S.nt0 : S.nt1;
+            const int2 r = dealt ? make_int2(static_cast<int>(blockIdx.x), ns * nt)
+                                 : plan_cta_range(S.pt, ns, nt, warp, total, blockIdx.x, gridDim.x);
             S.range[2 * warp] = r.x;
             S.range[2 * warp + 1] = r.y;
+            if (warp == 0) S.range[5] = dealt ? gridDim.x : 1;
         }
     }
 }
@@ -1350,7 +1357,7 @@ ffn_stream_kernel(const __grid_constant__ FfnParams p, const __grid_constant__ S
     int routed = 1;
     if (fused) routed = route_in_cta(p, S, reinterpret_cast<const uint16_t *>(x_s), act_s, off_s, ps);
     if (!routed) {  // the grid barrier gave up: stream nothing
-        if (threadIdx.x < 5) S.range[threadIdx.x] = 0;
+        if (threadIdx.x < 6) S.range[threadIdx.x] = threadIdx.x == 5;  // empty runs, stride 1
     } else if (routed == 1) {
         plan_in_cta(p, S, act_s, off_s);
     }
