@@ -62,7 +62,7 @@ constexpr int kBlockWarps = kComputeWarps + 2 + kGroups;
 constexpr int kBlockThreads = kBlockWarps * 32;
 constexpr int kND = 8;             // tiles in flight at most (full/empty barrier pairs)
 constexpr int kNR = 3;             // partial-sum buffers per group (compute warps -> epilogue)
-constexpr int kNB = 2;             // B-operand buffers (loader -> compute warps)
+constexpr int kNBMax = 4;          // B-operand buffers (loader -> compute warps) at most
 constexpr int kMaxTileBytes = 40 * 1024;  // a staged tile (codes, padding, scales) at most
 constexpr int kTileAlign = 1024;   // ring allocations start on a 128-byte-swizzle atom
 constexpr int kMaxK = 2048;
@@ -70,6 +70,10 @@ constexpr int kRedBytes = kWarps * 32 * 16;  // one item's partials: a float4 pe
 constexpr int kMaxSmemEntries = 2048;        // sorted slot ids kept in shared memory up to this many
 constexpr int kMaxExpertShare = 16;          // router rows a CTA computes when it routes the batch itself
 constexpr int kDealtMaxTokens = 2;          // tiles dealt out in turn up to this many tokens (plan_in_cta)
+
+// B-operand buffers: with dealt tiles every down tile has an operand of its
+// own, so the loader gets room to build several ahead (they are small then).
+__host__ __device__ __forceinline__ int n_bbufs(int T) { return T <= kDealtMaxTokens ? kNBMax : 2; }
 
 // ---------------------------------------------------------------------------
 // tile geometry
@@ -403,12 +407,13 @@ struct StreamSmem {
     uint8_t *ring;
     int ring_bytes;
     uint8_t *xall;           // all-token gate_up fragments (T <= kTokPerPass), else null
-    uint8_t *bbuf;           // [kNB][b_bytes]
+    uint8_t *bbuf;           // [nb][b_bytes]
     int b_bytes;
     float4 *red;             // [kGroups][kNR][kWarps * 32]
     uint64_t *full, *empty;  // [kND]: a tile's copies landed / every compute warp is done with it
     uint64_t *rfull, *rempty;  // [kGroups][kNR]: partials written / partials summed
-    uint64_t *bfull, *bempty;  // [kNB]: B operand built / every compute warp has moved past it
+    uint64_t *bfull, *bempty;  // [nb]: B operand built / every compute warp has moved past it
+    int nb, nb_log2;           // B-operand buffers (a power of two)
     int *abort;              // [0] set by a warp that gave up (every wait checks it); [1] grid barriers passed
     int *range;              // this CTA's tiles: [gs0, ge0), [gs1, ge1); then the slot count
     int *pst;                // producer: ring byte range [pst[d], pst[kND + d]) of the tile in descriptor d
@@ -811,16 +816,16 @@ __device__ __forceinline__ void run_compute(const FfnParams &p, StreamSmem &S, i
                 if (nk != key) {
                     ++kb;
                     key = nk;
-                    if (!mbar_wait_warp(&S.bfull[kb % kNB], (kb / kNB) & 1, S.abort, p.wait_limit)) {
+                    if (!mbar_wait_warp(&S.bfull[kb & (S.nb - 1)], (kb >> S.nb_log2) & 1, S.abort, p.wait_limit)) {
                         ok = false;
                         break;
                     }
                     if (kb > 0) {
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.bempty[(kb - 1) % kNB]);
+                        if (lane == 0) mbar_arrive(&S.bempty[(kb - 1) & (S.nb - 1)]);
                     }
                 }
-                xf = S.bbuf + static_cast<size_t>(kb % kNB) * S.b_bytes;
+                xf = S.bbuf + static_cast<size_t>(kb & (S.nb - 1)) * S.b_bytes;
                 ncol = min(tp, cnt - pass * tp);
             } else {  // every token is a column; the epilogue keeps the slot's
                 xf = S.xall + (bits == 8 ? 0 : p.T * xf_col_stride(p.w.H));
@@ -872,7 +877,7 @@ __device__ __forceinline__ void run_loader(const FfnParams &p, StreamSmem &S, Lo
             if (nk == key) continue;
             key = nk;
             ++kb;
-            if (!mbar_wait_warp(&S.bempty[kb % kNB], ((kb / kNB) & 1) ^ 1, S.abort, p.wait_limit)) {
+            if (!mbar_wait_warp(&S.bempty[kb & (S.nb - 1)], ((kb >> S.nb_log2) & 1) ^ 1, S.abort, p.wait_limit)) {
                 ok = false;
                 break;
             }
@@ -887,11 +892,11 @@ __device__ __forceinline__ void run_loader(const FfnParams &p, StreamSmem &S, Lo
                 }
                 ready = a;
             }
-            uint8_t *xf = S.bbuf + static_cast<size_t>(kb % kNB) * S.b_bytes;
+            uint8_t *xf = S.bbuf + static_cast<size_t>(kb & (S.nb - 1)) * S.b_bytes;
             const int ntok = min(tp, cnt - pass * tp);
             bad |= phase == 0 ? load_b_gu(p, S, a, pass, ntok, xf) : load_b_dn(p, S, a, pass, ntok, xf);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.bfull[kb % kNB]);
+            if (lane == 0) mbar_arrive(&S.bfull[kb & (S.nb - 1)]);
         }
     }
     ls.kb = kb;
@@ -1185,7 +1190,9 @@ __device__ __forceinline__ uint8_t *carve_stream_smem(uint8_t *smem, int ring_by
     q += xb;
     S.b_bytes = bbuf_bytes(H, I, T);
     S.bbuf = q;
-    q += kNB * S.b_bytes;
+    S.nb = n_bbufs(T);
+    S.nb_log2 = S.nb == 4 ? 2 : 1;
+    q += S.nb * S.b_bytes;
     S.red = reinterpret_cast<float4 *>(q);
     q += kGroups * kNR * kRedBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(q);
@@ -1194,8 +1201,8 @@ __device__ __forceinline__ uint8_t *carve_stream_smem(uint8_t *smem, int ring_by
     S.rfull = bars + 2 * kND;
     S.rempty = S.rfull + kGroups * kNR;
     S.bfull = S.rempty + kGroups * kNR;
-    S.bempty = S.bfull + kNB;
-    q = reinterpret_cast<uint8_t *>(S.bempty + kNB);
+    S.bempty = S.bfull + kNBMax;
+    q = reinterpret_cast<uint8_t *>(S.bempty + kNBMax);
     S.abort = reinterpret_cast<int *>(q);
     S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots, stride, flag (16-byte aligned)
     S.pst = S.abort + 12;
@@ -1218,9 +1225,9 @@ __device__ __forceinline__ uint8_t *carve_stream_smem(uint8_t *smem, int ring_by
 // Host mirror of carve_stream_smem: bytes past the ring.
 __host__ __forceinline__ size_t stream_smem_fixed(int H, int I, int T, int k, int max_slots) {
     const size_t n_srt = static_cast<size_t>(T) * k;
-    return static_cast<size_t>(xall_bytes(H, T)) + kNB * static_cast<size_t>(bbuf_bytes(H, I, T)) +
+    return static_cast<size_t>(xall_bytes(H, T)) + n_bbufs(T) * static_cast<size_t>(bbuf_bytes(H, I, T)) +
            kGroups * kNR * static_cast<size_t>(kRedBytes) +
-           (2 * kND + 2 * kGroups * kNR + 2 * kNB) * sizeof(uint64_t) + (12 + 2 * kND) * sizeof(int) +
+           (2 * kND + 2 * kGroups * kNR + 2 * kNBMax) * sizeof(uint64_t) + (12 + 2 * kND) * sizeof(int) +
            (MOE_MAX_TIERS + 1) * sizeof(TierPtrs) + 6 * sizeof(Geo) + 16 + plan_tab_bytes(max_slots) +
            (n_srt <= static_cast<size_t>(kMaxSmemEntries) ? (n_srt * sizeof(int) + 15) / 16 * 16 : 0);
 }
@@ -1237,7 +1244,7 @@ __device__ __forceinline__ void init_stream_smem(StreamSmem &S, int H, int I) {
             mbar_init(&S.rfull[i], kWarps);
             mbar_init(&S.rempty[i], 1);
         }
-        for (int i = 0; i < kNB; ++i) {
+        for (int i = 0; i < kNBMax; ++i) {
             mbar_init(&S.bfull[i], 1);
             mbar_init(&S.bempty[i], kComputeWarps);
         }
