@@ -1010,7 +1010,7 @@ __device__ __forceinline__ void run_epilogue(const FfnParams &p, StreamSmem &S, 
 // batch routed in the kernel the top-k candidates, choices, weights, slot
 // positions and a few ints of scan space.
 struct PrologueScratch {
-    size_t lists, x, cand, idx, w, pos, tmp, end;
+    size_t lists, x, cand, idx, w, pos, tmp, topk, end;
 };
 
 __host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
@@ -1029,25 +1029,42 @@ __host__ __device__ __forceinline__ PrologueScratch prologue_scratch(int H, int 
     ps.w = align16(ps.idx + (fused ? S_ * sizeof(int) : 0));
     ps.pos = align16(ps.w + (fused ? S_ * sizeof(float) : 0));
     ps.tmp = align16(ps.pos + (fused ? S_ * sizeof(int) : 0));
-    ps.end = ps.tmp + (fused ? 32 * sizeof(int) : 0);
+    // one token's top-k candidates: a key and an id per chunk of 32 logits and choice
+    ps.topk = align16(ps.tmp + (fused ? 32 * sizeof(int) : 0));
+    ps.end = ps.topk + (fused && T == 1 ? static_cast<size_t>((E + 31) / 32) * k * 8 : 0);
     return ps;
 }
 
-// One token (T == 1, k <= 31): warp 0 alone ends the routing from the grid's
-// logits and builds this CTA's schedule.  It writes what cta_topk_rows,
+// The top k of n candidate keys (at most 32 * NJ) held in shared memory.
+template <int NJ>
+__device__ __forceinline__ void warp_topk_candidates(const uint32_t *ckey, int n, int k, int &pos, float &w) {
+    const int lane = threadIdx.x & 31;
+    uint32_t key[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) key[j] = lane + 32 * j < n ? ckey[lane + 32 * j] : 0u;
+    warp_topk_rounds<NJ>(key, k, pos, w);
+}
+
+// One token (T == 1, k <= 31): warp 0 alone ends the routing from the top-k
+// candidates of the grid's logits and builds this CTA's schedule.  It writes what cta_topk_rows,
 // cta_group and plan_in_cta write (the choices and weights, the sorted slots,
 // their positions, the active list, the slot tables and the tile runs), with
 // the chosen experts held one per lane: the k choices of one token are
 // distinct, so each is one slot and its sorted position is its rank.  The
 // offsets are written only when fill_offsets.  The caller synchronises.
 __device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S, int *act_s, int *off_s, int *idx_s,
-                                               float *w_s, int *pos_s, bool fill_offsets) {
+                                               float *w_s, int *pos_s, const uint32_t *ckey, const int *cid,
+                                               bool fill_offsets) {
     const int lane = threadIdx.x & 31;
     const int E = p.E, k = p.k;
-    int e_r;
+    // the second stage of the top-k, over the candidates of cta_topk_candidates
+    const int n = (E + 31) / 32 * k;
+    int pos_r;
     float w_r;
-    if (E <= 512) warp_topk_redux<16>(p.route.logits, E, k, e_r, w_r);
-    else warp_topk_redux<32>(p.route.logits, E, k, e_r, w_r);
+    if (n <= 512) warp_topk_candidates<16>(ckey, n, k, pos_r, w_r);
+    else warp_topk_candidates<32>(ckey, n, k, pos_r, w_r);
+    // (position -1, as id -1 before, only when fewer than k keys are valid)
+    const int e_r = lane < k ? (pos_r >= 0 && pos_r < n ? cid[pos_r] : -1) : 0;
     int rank = 0;
     for (int j = 0; j < k; ++j) rank += __shfl_sync(0xffffffffu, e_r, j) < e_r;
     if (lane < k) {
@@ -1083,22 +1100,8 @@ __device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S
             for (int a = 0; a < k; ++a) c += __shfl_sync(0xffffffffu, e, a) < x0 + lane;
             if (x0 + lane <= E) off_s[x0 + lane] = c;
         }
+    // the tiles are dealt out in turn (below), so no tile costs are needed
     const int nt0 = S.nt0, nt1 = S.nt1;
-    long long tc0 = 0, tc1 = 0, v0 = 0, v1 = 0;
-    if (lane < ns) {
-        tc0 = tile_cost(pi.H, pi.I, 0, phase_bits(bits, 0), 1);
-        tc1 = tile_cost(pi.H, pi.I, 1, phase_bits(bits, 1), 1);
-        v0 = nt0 * tc0;
-        v1 = nt1 * tc1;
-    }
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const long long u0 = __shfl_up_sync(0xffffffffu, v0, o), u1 = __shfl_up_sync(0xffffffffu, v1, o);
-        if (lane >= o) {
-            v0 += u0;
-            v1 += u1;
-        }
-    }
     if (lane < ns) {
         const PlanTabs &t = S.pt;
         t.expert[lane] = e;
@@ -1107,10 +1110,6 @@ __device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S
         t.jloc[lane] = jl;
         t.first[lane] = first;
         t.count[lane] = 1;
-        t.tc0[lane] = tc0;
-        t.tc1[lane] = tc1;
-        t.pre0[lane] = v0;
-        t.pre1[lane] = v1;
     }
     // one token: every tile is a single pass, so the tiles are dealt out in
     // turn (tile g to CTA g mod grid; see plan_in_cta)
@@ -1138,7 +1137,7 @@ __device__ __forceinline__ int route_in_cta(const FfnParams &p, StreamSmem &S, c
     const int e1 = static_cast<int>(static_cast<long long>(E) * (blockIdx.x + 1) / gridDim.x);
     cta_logits(x_s, T, H, E, p.route.wr, p.route.bias, e0, e1,
                reinterpret_cast<float *>(S.ring + ps.cand), p.route.logits);
-    int *barrier_ok = S.range + 5;
+    int *barrier_ok = S.range + 7;
     __syncthreads();  // every thread's logits are written before thread 0 arrives
     if (threadIdx.x == 0) {
         const bool ok = grid_barrier(p.route.gbar, S.abort[1]++, S.abort, p.wait_limit);
@@ -1155,8 +1154,13 @@ __device__ __forceinline__ int route_in_cta(const FfnParams &p, StreamSmem &S, c
     int *pos_s = reinterpret_cast<int *>(S.ring + ps.pos);
     const bool one = T == 1 && k <= 31 && E <= 1024 && p.pi.max_count >= 1 && S.srt != nullptr;
     if (one) {
+        uint32_t *ckey = reinterpret_cast<uint32_t *>(S.ring + ps.topk);
+        int *cid = reinterpret_cast<int *>(ckey + (E + 31) / 32 * k);
+        cta_topk_candidates(p.route.logits, E, k, ckey, cid);
+        __syncthreads();
         if (threadIdx.x < 32)
-            route_plan_one(p, S, act_s, off_s, idx_s, w_s, pos_s, blockIdx.x == 0 && p.route.topk_idx != nullptr);
+            route_plan_one(p, S, act_s, off_s, idx_s, w_s, pos_s, ckey, cid,
+                           blockIdx.x == 0 && p.route.topk_idx != nullptr);
         __syncthreads();
     } else {
         cta_topk_rows(p.route.logits, T, E, k, idx_s, w_s);
@@ -1204,7 +1208,7 @@ __device__ __forceinline__ uint8_t *carve_stream_smem(uint8_t *smem, int ring_by
     S.bempty = S.bfull + kNBMax;
     q = reinterpret_cast<uint8_t *>(S.bempty + kNBMax);
     S.abort = reinterpret_cast<int *>(q);
-    S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots, stride, flag (16-byte aligned)
+    S.range = S.abort + 4;  // gs0, ge0, gs1, ge1, n_slots, stride, flag, routing flag (16-byte aligned)
     S.pst = S.abort + 12;
     q += (12 + 2 * kND) * sizeof(int);
     S.tp = reinterpret_cast<TierPtrs *>(q);

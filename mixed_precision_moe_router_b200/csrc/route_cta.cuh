@@ -72,17 +72,11 @@ __device__ __forceinline__ float key_value(uint32_t key) {
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
+// The k rounds on keys already held by the lanes (entry lane + 32 j in
+// key[j], 0 for none); the position of choice r is returned in lane r.
 template <int NJ>
-__device__ __forceinline__ void warp_topk_redux(const float *row, int E, int k, int &out_i, float &out_w) {
+__device__ __forceinline__ void warp_topk_rounds(uint32_t (&key)[NJ], int k, int &out_i, float &out_w) {
     const int lane = threadIdx.x & 31;
-    // key 0 marks an entry out of range or already taken (no float maps to 0
-    // but a NaN with every bit set)
-    uint32_t key[NJ];
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-        const int e = lane + 32 * j;
-        key[j] = e < E ? order_key(__ldcg(row + e) + 0.0f) : 0u;  // -0 keys as +0
-    }
     float my_v = 0.f;
     int my_i = 0;
     for (int r = 0; r < k; ++r) {
@@ -135,6 +129,48 @@ __device__ __forceinline__ void warp_topk_redux(const float *row, int E, int k, 
     const float sum = warp_sum(z);
     out_i = my_i;
     out_w = z / sum;
+}
+
+template <int NJ>
+__device__ __forceinline__ void warp_topk_redux(const float *row, int E, int k, int &out_i, float &out_w) {
+    const int lane = threadIdx.x & 31;
+    // key 0 marks an entry out of range or already taken (no float maps to 0
+    // but a NaN with every bit set)
+    uint32_t key[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const int e = lane + 32 * j;
+        key[j] = e < E ? order_key(__ldcg(row + e) + 0.0f) : 0u;  // -0 keys as +0
+    }
+    warp_topk_rounds<NJ>(key, k, out_i, out_w);
+}
+
+// Top-k of one row, first stage, by every warp of the CTA: warp w ranks the
+// 32 logits of each chunk c = w, w + warps, ... (ids 32c .. 32c + 31, one per
+// lane) and keeps its k best as candidates c * k .. c * k + k - 1, in rank
+// order (equal keys lowest id first; key 0 and id -1 past the chunk's
+// entries).  A row's top k are among its chunks' candidates, and because the
+// chunks follow the ids, a lower candidate position among equal keys is a
+// lower id: warp_topk_rounds over the candidate keys, with positions for ids,
+// then makes exactly the choices warp_topk_redux makes over the whole row.
+// k <= 31.
+__device__ __forceinline__ void cta_topk_candidates(const float *row, int E, int k, uint32_t *ckey, int *cid) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nc = (E + 31) / 32;
+    for (int c = warp; c < nc; c += nw) {
+        const int e = 32 * c + lane;
+        uint32_t key = e < E ? order_key(__ldcg(row + e) + 0.0f) : 0u;  // -0 keys as +0
+        for (int r = 0; r < k; ++r) {
+            const uint32_t wk = __reduce_max_sync(0xffffffffu, key);
+            const uint32_t id = (key != 0u && key == wk) ? static_cast<uint32_t>(e) : 0xffffffffu;
+            const uint32_t wi = __reduce_min_sync(0xffffffffu, id);
+            if (lane == r) {
+                ckey[c * k + r] = wk;
+                cid[c * k + r] = static_cast<int>(wi);
+            }
+            if (static_cast<uint32_t>(e) == wi) key = 0u;
+        }
+    }
 }
 
 // Top-k of T rows by a whole CTA: one warp per row (E <= 1024, k <= 32).
