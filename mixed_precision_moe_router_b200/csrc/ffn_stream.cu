@@ -283,20 +283,21 @@ __device__ __forceinline__ TileAcc warp_tile(const uint8_t *stage, const Geo G, 
                 if (g < (nt == 0 ? ncol0 : ncol1))
                     X[bb] = *reinterpret_cast<const uint4 *>(xg + nt * 8 * cs + (b + bb) * 64);
             }
-            // four independent products: two k16 halves of two blocks
-            float c[4][4] = {};
+            // a block's two k16 halves chained through the accumulator (the
+            // products are exact), the two blocks independent
+            float c[2][4] = {};
 #pragma unroll
             for (int bb = 0; bb < 2; ++bb) {
-                mma16816(c[2 * bb], PA[bb][0], PB[bb][0], PA[bb][1], PB[bb][1], X[bb].x, X[bb].y);
-                mma16816(c[2 * bb + 1], PA[bb][2], PB[bb][2], PA[bb][3], PB[bb][3], X[bb].z, X[bb].w);
+                mma16816(c[bb], PA[bb][0], PB[bb][0], PA[bb][1], PB[bb][1], X[bb].x, X[bb].y);
+                mma16816(c[bb], PA[bb][2], PB[bb][2], PA[bb][3], PB[bb][3], X[bb].z, X[bb].w);
             }
 #pragma unroll
             for (int bb = 0; bb < 2; ++bb) {
                 const float dA = bb ? da.y : da.x, dB = bb ? db.y : db.x;
-                acc[nt][0] = fmaf(dA, c[2 * bb][0] + c[2 * bb + 1][0], acc[nt][0]);
-                acc[nt][1] = fmaf(dA, c[2 * bb][1] + c[2 * bb + 1][1], acc[nt][1]);
-                acc[nt][2] = fmaf(dB, c[2 * bb][2] + c[2 * bb + 1][2], acc[nt][2]);
-                acc[nt][3] = fmaf(dB, c[2 * bb][3] + c[2 * bb + 1][3], acc[nt][3]);
+                acc[nt][0] = fmaf(dA, c[bb][0], acc[nt][0]);
+                acc[nt][1] = fmaf(dA, c[bb][1], acc[nt][1]);
+                acc[nt][2] = fmaf(dB, c[bb][2], acc[nt][2]);
+                acc[nt][3] = fmaf(dB, c[bb][3], acc[nt][3]);
             }
         }
     }
