@@ -1062,7 +1062,9 @@ __device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S
     const int n = (E + 31) / 32 * k;
     int pos_r;
     float w_r;
-    if (n <= 512) warp_topk_candidates<16>(ckey, n, k, pos_r, w_r);
+    // the fewest keys per lane that hold them (a smaller tree per round)
+    if (n <= 256) warp_topk_candidates<8>(ckey, n, k, pos_r, w_r);
+    else if (n <= 512) warp_topk_candidates<16>(ckey, n, k, pos_r, w_r);
     else warp_topk_candidates<32>(ckey, n, k, pos_r, w_r);
     // (position -1, as id -1 before, only when fewer than k keys are valid)
     const int e_r = lane < k ? (pos_r >= 0 && pos_r < n ? cid[pos_r] : -1) : 0;

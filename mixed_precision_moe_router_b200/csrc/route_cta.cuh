@@ -162,13 +162,15 @@ __device__ __forceinline__ void cta_topk_candidates(const float *row, int E, int
         uint32_t key = e < E ? order_key(__ldcg(row + e) + 0.0f) : 0u;  // -0 keys as +0
         for (int r = 0; r < k; ++r) {
             const uint32_t wk = __reduce_max_sync(0xffffffffu, key);
-            const uint32_t id = (key != 0u && key == wk) ? static_cast<uint32_t>(e) : 0xffffffffu;
-            const uint32_t wi = __reduce_min_sync(0xffffffffu, id);
+            // the ids rise with the lane: the lowest lane holding the maximum
+            // has the lowest id (-1 when no entry is left)
+            const unsigned m = __ballot_sync(0xffffffffu, key != 0u && key == wk);
+            const int wl = m ? __ffs(m) - 1 : -1;
             if (lane == r) {
                 ckey[c * k + r] = wk;
-                cid[c * k + r] = static_cast<int>(wi);
+                cid[c * k + r] = wl >= 0 ? 32 * c + wl : -1;
             }
-            if (static_cast<uint32_t>(e) == wi) key = 0u;
+            if (lane == wl) key = 0u;
         }
     }
 }
