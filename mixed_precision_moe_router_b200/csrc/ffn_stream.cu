@@ -262,43 +262,29 @@ __device__ __forceinline__ TileAcc warp_tile(const uint8_t *stage, const Geo G, 
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    // one pair of blocks per iteration: a larger unroll measured slower, its
-    // extra code competing with the other roles' for the instruction cache
+    // one block per iteration: the smallest loop body (a larger unroll
+    // measured slower, its code competing with the other roles' for the
+    // instruction cache)
 #pragma unroll 1
-    for (int b = b0; b < b1; b += 2) {
-        const float2 da = half2_to_float2(*reinterpret_cast<const uint32_t *>(scl + rA * G.sb + ((2 * b) ^ sxa)));
-        const float2 db = half2_to_float2(*reinterpret_cast<const uint32_t *>(scl + rB * G.sb + ((2 * b) ^ sxb)));
-        uint32_t PA[2][4], PB[2][4];
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-            dequant8<BITS, PAD>(stage, G, rA, xa, b + bb, t, PA[bb]);
-            dequant8<BITS, PAD>(stage, G, rB, xb, b + bb, t, PB[bb]);
-        }
+    for (int b = b0; b < b1; ++b) {
+        const float dA = __half2float(*reinterpret_cast<const __half *>(scl + rA * G.sb + ((2 * b) ^ sxa)));
+        const float dB = __half2float(*reinterpret_cast<const __half *>(scl + rB * G.sb + ((2 * b) ^ sxb)));
+        uint32_t PA[4], PB[4];
+        dequant8<BITS, PAD>(stage, G, rA, xa, b, t, PA);
+        dequant8<BITS, PAD>(stage, G, rB, xb, b, t, PB);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            uint4 X[2];
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                X[bb] = make_uint4(0u, 0u, 0u, 0u);
-                if (g < (nt == 0 ? ncol0 : ncol1))
-                    X[bb] = *reinterpret_cast<const uint4 *>(xg + nt * 8 * cs + (b + bb) * 64);
-            }
-            // a block's two k16 halves chained through the accumulator (the
-            // products are exact), the two blocks independent
-            float c[2][4] = {};
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                mma16816(c[bb], PA[bb][0], PB[bb][0], PA[bb][1], PB[bb][1], X[bb].x, X[bb].y);
-                mma16816(c[bb], PA[bb][2], PB[bb][2], PA[bb][3], PB[bb][3], X[bb].z, X[bb].w);
-            }
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                const float dA = bb ? da.y : da.x, dB = bb ? db.y : db.x;
-                acc[nt][0] = fmaf(dA, c[bb][0], acc[nt][0]);
-                acc[nt][1] = fmaf(dA, c[bb][1], acc[nt][1]);
-                acc[nt][2] = fmaf(dB, c[bb][2], acc[nt][2]);
-                acc[nt][3] = fmaf(dB, c[bb][3], acc[nt][3]);
-            }
+            uint4 X = make_uint4(0u, 0u, 0u, 0u);
+            if (g < (nt == 0 ? ncol0 : ncol1)) X = *reinterpret_cast<const uint4 *>(xg + nt * 8 * cs + b * 64);
+            // the block's two k16 halves chained through the accumulator (the
+            // products are exact)
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma16816(c, PA[0], PB[0], PA[1], PB[1], X.x, X.y);
+            mma16816(c, PA[2], PB[2], PA[3], PB[3], X.z, X.w);
+            acc[nt][0] = fmaf(dA, c[0], acc[nt][0]);
+            acc[nt][1] = fmaf(dA, c[1], acc[nt][1]);
+            acc[nt][2] = fmaf(dB, c[2], acc[nt][2]);
+            acc[nt][3] = fmaf(dB, c[3], acc[nt][3]);
         }
     }
     return out;
