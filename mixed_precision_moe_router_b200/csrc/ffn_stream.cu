@@ -189,11 +189,26 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
     return d;
 }
 
+// Byte offsets in a staged tile of thread t's codes of block b in row r: the
+// code word (8 bytes for 8-bit codes, 4 for 4-bit and FP4, the low-plane u16
+// for 3-bit) and, for 3-bit codes, the high-plane byte.
 template <int BITS, bool PAD>
-__device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int r, int xr, int b, int t,
-                                         uint32_t (&P)[4]) {
+__device__ __forceinline__ void code_offsets(const Geo &G, int r, int xr, int b, int t, int &o0, int &o1) {
     if constexpr (BITS == 8) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(tile + tile_off<PAD>(32 * b + 8 * t, r, G, xr));
+        o0 = tile_off<PAD>(32 * b + 8 * t, r, G, xr);
+    } else if constexpr (BITS == 4 || BITS == kBitsFp4) {
+        o0 = tile_off<PAD>(16 * b + 4 * t, r, G, xr);
+    } else {
+        o0 = tile_off<PAD>(8 * b + 2 * t, r, G, xr);
+        o1 = tile_off<PAD>(G.K / 4 + 4 * b + t, r, G, xr);
+    }
+}
+
+// The codes at those offsets as four half2 of exact integers q.
+template <int BITS>
+__device__ __forceinline__ void dequant8(const uint8_t *tile, int o0, int o1, uint32_t (&P)[4]) {
+    if constexpr (BITS == 8) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(tile + o0);
         const uint32_t u0 = w.x ^ 0x80808080u, u1 = w.y ^ 0x80808080u;  // c = q + 128
         constexpr uint32_t kBias = 0x64806480u;                         // 1024 + 128
         P[0] = hsub2(prmt(u0, 0x64646464u, 0x4140u), kBias);
@@ -202,7 +217,7 @@ __device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int 
         P[3] = hsub2(prmt(u1, 0x64646464u, 0x4342u), kBias);
     } else if constexpr (BITS == 4) {
         // nibble i of the word at byte 16b + 4t is weight 8t + i (c = q + 8)
-        const uint32_t v = *reinterpret_cast<const uint32_t *>(tile + tile_off<PAD>(16 * b + 4 * t, r, G, xr));
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(tile + o0);
         const uint32_t v8 = v >> 8;
         P[0] = hsub2((v & 0x000F000Fu) | 0x64006400u, 0x64086408u);   // 1024 + c - 1032
         P[1] = hsub2((v & 0x00F000F0u) | 0x54005400u, 0x54805480u);   // 64 + c - 72
@@ -211,12 +226,12 @@ __device__ __forceinline__ void dequant8(const uint8_t *tile, const Geo &G, int 
     } else if constexpr (BITS == kBitsFp4) {
         // FP4 codes in the 4-bit layout: nibble i of the word at byte 16b + 4t
         // is weight 8t + i
-        fp4_pairs(*reinterpret_cast<const uint32_t *>(tile + tile_off<PAD>(16 * b + 4 * t, r, G, xr)), P);
+        fp4_pairs(*reinterpret_cast<const uint32_t *>(tile + o0), P);
     } else {
         // low plane: bits 0-1 of weight 8t+i at bit 2i of the u16 at byte 8b+2t;
         // high plane: bit 2 at bit i of byte K/4 + 4b + t (c = q + 4)
-        const uint32_t lo16 = *reinterpret_cast<const uint16_t *>(tile + tile_off<PAD>(8 * b + 2 * t, r, G, xr));
-        const uint32_t hb = tile[tile_off<PAD>(G.K / 4 + 4 * b + t, r, G, xr)];
+        const uint32_t lo16 = *reinterpret_cast<const uint16_t *>(tile + o0);
+        const uint32_t hb = tile[o1];
         const uint32_t X = prmt(lo16, 0u, 0x4140u);  // weights i and i+4 16 bits apart
         const uint32_t Y = hb * 0x4004u;             // hb << 2 | hb << 14
         P[0] = hsub2((X & 0x00030003u) | (Y & 0x00040004u) | 0x64006400u, 0x64046404u);           // 1024 + c - 1028
@@ -253,10 +268,15 @@ __device__ __forceinline__ TileAcc warp_tile(const uint8_t *stage, const Geo G, 
     TileAcc out;
     float (&acc)[2][4] = out.acc;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int xa = row_x<PAD>(rA, G), xb = row_x<PAD>(rB, G);
+    const int xa = row_x<PAD>(rA, G);
+    // Rows rA and rB are a multiple of 8 rows apart, and every layout's
+    // swizzle of a row depends on the row mod 8: row rB's codes and scales
+    // sit a fixed distance after row rA's.
+    const int dcode = tile_off<PAD>(0, rB, G, row_x<PAD>(rB, G)) - tile_off<PAD>(0, rA, G, xa);
+    const uint8_t *stageB = stage + dcode;
     // scales: [row][sb] after the codes, swizzled at width Ws (or plain)
-    const uint8_t *scl = stage + G.cb;
-    const int sxa = G.Ws ? swz(rA, G.Ws) : 0, sxb = G.Ws ? swz(rB, G.Ws) : 0;
+    const uint8_t *sclA = stage + G.cb + rA * G.sb, *sclB = sclA + (rB - rA) * G.sb;
+    const int sxa = G.Ws ? swz(rA, G.Ws) : 0;
     const uint8_t *xg = xf + g * cs + t * 16;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -267,11 +287,14 @@ __device__ __forceinline__ TileAcc warp_tile(const uint8_t *stage, const Geo G, 
     // instruction cache)
 #pragma unroll 1
     for (int b = b0; b < b1; ++b) {
-        const float dA = __half2float(*reinterpret_cast<const __half *>(scl + rA * G.sb + ((2 * b) ^ sxa)));
-        const float dB = __half2float(*reinterpret_cast<const __half *>(scl + rB * G.sb + ((2 * b) ^ sxb)));
+        const int so = (2 * b) ^ sxa;
+        const float dA = __half2float(*reinterpret_cast<const __half *>(sclA + so));
+        const float dB = __half2float(*reinterpret_cast<const __half *>(sclB + so));
+        int o0, o1 = 0;
+        code_offsets<BITS, PAD>(G, rA, xa, b, t, o0, o1);
         uint32_t PA[4], PB[4];
-        dequant8<BITS, PAD>(stage, G, rA, xa, b, t, PA);
-        dequant8<BITS, PAD>(stage, G, rB, xb, b, t, PB);
+        dequant8<BITS>(stage, o0, o1, PA);
+        dequant8<BITS>(stageB, o0, o1, PB);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             uint4 X = make_uint4(0u, 0u, 0u, 0u);
