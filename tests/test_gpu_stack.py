@@ -128,3 +128,57 @@ def test_stack_tiny_configuration():
         torch.cuda.synchronize()
         _check_stream(got, x, res)
         x = res["x_next"].astype(np.float32)
+
+
+def test_one_token_top_k_ties_resolve_to_the_lowest_id(decode_layers):
+    """The one-token routing inside the kernels ranks 32-logit chunks first,
+    then their candidates.  Three experts in different chunks are given the
+    router row and bias of the k-th choice, so that they tie exactly for the
+    last place: the lowest id must take it ([P1] "step 4": the router picks
+    the best k; ties go to the lower id).  The stack and the fused layer path
+    are checked against the oracle's layer, which a wrong pick fails (another
+    expert's output)."""
+    cfg, layers, routers = decode_layers
+    k, E = cfg.k, cfg.E
+    wr0, bias0 = routers[0]
+    seed = inputs.layer_seed(cfg, 0)
+    for s in range(20):  # a token whose k-th logit is clear of its neighbours
+        x = inputs.activations(1, cfg.H, seed=inputs.X_SEED + 700 + s, device=DEV)
+        n = B.rmsnorm(x)
+        idx, _, lg = B.router_topk(n, wr0, bias0, k, want_logits=True)
+        lg = lg[0].double().cpu()
+        srt = torch.sort(lg, descending=True).values
+        gap = float(min(srt[k - 2] - srt[k - 1], srt[k - 1] - srt[k]))
+        if gap > 1e-3 * float(srt[k - 1].abs()) + 1e-4:
+            break
+    else:
+        pytest.skip("no token with a clear k-th logit")
+    chosen = set(idx[0].tolist())
+    ek = int(idx[0, k - 1])
+    others = [e for e in range(E) if e not in chosen and e // 32 != ek // 32]
+    ea, eb = others[0], others[-1]  # the lowest and highest ids outside ek's chunk
+    win = min(ea, ek, eb)
+    wr = wr0.clone()
+    wr[ea] = wr0[ek]
+    wr[eb] = wr0[ek]
+    bias = None
+    if bias0 is not None:
+        bias = bias0.clone()
+        bias[ea] = bias0[ek]
+        bias[eb] = bias0[ek]
+    xn = x.float().cpu().numpy()
+    nn = oracle.rms_norm(xn).astype(np.float32)
+    wrn, bn = wr.float().cpu().numpy(), None if bias is None else bias.cpu().numpy()
+    oidx, _ = oracle.select_topk(oracle.router_logits(nn, wrn, bn), k)
+    tied = {ea, ek, eb}
+    assert win in oidx[0] and not (tied - {win}) & set(oidx[0].tolist())  # the tie as built
+    ox = Hh.OracleExperts(cfg, seed, DEV)
+    ox.prefetch(list(oidx.reshape(-1)) + [E])
+    res = oracle.moe_layer(nn, wrn, bn, k, ox, ox.shared(), cfg.H, cfg.I, residual=xn)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    got = B.stack_forward(B.Stack([layers[0]], [(wr, bias)]), x, k, status=status)
+    _, x_next, _ = B.layer_forward(layers[0], wr, bias, n, k, residual=x, mode=B.FFN_GEMV, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    _check_stream(got, xn, res)
+    _check_stream(x_next, xn, res)
