@@ -1142,12 +1142,12 @@ __device__ __forceinline__ void route_plan_one(const FfnParams &p, StreamSmem &S
 // also writes the routing outputs.  Returns 0 when the grid barrier gave up,
 // 2 when the schedule is built too (one token), else 1.
 __device__ __forceinline__ int route_in_cta(const FfnParams &p, StreamSmem &S, const uint16_t *x_s, int *act_s,
-                                          int *off_s, const PrologueScratch &ps) {
+                                          int *off_s, const PrologueScratch &ps, const uint16_t *wr_s = nullptr) {
     const int T = p.T, E = p.E, k = p.k, H = p.w.H, S_ = T * k;
     // logits of experts [E * c / G, E * (c + 1) / G), all warps
     const int e0 = static_cast<int>(static_cast<long long>(E) * blockIdx.x / gridDim.x);
     const int e1 = static_cast<int>(static_cast<long long>(E) * (blockIdx.x + 1) / gridDim.x);
-    cta_logits(x_s, T, H, E, p.route.wr, p.route.bias, e0, e1,
+    cta_logits(x_s, T, H, E, p.route.wr, wr_s, p.route.bias, e0, e1,
                reinterpret_cast<float *>(S.ring + ps.cand), p.route.logits);
     int *barrier_ok = S.range + 7;
     __syncthreads();  // every thread's logits are written before thread 0 arrives
@@ -1626,6 +1626,7 @@ struct StackParams {
     long long wait_limit;
     int skip_publish;  // test hook, as in FfnParams (-1: none)
     int ring_bytes;
+    int wr_stage;      // ring offset of this CTA's router rows staged for the logits, or -1
 };
 
 // Bytes past the shared stream layout: this layer's parameters, its top-k
@@ -1750,6 +1751,16 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
         // descriptor below is read)
         for (int c = threadIdx.x; c < T * H / 8; c += blockDim.x)
             cp_async_16b(x_s + 8 * c, xl + 8 * static_cast<size_t>(c));
+        // and this CTA's router rows (they do not depend on x), so that the
+        // logits read them from shared memory after the norm
+        const int re0 = static_cast<int>(static_cast<long long>(E) * blockIdx.x / gridDim.x);
+        const int re1 = static_cast<int>(static_cast<long long>(E) * (blockIdx.x + 1) / gridDim.x);
+        uint16_t *wr_s = P.wr_stage >= 0 ? reinterpret_cast<uint16_t *>(S.ring + P.wr_stage) : nullptr;
+        if (wr_s) {
+            const uint16_t *rows = Ld.wr + static_cast<size_t>(re0) * H;
+            for (int c = threadIdx.x; c < (re1 - re0) * H / 8; c += blockDim.x)
+                cp_async_16b(wr_s + 8 * c, rows + 8 * static_cast<size_t>(c));
+        }
         // this layer's weights descriptor, the schedule's view of its shelves and
         // their table pointers into shared memory (a word per thread, one round)
         {
@@ -1774,7 +1785,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) stack_kernel(const __grid_co
             const bool xbad = build_xall(p, reinterpret_cast<const uint8_t *>(x_s), S.xall);
             if (__any_sync(0xffffffffu, xbad) && (threadIdx.x & 31) == 0) status_or(P.status, MOE_STATUS_FP16_RANGE);
         }
-        const int routed = route_in_cta(p, S, x_s, act_s, off_s, ps);
+        const int routed = route_in_cta(p, S, x_s, act_s, off_s, ps, wr_s);
         if (!routed) {
             alive = false;
             break;
@@ -1954,6 +1965,18 @@ cudaError_t moe_launch_stack(const void *layers, int n_layers, int T, int k, int
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if ((E + sms - 1) / sms > moe::kMaxExpertShare) return cudaErrorInvalidConfiguration;
+    // the router rows of a CTA (at most ceil(E / grid)) staged in the ring's
+    // scratch after the routing lists, when they fit, for one or two tokens
+    // (with more, the norm already covers their latency and the extra copies
+    // measured slower)
+    if (T > 2) {
+        P.wr_stage = -1;
+    } else {
+        const int max_slots = (T * k < E ? T * k : E) + 1;
+        const size_t at = moe::align16(moe::prologue_scratch(H, T, k, E, max_slots, true).end);
+        const size_t need = at + static_cast<size_t>((E + sms - 1) / sms) * H * sizeof(uint16_t);
+        P.wr_stage = need <= static_cast<size_t>(ring) ? static_cast<int>(at) : -1;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(moe::kBlockThreads);

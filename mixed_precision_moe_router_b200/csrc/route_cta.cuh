@@ -199,15 +199,18 @@ __device__ __forceinline__ void cta_topk_rows(const float *logits, int T, int E,
 //   x_s bf16 [T][H] in shared memory; part: 4 * (e1 - e0) * NT floats of
 //   shared scratch; logits fp32 [T][E] (global).  Ends with a barrier.
 // ---------------------------------------------------------------------------
-template <int NT>
-__device__ __forceinline__ void cta_logits_nt(const uint16_t *x_s, int T, int H, int E, const uint16_t *wr,
+// rows: the router rows e0 .. e1 - 1 (row e0 at rows[0]), in global memory or,
+// with SMEM, staged in shared memory; the values and their order of use are
+// the same either way.
+template <int NT, bool SMEM>
+__device__ __forceinline__ void cta_logits_nt(const uint16_t *x_s, int T, int H, int E, const uint16_t *rows,
                                               const float *bias, int e0, int e1, float *part, float *logits) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int vec = H / 8, qv = vec / 4;  // 16-byte chunks per row and per quarter
     const int ntask = 4 * (e1 - e0);
     for (int task = warp; task < ntask; task += nwarps) {
         const int el = task >> 2, q = task & 3;
-        const uint16_t *row = wr + static_cast<size_t>(e0 + el) * H;
+        const uint16_t *row = rows + static_cast<size_t>(el) * H;
         float acc[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[t] = 0.f;
@@ -216,7 +219,8 @@ __device__ __forceinline__ void cta_logits_nt(const uint16_t *x_s, int T, int H,
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int c = c0 + lane + 32 * u;
-                wv[u] = c < (q + 1) * qv ? ld_stream_v4(row + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+                wv[u] = c < (q + 1) * qv ? (SMEM ? *reinterpret_cast<const uint4 *>(row + 8 * c) : ld_stream_v4(row + 8 * c))
+                                         : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -259,14 +263,27 @@ __device__ __forceinline__ void cta_logits_nt(const uint16_t *x_s, int T, int H,
 
 __host__ __device__ __forceinline__ int cta_logits_nt_for(int T) { return T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : (T <= 8 ? 8 : 16))); }
 
+// wr_s: this CTA's rows staged in shared memory, or null to read wr.
 __device__ __forceinline__ void cta_logits(const uint16_t *x_s, int T, int H, int E, const uint16_t *wr,
-                                           const float *bias, int e0, int e1, float *part, float *logits) {
+                                           const uint16_t *wr_s, const float *bias, int e0, int e1, float *part,
+                                           float *logits) {
+    const uint16_t *rows = wr + static_cast<size_t>(e0) * H;
+    if (wr_s) {
+        switch (cta_logits_nt_for(T)) {
+            case 1: cta_logits_nt<1, true>(x_s, T, H, E, wr_s, bias, e0, e1, part, logits); break;
+            case 2: cta_logits_nt<2, true>(x_s, T, H, E, wr_s, bias, e0, e1, part, logits); break;
+            case 4: cta_logits_nt<4, true>(x_s, T, H, E, wr_s, bias, e0, e1, part, logits); break;
+            case 8: cta_logits_nt<8, true>(x_s, T, H, E, wr_s, bias, e0, e1, part, logits); break;
+            default: cta_logits_nt<16, true>(x_s, T, H, E, wr_s, bias, e0, e1, part, logits); break;
+        }
+        return;
+    }
     switch (cta_logits_nt_for(T)) {
-        case 1: cta_logits_nt<1>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
-        case 2: cta_logits_nt<2>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
-        case 4: cta_logits_nt<4>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
-        case 8: cta_logits_nt<8>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
-        default: cta_logits_nt<16>(x_s, T, H, E, wr, bias, e0, e1, part, logits); break;
+        case 1: cta_logits_nt<1, false>(x_s, T, H, E, rows, bias, e0, e1, part, logits); break;
+        case 2: cta_logits_nt<2, false>(x_s, T, H, E, rows, bias, e0, e1, part, logits); break;
+        case 4: cta_logits_nt<4, false>(x_s, T, H, E, rows, bias, e0, e1, part, logits); break;
+        case 8: cta_logits_nt<8, false>(x_s, T, H, E, rows, bias, e0, e1, part, logits); break;
+        default: cta_logits_nt<16, false>(x_s, T, H, E, rows, bias, e0, e1, part, logits); break;
     }
 }
 
