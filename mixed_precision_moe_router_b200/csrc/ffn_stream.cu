@@ -70,6 +70,7 @@ constexpr int kRedBytes = kWarps * 32 * 16;  // one item's partials: a float4 pe
 constexpr int kMaxSmemEntries = 2048;        // sorted slot ids kept in shared memory up to this many
 constexpr int kMaxExpertShare = 16;          // router rows a CTA computes when it routes the batch itself
 constexpr int kDealtMaxTokens = 2;          // tiles dealt out in turn up to this many tokens (plan_in_cta)
+constexpr long long kFirstTileHeadStart = 4000;  // cycles the producer gives a layer's first tiles (run_producer)
 
 // B-operand buffers: with dealt tiles every down tile has an operand of its
 // own, so the loader gets room to build several ahead (they are small then).
@@ -749,6 +750,10 @@ __device__ __forceinline__ void run_producer(const FfnParams &p, const StreamMap
             const int d = (i0 + j) % kND;
             st[d] = end - sz;
             en[d] = end;
+            // the first tile of each compute group goes first; the rest follow
+            // once the first has landed (at most about 2 us later), so that
+            // compute starts before the whole burst of every CTA has arrived
+            if (j >= kGroups) mbar_wait_limit(&S.full[i0 % kND], (i0 / kND) & 1, kFirstTileHeadStart);
             issue_tile(p, M, S, phase, a, b, S.ring + (end - sz), &S.full[d]);
         }
     }
