@@ -70,7 +70,7 @@ constexpr int kRedBytes = kWarps * 32 * 16;  // one item's partials: a float4 pe
 constexpr int kMaxSmemEntries = 2048;        // sorted slot ids kept in shared memory up to this many
 constexpr int kMaxExpertShare = 16;          // router rows a CTA computes when it routes the batch itself
 constexpr int kDealtMaxTokens = 2;          // tiles dealt out in turn up to this many tokens (plan_in_cta)
-constexpr long long kFirstTileHeadStart = 4000;  // cycles the producer gives a layer's first tiles (run_producer)
+constexpr long long kFirstTileHeadStart = 8000;  // cycles the producer gives a layer's first tiles (run_producer)
 
 // B-operand buffers: with dealt tiles every down tile has an operand of its
 // own, so the loader gets room to build several ahead (they are small then).
