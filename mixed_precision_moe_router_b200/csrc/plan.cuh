@@ -11,6 +11,8 @@
 // Numbering the tiles of a phase globally as g = slot * nt + tile, each CTA
 // takes the contiguous run of tiles whose start falls in its equal share of
 // the phase's total cost, first of gate_up (phase 0), then of down (phase 1).
+// (For one or two tokens the streaming kernel deals the tiles out in turn
+// instead, CTA c taking g = c, c + grid, ...; see plan_in_cta.)
 #pragma once
 #include "common.cuh"
 
