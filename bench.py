@@ -348,6 +348,13 @@ def stack_touched_bytes(run, layers, routers, stream):
     return ex, rt
 
 
+def decode_config(world, T):
+    """The decode workload as both arms report it."""
+    return {"workload": f"decode: {N_LAYERS} stacked MoE layers (H=2048, I=512, E=512, top-10 + 1 shared, "
+                        "shelves 128x8-bit/192x4-bit/192x3-bit, Zipf routing), 1 token per step per GPU",
+            "global_batch": world * T, "layers": N_LAYERS, "parallelism": f"replicas{world}"}
+
+
 def run_native(args, rank, world):
     from mixed_precision_moe_router_b200 import binding as B
     device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -439,11 +446,9 @@ def run_native(args, rank, world):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "int codes x fp16 activations, fp32 accumulation; bf16 residual stream",
         "data": "synthetic",
-        "config": {"workload": f"decode: {N_LAYERS} stacked MoE layers (H=2048, I=512, E=512, top-10 + 1 shared, "
-                               "shelves 128x8-bit/192x4-bit/192x3-bit, Zipf routing), 1 token per step per GPU",
-                   "global_batch": world * T, "layers": N_LAYERS, "parallelism": f"replicas{world}",
-                   "l2": f"inputs larger than L2: {sum(ex) / 1e9:.2f} GB of expert blocks touched per step",
-                   "launch": f"one launch of the persistent stack kernel per step (all {N_LAYERS} layers)"},
+        "config": dict(decode_config(world, T),
+                       l2=f"inputs larger than L2: {sum(ex) / 1e9:.2f} GB of expert blocks touched per step",
+                       launch=f"one launch of the persistent stack kernel per step (all {N_LAYERS} layers)"),
         "roofline": {"bound": "hbm", "kernel": f"stack kernel: one decode step through {N_LAYERS} layers",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": traffic, "peak_kind": peak_kind,
@@ -682,7 +687,7 @@ def main():
             "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / v, 3) if v else None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": "decode: 48 stacked MoE layers, 1 token (oracle sample)"},
+            "data": "synthetic", "config": decode_config(1, 1),
             "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
