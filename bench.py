@@ -40,23 +40,38 @@ N_LAYERS = inputs.N_STACK  # --layers changes it (profiling runs only)
 # Sources the persistent decode kernel is compiled from.  The DRAM traffic
 # below was captured (ncu dram__bytes_read.sum + dram__bytes_write.sum, cold
 # L2, one launch of a 4-layer stack, one token) for the sources with this
-# digest; when they change, the bench reports traffic as null until the
-# capture is taken again.
+# digest (of their code, comments ignored); when the code changes, the bench
+# reports traffic as null until the capture is taken again.
 STACK_SOURCES = ("csrc/ffn_stream.cu", "csrc/ffn.cuh", "csrc/plan.cuh", "csrc/route_cta.cuh", "csrc/sync.cuh",
                  "csrc/common.cuh")
-STACK_TRAFFIC = {"digest": "32c72f17e5f3b04c", "dram_bytes": 120261120 + 4708352, "algorithmic_bytes": 118497280, "layers": 4}
+STACK_TRAFFIC = {"digest": "02ebced11b752ae5", "dram_bytes": 120261120 + 4708352, "algorithmic_bytes": 118497280, "layers": 4}
 # The same for the prefill FFN call's two GEMM launches (gate_up and down; ncu
 # DRAM read + write of one call of the 4096-token workload).
 PREFILL_SOURCES = ("csrc/ffn_gemm_sm100.cu", "csrc/ffn.cuh", "csrc/plan.cuh", "csrc/sync.cuh", "csrc/common.cuh")
-PREFILL_TRAFFIC = {"digest": "4d2e09ea5eba988b", "dram_bytes": 765532672 + 40060416 + 391464192 + 315183104}
+PREFILL_TRAFFIC = {"digest": "929055e67f191e37", "dram_bytes": 765532672 + 40060416 + 391464192 + 315183104}
 
 
-def source_digest(files):
+def strip_comments(src):
+    """C++ source without its comments and blank lines (what the compiler sees
+    of it, up to layout), so that a comment edit keeps a capture valid."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
+def source_digest(files, read=None):
+    """Digest of the kernel sources' code (comments ignored).  read(f) gives a
+    file's text; by default the working tree's."""
     import hashlib
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "mixed_precision_moe_router_b200", f), "rb") as fh:
-            h.update(fh.read())
+        if read is None:
+            with open(os.path.join(ROOT, "mixed_precision_moe_router_b200", f), encoding="utf-8") as fh:
+                text = fh.read()
+        else:
+            text = read(f)
+        h.update(strip_comments(text).encode())
     return h.hexdigest()[:16]
 
 
