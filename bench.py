@@ -561,7 +561,9 @@ def tier_planner_curve(layer0, router, stream, fractions=(0.75, 1.0, 1.3, 1.6)):
     each byte budget (a fraction of the configured 128/192/192 shelves), and
     that plan's layer built (experts renumbered so that each shelf is one
     contiguous id range) and its one-token FFN call timed, next to the
-    configured shelves' own."""
+    configured shelves' own.  Then the pages' down ladder planned at the
+    configured size: levels that pair a gate_up with a down format (3-bit
+    with FP4, 4/4, 8/8), errors per matrix from the same quantiser."""
     from mixed_precision_moe_router_b200 import binding as B
     from mixed_precision_moe_router_b200 import ep, planner
     cfg = inputs.DECODE
@@ -605,10 +607,36 @@ def tier_planner_curve(layer0, router, stream, fractions=(0.75, 1.0, 1.3, 1.6)):
                     "permuted_ids": order != list(range(cfg.E))})
         del layer
         out.append(row)
+    # the pages' ladder: each level a (gate_up, down) format pair, the rarest
+    # experts with 3-bit gate_up and FP4 down, planned at the configured size
+    ladder = ((3, B.FP4), (4, 4), (8, 8))
+    sqm = {}
+    for fmt in (3, 4, 8, B.FP4):
+        for name, w in (("gu", wgu.contiguous()), ("dn", wdn.contiguous())):
+            qs, sc = B.quantize(w, fmt)
+            back, _ = B.dequantize(qs, sc, w.shape[1], fmt)
+            sqm[(name, fmt)] = float(((back - w).double() ** 2).sum())
+    lerr = [{lv: sqm[("gu", lv[0])] + sqm[("dn", lv[1])] for lv in ladder} for _ in range(cfg.E)]
+    lnb = {lv: ep.expert_bytes(cfg.H, cfg.I, lv) for lv in ladder}
+    ladder_rows = []
+    for frac in (0.75, 1.0):
+        plan = planner.plan_tiers(freq, lerr, lnb, frac * ref_bytes, bits=ladder)
+        order, shelves = planner.shelves_from_bits(plan)
+        perm = torch.tensor(order, device=dev)
+        src = (lambda c, sd, e, d, order=order: inputs.expert_source(c, sd, order[e] if e < c.E else e, d))
+        layer = B.build_layer(cfg, seed, dev, source=src, tier_ranges=shelves)
+        prouter = (wr[perm].contiguous(), None if bias is None else bias[perm].contiguous())
+        fpl = ffn_profile([layer] * len(tokens), [prouter] * len(tokens), tokens, stream)
+        del layer
+        ladder_rows.append({
+            "budget_gb": round(frac * ref_bytes / 1e9, 3), "layer_gb": round(planner.plan_bytes(plan, lnb) / 1e9, 3),
+            "shelves": {f"{g}/{'fp4' if d == B.FP4 else d} (gate_up/down)": n for (g, d), _, n in shelves},
+            "expected_error_vs_configured": round(planner.expected_error(plan, freq, lerr) / ref_err, 4),
+            "ffn_us_T1": round(fpl["ms"] * 1e3, 2), "touched_mb_T1": round(fpl["bytes"] / 1e6, 2)})
     fp = ffn_profile([layer0] * len(tokens), [router] * len(tokens), tokens, stream)
     return {"configured": {"layer_gb": round(ref_bytes / 1e9, 3), "shelves": {f"{b}-bit": n for b, _, n in cfg.tier_ranges()},
                            "ffn_us_T1": round(fp["ms"] * 1e3, 2), "touched_mb_T1": round(fp["bytes"] / 1e6, 2)},
-            "plans": out}
+            "plans": out, "down_ladder_plans": ladder_rows}
 
 
 class OracleStack:

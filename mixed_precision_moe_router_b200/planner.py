@@ -20,6 +20,12 @@ The library stores each precision as one shelf covering a contiguous id range
 and returns the permutation together with the shelf ranges; when the
 planned precisions already fall with the expert id (hot experts first, as
 their ids are popularity ranks) the permutation is the identity.
+
+A level need not be one width: the pages' repacker gives the down
+projections a ladder of their own (`--gu Q6_K,IQ4_XS,IQ3_XXS` beside `--dn
+Q8_0,IQ4_NL,MXFP4`), so a level can be a (gate_up, down) format pair such as
+(3, 5) for 3-bit gate_up with FP4 down; err and nbytes are then keyed by the
+pairs, and the levels are ranked by their bytes.
 """
 import heapq
 
@@ -32,7 +38,7 @@ def plan_tiers(freq, err, nbytes, budget, bits=BITS):
     expert's expected error and bytes.  Raises if even the lowest precision
     does not fit."""
     E = len(freq)
-    bits = tuple(sorted(bits))
+    bits = tuple(sorted(bits, key=lambda b: nbytes[b]))  # ascending bytes
     level = [0] * E
     used = sum(nbytes[bits[0]] for _ in range(E))
     if used > budget:
@@ -73,9 +79,11 @@ def expected_error(plan, freq, err):
 
 def shelves_from_bits(plan):
     """(order, shelves): order[new_id] = old expert id, sorted by precision
-    (highest first) then id; shelves = [(bits, first, count)] over the new ids,
-    one per precision in use."""
-    order = sorted(range(len(plan)), key=lambda e: (-plan[e], e))
+    (highest first, widths or format pairs compared as values) then id;
+    shelves = [(bits, first, count)] over the new ids, one per precision in
+    use."""
+    # a stable sort in descending order keeps equal precisions in id order
+    order = sorted(range(len(plan)), key=lambda e: plan[e], reverse=True)
     shelves = []
     for new, e in enumerate(order):
         b = plan[e]

@@ -102,3 +102,36 @@ def test_beats_the_configured_split_at_its_size():
     plan = planner.plan_tiers(f, err, NB, planner.plan_bytes(split, NB))
     assert planner.plan_bytes(plan, NB) <= planner.plan_bytes(split, NB)
     assert planner.expected_error(plan, f, err) < planner.expected_error(split, f, err)
+
+
+def test_format_pair_levels_plan_the_down_ladder():
+    """Levels that are (gate_up, down) format pairs, as in the pages' repacker
+    ladder (3-bit gate_up with FP4 down, 4/4, 8/8): the plan fits the
+    budget, is maximal, falls with the id under equal error models, and its
+    shelves are format-pair ranges in the library's order."""
+    FP4 = 5
+    levels = ((3, FP4), (4, 4), (8, 8))
+    nb = {lv: ep.expert_bytes(H, I, lv) for lv in levels}
+    assert nb[(3, FP4)] < nb[(4, 4)] < nb[(8, 8)]
+    qerr = {3: 1 / 9, 4: 1 / 49, 8: 1 / 127 ** 2, FP4: 1 / 40}  # per weight, in units of amax^2
+    E = 96
+    f = _zipf(E)
+    err = [{lv: 2 * qerr[lv[0]] + qerr[lv[1]] for lv in levels} for _ in range(E)]
+    lo, hi = E * nb[(3, FP4)], E * nb[(8, 8)]
+    B = lo + 0.4 * (hi - lo)
+    plan = planner.plan_tiers(f, err, nb, B, bits=levels)
+    assert planner.plan_bytes(plan, nb) <= B
+    spare = B - planner.plan_bytes(plan, nb)
+    steps = [nb[levels[levels.index(lv) + 1]] - nb[lv] for lv in plan if lv != levels[-1]]
+    assert not steps or min(steps) > spare
+    rank = [levels.index(lv) for lv in plan]
+    assert all(a >= b for a, b in zip(rank, rank[1:]))
+    order, shelves = planner.shelves_from_bits(plan)
+    assert order == list(range(E))
+    assert [lv for lv, _, _ in shelves] == sorted({lv for lv in plan}, reverse=True)
+    assert sum(n for _, _, n in shelves) == E
+    # an unpopular expert with a large error model is lifted and renumbered first
+    err[E - 1] = {lv: 50 * v for lv, v in err[E - 1].items()}
+    plan = planner.plan_tiers(f, err, nb, B, bits=levels)
+    order, shelves = planner.shelves_from_bits(plan)
+    assert plan[E - 1] != levels[0] and order.index(E - 1) < order.index(E - 2)
