@@ -571,3 +571,35 @@ def test_fp4_codes_are_the_nearest_of_all_sixteen():
             even = [c for c in best if (c & 7) % 2 == 0]
             assert codes[r, i] == (even or best)[0], (r, i, v, best)
             assert abs(v - grid[codes[r, i]]) <= (1.0 if abs(v) <= 6 else 2.0)
+
+
+def test_fp4_scale_puts_the_block_max_in_the_top_binade():
+    """The MX scale of a block with E2M1 elements (largest binade [4, 6]) is
+    the power of two X with amax / X in [4, 8): the block's largest weight
+    lands in the elements' top binade or just above it (saturating to 6).  A
+    scale exponent one off in either direction fails this."""
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((64, 256)) * 10.0 ** rng.uniform(-4, 3, size=(64, 1))).astype(np.float32)
+    _, d = oracle.quantize_rows_fp4(w)
+    amax = np.abs(w.reshape(64, 8, 32)).max(axis=2).astype(np.float64)
+    X = 2.0 * d.astype(np.float64)
+    ratio = amax / X
+    assert np.all((ratio >= 4.0) & (ratio < 8.0)), ratio.min()
+    assert np.all(np.log2(X) == np.round(np.log2(X)))  # powers of two
+
+
+def test_fp4_sign_symmetry_and_power_of_two_equivariance():
+    """Negating a block flips the sign bit of every nonzero code and keeps
+    the scale; scaling it by 2^j keeps the codes and scales d by 2^j (away
+    from the scale's clamps)."""
+    rng = np.random.default_rng(9)
+    w = (rng.standard_normal((8, 128)) * 0.05).astype(np.float32)
+    c, d = oracle.quantize_rows_fp4(w)
+    cn, dn = oracle.quantize_rows_fp4(-w)
+    assert np.array_equal(dn, d)
+    nz = (c & 7) != 0
+    assert np.array_equal(cn[nz], c[nz] ^ 8) and np.array_equal(cn[~nz], c[~nz])
+    for j in (-3, 1, 5):
+        cj, dj = oracle.quantize_rows_fp4((w * np.float32(2.0 ** j)).astype(np.float32))
+        assert np.array_equal(cj, c)
+        assert np.array_equal(dj.astype(np.float64), d.astype(np.float64) * 2.0 ** j)
